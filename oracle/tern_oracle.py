@@ -1,0 +1,243 @@
+"""CPU oracle for the weight-only ternary linear layer (W1.58A16).
+
+TEST INFRASTRUCTURE ONLY. Only the tests, the package entry's smoke check and the
+bench's CPU-baseline leg may import this module. The CUDA library never calls it,
+and it shares no code, table or constant generator with the CUDA sources.
+
+Everything here is the plain definition, written out in float64 (or exact
+integers) with numpy, with no blocking, fusion or reordering:
+
+* The representation (what a ternarized weight is):
+  - "Post-Training Ternarization of Qwen3-4B: Capability, Effective Bit Budget,
+    Storage Compression, and Deployment" (arXiv 2609.01962v1), section 4.3
+    (order-2 residual ternarization: ternary planes, each with its own scales),
+    section 4.4 (a salience-selected subset of weights gets a second plane),
+    section 4.5 (block and group size 128) and section 3.1 (weight-only: the
+    activations stay 16-bit).
+  - the Qwen3-8B scale-up paper (arXiv 2609.09240), its representation
+    paragraph: one ternary plane for most weights, a second plane on a
+    salience-selected subset, with per-group scales.
+  The row form of the subset (whole output rows carry the second plane) and
+  the absence of the per-group offset are the readings this library builds;
+  the CUDA path follows the same reading.
+* The product: with weights in {-1, 0, +1} the matrix product reduces to adding
+  and subtracting activations ("Can Ternary LLMs Hit 1.58 Bits per Weight?",
+  promptzone, section "What It Is and How It Works"); the oracle computes it
+  as the dense float64 product of x with the dequantised W (library matmul),
+  which equals that sum of signed activations exactly up to rounding order.
+* Packing: the pages say only that the packed format persists the ternary
+  planes and scales losslessly (4B paper, section 9.1, Table 6; 8B paper,
+  storage discussion). The two byte layouts (2-bit execution codes and
+  base-3 storage bytes) are this library's own and are defined here by their
+  closed forms.
+* Bit accounting: the 4B paper, sections 3.2, 4.4 and 7.1 (1.641 effective
+  bits per weight against the ideal log2 3 = 1.585), and the 8B paper's
+  effective-bits equation (lost in extraction; read here as log2 3 per plane
+  symbol, with a fraction f2 of weights carrying a second plane).
+
+Every function was pinned against something other than itself by the
+``-m "not gpu"`` tests (brute force with exact rationals, closed forms,
+Python's own base conversion, page figures).
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+GROUP = 128          # scales are per (row, 128 consecutive K columns); 4B paper section 4.5
+CODES_PER_WORD = 16  # 2-bit execution codes per uint32 word
+TRITS_PER_BYTE = 5   # base-3 storage: 3**5 = 243 <= 256
+HEADER_BITS = 512    # a 64-byte container header, counted by the bit accounting
+
+
+# --------------------------------------------------------------------------------------
+# 2-bit execution plane: code c = t + 1 in {0, 1, 2}; 16 codes per uint32 word,
+# trit k of a row at bits 2*(k % 16) of word k // 16 (least significant first).
+# --------------------------------------------------------------------------------------
+
+def pack_exec(trits: np.ndarray) -> tuple[np.ndarray, int]:
+    """int8 trits [rows, K] -> uint32 words [rows, K/16].
+
+    Returns (words, n_invalid). An entry outside {-1, 0, +1} is counted as
+    invalid and encoded as the code of 0, which is what the CUDA path writes
+    too.
+    """
+    t = np.asarray(trits, dtype=np.int8)
+    rows, K = t.shape
+    if K % CODES_PER_WORD:
+        raise ValueError("K must be a multiple of 16")
+    invalid = (t < -1) | (t > 1)
+    codes = np.where(invalid, 1, t.astype(np.int64) + 1).astype(np.uint32)
+    codes = codes.reshape(rows, K // CODES_PER_WORD, CODES_PER_WORD)
+    words = np.zeros((rows, K // CODES_PER_WORD), dtype=np.uint32)
+    for i in range(CODES_PER_WORD):
+        words |= codes[:, :, i] << np.uint32(2 * i)
+    return words, int(invalid.sum())
+
+
+def unpack_exec(words: np.ndarray, K: int) -> tuple[np.ndarray, int]:
+    """uint32 words [rows, K/16] -> int8 trits [rows, K].
+
+    Code 3 has no trit: it is counted as invalid and decoded as 0.
+    """
+    w = np.asarray(words, dtype=np.uint32)
+    rows = w.shape[0]
+    if w.shape[1] * CODES_PER_WORD != K:
+        raise ValueError("words do not hold K codes per row")
+    shifts = (2 * np.arange(CODES_PER_WORD, dtype=np.uint32))
+    codes = (w[:, :, None] >> shifts[None, None, :]) & np.uint32(3)
+    invalid = codes == 3
+    t = np.where(invalid, 0, codes.astype(np.int64) - 1).astype(np.int8)
+    return t.reshape(rows, K), int(invalid.sum())
+
+
+# --------------------------------------------------------------------------------------
+# Base-3 storage plane: byte j of a row = sum_{i<5} (t[5j+i] + 1) * 3**i; a row holds
+# ceil(K/5) bytes; positions past K in the last byte hold trit 0 (digit 1).
+# --------------------------------------------------------------------------------------
+
+def store_row_bytes(K: int) -> int:
+    return -(-K // TRITS_PER_BYTE)
+
+
+def pack_store(trits: np.ndarray) -> tuple[np.ndarray, int]:
+    """int8 trits [rows, K] -> uint8 bytes [rows, ceil(K/5)]; returns (bytes, n_invalid)."""
+    t = np.asarray(trits, dtype=np.int8)
+    rows, K = t.shape
+    nb = store_row_bytes(K)
+    invalid = (t < -1) | (t > 1)
+    digits = np.ones((rows, nb * TRITS_PER_BYTE), dtype=np.int64)   # pad digit 1 = trit 0
+    digits[:, :K] = np.where(invalid, 1, t.astype(np.int64) + 1)
+    digits = digits.reshape(rows, nb, TRITS_PER_BYTE)
+    value = np.zeros((rows, nb), dtype=np.int64)
+    for i in range(TRITS_PER_BYTE):
+        value += digits[:, :, i] * (3 ** i)
+    return value.astype(np.uint8), int(invalid.sum())
+
+
+def unpack_store(data: np.ndarray, K: int) -> tuple[np.ndarray, int]:
+    """uint8 bytes [rows, ceil(K/5)] -> int8 trits [rows, K].
+
+    A byte >= 243 is not a base-3 number of five digits: it is counted invalid and
+    all five of its trits decode as 0. A padding digit (position >= K) other than
+    1 is a non-canonical encoding and is counted invalid too (the decoded trits
+    are unaffected).
+    """
+    b = np.asarray(data, dtype=np.uint8)
+    rows, nb = b.shape
+    if nb != store_row_bytes(K):
+        raise ValueError("row length does not match K")
+    bad_byte = b >= 243
+    v = b.astype(np.int64)
+    digits = np.empty((rows, nb, TRITS_PER_BYTE), dtype=np.int64)
+    for i in range(TRITS_PER_BYTE):
+        digits[:, :, i] = v % 3
+        v //= 3
+    digits[bad_byte] = 1
+    flat = digits.reshape(rows, nb * TRITS_PER_BYTE)
+    bad_pad = (flat[:, K:] != 1).any(axis=1) & ~bad_byte[:, -1] if nb * TRITS_PER_BYTE > K else np.zeros(rows, bool)
+    t = (flat[:, :K] - 1).astype(np.int8)
+    return t, int(bad_byte.sum()) + int(bad_pad.sum())
+
+
+# --------------------------------------------------------------------------------------
+# Residual-row metadata
+# --------------------------------------------------------------------------------------
+
+def slot_map(N: int, res_rows: np.ndarray) -> np.ndarray:
+    """int32 [N]: -1 for a row with one plane, else the row's index in res_rows."""
+    slot = np.full(N, -1, dtype=np.int32)
+    slot[np.asarray(res_rows, dtype=np.int64)] = np.arange(len(res_rows), dtype=np.int32)
+    return slot
+
+
+def row_bitmap(N: int, res_rows: np.ndarray) -> np.ndarray:
+    """uint8 [ceil(N/8)]: bit n % 8 of byte n // 8 is set when row n carries a second plane."""
+    bits = np.zeros(N, dtype=np.uint8)
+    bits[np.asarray(res_rows, dtype=np.int64)] = 1
+    return np.packbits(bits, bitorder="little")
+
+
+# --------------------------------------------------------------------------------------
+# Dequantisation and the linear layer
+# --------------------------------------------------------------------------------------
+
+def dequant(T1, s1, res_rows, T2, s2, rows=None) -> np.ndarray:
+    """Dense float64 W [N, K] (or the listed rows of it).
+
+    W[n, k] = s1[n, k // 128] * T1[n, k]
+              + [n in R] * s2[rho(n), k // 128] * T2[rho(n), k],
+    rho(n) = position of n in the sorted residual-row list R.
+    fp16 -> float64 is exact, so W is exact in float64.
+    """
+    T1 = np.asarray(T1)
+    N, K = T1.shape
+    if K % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    rows = np.arange(N) if rows is None else np.asarray(rows, dtype=np.int64)
+    s1_cols = np.repeat(np.asarray(s1, dtype=np.float64)[rows], GROUP, axis=1)   # s1[n, k // 128]
+    W = s1_cols * T1[rows].astype(np.float64)
+    res_rows = np.asarray(res_rows, dtype=np.int64)
+    if len(res_rows):
+        rho = slot_map(N, res_rows)[rows]
+        has2 = rho >= 0
+        if has2.any():
+            s2_cols = np.repeat(np.asarray(s2, dtype=np.float64)[rho[has2]], GROUP, axis=1)
+            W[has2] += s2_cols * np.asarray(T2)[rho[has2]].astype(np.float64)
+    return W
+
+
+def linear(x, T1, s1, res_rows, T2, s2, cols=None) -> np.ndarray:
+    """y_ref [M, N] (or [M, len(cols)]) = x . W^T in float64 (x fp16 -> float64 is exact)."""
+    W = dequant(T1, s1, res_rows, T2, s2, rows=cols)
+    return np.asarray(x, dtype=np.float64) @ W.T
+
+
+def round_fp16(y: np.ndarray) -> np.ndarray:
+    """One round-to-nearest-even conversion of float64 values to fp16."""
+    return np.asarray(y, dtype=np.float64).astype(np.float16)
+
+
+def rel_err(y, y_ref) -> float:
+    """max |y - y_ref| / max |y_ref|, the parity measure for fp16 outputs."""
+    y = np.asarray(y, dtype=np.float64)
+    y_ref = np.asarray(y_ref, dtype=np.float64)
+    denom = float(np.max(np.abs(y_ref))) if y_ref.size else 0.0
+    num = float(np.max(np.abs(y - y_ref))) if y_ref.size else 0.0
+    if denom == 0.0:
+        return num
+    return num / denom
+
+
+# --------------------------------------------------------------------------------------
+# Bit accounting
+# --------------------------------------------------------------------------------------
+
+def bits(N: int, K: int, r: int, group: int = GROUP) -> dict:
+    """Bits of one ternarized tensor in its three forms.
+
+    info  : log2(3) per plane symbol, (N + r) * K symbols; per weight this is
+            log2(3) * (1 + f2) with f2 = r / N, the fraction of weights with a second plane.
+    store : base-3 planes (8 * ceil(K/5) bits per plane row) + fp16 scales per plane row and
+            group + the residual-row bitmap (whole bytes) + a 64-byte header.
+    exec  : 2-bit planes (2 bits per symbol) + fp16 scales + the int32 slot map [N] + header.
+    """
+    if K % group:
+        raise ValueError("K must be a multiple of the group size")
+    G = K // group
+    weights = N * K
+    plane_rows = N + r
+    plane_trits = plane_rows * K
+    store_bits = 8 * plane_rows * store_row_bytes(K) + 16 * plane_rows * G + 8 * (-(-N // 8)) + HEADER_BITS
+    exec_bits = 2 * plane_trits + 16 * plane_rows * G + 32 * N + HEADER_BITS
+    return {
+        "weights": weights,
+        "plane_trits": plane_trits,
+        "store_bits": store_bits,
+        "exec_bits": exec_bits,
+        "bpw_info": math.log2(3) * plane_trits / weights,
+        "bpw_store": store_bits / weights,
+        "bpw_exec": exec_bits / weights,
+    }

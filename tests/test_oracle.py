@@ -1,0 +1,313 @@
+"""Pins for the CPU oracle, each independent of the oracle's own code.
+
+* packing: Python's own base-4 / base-3 number conversion, exhaustive over the
+  byte and word patterns that matter;
+* dequant + product: a second implementation with exact rationals
+  (fractions.Fraction) written from the definition, per output element,
+  without a dense W or a matmul;
+* the add/subtract identity for ternary weights (promptzone article, "What It
+  Is and How It Works": with weights in {-1, 0, +1} the product is additions and
+  subtractions of activations);
+* closed-form special cases (zero plane, single nonzero, all +1, r = N);
+* planted mistakes: variants of the oracle with a plausible bug each (a
+  dropped residual term, a transposed scale index, a wrong group width, a
+  flipped sign, an off-by-one residual slot) must all fail the rational check.
+"""
+
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import tern_oracle as O
+from ternary_weight_only_tern_b200 import synth
+
+
+# ----------------------------------------------------------------------------- packing
+
+def test_pack_exec_matches_python_base4():
+    rng = np.random.default_rng(11)
+    t = rng.integers(-1, 2, size=(7, 64)).astype(np.int8)
+    words, bad = oracle.pack_exec(t)
+    assert bad == 0 and words.shape == (7, 4) and words.dtype == np.uint32
+    for r in range(7):
+        for w in range(4):
+            codes = [int(v) + 1 for v in t[r, 16 * w:16 * w + 16]]
+            # code of trit k is base-4 digit k (least significant first)
+            expect = int("".join(str(c) for c in reversed(codes)), 4)
+            assert int(words[r, w]) == expect
+
+
+def test_unpack_exec_every_byte_pattern():
+    # all 256 byte values at each of the four byte positions of a word
+    vals = np.arange(256, dtype=np.uint32)
+    for pos in range(4):
+        words = (vals << np.uint32(8 * pos)) | np.uint32(0x55555555 & ~(0xFF << (8 * pos)))
+        t, bad = oracle.unpack_exec(words.reshape(256, 1), 16)
+        n_bad = 0
+        for v in range(256):
+            digits = [int(d) for d in reversed(np.base_repr(v, 4).zfill(4))]
+            for i, d in enumerate(digits):
+                k = 4 * pos + i
+                if d == 3:
+                    n_bad += 1
+                    assert t[v, k] == 0
+                else:
+                    assert t[v, k] == d - 1
+            others = [k for k in range(16) if not (4 * pos <= k < 4 * pos + 4)]
+            assert (t[v, others] == 0).all()     # code 1 elsewhere is trit 0
+        # each of the 4 digits is 3 in 64 of the 256 bytes; 3**4 = 81 bytes hold no 3 at all
+        assert bad == n_bad == 4 * 64
+        assert sum(1 for v in range(256) if '3' not in np.base_repr(v, 4)) == 81
+
+
+def test_pack_store_exhaustive_243():
+    combos = np.array(np.meshgrid(*[np.arange(-1, 2)] * 5, indexing="ij")).reshape(5, -1).T.astype(np.int8)
+    assert combos.shape == (243, 5)
+    b, bad = oracle.pack_store(combos)
+    assert bad == 0 and b.shape == (243, 1)
+    for row, trits in zip(b[:, 0], combos):
+        expect = int("".join(str(int(v) + 1) for v in reversed(trits)), 3)
+        assert int(row) == expect
+    assert sorted(int(v) for v in b[:, 0]) == list(range(243))   # a bijection onto 0..242
+    t, bad = oracle.unpack_store(b, 5)
+    assert bad == 0 and np.array_equal(t, combos)
+
+
+def test_unpack_store_rejects_high_bytes():
+    b = np.arange(256, dtype=np.uint8).reshape(256, 1)
+    t, bad = oracle.unpack_store(b, 5)
+    assert bad == 13
+    assert (t[243:] == 0).all()
+    for v in range(243):
+        digits = [int(d) for d in reversed(np.base_repr(v, 3).zfill(5))]
+        assert list(t[v]) == [d - 1 for d in digits]
+
+
+@pytest.mark.parametrize("K", [1, 4, 5, 6, 127, 128, 2560, 2563])
+def test_store_padding_and_roundtrip(K):
+    rng = np.random.default_rng(K)
+    t = rng.integers(-1, 2, size=(5, K)).astype(np.int8)
+    b, bad = oracle.pack_store(t)
+    assert bad == 0 and b.shape == (5, -(-K // 5))
+    back, bad = oracle.unpack_store(b, K)
+    assert bad == 0 and np.array_equal(back, t)
+    if K % 5:
+        # the padding digits of the last byte are 1 (trit 0): the last byte's value is below 3**(K%5) * ... +
+        last = b[:, -1].astype(int)
+        tail = K % 5
+        assert all(v // 3 ** tail == sum(3 ** i for i in range(5 - tail)) for v in last)
+        # a non-canonical padding digit is reported
+        bb = b.copy()
+        bb[0, -1] = int(bb[0, -1]) - 3 ** tail if bb[0, -1] >= 3 ** tail else int(bb[0, -1]) + 3 ** tail
+        _, bad = oracle.unpack_store(bb, K)
+        assert bad == 1
+
+
+def test_exec_roundtrip_and_invalid_trits():
+    rng = np.random.default_rng(3)
+    t = rng.integers(-1, 2, size=(9, 256)).astype(np.int8)
+    w, bad = oracle.pack_exec(t)
+    back, bad2 = oracle.unpack_exec(w, 256)
+    assert bad == bad2 == 0 and np.array_equal(back, t)
+    t2 = t.copy()
+    t2[0, 5] = 2
+    t2[3, 17] = -7
+    w2, bad = oracle.pack_exec(t2)
+    assert bad == 2
+    back, _ = oracle.unpack_exec(w2, 256)
+    assert back[0, 5] == 0 and back[3, 17] == 0
+
+
+# ----------------------------------------------------------------------------- linear
+
+def brute_linear(x, T1, s1, res_rows, T2, s2):
+    """Exact rational y[m][n] = sum_k x[m,k] * (s1[n,k//128] T1[n,k] + [n in R] s2[rho(n),k//128] T2[rho(n),k])."""
+    M, K = x.shape
+    N = T1.shape[0]
+    rho = {int(n): i for i, n in enumerate(res_rows)}
+    y = [[Fraction(0)] * N for _ in range(M)]
+    for m in range(M):
+        for n in range(N):
+            acc = Fraction(0)
+            for k in range(K):
+                g = k // 128
+                w = Fraction(float(s1[n][g])) * int(T1[n][k])
+                if n in rho:
+                    w += Fraction(float(s2[rho[n]][g])) * int(T2[rho[n]][k])
+                acc += Fraction(float(x[m][k])) * w
+            y[m][n] = acc
+    return y
+
+
+def check_against_brute(lin, case):
+    x, T1, s1, rr, T2, s2 = case
+    y = lin(x, T1, s1, rr, T2, s2)
+    yb = brute_linear(x, T1, s1, rr, T2, s2)
+    M, N = y.shape
+    for m in range(M):
+        for n in range(N):
+            scale = sum(abs(float(x[m][k])) for k in range(x.shape[1])) * 0.05 + 1e-30
+            if abs(Fraction(float(y[m, n])) - yb[m][n]) > Fraction(scale * 1e-14):
+                return False
+    return True
+
+
+def tiny_cases():
+    rng = np.random.default_rng(2024)
+    cases = []
+    for (N, K, M, r) in [(5, 128, 1, 2), (8, 256, 3, 3), (6, 256, 2, 6), (7, 128, 2, 0)]:
+        t = synth.draw_tensor(rng, "tiny", N, K, M, p_zero=0.4, res_pct=0)
+        res_rows = np.sort(rng.choice(N, size=r, replace=False)).astype(np.int32)
+        T2 = synth.draw_trits(rng, (r, K), 0.4)
+        s2 = synth.draw_scales(rng, r, K, 0.001, 0.005)
+        cases.append((t.x, t.T1, t.s1, res_rows, T2, s2))
+    return cases
+
+
+@pytest.mark.parametrize("idx", range(4))
+def test_linear_matches_exact_rationals(idx):
+    assert check_against_brute(oracle.linear, tiny_cases()[idx])
+
+
+def test_dequant_matches_definition_elementwise():
+    x, T1, s1, rr, T2, s2 = tiny_cases()[1]
+    W = oracle.dequant(T1, s1, rr, T2, s2)
+    rho = {int(n): i for i, n in enumerate(rr)}
+    for n in range(T1.shape[0]):
+        for k in range(T1.shape[1]):
+            w = float(s1[n, k // 128]) * int(T1[n, k])
+            if n in rho:
+                w += float(s2[rho[n], k // 128]) * int(T2[rho[n], k])
+            assert W[n, k] == w
+
+
+def test_add_subtract_identity():
+    rng = np.random.default_rng(5)
+    N, K, M = 16, 384, 4
+    x = rng.integers(-20, 21, size=(M, K)).astype(np.float16)      # integer x: both sides exact
+    T1 = synth.draw_trits(rng, (N, K), 0.4)
+    s1 = np.ones((N, K // 128), dtype=np.float16)
+    y = oracle.linear(x, T1, s1, np.zeros(0, np.int32), np.zeros((0, K), np.int8), np.zeros((0, K // 128), np.float16))
+    xf = x.astype(np.float64)
+    for m in range(M):
+        for n in range(N):
+            plus = xf[m][T1[n] == 1].sum()
+            minus = xf[m][T1[n] == -1].sum()
+            assert y[m, n] == plus - minus
+
+
+def test_special_cases():
+    rng = np.random.default_rng(9)
+    N, K, M = 8, 256, 2
+    x = synth.draw_x(rng, M, K)
+    s1 = synth.draw_scales(rng, N, K, 0.005, 0.02)
+    none_r = np.zeros(0, np.int32)
+    z2 = np.zeros((0, K), np.int8)
+    zs = np.zeros((0, K // 128), np.float16)
+    # zero plane -> zero output
+    assert (oracle.linear(x, np.zeros((N, K), np.int8), s1, none_r, z2, zs) == 0).all()
+    # one nonzero per row -> +-s*x_k exactly
+    T = np.zeros((N, K), np.int8)
+    ks = rng.integers(0, K, size=N)
+    sg = rng.choice([-1, 1], size=N)
+    T[np.arange(N), ks] = sg
+    y = oracle.linear(x, T, s1, none_r, z2, zs)
+    for n in range(N):
+        for m in range(M):
+            assert y[m, n] == sg[n] * float(s1[n, ks[n] // 128]) * float(x[m, ks[n]])
+    # all +1 -> sum over groups of s * (sum of x in the group)
+    y = oracle.linear(x, np.ones((N, K), np.int8), s1, none_r, z2, zs)
+    gx = x.astype(np.float64).reshape(M, K // 128, 128).sum(axis=2)
+    assert np.allclose(y, gx @ s1.astype(np.float64).T, rtol=1e-13, atol=1e-13)
+    # r = N with T2 = T1, s2 = s1 doubles the output; r = 0 leaves it alone
+    T1 = synth.draw_trits(rng, (N, K), 0.4)
+    y1 = oracle.linear(x, T1, s1, none_r, z2, zs)
+    y2 = oracle.linear(x, T1, s1, np.arange(N, dtype=np.int32), T1, s1)
+    assert np.allclose(y2, 2 * y1, rtol=1e-13, atol=1e-13)
+
+
+def test_sampled_columns_match_full():
+    rng = np.random.default_rng(1)
+    t = synth.draw_tensor(rng, "s", 40, 256, 3, p_zero=0.4, res_pct=25)
+    full = oracle.linear(t.x, t.T1, t.s1, t.res_rows, t.T2, t.s2)
+    cols = np.array([0, 3, 17, 39, int(t.res_rows[0])])
+    part = oracle.linear(t.x, t.T1, t.s1, t.res_rows, t.T2, t.s2, cols=cols)
+    assert np.array_equal(part, full[:, cols])
+
+
+# ------------------------------------------------------------------ planted mistakes
+
+def _mut_drop_residual(x, T1, s1, rr, T2, s2):
+    return O.linear(x, T1, s1, np.zeros(0, np.int32), T2[:0], s2[:0])
+
+
+def _mut_scale_index(x, T1, s1, rr, T2, s2):
+    # scale indexed by k % G instead of k // 128 (a transposed/misread index)
+    N, K = T1.shape
+    G = K // 128
+    idx = np.arange(K) % G
+    W = s1.astype(np.float64)[:, idx] * T1
+    if len(rr):
+        W[rr] += s2.astype(np.float64)[:, idx] * T2
+    return x.astype(np.float64) @ W.T
+
+
+def _mut_group_width(x, T1, s1, rr, T2, s2):
+    N, K = T1.shape
+    idx = np.minimum(np.arange(K) // 64, K // 128 - 1)
+    W = s1.astype(np.float64)[:, idx] * T1
+    if len(rr):
+        W[rr] += s2.astype(np.float64)[:, idx] * T2
+    return x.astype(np.float64) @ W.T
+
+
+def _mut_sign(x, T1, s1, rr, T2, s2):
+    W = O.dequant(T1, s1, rr, T2, s2)
+    if len(rr):
+        W[rr] -= 2 * np.repeat(s2.astype(np.float64), 128, axis=1) * T2
+    return x.astype(np.float64) @ W.T
+
+
+def _mut_slot_shift(x, T1, s1, rr, T2, s2):
+    if len(rr) < 2:
+        return O.linear(x, T1, s1, rr, T2, s2) + 1.0
+    return O.linear(x, T1, s1, rr, np.roll(T2, 1, axis=0), np.roll(s2, 1, axis=0))
+
+
+@pytest.mark.parametrize("mutant", [_mut_drop_residual, _mut_scale_index, _mut_group_width, _mut_sign,
+                                    _mut_slot_shift])
+def test_planted_mistakes_are_caught(mutant):
+    cases = tiny_cases()
+    assert not all(check_against_brute(mutant, c) for c in cases[:3])
+
+
+# ----------------------------------------------------------------------------- exact case
+
+def test_exact_inputs_are_exact_in_fp32_sums():
+    rng = np.random.default_rng(4)
+    t = synth.draw_exact_tensor(rng, 12, 512, 3, 4)
+    y = oracle.linear(t.x, t.T1, t.s1, t.res_rows, t.T2, t.s2)
+    yb = brute_linear(t.x, t.T1, t.s1, t.res_rows, t.T2, t.s2)
+    for m in range(3):
+        for n in range(12):
+            assert Fraction(float(y[m, n])) == yb[m][n]                # float64 exact
+            assert (yb[m][n] * 64).denominator == 1                    # multiple of 2^-6
+            assert abs(yb[m][n]) < 2 ** 18
+    # s1*t1 + s2*t2 exact in fp16
+    W = oracle.dequant(t.T1, t.s1, t.res_rows, t.T2, t.s2)
+    assert np.array_equal(W.astype(np.float16).astype(np.float64), W)
+
+
+def test_round_fp16_is_round_to_nearest_even():
+    # 1 + 2^-11 is halfway between 1 and the next fp16 (1 + 2^-10): ties to even -> 1
+    assert float(oracle.round_fp16(np.array([1 + 2 ** -11]))[0]) == 1.0
+    assert float(oracle.round_fp16(np.array([1 + 3 * 2 ** -11]))[0]) == 1 + 2 ** -9
+    assert float(oracle.round_fp16(np.array([1 + 2 ** -11 + 2 ** -30]))[0]) == 1 + 2 ** -10
+
+
+def test_rel_err():
+    assert oracle.rel_err(np.array([1.0, 2.0]), np.array([1.0, 2.0])) == 0.0
+    assert math.isclose(oracle.rel_err(np.array([1.0, 2.002]), np.array([1.0, 2.0])), 0.001)
