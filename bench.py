@@ -1,0 +1,497 @@
+"""Benchmark of the W1.58A16 ternary linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--quick]
+
+A step is one decode pass (M = 1) over the 252 ternarized linear tensors of a 36-layer
+Qwen3-8B-shaped stack (q, k, v, o, gate, up, down per layer; 15% of rows carry a residual
+plane), i.e. 252 tern_linear calls, replayed from a CUDA graph. Weights come from a pool of
+8 distinct layers (about 470 MB of packed planes, several times the 126 MB L2), assigned to
+the 36 layer slots round-robin, so every call streams its weights from HBM.
+
+value     : packed-weight GB/s = (2-bit planes + fp16 scales + slot map) bytes per step / time.
+roofline  : the dominant op (the gate projection's tern_linear at M = 1), algorithmic bytes
+            (packed weight + activations) per call / its average call time, against the
+            measured HBM copy bandwidth.
+e2e       : the same metric through the Python API with the step's activations copied from
+            pinned host memory and its outputs copied back, every step.
+cpu_baseline / --impl reference: the CPU oracle (numpy float64) on a bounded sample.
+extra     : per-projection and per-M decode figures, the M = 2048 prefill GEMM in TFLOP/s,
+            packing throughput, bit accounting, and dense fp16 cuBLAS on the same shapes.
+
+For --gpus N > 1 (torchrun) every rank runs the same workload on its own GPU (replicas; the
+path has no data exchange), the timed region is bracketed by barriers, and the time is the
+max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "W1.58A16 GEMV packed-weight GB/s (% of HBM peak); GEMM TFLOP/s at M=2048"
+WORKLOAD = "qwen3-8b-decode-stack-m1"
+RES_PCT = 15
+POOL_LAYERS = 8
+LAYERS = 36
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        time.sleep(0.1)
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        mx = max(r[1] for r in rows)
+        load = [r for r in rows] or rows
+        sm = float(np.median([r[0] for r in load]))
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i, v in enumerate(r[2]) if v.lower().startswith("active")})
+        return {"sm_mhz": sm, "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_uuid(torch, dev):
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev.index or 0)
+
+
+# ------------------------------------------------------------------------------ workload
+def draw_layer_on_device(torch, api, shapes, dev, seed):
+    """One layer's projections, drawn on the device with a seeded torch generator (same
+    distributions as the host recipe: P(0) = 0.4, P(+-1) = 0.3; s1 ~ U[0.005, 0.02];
+    s2 ~ U[0.001, 0.005]; 15% residual rows uniformly without replacement) and packed with
+    tern_pack_exec."""
+    from ternary_weight_only_tern_b200.synth import residual_count
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    out = {}
+    for name, N, K in shapes:
+        G = K // 128
+
+        def trits(rows):
+            u = torch.randint(0, 10, (rows, K), dtype=torch.uint8, generator=g, device=dev)
+            return (u >= 7).to(torch.int8) - (u < 3).to(torch.int8)
+
+        T1 = trits(N)
+        s1 = (torch.rand((N, G), generator=g, device=dev) * 0.015 + 0.005).half()
+        r = residual_count(N, RES_PCT)
+        rows = torch.randperm(N, generator=g, device=dev)[:r].sort().values.to(torch.int32)
+        T2 = trits(r)
+        s2 = (torch.rand((r, G), generator=g, device=dev) * 0.004 + 0.001).half()
+        out[name] = api.TernWeight.from_trits(T1, s1, rows, T2, s2)
+        del T1, T2
+    return out
+
+
+def packed_bytes(w) -> int:
+    return w.nbytes()
+
+
+def time_graph(torch, graph, reps, stream):
+    """Seconds for `reps` replays; the graph is launched on `stream` (replay() uses the current
+    stream), bracketed by events on that same stream."""
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        s.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e.record(stream)
+    e.synchronize()
+    return s.elapsed_time(e) / 1e3
+
+
+def capture(torch, fn, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        fn()                     # eager warm-up of this exact sequence
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+def oracle_sample(seconds_budget=12.0):
+    """The oracle on one 8B-shaped decoder layer's 7 projections at M = 1 (numpy inputs drawn
+    with the host recipe). Returns (packed bytes, seconds, threads, description)."""
+    import oracle
+    from ternary_weight_only_tern_b200 import synth
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    tensors = list(synth.draw_workload(synth.WORKLOADS[4]))
+    nbytes, secs, calls = 0, 0.0, 0
+    while secs < seconds_budget:
+        t = tensors[calls % len(tensors)]
+        t0 = time.perf_counter()
+        oracle.linear(t.x[:1], t.T1, t.s1, t.res_rows, t.T2, t.s2)
+        secs += time.perf_counter() - t0
+        nbytes += (t.N + t.r) * t.K // 4 + 2 * (t.N + t.r) * (t.K // 128) + 4 * t.N
+        calls += 1
+    return nbytes, secs, threads, f"oracle.linear (numpy float64 dequant + matmul) cycling the 7 projections of " \
+                                  f"one Qwen3-8B-shaped layer at M=1, 15% residual rows ({calls} calls, " \
+                                  f"{secs:.1f} s)"
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle as it stands, on rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    from ternary_weight_only_tern_b200 import synth
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    tensors = list(synth.draw_workload(synth.WORKLOADS[4]))
+
+    def step(i):
+        t = tensors[i % len(tensors)]
+        oracle.linear(t.x[:1], t.T1, t.s1, t.res_rows, t.T2, t.s2)
+        return (t.N + t.r) * t.K // 4 + 2 * (t.N + t.r) * (t.K // 128) + 4 * t.N
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    nbytes = sum(step(args.warmup + i) for i in range(args.steps))
+    secs = time.perf_counter() - t0
+    val = nbytes / secs / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(1, args.steps) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (numpy PCG64, seed 3: the 8B projection recipe)",
+        "config": {"workload": WORKLOAD, "sample": "one 8B projection per step, cycling q,k,v,o,gate,up,down",
+                   "M": 1, "residual_pct": RES_PCT},
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": "one Qwen3-8B-shaped projection per step at M=1 (cycling the 7)"},
+        "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------ main arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true", help="skip the extra measurements")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from ternary_weight_only_tern_b200 import _lib, api, synth
+
+    _lib.load()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks, peak_kind = load_peaks()
+    shapes = list(synth.WORKLOADS[4].shapes)
+    pool = [draw_layer_on_device(torch, api, shapes, dev, seed=1000 + i) for i in range(POOL_LAYERS)]
+    torch.cuda.synchronize()
+    names = [s[0] for s in shapes]
+    Kmax = max(K for _, _, K in shapes)
+    ws = torch.empty(max(api.workspace_bytes(pool[0][n], 16) for n in names) + 256, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+
+    def make_io(M):
+        xs = {n: torch.randn((M, K), generator=gen, device=dev).half() for n, _, K in shapes}
+        ys = [{n: torch.empty((M, N), dtype=torch.float16, device=dev) for n, N, _ in shapes} for _ in range(LAYERS)]
+        return xs, ys
+
+    def step_fn(M, xs, ys, only=None):
+        def fn():
+            for layer in range(LAYERS):
+                W = pool[layer % POOL_LAYERS]
+                for n in names:
+                    if only is None or n == only:
+                        api.linear(xs[n], W[n], out=ys[layer][n], workspace=ws)
+        return fn
+
+    def step_bytes(M, only=None):
+        wb = sum(packed_bytes(pool[l % POOL_LAYERS][n]) for l in range(LAYERS) for n in names
+                 if only is None or n == only)
+        ab = sum(2 * M * (K + N) for l in range(LAYERS) for (n, N, K) in shapes if only is None or n == only)
+        return wb, ab
+
+    # ---------------- the timed region: K graph replays of the full M = 1 step
+    xs1, ys1 = make_io(1)
+    g_step = capture(torch, step_fn(1, xs1, ys1), stream)
+    launches_per_step = sum(2 if pool[l % POOL_LAYERS][n].r > 0 else 1 for l in range(LAYERS) for n in names)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            g_step.replay()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_uuid(torch, dev)) as clk:
+        secs = time_graph(torch, g_step, args.steps, stream)
+    torch.cuda.synchronize()
+    barrier()
+    secs = max_over_ranks(secs)
+    wb, ab = step_bytes(1)
+    value = world * wb * args.steps / secs / 1e9
+    ms_per_step = secs / args.steps * 1e3
+
+    # ---------------- the dominant op: the gate projection's tern_linear at M = 1
+    g_gate = capture(torch, step_fn(1, xs1, ys1, only="gate"), stream)
+    with torch.cuda.stream(stream):
+        for _ in range(5):
+            g_gate.replay()
+    reps = max(20, min(400, args.steps // 10))
+    t_gate = time_graph(torch, g_gate, reps, stream) / (reps * LAYERS)
+    gw, ga = step_bytes(1, only="gate")
+    gate_bytes = (gw + ga) / LAYERS
+    achieved = gate_bytes / t_gate / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "op": "tern_linear gate 12288x4096 (+1843 residual rows) M=1, both passes",
+                "us_per_call": t_gate * 1e6, "bytes_per_call": gate_bytes, "peak_kind": peak_kind,
+                "frac_of_8000": achieved / 8000.0}
+
+    extra = {}
+    if not args.quick and world == 1:
+        extra = extras(torch, api, synth, pool, shapes, names, stream, dev, ws, step_fn, step_bytes, make_io, peaks,
+                       time_graph, capture)
+
+    # ---------------- e2e through the Python API with host buffers
+    e2e_steps = max(3, min(20, args.steps // 100))
+    xh = {n: torch.randn((1, K)).half().pin_memory() for n, _, K in shapes}
+    yh = [{n: torch.empty((1, N), dtype=torch.float16).pin_memory() for n, N, _ in shapes} for _ in range(LAYERS)]
+    h2d = sum(2 * K for _, _, K in shapes)
+    d2h = LAYERS * sum(2 * N for _, N, _ in shapes)
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            for n in names:
+                xs1[n].copy_(xh[n], non_blocking=True)
+            step_fn(1, xs1, ys1)()
+            for layer in range(LAYERS):
+                for n in names:
+                    yh[layer][n].copy_(ys1[layer][n], non_blocking=True)
+        stream.synchronize()
+
+    e2e_step()
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e2e_secs = max_over_ranks(time.perf_counter() - t0)
+    e2e = {"value": world * wb * e2e_steps / e2e_secs / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+           "note": "252 api.linear calls per step from Python (ctypes), activations copied in and outputs out"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        nb, cs, threads, desc = oracle_sample()
+        cpu = {"value": nb / cs / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": cs}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic: trits P(0)=0.4, P(+-1)=0.3, fp16 group-128 scales, seeded torch generator per pool layer",
+        "config": {"workload": WORKLOAD, "layers": LAYERS, "projections": names, "M": 1, "residual_pct": RES_PCT,
+                   "pool_layers": POOL_LAYERS, "packed_bytes_per_step": wb, "activation_bytes_per_step": ab,
+                   "l2": f"inputs larger than L2: {POOL_LAYERS}-layer weight pool of "
+                         f"{sum(packed_bytes(w) for L in pool for w in L.values()) / 1e6:.0f} MB rotated through",
+                   "parallelism": f"replicas x{world}", "frac_of_measured_hbm": value / peaks["hbm_gbs"],
+                   "frac_of_8000": value / 8000.0},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(), "extra": extra,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def extras(torch, api, synth, pool, shapes, names, stream, dev, ws, step_fn, step_bytes, make_io, peaks,
+           time_graph, capture):
+    out = {}
+    hbm = peaks["hbm_gbs"]
+    # per projection at M = 1
+    xs1, ys1 = make_io(1)
+    per = {}
+    for n in names:
+        g = capture(torch, step_fn(1, xs1, ys1, only=n), stream)
+        t = time_graph(torch, g, 50, stream) / (50 * LAYERS)
+        wb, ab = step_bytes(1, only=n)
+        per[n] = {"us": t * 1e6, "packed_gbs": wb / LAYERS / t / 1e9, "frac": (wb + ab) / LAYERS / t / 1e9 / hbm}
+        del g
+    out["per_projection_m1"] = per
+    # per M over the whole stack
+    perm = {}
+    for M in (1, 4, 8, 16):
+        xs, ys = make_io(M)
+        g = capture(torch, step_fn(M, xs, ys), stream)
+        t = time_graph(torch, g, 30, stream) / 30
+        wb, ab = step_bytes(M)
+        perm[str(M)] = {"us_per_step": t * 1e6, "packed_gbs": wb / t / 1e9, "frac": (wb + ab) / t / 1e9 / hbm}
+        del g, xs, ys
+    out["per_M_stack"] = perm
+    # prefill GEMM at M = 2048 on the gate/up/down shapes
+    gemm = {}
+    for n in ("gate", "up", "down"):
+        N, K = [(s[1], s[2]) for s in shapes if s[0] == n][0]
+        x = torch.randn((2048, K), device=dev).half()
+        y = torch.empty((2048, N), dtype=torch.float16, device=dev)
+        wsg = torch.empty(api.workspace_bytes(pool[0][n], 2048) + 256, dtype=torch.uint8, device=dev)
+
+        def fn(n=n, x=x, y=y, wsg=wsg):
+            for i in range(4):
+                api.linear(x, pool[i][n], out=y, workspace=wsg)
+        g = capture(torch, fn, stream)
+        t = time_graph(torch, g, 5, stream) / 20
+        fl = 2.0 * 2048 * N * K
+        gemm[n] = {"us": t * 1e6, "tflops": fl / t / 1e12, "frac_burst": fl / t / 1e12 / peaks["bf16_tflops"],
+                   "frac_sustained": fl / t / 1e12 / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])}
+        del g, x, y, wsg
+    out["gemm_m2048"] = gemm
+    # packing throughput on the gate shape
+    u = torch.randint(0, 3, (12288, 4096), dtype=torch.int8, device=dev) - 1
+    for fn_name, fn in (("pack_exec", api.pack_exec), ("pack_store", api.pack_store)):
+        fn(u)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(5):
+            r = fn(u)
+        dt = (time.perf_counter() - t0) / 5
+        out[fn_name] = {"ms": dt * 1e3, "in_gbs": u.numel() / dt / 1e9, "out_bytes": r.numel() * r.element_size(),
+                        "note": "synchronous call incl. status read-back"}
+    del u
+    # bit accounting of the 252-tensor 8B stack
+    tot = {"weights": 0, "store_bits": 0, "exec_bits": 0, "plane_trits": 0}
+    for (n, N, K) in shapes:
+        b = api.bits(N, K, synth.residual_count(N, RES_PCT))
+        for k in tot:
+            tot[k] += LAYERS * b[k]
+    out["bits_8b_stack"] = {"bpw_info": 1.584962500721156 * tot["plane_trits"] / tot["weights"],
+                            "bpw_store": tot["store_bits"] / tot["weights"],
+                            "bpw_exec": tot["exec_bits"] / tot["weights"],
+                            "store_gib": tot["store_bits"] / 8 / 2 ** 30}
+    # dense fp16 cuBLAS on the gate shape (context, as in the pages' comparison)
+    Wd = [torch.randn((12288, 4096), device=dev).half() for _ in range(4)]
+    x1 = torch.randn((1, 4096), device=dev).half()
+    xb = torch.randn((2048, 4096), device=dev).half()
+
+    def dense1():
+        for w in Wd:
+            torch.matmul(x1, w.t())
+
+    def dense2():
+        for w in Wd:
+            torch.matmul(xb, w.t())
+    g1 = capture(torch, dense1, stream)
+    t1 = time_graph(torch, g1, 50, stream) / 200
+    g2 = capture(torch, dense2, stream)
+    t2 = time_graph(torch, g2, 5, stream) / 20
+    out["context_fp16_cublas_gate"] = {"m1_us": t1 * 1e6, "m1_gbs": 12288 * 4096 * 2 / t1 / 1e9,
+                                       "m2048_us": t2 * 1e6, "m2048_tflops": 2 * 2048 * 12288 * 4096 / t2 / 1e12}
+    return out
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,160 @@
+/*
+ * tern.h -- C ABI of libtern.so: the weight-only ternary linear layer (W1.58A16) on
+ * NVIDIA B200 (sm_100a).
+ *
+ * What is computed (the representation of the ternarized weights):
+ *   y[m, n] = sum_g s1[n, g] * sum_{k in g} T1[n, k] * x[m, k]
+ *           + [n in R] * sum_g s2[rho(n), g] * sum_{k in g} T2[rho(n), k] * x[m, k]
+ *   - T1, T2 hold trits in {-1, 0, +1}; each s is an fp16 scale per (row, 128-wide K group).
+ *     "Post-Training Ternarization of Qwen3-4B: Capability, Effective Bit Budget, Storage
+ *     Compression, and Deployment" (arXiv 2609.01962v1), section 4.3 (ternary planes with
+ *     scales; an order-2 residual plane), section 4.5 (group size 128).
+ *   - R is a salience-selected subset that carries the second plane (4B paper, section 4.4;
+ *     the Qwen3-8B scale-up paper, arXiv 2609.09240, representation paragraph). This
+ *     library takes the subset as whole output rows; rho(n) is n's index in the sorted R.
+ *     The pages' per-group offset is not part of this operation.
+ *   - x and y stay fp16 (weight-only quantisation, 4B paper section 3.1); the sums are
+ *     accumulated in fp32 and rounded to fp16 once.
+ *   - With weights in {-1, 0, +1} the product is additions and subtractions of activations
+ *     (promptzone, "Can Ternary LLMs Hit 1.58 Bits per Weight?", section "What It Is and
+ *     How It Works"); the kernels feed exact +-x or 0 products to fp32 accumulators.
+ *
+ * Layouts (all row-major, no padding between rows):
+ *   exec plane : uint32 [rows, K/16]; trit k of a row is code c = t + 1 in {0,1,2} at
+ *                bits 2*(k % 16) of word k/16 (code 3 is invalid).
+ *   store plane: uint8 [rows, ceil(K/5)]; byte j = sum_{i<5} (t[5j+i] + 1) * 3^i, the
+ *                positions past K in a row's last byte hold trit 0 (digit 1); bytes >= 243
+ *                are invalid.
+ *   scales     : fp16 (IEEE binary16 bit patterns, tern_half) [rows, K/128].
+ *   x, y       : fp16 [M, K] and [M, N].
+ *   Persisting the discrete planes and scales (not a floating reconstruction) is what the
+ *   pages' lossless packing does (4B paper, section 9.1 and Table 6; 8B paper, storage
+ *   discussion); the two byte layouts are this library's own.
+ *
+ * Conventions:
+ *   - Pointers marked "device" point to device memory of the current CUDA device; the
+ *     caller owns every buffer. tern_linear allocates nothing: its only scratch is the
+ *     caller's workspace.
+ *   - Arguments are validated on the host before any launch; on a host-side error nothing
+ *     is launched and nothing is written.
+ *   - tern_linear is asynchronous on the given stream and can be captured in a CUDA graph.
+ *     The pack and unpack calls are synchronous on their stream: they return only after
+ *     the stream has drained, so that they can report invalid codes found on the device.
+ *   - `stream` is a cudaStream_t (0 = the legacy default stream).
+ */
+#ifndef TERN_H
+#define TERN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t tern_half;               /* IEEE binary16 bit pattern */
+typedef struct CUstream_st* tern_stream;  /* the same type as cudaStream_t */
+
+typedef enum {
+    TERN_OK = 0,
+    TERN_ERR_NULL = 1,       /* a required pointer is NULL */
+    TERN_ERR_SHAPE = 2,      /* a size is negative, K is not a multiple of 128 (16 for the exec
+                                plane), group != 128, r > N, or a size is too large */
+    TERN_ERR_ALIGN = 3,      /* a pointer is not 16-byte aligned */
+    TERN_ERR_BAD_TRIT = 4,   /* pack: an input int8 is outside {-1, 0, +1} */
+    TERN_ERR_BAD_CODE = 5,   /* unpack / validate: a 2-bit code 3, a byte >= 243, or a
+                                non-canonical padding digit */
+    TERN_ERR_RESIDUAL = 6,   /* validate: residual rows not strictly increasing, out of range,
+                                or inconsistent with the slot map */
+    TERN_ERR_WORKSPACE = 7,  /* workspace smaller than tern_linear_workspace_bytes() or NULL */
+    TERN_ERR_CUDA = 8,       /* a CUDA runtime call failed (launch error, no device, ...) */
+    TERN_ERR_TIMEOUT = 9     /* reserved: a bounded device-side wait ran out */
+} tern_status;
+
+/* A ternarized weight W [N, K] in execution form. Every pointer is device memory,
+ * caller-owned, 16-byte aligned.                                                       */
+typedef struct {
+    int64_t N, K;                /* output and input features; K % 128 == 0            */
+    int32_t group;               /* scale group width along K; must be 128             */
+    const uint32_t* plane1;      /* [N, K/16]   exec codes of T1                        */
+    const tern_half* scale1;     /* [N, K/128]  s1                                      */
+    int64_t r;                   /* rows with a second plane, 0 <= r <= N               */
+    const int32_t* res_rows;     /* [r] strictly increasing row indices (R); read only by
+                                    tern_weight_validate                                 */
+    const int32_t* res_slot;     /* [N] -1, or rho(n) for n in R                        */
+    const uint32_t* plane2;      /* [r, K/16]   exec codes of T2                        */
+    const tern_half* scale2;     /* [r, K/128]  s2                                      */
+} tern_weight;
+
+/* ---------------------------------------------------------------- packing (offline) */
+
+/* int8 trits t [rows, K] (device) -> exec plane out [rows, K/16] (device). K % 16 == 0.
+ * An input outside {-1,0,+1} is encoded as the code of 0 and the call returns
+ * TERN_ERR_BAD_TRIT (the rest of `out` is written as usual). Synchronous on `stream`. */
+tern_status tern_pack_exec(const int8_t* t, int64_t rows, int64_t K, uint32_t* out, tern_stream stream);
+
+/* exec plane p [rows, K/16] (device) -> int8 trits out [rows, K] (device). A code 3 decodes
+ * as 0 and the call returns TERN_ERR_BAD_CODE. Synchronous on `stream`.               */
+tern_status tern_unpack_exec(const uint32_t* p, int64_t rows, int64_t K, int8_t* out, tern_stream stream);
+
+/* int8 trits t [rows, K] (device) -> store plane out [rows, ceil(K/5)] (device). Any K >= 0.
+ * Invalid trits: as for tern_pack_exec. Synchronous on `stream`.                        */
+tern_status tern_pack_store(const int8_t* t, int64_t rows, int64_t K, uint8_t* out, tern_stream stream);
+
+/* store plane b [rows, ceil(K/5)] (device) -> int8 trits out [rows, K] (device). A byte
+ * >= 243 decodes as five 0 trits; a padding digit other than 1 is non-canonical; both
+ * return TERN_ERR_BAD_CODE. Synchronous on `stream`.                                    */
+tern_status tern_unpack_store(const uint8_t* b, int64_t rows, int64_t K, int8_t* out, tern_stream stream);
+
+/* Checks a weight descriptor's device data: every code of plane1/plane2 is in {0,1,2},
+ * res_rows is strictly increasing in [0, N), and res_slot[n] == i exactly when
+ * res_rows[i] == n (else -1). Returns TERN_OK, TERN_ERR_BAD_CODE or TERN_ERR_RESIDUAL.
+ * Synchronous on `stream`. tern_linear does not repeat these checks; it only keeps its
+ * own memory accesses in bounds when a slot is out of range.                            */
+tern_status tern_weight_validate(const tern_weight* w, tern_stream stream);
+
+/* ---------------------------------------------------------------- the linear layer */
+
+/* Bytes of workspace tern_linear needs for this weight and batch size (0 if none). */
+size_t tern_linear_workspace_bytes(const tern_weight* w, int64_t M);
+
+/* y [M, N] = x [M, K] . W^T for the ternary W above (x, y device, fp16, row-major).
+ * M <= 16 runs the decode GEMV (split along K over a thread-block cluster); larger M
+ * runs the dequantise-into-tcgen05 GEMM. M == 0 is a no-op returning TERN_OK.
+ * x and y must not overlap. Asynchronous on `stream`; capturable in a CUDA graph.
+ * workspace: device scratch of at least tern_linear_workspace_bytes(w, M) bytes, owned
+ * by the caller, not used by another call that runs at the same time.                  */
+tern_status tern_linear(const tern_weight* w, const tern_half* x, int64_t M, tern_half* y,
+                        void* workspace, size_t workspace_bytes, tern_stream stream);
+
+/* ---------------------------------------------------------------- bit accounting */
+
+typedef struct {
+    uint64_t weights;       /* N*K                                                      */
+    uint64_t plane_trits;   /* (N+r)*K symbols in the ternary planes                    */
+    uint64_t store_bits;    /* 8*(N+r)*ceil(K/5) + 16*(N+r)*G + 8*ceil(N/8) + 512       */
+    uint64_t exec_bits;     /* 2*(N+r)*K + 16*(N+r)*G + 32*N + 512                      */
+    double bpw_info;        /* log2(3) * plane_trits / weights = log2(3) * (1 + r/N)    */
+    double bpw_store;       /* store_bits / weights                                     */
+    double bpw_exec;        /* exec_bits / weights                                      */
+} tern_bits_report;
+
+/* Bits per weight of one ternarized tensor: the information rate of its planes (log2 3 per
+ * symbol, with a fraction f2 = r/N of weights carrying a second plane), and the exact bit
+ * totals of its storage form (base-3 planes, fp16 scales, the residual-row bitmap, a
+ * 64-byte header) and of its execution form (2-bit planes, fp16 scales, the int32 slot map,
+ * a 64-byte header). 4B paper, sections 3.2, 4.4 and 7.1 (1.641 effective bits against the
+ * ideal 1.585); 8B paper, effective-bits equation. Pure host function.                  */
+tern_status tern_bits(int64_t N, int64_t K, int64_t r, int32_t group, tern_bits_report* out);
+
+/* A static, human-readable name for a status code. */
+const char* tern_status_string(tern_status s);
+
+/* The library's version as major*10000 + minor*100 + patch. */
+int tern_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TERN_H */

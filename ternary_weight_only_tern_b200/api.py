@@ -1,0 +1,179 @@
+"""Torch-tensor front end of libtern.so: checks dtypes, devices and contiguity, allocates the
+outputs with PyTorch, and passes raw pointers and the current CUDA stream to the C ABI.
+No arithmetic of the method happens here; every step runs in the library's kernels."""
+
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+
+GROUP = 128
+
+
+def _stream(device: torch.device | None = None) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype, name: str, ndim: int = 2):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _ptr(t: torch.Tensor | None):
+    return ctypes.c_void_p(t.data_ptr() if t is not None and t.numel() else None)
+
+
+# ------------------------------------------------------------------------------ packing
+
+def pack_exec(trits: torch.Tensor) -> torch.Tensor:
+    """int8 [rows, K] -> exec plane as int32 [rows, K/16] (uint32 bit patterns)."""
+    _need(trits, torch.int8, "trits")
+    rows, K = trits.shape
+    out = torch.empty((rows, K // 16), dtype=torch.int32, device=trits.device)
+    _lib.check("tern_pack_exec", _lib.load().tern_pack_exec(_ptr(trits), rows, K, _ptr(out), _stream(trits.device)))
+    return out
+
+
+def unpack_exec(words: torch.Tensor, K: int) -> torch.Tensor:
+    _need(words, torch.int32, "words")
+    rows = words.shape[0]
+    if words.shape[1] * 16 != K:
+        raise ValueError("words must hold K/16 words per row")
+    out = torch.empty((rows, K), dtype=torch.int8, device=words.device)
+    _lib.check("tern_unpack_exec", _lib.load().tern_unpack_exec(_ptr(words), rows, K, _ptr(out), _stream(words.device)))
+    return out
+
+
+def pack_store(trits: torch.Tensor) -> torch.Tensor:
+    """int8 [rows, K] -> base-3 store plane uint8 [rows, ceil(K/5)]."""
+    _need(trits, torch.int8, "trits")
+    rows, K = trits.shape
+    out = torch.empty((rows, -(-K // 5)), dtype=torch.uint8, device=trits.device)
+    _lib.check("tern_pack_store", _lib.load().tern_pack_store(_ptr(trits), rows, K, _ptr(out), _stream(trits.device)))
+    return out
+
+
+def unpack_store(data: torch.Tensor, K: int) -> torch.Tensor:
+    _need(data, torch.uint8, "data")
+    rows = data.shape[0]
+    if data.shape[1] != -(-K // 5):
+        raise ValueError("data must hold ceil(K/5) bytes per row")
+    out = torch.empty((rows, K), dtype=torch.int8, device=data.device)
+    _lib.check("tern_unpack_store", _lib.load().tern_unpack_store(_ptr(data), rows, K, _ptr(out), _stream(data.device)))
+    return out
+
+
+# ------------------------------------------------------------------------------ weights
+
+@dataclass
+class TernWeight:
+    """A ternarized weight W [N, K] in execution form, on one CUDA device."""
+    N: int
+    K: int
+    plane1: torch.Tensor     # int32 [N, K/16]
+    scale1: torch.Tensor     # float16 [N, K/128]
+    res_rows: torch.Tensor   # int32 [r]
+    res_slot: torch.Tensor   # int32 [N]
+    plane2: torch.Tensor     # int32 [r, K/16]
+    scale2: torch.Tensor     # float16 [r, K/128]
+
+    @property
+    def r(self) -> int:
+        return int(self.res_rows.numel())
+
+    @property
+    def device(self) -> torch.device:
+        return self.plane1.device
+
+    def c_struct(self) -> _lib.TernWeightC:
+        c = getattr(self, "_c", None)
+        if c is None:
+            c = _lib.TernWeightC(
+                self.N, self.K, GROUP, self.plane1.data_ptr(), self.scale1.data_ptr(), self.r,
+                self.res_rows.data_ptr() if self.r else None, self.res_slot.data_ptr(),
+                self.plane2.data_ptr() if self.r else None, self.scale2.data_ptr() if self.r else None)
+            object.__setattr__(self, "_c", c)
+        return c
+
+    def nbytes(self) -> int:
+        """Bytes the decode kernels stream per call: both planes, their scales and the slot map."""
+        return sum(t.numel() * t.element_size() for t in (self.plane1, self.scale1, self.plane2, self.scale2,
+                                                           self.res_slot))
+
+    @classmethod
+    def from_trits(cls, T1: torch.Tensor, s1: torch.Tensor, res_rows: torch.Tensor | None = None,
+                   T2: torch.Tensor | None = None, s2: torch.Tensor | None = None) -> "TernWeight":
+        """Packs int8 planes on the device (tern_pack_exec) and builds the residual-row slot map."""
+        _need(T1, torch.int8, "T1")
+        _need(s1, torch.float16, "s1")
+        N, K = T1.shape
+        dev = T1.device
+        if res_rows is None or res_rows.numel() == 0:
+            res_rows = torch.zeros(0, dtype=torch.int32, device=dev)
+            T2 = torch.zeros((0, K), dtype=torch.int8, device=dev)
+            s2 = torch.zeros((0, K // GROUP), dtype=torch.float16, device=dev)
+        res_rows = res_rows.to(device=dev, dtype=torch.int32).contiguous()
+        r = int(res_rows.numel())
+        slot = torch.full((N,), -1, dtype=torch.int32, device=dev)
+        if r:
+            slot[res_rows.long()] = torch.arange(r, dtype=torch.int32, device=dev)
+        plane2 = pack_exec(T2) if r else torch.zeros((0, K // 16), dtype=torch.int32, device=dev)
+        return cls(N, K, pack_exec(T1), s1.contiguous(), res_rows, slot, plane2,
+                   s2.contiguous() if r else torch.zeros((0, K // GROUP), dtype=torch.float16, device=dev))
+
+    @classmethod
+    def from_numpy(cls, T1, s1, res_rows, T2, s2, device="cuda") -> "TernWeight":
+        t = lambda a, dt: torch.from_numpy(a).to(device=device, dtype=dt).contiguous()  # noqa: E731
+        return cls.from_trits(t(T1, torch.int8), t(s1, torch.float16), t(res_rows, torch.int32),
+                              t(T2, torch.int8), t(s2, torch.float16))
+
+
+def weight_validate(w: TernWeight) -> None:
+    _lib.check("tern_weight_validate", _lib.load().tern_weight_validate(ctypes.byref(w.c_struct()),
+                                                                         _stream(w.device)))
+
+
+# ------------------------------------------------------------------------------ linear
+
+def workspace_bytes(w: TernWeight, M: int) -> int:
+    return int(_lib.load().tern_linear_workspace_bytes(ctypes.byref(w.c_struct()), M))
+
+
+def linear(x: torch.Tensor, w: TernWeight, out: torch.Tensor | None = None,
+           workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """y [M, N] = x [M, K] . W^T (fp16 in, fp32 accumulation, fp16 out)."""
+    _need(x, torch.float16, "x")
+    M, K = x.shape
+    if K != w.K:
+        raise ValueError(f"x has K={K}, weight has K={w.K}")
+    if out is None:
+        out = torch.empty((M, w.N), dtype=torch.float16, device=x.device)
+    else:
+        _need(out, torch.float16, "out")
+        if tuple(out.shape) != (M, w.N):
+            raise ValueError(f"out must have shape {(M, w.N)}, got {tuple(out.shape)}")
+    need = workspace_bytes(w, M)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _lib.check("tern_linear", _lib.load().tern_linear(
+        ctypes.byref(w.c_struct()), _ptr(x), M, _ptr(out), _ptr(workspace), ws_bytes, _stream(x.device)))
+    return out
+
+
+# ------------------------------------------------------------------------------ bits
+
+def bits(N: int, K: int, r: int, group: int = GROUP) -> dict:
+    rep = _lib.TernBitsReport()
+    _lib.check("tern_bits", _lib.load().tern_bits(N, K, r, group, ctypes.byref(rep)))
+    return {f: getattr(rep, f) for f, _ in rep._fields_}

@@ -1,0 +1,78 @@
+// C ABI of libtern.so: argument validation and dispatch of tern_linear.
+//
+// tern_linear computes y = x . W^T for a ternarized W (planes T1, T2 with fp16 group-128
+// scales; "Post-Training Ternarization of Qwen3-4B", arXiv 2609.01962v1, sections 4.3-4.5)
+// on fp16 activations. M <= 16 (decode) runs the split-K GEMV on the packed planes; larger
+// M (prefill) runs the dequantise-into-tcgen05 GEMM. Both read the packed planes directly,
+// never a floating reconstruction of W (section 14: native kernels consume the ternary
+// planes; section 15: a lossless native kernel).
+#include <mutex>
+
+#include "tern_internal.cuh"
+
+namespace tern {
+
+int sm_count() {
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!cache[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+namespace {
+
+constexpr int64_t kMaxRows = int64_t(1) << 22;    // grid limits of the kernels
+constexpr int64_t kMaxK = int64_t(1) << 20;
+constexpr int64_t kGemvMaxM = 16;
+
+tern_status check_weight(const tern_weight* w) {
+    if (!w) return TERN_ERR_NULL;
+    if (w->N <= 0 || w->K <= 0 || w->K % kGroup || w->group != kGroup) return TERN_ERR_SHAPE;
+    if (w->N > kMaxRows || w->K > kMaxK || w->r < 0 || w->r > w->N) return TERN_ERR_SHAPE;
+    if (!w->plane1 || !w->scale1) return TERN_ERR_NULL;
+    if (w->r > 0 && (!w->plane2 || !w->scale2 || !w->res_slot)) return TERN_ERR_NULL;
+    if (!aligned16(w->plane1) || !aligned16(w->scale1)) return TERN_ERR_ALIGN;
+    if (w->r > 0 && (!aligned16(w->plane2) || !aligned16(w->scale2) || !aligned16(w->res_slot)))
+        return TERN_ERR_ALIGN;
+    return TERN_OK;
+}
+
+}  // namespace
+}  // namespace tern
+
+using namespace tern;
+
+extern "C" size_t tern_linear_workspace_bytes(const tern_weight* w, int64_t M) {
+    if (check_weight(w) != TERN_OK || M <= 0) return 0;
+    const size_t b = M <= kGemvMaxM ? gemv_workspace_bytes(*w, M) : gemm_workspace_bytes(*w, M);
+    return (b + 255) & ~size_t(255);
+}
+
+extern "C" tern_status tern_linear(const tern_weight* w, const tern_half* x, int64_t M, tern_half* y,
+                                   void* workspace, size_t workspace_bytes, tern_stream stream) {
+    const tern_status ws = check_weight(w);
+    if (ws != TERN_OK) return ws;
+    if (M < 0 || M > (int64_t(1) << 31)) return TERN_ERR_SHAPE;
+    if (M == 0) return TERN_OK;
+    if (!x || !y) return TERN_ERR_NULL;
+    if (!aligned16(x) || !aligned16(y)) return TERN_ERR_ALIGN;
+    const size_t need = tern_linear_workspace_bytes(w, M);
+    if (need && (!workspace || workspace_bytes < need)) return TERN_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return TERN_ERR_ALIGN;
+    // x and y must not overlap
+    const uintptr_t xb = reinterpret_cast<uintptr_t>(x), yb = reinterpret_cast<uintptr_t>(y);
+    const uintptr_t xe = xb + size_t(M) * size_t(w->K) * 2, ye = yb + size_t(M) * size_t(w->N) * 2;
+    if (xb < ye && yb < xe) return TERN_ERR_SHAPE;
+    cudaStream_t st = as_cuda(stream);
+    const __half* xh = reinterpret_cast<const __half*>(x);
+    __half* yh = reinterpret_cast<__half*>(y);
+    if (M <= kGemvMaxM) return gemv_launch(*w, xh, int(M), yh, static_cast<float*>(workspace), st);
+    return gemm_launch(*w, xh, M, yh, workspace, st);
+}

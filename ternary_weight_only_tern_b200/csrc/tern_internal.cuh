@@ -1,0 +1,38 @@
+// Internal declarations shared by the libtern.so translation units (not installed).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/tern.h"
+
+namespace tern {
+
+constexpr int kGroup = 128;          // K columns per scale group
+constexpr int kCodesPerWord = 16;    // 2-bit codes per uint32 of the exec plane
+constexpr int kWordsPerGroup = kGroup / kCodesPerWord;
+constexpr int kTritsPerByte = 5;     // base-3 storage
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t as_cuda(tern_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Device-side status words for the synchronous pack/unpack/validate calls (tern_pack.cu).
+// Returns a device pointer to a zeroed slot, or nullptr on a CUDA error.
+unsigned int* acquire_flag_slot(cudaStream_t stream);
+tern_status read_flag_slot(unsigned int* slot, cudaStream_t stream, unsigned int* value);
+
+// Decode GEMV (tern_gemv.cu), M in [1, 16].
+tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y, float* res_ws,
+                        cudaStream_t stream);
+size_t gemv_workspace_bytes(const tern_weight& w, int64_t M);
+
+// Prefill GEMM on tcgen05 (tern_gemm_sm100.cu), M > 16.
+tern_status gemm_launch(const tern_weight& w, const __half* x, int64_t M, __half* y, void* workspace,
+                        cudaStream_t stream);
+size_t gemm_workspace_bytes(const tern_weight& w, int64_t M);
+
+int sm_count();   // of the current device, cached per device
+
+}  // namespace tern

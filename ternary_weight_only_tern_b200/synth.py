@@ -13,6 +13,7 @@ x, T1, s1, residual rows, T2, s2):
   (row, 128-wide K group).
 * residual rows: r = round-half-up(pct% of N) rows drawn uniformly without
   replacement, then sorted.
+* a stack of layers draws layer l from PCG64(SeedSequence([seed, l])).
 
 The projection shapes are those of Qwen3-4B (hidden 2560, intermediate 9728)
 and Qwen3-8B (hidden 4096, intermediate 12288), 36 decoder layers each with the
@@ -134,16 +135,28 @@ WORKLOADS = {
 }
 
 
-def draw_workload(w: Workload, layers: int | None = None, only=None):
+def layer_rng(w: Workload, layer: int) -> np.random.Generator:
+    """PCG64(seed) for a one-layer workload; PCG64(SeedSequence([seed, layer])) per layer of a stack,
+    so that any layer can be drawn on its own."""
+    if w.layers == 1:
+        return np.random.Generator(np.random.PCG64(w.seed))
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([w.seed, layer])))
+
+
+def draw_workload(w: Workload, layers=None, only=None):
     """Yield TernTensor for every (layer, projection) of a workload, x drawn at max(Ms) rows.
 
-    ``layers`` caps the number of layers drawn; ``only`` restricts to projection names
-    (the skipped projections are still drawn, so a projection's arrays do not depend on it).
+    ``layers`` is a count (the first n layers) or a list of layer indices; ``only`` restricts
+    to projection names (the skipped projections are still drawn, so a projection's arrays do
+    not depend on it).
     """
-    rng = np.random.Generator(np.random.PCG64(w.seed))
-    n_layers = w.layers if layers is None else min(layers, w.layers)
+    if layers is None or isinstance(layers, int):
+        layer_ids = range(w.layers if layers is None else min(layers, w.layers))
+    else:
+        layer_ids = list(layers)
     M = max(w.Ms)
-    for layer in range(n_layers):
+    for layer in layer_ids:
+        rng = layer_rng(w, layer)
         for (name, N, K) in w.shapes:
             t = draw_tensor(rng, name, N, K, M, p_zero=w.p_zero, res_pct=w.res_pct,
                             s1_range=w.s1_range, s2_range=w.s2_range)

@@ -1,0 +1,127 @@
+"""The C-ABI library loads and exports every function include/tern.h declares; host-side
+logic (bit accounting, argument validation) needs no GPU and is checked here."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from ternary_weight_only_tern_b200 import _lib, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "tern.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tern_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from ternary_weight_only_tern_b200 import build
+        build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_boundary():
+    fns = header_functions()
+    for name in ["tern_pack_exec", "tern_unpack_exec", "tern_pack_store", "tern_unpack_store",
+                 "tern_linear_workspace_bytes", "tern_linear", "tern_bits", "tern_status_string"]:
+        assert name in fns
+    assert set(fns) == set(_lib.EXPORTS), "ctypes declarations and header disagree"
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+    assert lib.tern_version() >= 100
+
+
+def test_status_strings(lib):
+    for code in range(10):
+        assert lib.tern_status_string(code)
+    assert lib.tern_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("N,K,r", [(4096, 2560, 0), (9728, 2560, 973), (12288, 4096, 1843), (13, 384, 13),
+                                   (1024, 12288, 154), (1, 128, 1)])
+def test_tern_bits_equals_oracle(lib, N, K, r):
+    rep = _lib.TernBitsReport()
+    assert lib.tern_bits(N, K, r, 128, ctypes.byref(rep)) == 0
+    ref = oracle.bits(N, K, r)
+    for f in ("weights", "plane_trits", "store_bits", "exec_bits"):
+        assert getattr(rep, f) == ref[f], f
+    for f in ("bpw_info", "bpw_store", "bpw_exec"):
+        assert getattr(rep, f) == pytest.approx(ref[f], rel=1e-15, abs=0), f
+
+
+def test_tern_bits_whole_stack(lib):
+    # the 252 targeted tensors of the 4B model at 10% residual rows: sum of per-tensor integers
+    rep = _lib.TernBitsReport()
+    tot = {"weights": 0, "store_bits": 0, "exec_bits": 0}
+    for (_, N, K) in synth.WORKLOADS[3].shapes:
+        r = synth.residual_count(N, 10)
+        assert lib.tern_bits(N, K, r, 128, ctypes.byref(rep)) == 0
+        for k in tot:
+            tot[k] += synth.N_LAYERS * getattr(rep, k)
+    assert tot["weights"] == 3_633_315_840       # = 36 * (4096+2048)*2560 + 2560*4096 + 3*9728*2560 ...
+    assert 1.7 < tot["store_bits"] / tot["weights"] < 2.0
+
+
+def test_tern_bits_rejects(lib):
+    rep = _lib.TernBitsReport()
+    S = _lib.STATUS
+    assert lib.tern_bits(0, 128, 0, 128, ctypes.byref(rep)) == S["TERN_ERR_SHAPE"]
+    assert lib.tern_bits(16, 100, 0, 128, ctypes.byref(rep)) == S["TERN_ERR_SHAPE"]
+    assert lib.tern_bits(16, 128, 0, 64, ctypes.byref(rep)) == S["TERN_ERR_SHAPE"]
+    assert lib.tern_bits(16, 128, 17, 128, ctypes.byref(rep)) == S["TERN_ERR_SHAPE"]
+    assert lib.tern_bits(16, 128, 0, 128, None) == S["TERN_ERR_NULL"]
+
+
+def test_linear_host_validation(lib):
+    """Every check here fails before a launch, so no device is touched."""
+    S = _lib.STATUS
+    fake = 1 << 20         # an aligned non-null address that is never dereferenced on these paths
+    w = _lib.TernWeightC(64, 256, 128, fake, fake, 0, None, fake, None, None)
+    call = lambda w, x, M, y, ws=None, wsb=0: lib.tern_linear(  # noqa: E731
+        ctypes.byref(w) if w is not None else None, x, M, y, ws, wsb, None)
+    assert call(None, fake, 1, fake) == S["TERN_ERR_NULL"]
+    assert call(w, fake, 0, fake) == S["TERN_OK"]                 # M == 0 is a no-op
+    assert call(w, None, 1, fake) == S["TERN_ERR_NULL"]
+    assert call(w, fake + 2, 1, fake * 4) == S["TERN_ERR_ALIGN"]
+    assert call(w, fake, 1, fake) == S["TERN_ERR_SHAPE"]          # x and y overlap
+    assert call(w, fake, -1, fake) == S["TERN_ERR_SHAPE"]
+    bad = _lib.TernWeightC(64, 200, 128, fake, fake, 0, None, fake, None, None)
+    assert call(bad, fake, 1, fake * 4) == S["TERN_ERR_SHAPE"]
+    bad = _lib.TernWeightC(64, 256, 64, fake, fake, 0, None, fake, None, None)
+    assert call(bad, fake, 1, fake * 4) == S["TERN_ERR_SHAPE"]
+    bad = _lib.TernWeightC(64, 256, 128, fake, fake, 65, fake, fake, fake, fake)
+    assert call(bad, fake, 1, fake * 4) == S["TERN_ERR_SHAPE"]    # r > N
+    bad = _lib.TernWeightC(64, 256, 128, fake, fake, 4, fake, fake, None, fake)
+    assert call(bad, fake, 1, fake * 4) == S["TERN_ERR_NULL"]     # residual plane missing
+    bad = _lib.TernWeightC(64, 256, 128, fake + 4, fake, 0, None, fake, None, None)
+    assert call(bad, fake, 1, fake * 4) == S["TERN_ERR_ALIGN"]
+    # a residual weight needs workspace for the decode path
+    wr = _lib.TernWeightC(64, 256, 128, fake, fake, 4, fake, fake, fake, fake)
+    need = lib.tern_linear_workspace_bytes(ctypes.byref(wr), 3)
+    assert need >= 3 * 4 * 4 and need % 256 == 0
+    assert call(wr, fake, 3, fake * 4) == S["TERN_ERR_WORKSPACE"]
+    assert call(wr, fake, 3, fake * 4, fake * 8, need - 1) == S["TERN_ERR_WORKSPACE"]
+    assert lib.tern_linear_workspace_bytes(ctypes.byref(w), 16) == 0
+
+
+def test_pack_host_validation(lib):
+    S = _lib.STATUS
+    fake = 1 << 20
+    assert lib.tern_pack_exec(fake, 4, 17, fake * 2, None) == S["TERN_ERR_SHAPE"]
+    assert lib.tern_pack_exec(None, 4, 16, fake, None) == S["TERN_ERR_NULL"]
+    assert lib.tern_pack_exec(fake + 1, 4, 16, fake * 2, None) == S["TERN_ERR_ALIGN"]
+    assert lib.tern_pack_exec(fake, 0, 16, fake * 2, None) == S["TERN_OK"]
+    assert lib.tern_unpack_exec(fake, -1, 16, fake * 2, None) == S["TERN_ERR_SHAPE"]
+    assert lib.tern_pack_store(None, 4, 7, fake, None) == S["TERN_ERR_NULL"]
+    assert lib.tern_unpack_store(fake, 4, -7, fake, None) == S["TERN_ERR_SHAPE"]
+    assert lib.tern_weight_validate(None, None) == S["TERN_ERR_NULL"]

@@ -1,0 +1,183 @@
+"""GPU parity of tern_linear against the float64 oracle.
+
+Bar: max|y - y_ref| / max|y_ref| <= 2e-3 with no NaN/Inf on seeded synthetic inputs, and
+bit-exact equality with the oracle's single fp16 rounding on inputs where fp32 accumulation is
+exact. Full-size shapes of all five workloads run in the launch configuration the bench times;
+where the oracle would be slow (the 36-layer stack, M = 2048) it computes sampled output
+columns for every token.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from ternary_weight_only_tern_b200 import api, synth
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3
+
+
+def run(t: synth.TernTensor, M: int, weight=None):
+    w = weight or api.TernWeight.from_numpy(t.T1, t.s1, t.res_rows, t.T2, t.s2)
+    x = torch.from_numpy(np.ascontiguousarray(t.x[:M])).cuda()
+    y = api.linear(x, w)
+    torch.cuda.synchronize()
+    return y.cpu().numpy(), w
+
+
+def check(y, y_ref, tol=TOL):
+    assert np.isfinite(y).all()
+    err = oracle.rel_err(y.astype(np.float64), y_ref)
+    assert err <= tol, f"rel err {err:.3e}"
+    return err
+
+
+def test_config1_single_gemv():
+    t = next(synth.draw_workload(synth.WORKLOADS[1]))
+    y, _ = run(t, 1)
+    check(y, oracle.linear(t.x[:1], t.T1, t.s1, t.res_rows, t.T2, t.s2))
+
+
+@pytest.mark.parametrize("name", list(synth.QWEN3_4B))
+def test_config2_4b_layer(name):
+    t = next(synth.draw_workload(synth.WORKLOADS[2], only=[name]))
+    y, _ = run(t, 1)
+    check(y, oracle.linear(t.x[:1], t.T1, t.s1, t.res_rows, t.T2, t.s2))
+
+
+@pytest.mark.parametrize("name", list(synth.QWEN3_8B))
+def test_config4_8b_projections_all_M(name):
+    t = next(synth.draw_workload(synth.WORKLOADS[4], only=[name]))
+    y_ref = oracle.linear(t.x, t.T1, t.s1, t.res_rows, t.T2, t.s2)       # 16 tokens
+    w = None
+    for M in synth.WORKLOADS[4].Ms:
+        y, w = run(t, M, w)
+        check(y, y_ref[:M])
+
+
+@pytest.mark.parametrize("layer", [0, 17, 35])
+def test_config3_4b_stack_sampled(layer):
+    rng = np.random.default_rng(layer)
+    for t in synth.draw_workload(synth.WORKLOADS[3], layers=[layer]):
+        cols = np.unique(np.concatenate([rng.choice(t.N, 48, replace=False), t.res_rows[:16]]))
+        y_ref = oracle.linear(t.x, t.T1, t.s1, t.res_rows, t.T2, t.s2, cols=cols)
+        w = None
+        for M in synth.WORKLOADS[3].Ms:
+            y, w = run(t, M, w)
+            check(y[:, cols], y_ref[:M])
+
+
+@pytest.mark.parametrize("name", ["gate", "down"])
+def test_config5_prefill_sampled(name):
+    t = next(synth.draw_workload(synth.WORKLOADS[5], only=[name]))
+    rng = np.random.default_rng(5)
+    cols = np.unique(np.concatenate([rng.choice(t.N, 40, replace=False), t.res_rows[:24]]))
+    y_ref = oracle.linear(t.x, t.T1, t.s1, t.res_rows, t.T2, t.s2, cols=cols)
+    y, _ = run(t, 2048)
+    check(y[:, cols], y_ref)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 9, 15, 16, 17, 100, 511, 513])
+def test_odd_M(M):
+    rng = np.random.default_rng(100 + M)
+    t = synth.draw_tensor(rng, "odd", 320, 1152, M, p_zero=0.4, res_pct=10)
+    y, _ = run(t, M)
+    check(y, oracle.linear(t.x, t.T1, t.s1, t.res_rows, t.T2, t.s2))
+
+
+@pytest.mark.parametrize("N,K,r", [(100, 128, 7), (1, 128, 1), (1000 + 7, 384, 0), (77, 12288, 77), (64, 256, 64),
+                                   (4096 + 48, 2560, 300)])
+def test_ragged_and_degenerate_shapes(N, K, r):
+    rng = np.random.default_rng(N + K + r)
+    t = synth.draw_tensor(rng, "rag", N, K, 16, p_zero=0.4, res_pct=0)
+    rr = np.sort(rng.choice(N, r, replace=False)).astype(np.int32)
+    T2 = synth.draw_trits(rng, (r, K), 0.4)
+    s2 = synth.draw_scales(rng, r, K, 0.001, 0.005)
+    t = synth.TernTensor("rag", N, K, t.x, t.T1, t.s1, rr, T2, s2)
+    y_ref = oracle.linear(t.x, t.T1, t.s1, rr, T2, s2)
+    w = None
+    for M in (1, 7, 16):
+        y, w = run(t, M, w)
+        check(y, y_ref[:M])
+
+
+@pytest.mark.parametrize("M", [1, 4, 8, 16, 24, 300])
+@pytest.mark.parametrize("N,K,r", [(256, 512, 40), (1024, 4096, 154), (130, 12288, 13)])
+def test_exact_case_bit_exact(M, N, K, r):
+    rng = np.random.default_rng(M * 31 + N + K)
+    t = synth.draw_exact_tensor(rng, N, K, M, r)
+    y, _ = run(t, M)
+    y_ref = oracle.round_fp16(oracle.linear(t.x, t.T1, t.s1, t.res_rows, t.T2, t.s2))
+    assert np.array_equal(y.view(np.uint16), y_ref.view(np.uint16))
+
+
+def test_special_cases():
+    rng = np.random.default_rng(77)
+    N, K, M = 192, 512, 16
+    x = synth.draw_x(rng, M, K)
+    s1 = synth.draw_scales(rng, N, K, 0.005, 0.02)
+    none = (np.zeros(0, np.int32), np.zeros((0, K), np.int8), np.zeros((0, K // 128), np.float16))
+    # zero plane -> exactly zero
+    t = synth.TernTensor("z", N, K, x, np.zeros((N, K), np.int8), s1, *none)
+    y, _ = run(t, M)
+    assert (y == 0).all()
+    # all +1: s times group sums
+    t = synth.TernTensor("p", N, K, x, np.ones((N, K), np.int8), s1, *none)
+    y, _ = run(t, M)
+    check(y, oracle.linear(x, t.T1, s1, *none))
+    # r = N with T2 = T1, s2 = s1 doubles the r = 0 result
+    T1 = synth.draw_trits(rng, (N, K), 0.4)
+    y1, _ = run(synth.TernTensor("a", N, K, x, T1, s1, *none), M)
+    y2, _ = run(synth.TernTensor("b", N, K, x, T1, s1, np.arange(N, dtype=np.int32), T1, s1), M)
+    check(y2, 2 * y1.astype(np.float64), tol=1e-3)
+
+
+def test_out_shape_is_checked():
+    t = next(synth.draw_workload(synth.WORKLOADS[1]))
+    w = api.TernWeight.from_numpy(t.T1, t.s1, t.res_rows, t.T2, t.s2)
+    x = torch.from_numpy(t.x).cuda()
+    with pytest.raises(ValueError):
+        api.linear(x, w, out=torch.empty((2, t.N), dtype=torch.float16, device="cuda"))
+
+
+def test_deterministic_and_m0():
+    t = next(synth.draw_workload(synth.WORKLOADS[4], only=["q"]))
+    y1, w = run(t, 16)
+    y2, _ = run(t, 16, w)
+    assert np.array_equal(y1.view(np.uint16), y2.view(np.uint16))
+    x = torch.empty((0, t.K), dtype=torch.float16, device="cuda")
+    assert api.linear(x, w).shape == (0, t.N)
+
+
+@pytest.mark.parametrize("M", [3, 40])
+def test_non_finite_activations_propagate(M):
+    """A token with an inf or NaN activation gets non-finite outputs (the oracle's IEEE sums give
+    +-inf or NaN there); the other tokens stay finite and within tolerance."""
+    rng = np.random.default_rng(3)
+    t = synth.draw_tensor(rng, "nan", 64, 256, M, p_zero=0.4, res_pct=10)
+    x = t.x.copy()
+    x[0, 5] = np.inf
+    x[1, 7] = np.nan
+    t = synth.TernTensor("n", 64, 256, x, t.T1, t.s1, t.res_rows, t.T2, t.s2)
+    y, _ = run(t, M)
+    with np.errstate(invalid="ignore"):
+        y_ref = oracle.linear(x, t.T1, t.s1, t.res_rows, t.T2, t.s2)
+    assert not np.isfinite(y_ref[:2]).any()
+    assert not np.isfinite(y[:2]).any()
+    check(y[2:], y_ref[2:])
+
+
+def test_workspace_and_output_untouched_outside_bounds():
+    t = next(synth.draw_workload(synth.WORKLOADS[4], only=["k"]))
+    w = api.TernWeight.from_numpy(t.T1, t.s1, t.res_rows, t.T2, t.s2)
+    M = 16
+    assert t.x.shape[0] == M
+    need = api.workspace_bytes(w, M)
+    ws = torch.full((need + 4096,), 0xA5, dtype=torch.uint8, device="cuda")
+    yb = torch.full((M * t.N + 4096,), 7.0, dtype=torch.float16, device="cuda")
+    x = torch.from_numpy(t.x[:M]).cuda()
+    api.linear(x, w, out=yb[: M * t.N].view(M, t.N), workspace=ws)
+    torch.cuda.synchronize()
+    assert (ws[need:] == 0xA5).all() and (yb[M * t.N:] == 7.0).all()
+    check(yb[: M * t.N].view(M, t.N).cpu().numpy(), oracle.linear(t.x[:M], t.T1, t.s1, t.res_rows, t.T2, t.s2))
