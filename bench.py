@@ -121,6 +121,23 @@ def gpu_uuid(torch, dev):
         return str(dev.index or 0)
 
 
+# ------------------------------------------------------------------------------ replicas
+def max_over_ranks_of(dist, v: float, device=None) -> float:
+    """The largest of every rank's v (all ranks call it, in the same order); v itself on one rank."""
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_value(world: int, units_per_rank: float, max_secs: float) -> float:
+    """Whole-job throughput of `world` replicas that each processed `units_per_rank` units,
+    timed as the slowest rank."""
+    return world * units_per_rank / max_secs
+
+
 # ------------------------------------------------------------------------------ workload
 def draw_layer_on_device(torch, api, shapes, dev, seed):
     """One layer's projections, drawn on the device with a seeded torch generator (same
@@ -144,7 +161,9 @@ def draw_layer_on_device(torch, api, shapes, dev, seed):
         rows = torch.randperm(N, generator=g, device=dev)[:r].sort().values.to(torch.int32)
         T2 = trits(r)
         s2 = (torch.rand((r, G), generator=g, device=dev) * 0.004 + 0.001).half()
-        out[name] = api.TernWeight.from_trits(T1, s1, rows, T2, s2)
+        w = api.TernWeight.from_trits(T1, s1, rows, T2, s2)
+        w.static = True            # model weights: nothing queued before a call writes them
+        out[name] = w
         del T1, T2
     return out
 
@@ -249,6 +268,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="skip the extra measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline")
+    ap.add_argument("--profile", choices=["gemv", "gemm"], default=None,
+                    help="run a few calls of one op on one pool layer and exit (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -277,19 +298,18 @@ def main():
             dist.barrier()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks_of(dist if world > 1 else None, v, dev)
 
     peaks, peak_kind = load_peaks()
     shapes = list(synth.WORKLOADS[4].shapes)
+    if args.profile:
+        return profile_case(torch, api, shapes, dev, args.profile)
     pool = [draw_layer_on_device(torch, api, shapes, dev, seed=1000 + i) for i in range(POOL_LAYERS)]
     torch.cuda.synchronize()
     names = [s[0] for s in shapes]
     Kmax = max(K for _, _, K in shapes)
     ws = torch.empty(max(api.workspace_bytes(pool[0][n], 16) for n in names) + 256, dtype=torch.uint8, device=dev)
+    launches_per_call = 1
     stream = torch.cuda.Stream(device=dev)
     gen = torch.Generator(device=dev)
     gen.manual_seed(7)
@@ -317,7 +337,7 @@ def main():
     # ---------------- the timed region: K graph replays of the full M = 1 step
     xs1, ys1 = make_io(1)
     g_step = capture(torch, step_fn(1, xs1, ys1), stream)
-    launches_per_step = sum(2 if pool[l % POOL_LAYERS][n].r > 0 else 1 for l in range(LAYERS) for n in names)
+    launches_per_step = LAYERS * len(names) * launches_per_call
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             g_step.replay()
@@ -330,7 +350,7 @@ def main():
     barrier()
     secs = max_over_ranks(secs)
     wb, ab = step_bytes(1)
-    value = world * wb * args.steps / secs / 1e9
+    value = replica_value(world, wb * args.steps, secs) / 1e9
     ms_per_step = secs / args.steps * 1e3
 
     # ---------------- the dominant op: the gate projection's tern_linear at M = 1
@@ -406,6 +426,23 @@ def main():
         "gpu_launches": launches_per_step * args.steps, "clocks": clk.summary(), "extra": extra,
     }
     print(json.dumps(line), flush=True)
+
+
+def profile_case(torch, api, shapes, dev, which):
+    """A minimal run for ncu: the 7 projections of two layers at M = 1 (gemv), or gate, up and
+    down at M = 2048 (gemm), each called three times in the order q, k, v, o, gate, up, down."""
+    pool = [draw_layer_on_device(torch, api, shapes, dev, seed=1000 + i) for i in range(2)]
+    names = ["q", "k", "v", "o", "gate", "up", "down"] if which == "gemv" else ["gate", "up", "down"]
+    M = 1 if which == "gemv" else 2048
+    xs = {n: torch.randn((M, K), device=dev).half() for n, _, K in shapes}
+    ys = {n: torch.empty((M, N), dtype=torch.float16, device=dev) for n, N, _ in shapes}
+    torch.cuda.synchronize()
+    for _ in range(3):
+        for layer in pool:
+            for n in names:
+                api.linear(xs[n], layer[n], out=ys[n])
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": which, "calls": 3 * len(pool) * len(names)}))
 
 
 def extras(torch, api, synth, pool, shapes, names, stream, dev, ws, step_fn, step_bytes, make_io, peaks,

@@ -68,7 +68,7 @@ typedef enum {
                                 or inconsistent with the slot map */
     TERN_ERR_WORKSPACE = 7,  /* workspace smaller than tern_linear_workspace_bytes() or NULL */
     TERN_ERR_CUDA = 8,       /* a CUDA runtime call failed (launch error, no device, ...) */
-    TERN_ERR_TIMEOUT = 9     /* reserved: a bounded device-side wait ran out */
+    TERN_ERR_TIMEOUT = 9     /* a bounded device-side wait ran out (see tern_device_status) */
 } tern_status;
 
 /* A ternarized weight W [N, K] in execution form. Every pointer is device memory,
@@ -84,7 +84,14 @@ typedef struct {
     const int32_t* res_slot;     /* [N] -1, or rho(n) for n in R                        */
     const uint32_t* plane2;      /* [r, K/16]   exec codes of T2                        */
     const tern_half* scale2;     /* [r, K/128]  s2                                      */
+    uint32_t flags;              /* 0 or TERN_WEIGHT_STATIC                             */
 } tern_weight;
+
+/* tern_weight.flags: the planes, scales and slot map are not written by work queued before
+ * the call on its stream (model weights). tern_linear may then start reading them while the
+ * previous kernel on the stream is still running (programmatic dependent launch); x is
+ * always read only after that kernel has finished.                                      */
+#define TERN_WEIGHT_STATIC 1u
 
 /* ---------------------------------------------------------------- packing (offline) */
 
@@ -146,6 +153,11 @@ typedef struct {
  * a 64-byte header). 4B paper, sections 3.2, 4.4 and 7.1 (1.641 effective bits against the
  * ideal 1.585); 8B paper, effective-bits equation. Pure host function.                  */
 tern_status tern_bits(int64_t N, int64_t K, int64_t r, int32_t group, tern_bits_report* out);
+
+/* Reports, and clears, the current device's sticky status word for asynchronous work: returns
+ * TERN_ERR_TIMEOUT if a tern_linear kernel since the last call gave up a bounded device-side
+ * wait (its output is then undefined), else TERN_OK. Synchronous on `stream`.            */
+tern_status tern_device_status(tern_stream stream);
 
 /* A static, human-readable name for a status code. */
 const char* tern_status_string(tern_status s);

@@ -86,6 +86,7 @@ class TernWeight:
     res_slot: torch.Tensor   # int32 [N]
     plane2: torch.Tensor     # int32 [r, K/16]
     scale2: torch.Tensor     # float16 [r, K/128]
+    static: bool = False     # weights not written by queued work: tern_linear may prefetch them early
 
     @property
     def r(self) -> int:
@@ -101,7 +102,8 @@ class TernWeight:
             c = _lib.TernWeightC(
                 self.N, self.K, GROUP, self.plane1.data_ptr(), self.scale1.data_ptr(), self.r,
                 self.res_rows.data_ptr() if self.r else None, self.res_slot.data_ptr(),
-                self.plane2.data_ptr() if self.r else None, self.scale2.data_ptr() if self.r else None)
+                self.plane2.data_ptr() if self.r else None, self.scale2.data_ptr() if self.r else None,
+                _lib.WEIGHT_STATIC if self.static else 0)
             object.__setattr__(self, "_c", c)
         return c
 

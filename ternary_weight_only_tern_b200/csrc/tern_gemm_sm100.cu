@@ -1,20 +1,532 @@
-// Prefill path (M > 16). Placeholder: runs the decode GEMV on 16-row chunks of x.
+// Prefill GEMM (M > 16): y[M, N] = x[M, K] . W^T on tcgen05 tensor cores, W dequantised from
+// the packed ternary planes straight into shared memory.
+//
+// The operation is that of "Post-Training Ternarization of Qwen3-4B" (arXiv 2609.01962v1),
+// sections 4.3-4.5: W = s1 (.) T1, plus s2 (.) T2 on the residual rows, fp16 activations
+// (section 3.1). At M in the thousands it is a dense contraction, so it runs on the tensor
+// cores; the weights are never reconstructed in global memory (section 14: native kernels
+// consume the ternary planes directly).
+//
+// One CTA computes a 128 (tokens) x 256 (weight rows) tile with one tcgen05.mma
+// (kind::f16, M = 128, N = 256, K = 16, fp32 accumulator in TMEM) per 16 columns of K:
+//  * warp 0, one thread: TMA loads of the x tile (128 x 64 fp16, 128-byte swizzle) into a
+//    3-stage ring, and TMA loads of the packed codes of the tile's 256 weight rows (16 bytes
+//    per row per K block) and of its residual rows into an 8-stage ring that runs ahead;
+//  * warp 1, one thread: issues the MMAs and commits each stage back to the producers;
+//  * warps 2-9 (256 threads, one weight row each): per 64-wide K block, read the row's 16
+//    bytes of 2-bit codes from shared memory, decode them to exact fp16 s1 * t1 (two trits
+//    per LOP3 into fp16 magic values, one subtract, one multiply), and store the row's 128
+//    bytes in the 128-byte swizzled K-major layout the MMA reads. Rows of the residual set
+//    then get RN(s1*t1 + s2*t2) with one fused multiply-add. Scales are loaded two groups
+//    ahead. After the K loop the same warps read the accumulator from TMEM and write y.
+//  * every wait is bounded: after about two seconds the kernel records TERN_ERR_TIMEOUT in
+//    a device status word, drains its own copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "tern_internal.cuh"
 
 namespace tern {
+namespace {
 
-size_t gemm_workspace_bytes(const tern_weight& w, int64_t M) {
-    return gemv_workspace_bytes(w, M < 16 ? M : 16);
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int kStages = 3;                          // x tile + dequantised W tile
+constexpr int kStagesP = 8;                         // packed codes
+constexpr int kDequantThreads = 256;
+constexpr int kThreads = 64 + kDequantThreads;
+constexpr int kABytes = BM * BK * 2;
+constexpr int kBBytes = BN * BK * 2;
+constexpr int kPBytes = BN * 16;                    // 16 bytes (64 trits) of codes per row
+constexpr int kResBox = 32;                         // residual rows per TMA box
+constexpr int kTmemCols = 256;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // bounded waits give up after ~2 s
+constexpr unsigned kTimeoutBit = 1u;
+
+struct GemmArgs {
+    const uint32_t* plane1;
+    const __half* scale1;
+    const uint32_t* plane2;
+    const __half* scale2;
+    const int32_t* res_slot;
+    int64_t N, K, r, M;
+    int32_t G;
+    __half* y;
+    unsigned int* status;
+};
+
+struct SmemLayout {
+    static constexpr int a_off = 0;
+    static constexpr int b_off = a_off + kStages * kABytes;
+    static constexpr int p1_off = b_off + kStages * kBBytes;                    // [kStagesP][256][16 B]
+    static constexpr int p2_off = p1_off + kStagesP * kPBytes;                  // [kStagesP][256][16 B]
+    static constexpr int bar_off = p2_off + kStagesP * kPBytes;
+    static constexpr int nbar = 3 * kStages + 2 * kStagesP + 1;
+    static constexpr int tmem_off = bar_off + nbar * 8;
+    static constexpr int cnt_off = tmem_off + 16;                               // 8 warp counts + total
+    static constexpr int list_off = cnt_off + 48;                               // int2 [BN]
+    static constexpr int bytes = list_off + BN * 8;
+};
+constexpr size_t kSmemBytes = SmemLayout::bytes + 1024;                          // + alignment slack
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+
+// ------------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-tern_status gemm_launch(const tern_weight& w, const __half* x, int64_t M, __half* y, void* workspace,
-                        cudaStream_t stream) {
-    for (int64_t m0 = 0; m0 < M; m0 += 16) {
-        const int mc = int(M - m0 < 16 ? M - m0 : 16);
-        const tern_status st = gemv_launch(w, x + m0 * w.K, mc, y + m0 * w.N, static_cast<float*>(workspace), stream);
-        if (st != TERN_OK) return st;
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait for the phase of the given parity: false after about two seconds.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    const uint32_t addr = smem_u32(bar);
+    uint64_t t0 = 0;
+    for (uint32_t i = 0;; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(addr), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if ((i & 255u) == 0) {
+            const uint64_t t = global_ns();
+            if (i == 0) t0 = t;
+            else if (t - t0 > kWaitLimitNs) return false;
+        }
     }
-    return TERN_OK;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t umma_desc_sw128(const void* p) {
+    const uint64_t addr = smem_u32(p);
+    return ((addr & 0x3FFFFull) >> 4) | (1ull << 16) | (uint64_t(1024 >> 4) << 32) | (1ull << 46) |
+           (2ull << 61);
+}
+
+// Instruction descriptor: kind::f16, A = B = fp16, D = fp32, both K-major, M = BM, N = BN.
+constexpr uint32_t kIdesc = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t a_desc, uint64_t b_desc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(a_desc), "l"(b_desc), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// AND of `pred` over the 256 dequantising threads (named barrier 1); every one of them must call it.
+__device__ __forceinline__ bool dequant_all(bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.and.pred q, 1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(uint32_t(pred)), "n"(kDequantThreads)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(magic));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// Eight consecutive trits (the codes in the low 16 bits of v) as four fp16x2 pairs of exact t,
+// natural order: (t0, t1), (t2, t3), (t4, t5), (t6, t7). Spreading v | v << 14 puts the codes of
+// trits 2j and 2j+1 at bits 4j and 16 + 4j; a LOP3 writes them into the mantissa of a power of
+// two B (1024 + c, 64 + c, 4 + c), and subtracting B + 1 leaves t = c - 1 exactly.
+__device__ __forceinline__ void decode8(uint32_t v, __half2 (&t)[4]) {
+    const uint32_t u = v | (v << 14);
+    t[0] = __hsub2(bits_h2(lop3_and_or(u, 0x00030003u, 0x64006400u)), bits_h2(0x64016401u));       // 1024 + 1
+    t[1] = __hsub2(bits_h2(lop3_and_or(u, 0x00300030u, 0x54005400u)), bits_h2(0x54105410u));       // 64 + 1
+    t[2] = __hsub2(bits_h2(lop3_and_or(u, 0x03000300u, 0x44004400u)), bits_h2(0x45004500u));       // 4 + 1
+    t[3] = __hsub2(bits_h2(lop3_and_or(u >> 4, 0x03000300u, 0x44004400u)), bits_h2(0x45004500u));
+}
+
+// Byte offset of 16-byte chunk c (K columns 8c .. 8c+7) of row n in a 128-byte swizzled tile.
+__device__ __forceinline__ uint32_t sw128_offset(int n, int c) {
+    return uint32_t(n) * 128u + uint32_t((c ^ (n & 7)) << 4);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                                                           const __grid_constant__ CUtensorMap tmap_p1,
+                                                           const __grid_constant__ CUtensorMap tmap_p2,
+                                                           const GemmArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem_a = smem + SmemLayout::a_off;
+    uint8_t* smem_b = smem + SmemLayout::b_off;
+    uint8_t* smem_p1 = smem + SmemLayout::p1_off;
+    uint8_t* smem_p2 = smem + SmemLayout::p2_off;
+    uint64_t* full_a = reinterpret_cast<uint64_t*>(smem + SmemLayout::bar_off);
+    uint64_t* full_b = full_a + kStages;
+    uint64_t* empty = full_b + kStages;
+    uint64_t* full_p = empty + kStages;
+    uint64_t* empty_p = full_p + kStagesP;
+    uint64_t* tmem_full = empty_p + kStagesP;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SmemLayout::tmem_off);
+    int* counts = reinterpret_cast<int*>(smem + SmemLayout::cnt_off);
+    int2* res_list = reinterpret_cast<int2*>(smem + SmemLayout::list_off);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t n0 = int64_t(blockIdx.x) * BN;
+    const int64_t m0 = int64_t(blockIdx.y) * BM;
+    const int num_kb = int(a.K / BK);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full_a[s], 1);
+            mbar_init(&full_b[s], kDequantThreads);
+            mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < kStagesP; ++s) {
+            mbar_init(&full_p[s], 1);
+            mbar_init(&empty_p[s], kDequantThreads);
+        }
+        mbar_init(tmem_full, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_async_smem();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    // Residual rows of this tile: (local row, slot) in row order. Their slots are contiguous
+    // (R is sorted), so their codes come in with TMA boxes starting at the first slot.
+    int my_slot = -1;
+    unsigned res_ballot = 0;
+    if (warp >= 2) {
+        const int t = threadIdx.x - 64;
+        const int64_t n = n0 + t;
+        if (a.r > 0 && n < a.N) {
+            const int s = a.res_slot[n];
+            if (s >= 0 && s < a.r) my_slot = s;
+        }
+        res_ballot = __ballot_sync(0xffffffffu, my_slot >= 0);
+        if (lane == 0) counts[warp - 2] = __popc(res_ballot);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    int n_res = 0;
+    for (int w = 0; w < 8; ++w) n_res += counts[w];
+    if (warp >= 2 && my_slot >= 0) {
+        int base = 0;
+        for (int w = 0; w < warp - 2; ++w) base += counts[w];
+        const int pos = base + __popc(res_ballot & ((1u << lane) - 1u));
+        res_list[pos] = make_int2(threadIdx.x - 64, my_slot);
+    }
+    __syncthreads();
+    const int s_lo = n_res > 0 ? res_list[0].y : 0;
+    const int res_boxes = (n_res + kResBox - 1) / kResBox;
+
+    bool ok = true;
+    if (warp == 0) {
+        if (lane == 0) {
+            int issued = 0, p_issued = 0;
+            for (int kb = 0; kb < num_kb && ok; ++kb) {
+                // codes run up to kStagesP blocks ahead of x
+                for (; p_issued < num_kb && p_issued < kb + kStagesP && ok; ++p_issued) {
+                    const int sp = p_issued % kStagesP;
+                    if (p_issued >= kStagesP) ok = mbar_wait(&empty_p[sp], ((p_issued / kStagesP) - 1) & 1);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&full_p[sp], uint32_t(kPBytes + res_boxes * kResBox * 16));
+                    tma_load_2d(smem_p1 + sp * kPBytes, &tmap_p1, p_issued * (BK / kCodesPerWord), int(n0), &full_p[sp]);
+                    for (int j = 0; j < res_boxes; ++j)
+                        tma_load_2d(smem_p2 + sp * kPBytes + j * kResBox * 16, &tmap_p2,
+                                    p_issued * (BK / kCodesPerWord), s_lo + j * kResBox, &full_p[sp]);
+                }
+                if (!ok) break;
+                const int s = kb % kStages;
+                if (kb >= kStages) ok = mbar_wait(&empty[s], ((kb / kStages) - 1) & 1);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&full_a[s], kABytes);
+                tma_load_2d(smem_a + s * kABytes, &tmap_x, kb * BK, int(m0), &full_a[s]);
+                issued = kb + 1;
+            }
+            // drain: every issued copy lands before the CTA may exit
+            for (int kb = issued - 1; kb >= 0 && kb >= issued - kStages; --kb)
+                if (!mbar_wait(&full_a[kb % kStages], (kb / kStages) & 1)) ok = false;
+            for (int kb = p_issued - 1; kb >= 0 && kb >= p_issued - kStagesP; --kb)
+                if (!mbar_wait(&full_p[kb % kStagesP], (kb / kStagesP) & 1)) ok = false;
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            for (int kb = 0; kb < num_kb && ok; ++kb) {
+                const int s = kb % kStages;
+                const uint32_t par = (kb / kStages) & 1;
+                ok = mbar_wait(&full_a[s], par) && mbar_wait(&full_b[s], par);
+                if (!ok) break;
+                tc_fence_after();
+                const uint8_t* as = smem_a + s * kABytes;
+                const uint8_t* bs = smem_b + s * kBBytes;
+#pragma unroll
+                for (int k = 0; k < BK / 16; ++k)
+                    umma_f16(tmem_base, umma_desc_sw128(as + 32 * k), umma_desc_sw128(bs + 32 * k),
+                             (kb > 0 || k > 0) ? 1u : 0u);
+                umma_commit(&empty[s]);
+            }
+            umma_commit(tmem_full);          // also on a timeout: every issued MMA retires first
+            if (!mbar_wait(tmem_full, 0)) ok = false;
+        }
+    } else {
+        // ---------------- dequantise W into the swizzled B stages
+        const int t = threadIdx.x - 64;
+        const int64_t n = n0 + t;
+        const bool valid = n < a.N;
+        const __half* srow = a.scale1 + (valid ? n : 0) * int64_t(a.G);
+        // scales of this row two groups ahead; residual items (row i = item / 8, chunk item % 8)
+        // of this thread: items t and t + 256 carry their scale two groups ahead too
+        __half sq[3];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) sq[j] = (valid && j < a.G) ? srow[j] : __float2half(0.f);
+        const int item0 = t, item1 = t + kDequantThreads;
+        const bool has0 = item0 < n_res * 8, has1 = item1 < n_res * 8;
+        const __half* s2row0 = has0 ? a.scale2 + int64_t(res_list[item0 >> 3].y) * a.G : a.scale2;
+        const __half* s2row1 = has1 ? a.scale2 + int64_t(res_list[item1 >> 3].y) * a.G : a.scale2;
+        __half rq0[3], rq1[3];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+            rq0[j] = (has0 && j < a.G) ? s2row0[j] : __float2half(0.f);
+            rq1[j] = (has1 && j < a.G) ? s2row1[j] : __float2half(0.f);
+        }
+        for (int kb = 0; kb < num_kb; ++kb) {
+            const int s = kb % kStages, sp = kb % kStagesP;
+            const int g = kb / 2;
+            if ((kb & 1) == 0 && kb > 0) {   // a new group: shift the scale queues, load two ahead
+                sq[0] = sq[1]; sq[1] = sq[2];
+                rq0[0] = rq0[1]; rq0[1] = rq0[2];
+                rq1[0] = rq1[1]; rq1[1] = rq1[2];
+                const int g2 = g + 2;
+                if (g2 < a.G) {
+                    sq[2] = valid ? srow[g2] : __float2half(0.f);
+                    if (has0) rq0[2] = s2row0[g2];
+                    if (has1) rq1[2] = s2row1[g2];
+                }
+            }
+            // every dequantising thread takes the same decision, so the named barriers below match
+            ok = dequant_all(mbar_wait(&full_p[sp], (kb / kStagesP) & 1) &&
+                             (kb < kStages || mbar_wait(&empty[s], ((kb / kStages) - 1) & 1)));
+            if (!ok) break;
+            uint8_t* bs = smem_b + s * kBBytes;
+            const uint4 cur = *reinterpret_cast<const uint4*>(smem_p1 + sp * kPBytes + t * 16);
+            const __half2 s2 = __half2half2(valid ? sq[0] : __float2half(0.f));
+            const uint32_t words[4] = {cur.x, cur.y, cur.z, cur.w};
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint32_t v = (c & 1) ? (words[c >> 1] >> 16) : (words[c >> 1] & 0xFFFFu);
+                __half2 tt[4];
+                decode8(v, tt);
+                uint4 o;
+                o.x = h2_bits(__hmul2(tt[0], s2));
+                o.y = h2_bits(__hmul2(tt[1], s2));
+                o.z = h2_bits(__hmul2(tt[2], s2));
+                o.w = h2_bits(__hmul2(tt[3], s2));
+                *reinterpret_cast<uint4*>(bs + sw128_offset(t, c)) = o;
+            }
+            if (n_res > 0) {
+                asm volatile("bar.sync 1, %0;" ::"n"(kDequantThreads) : "memory");
+                for (int i = t; i < n_res * 8; i += kDequantThreads) {
+                    const int row = i >> 3, c = i & 7;
+                    const int2 e = res_list[row];
+                    const uint32_t w2 =
+                        *reinterpret_cast<const uint32_t*>(smem_p2 + sp * kPBytes + row * 16 + (c >> 1) * 4);
+                    const __half sc2 = (i == item0) ? rq0[0] : (i == item1) ? rq1[0]
+                                                                            : a.scale2[int64_t(e.y) * a.G + g];
+                    const __half2 s22 = __half2half2(sc2);
+                    __half2 tt[4];
+                    decode8((c & 1) ? (w2 >> 16) : (w2 & 0xFFFFu), tt);
+                    uint4* dst = reinterpret_cast<uint4*>(bs + sw128_offset(e.x, c));
+                    uint4 o = *dst;
+                    o.x = h2_bits(__hfma2(tt[0], s22, bits_h2(o.x)));
+                    o.y = h2_bits(__hfma2(tt[1], s22, bits_h2(o.y)));
+                    o.z = h2_bits(__hfma2(tt[2], s22, bits_h2(o.z)));
+                    o.w = h2_bits(__hfma2(tt[3], s22, bits_h2(o.w)));
+                    *dst = o;
+                }
+            }
+            fence_async_smem();
+            mbar_arrive(&full_b[s]);
+            mbar_arrive(&empty_p[sp]);
+        }
+        // ---------------- epilogue: TMEM -> fp16 y (tcgen05.ld is warp-collective: ok is made warp-uniform)
+        if (ok) ok = mbar_wait(tmem_full, 0);
+        ok = __all_sync(0xffffffffu, ok);
+        tc_fence_after();
+        if (ok) {
+            const int lq = warp & 3;                         // TMEM lanes 32*lq .. 32*lq+31
+            const int col0 = ((warp - 2) >> 2) * (BN / 2);   // columns 0..127 or 128..255
+            const int64_t m = m0 + lq * 32 + lane;
+#pragma unroll 1
+            for (int cc = 0; cc < BN / 2; cc += 32) {
+                uint32_t r[32];
+                const uint32_t taddr = tmem_base + (uint32_t(lq * 32) << 16) + uint32_t(col0 + cc);
+                asm volatile(
+                    "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+                    "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
+                    "[%32];"
+                    : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                      "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                      "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+                      "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+                      "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                    : "r"(taddr));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                if (m < a.M) {
+                    const int64_t nc = n0 + col0 + cc;
+                    __half* dst = a.y + m * a.N + nc;
+                    uint32_t h[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        h[j] = h2_bits(__floats2half2_rn(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])));
+                    const bool vec = (nc + 32 <= a.N) && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
+                    if (vec) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            reinterpret_cast<uint4*>(dst)[j] = make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+                    } else {
+                        for (int j = 0; j < 32 && nc + j < a.N; ++j)
+                            dst[j] = __ushort_as_half(static_cast<unsigned short>((j & 1) ? (h[j >> 1] >> 16)
+                                                                                          : (h[j >> 1] & 0xFFFFu)));
+                    }
+                }
+            }
+        }
+    }
+    __syncwarp();
+    if (!ok && a.status) atomicOr(a.status, kTimeoutBit);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+}  // namespace
+
+size_t gemm_workspace_bytes(const tern_weight&, int64_t) { return 0; }
+
+tern_status gemm_launch(const tern_weight& w, const __half* x, int64_t M, __half* y, void*, cudaStream_t stream) {
+    if (M > (int64_t(1) << 31) - BM || w.K % BK) return TERN_ERR_SHAPE;
+    const int64_t n_tiles = (w.N + BN - 1) / BN, m_tiles = (M + BM - 1) / BM;
+    if (n_tiles > 0x7FFFFFFF || m_tiles > 65535) return TERN_ERR_SHAPE;
+    auto enc = encode_fn();
+    if (!enc) return TERN_ERR_CUDA;
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {cuuint64_t(w.K), cuuint64_t(M)};
+    const cuuint64_t strides[1] = {cuuint64_t(w.K) * sizeof(__half)};
+    const cuuint32_t box[2] = {BK, BM};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(x), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return TERN_ERR_CUDA;
+    // packed codes: [rows, K/16] uint32, boxes of 4 words (one 64-wide K block) x 256 or 32 rows
+    CUtensorMap map_p1, map_p2;
+    auto plane_map = [&](CUtensorMap* m, const uint32_t* plane, int64_t rows, uint32_t box_rows) {
+        const cuuint64_t pd[2] = {cuuint64_t(w.K / kCodesPerWord), cuuint64_t(rows > 0 ? rows : 1)};
+        const cuuint64_t ps[1] = {cuuint64_t(w.K / kCodesPerWord) * 4};
+        const cuuint32_t pb[2] = {BK / kCodesPerWord, box_rows};
+        return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(plane), pd, ps, pb, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    };
+    if (!plane_map(&map_p1, w.plane1, w.N, BN)) return TERN_ERR_CUDA;
+    if (!plane_map(&map_p2, w.r > 0 ? w.plane2 : w.plane1, w.r > 0 ? w.r : w.N, kResBox)) return TERN_ERR_CUDA;
+    static std::mutex mu;
+    static bool configured[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TERN_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!configured[dev]) {
+            if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes)) !=
+                cudaSuccess)
+                return TERN_ERR_CUDA;
+            configured[dev] = true;
+        }
+    }
+    GemmArgs a;
+    a.plane1 = w.plane1;
+    a.scale1 = reinterpret_cast<const __half*>(w.scale1);
+    a.plane2 = w.plane2;
+    a.scale2 = reinterpret_cast<const __half*>(w.scale2);
+    a.res_slot = w.r > 0 ? w.res_slot : nullptr;
+    a.N = w.N;
+    a.K = w.K;
+    a.r = w.r;
+    a.M = M;
+    a.G = int32_t(w.K / kGroup);
+    a.y = y;
+    a.status = async_status_word();
+    gemm_kernel<<<dim3(unsigned(n_tiles), unsigned(m_tiles)), kThreads, kSmemBytes, stream>>>(map, map_p1, map_p2, a);
+    return cudaGetLastError() == cudaSuccess ? TERN_OK : TERN_ERR_CUDA;
 }
 
 }  // namespace tern

@@ -7,30 +7,39 @@
 // exact, so the layer is a signed sum of activations ("Can Ternary LLMs Hit 1.58 Bits per
 // Weight?", promptzone, "What It Is and How It Works"), accumulated here in fp32.
 //
-// Design (B200, memory-bound at 0.266 bytes per weight):
-//  * One CTA = 4 warps = 64 output rows (one 16-row strip per warp) x one K-slice. The
-//    K-slices of a row block form a thread-block cluster; partial sums are reduced over
-//    distributed shared memory in a fixed order (no global workspace, no atomics, no
-//    spin-waits), and the CTA of rank c writes rows [c*64/S, (c+1)*64/S) of the block.
-//  * The signed sums run on the tensor pipe as mma.sync m16n8k16 (fp16 in, fp32
-//    accumulate): A = 16 weight rows x 16 K of decoded trits, B = the activations of up to
-//    8 tokens. The products are exact (+-x or 0), so this is the fp32-accumulated
-//    add/subtract of the method, with the decode cost independent of M.
+// Design (B200; memory-bound at 0.266 bytes per weight):
+//  * A CTA owns 64 output rows x one K-slice of at most 8 groups. Its first act is to issue
+//    2D TMA loads of its whole weight tile (64 rows x 128 bytes of codes per box, 128-byte
+//    swizzle), of the residual-plane rows that belong to those 64 rows and of their scales,
+//    so the HBM stream starts at once and no later step waits on another global round trip
+//    except the read of x.
+//  * The K-slices of a 64-row block form a thread-block cluster. Partial sums meet in
+//    distributed shared memory in a fixed order (no global partials, no atomics, no
+//    spin-waits on other CTAs); the CTA of cluster rank c writes rows [c*64/S, (c+1)*64/S).
+//  * Warps 0-3 each own a 16-row strip of the main plane. Warp 4 owns the residual rows of the
+//    block: since R is sorted, they are the contiguous slots [s_lo, s_lo + nres) of the
+//    residual plane, taken 16 rows at a time. Their sums join the main rows' sums before the
+//    single rounding to fp16.
+//  * The signed sums run on the tensor pipe as mma.sync m16n8k16 (fp16 in, fp32 accumulate):
+//    A = 16 weight rows x 16 K of decoded trits, B = the activations of up to 8 tokens. The
+//    products are exact (+-x or 0), so this is the fp32-accumulated add/subtract of the
+//    method, and the decode cost does not grow with M.
 //  * Decode is branch-free: one LOP3 turns two 2-bit codes (bits p and p+16 of a word) into
 //    an fp16 pair (B_p + c) by writing the code into the mantissa of a power of two B_p; a
 //    shift by 6 either way moves the codes of bits 0-3 and 10-15 into mantissa positions,
-//    so a word of 16 trits costs 2 shifts and 8 LOP3. Since c = t + 1, the MMA then sums
+//    so a word of 16 trits costs 2 shifts and 8 LOP3. Since c = t + 1, the MMA sums
 //    (B_p + 1 + t) * x from zero, and C = sum (B_p + 1) * x is subtracted once per group. C is
 //    computed once per CTA by the same MMA on the constant pattern B_p + 1 in the same K
-//    order, so a zero plane cancels bit for bit. The bases are 4, 16 and 64, so the offsets
+//    order (hidden behind the weight loads), so a zero plane cancels bit for bit. The bases are 4, 16 and 64, so the offsets
 //    are small and every partial sum is exact on integer inputs. A non-finite activation
 //    makes every output of its token non-finite (NaN where the dense product has +-inf).
 //  * The contraction order over K is free, so the MMA's K order follows the packed words
-//    (pair j = trits j and j+8 of a word); the activations of the slice are staged in
-//    shared memory in that order once per CTA.
-//  * Rows of the residual plane T2 run as a first pass of the same kernel that writes fp32
-//    sums to the workspace; the main pass adds them to the rows of R before its single
-//    rounding to fp16.
+//    (pair j = trits j and j+8 of a word); x is staged in shared memory in that order.
+//  * Launches use programmatic dependent launch: a kernel may start while the previous one on
+//    the stream drains; it reads x (and, unless the weight is flagged static, the weight)
+//    only after griddepcontrol.wait, and writes nothing before it.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <stdlib.h>
 
 #include <algorithm>
@@ -41,32 +50,57 @@
 namespace tern {
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kThreads = kWarps * 32;
-constexpr int kRowsPerCta = 16 * kWarps;
+constexpr int kMainWarps = 4;
+constexpr int kThreads = (kMainWarps + 1) * 32;     // + one warp for the residual rows
+constexpr int kRowsPerCta = 16 * kMainWarps;        // 64
+constexpr int kChunkGroups = 4;                     // groups per TMA box: 32 words = 128 bytes per row
+constexpr int kMaxGpc = 8;                          // groups per K-slice
+constexpr int kMaxChunks = kMaxGpc / kChunkGroups;
+constexpr int kStrip = 16;
+constexpr int kResStrips = 2;                       // residual strips resident at once
+constexpr int kMaxResRows = kRowsPerCta;            // residual rows of one block (all of them)
 constexpr int kMaxSplit = 16;
-constexpr int kPrefetch = 4;                  // groups of packed words in flight per warp
-constexpr int kSmemBudget = 96 * 1024;        // activations staged per CTA (bytes)
-constexpr int kNegcStride = 16;               // floats per group (one per token)
+constexpr int kMainChunkBytes = kRowsPerCta * 128;  // 8 KB
+constexpr int kStripBytes = kStrip * 128;           // 2 KB
+constexpr int kResChunkBytes = kResStrips * kStripBytes;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // bounded waits give up after ~2 s
 
 struct GemvArgs {
-    const uint32_t* plane;     // [rows, K/16]
-    const __half* scale;       // [rows, G]
+    const __half* scale1;      // [N, G]
+    const __half* scale2;      // [r, G]
+    const int32_t* res_slot;   // [N] or nullptr
     const __half* x;           // [M, K]
-    int64_t rows;
-    int64_t K;
-    int32_t G;
-    int32_t M;
+    __half* y;                 // [M, N]
+    unsigned int* status;      // sticky timeout word
+    int64_t N, r, K;
+    int32_t G, M;
     int32_t gpc;               // groups per K-slice
-    int32_t split;             // K-slices (= cluster size along x)
-    __half* y;                 // main pass: [M, rows]
-    float* res_out;            // residual pass: [M, rows] fp32 sums
-    const float* res_in;       // main pass: [M, r] residual sums, or nullptr
-    const int32_t* res_slot;   // main pass: [rows] slot map, or nullptr
-    int64_t r;
+    int32_t split;             // K-slices = cluster size
+    int32_t static_weights;    // planes may be read before griddepcontrol.wait
 };
 
+struct Smem {
+    static constexpr int wt1 = 0;                                          // [chunk][64 rows][128 B]
+    static constexpr int wt2 = wt1 + kMaxChunks * kMainChunkBytes;        // [chunk][2 strips][16][128 B]
+    static constexpr int bar = wt2 + kMaxChunks * kResChunkBytes;         // mbar1[chunks], mbar2[chunks]
+    static constexpr int misc = bar + 2 * kMaxChunks * 8;                  // s_lo, nres
+    static constexpr int sc1 = misc + 16;                                  // half [64][kMaxGpc]
+    static constexpr int sc2 = sc1 + kRowsPerCta * kMaxGpc * 2;            // half [64][kMaxGpc]
+    static constexpr int bslot = sc2 + kMaxResRows * kMaxGpc * 2;          // int [64]: slot - s_lo, or -1
+    static constexpr int cofs = bslot + kRowsPerCta * 4;                   // float [kMaxGpc][16]
+    static constexpr int xzero = cofs + kMaxGpc * 16 * 4;                  // half [kMaxGpc * 128]: zeros
+    static constexpr int red = xzero + kMaxGpc * kGroup * 2;               // float [128][M], then xs
+};
+size_t smem_bytes(int M) {
+    return size_t(Smem::red) + size_t(kRowsPerCta + kMaxResRows) * M * 4 + size_t(M) * kMaxGpc * kGroup * 2 + 1024;
+}
+static_assert(Smem::xzero % 16 == 0 && Smem::red % 16 == 0, "16-byte aligned activation rows");
+
 // ------------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
 __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
     uint32_t d;
     asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(magic));   // (a & b) | c
@@ -79,18 +113,57 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return d;
 }
 
-__device__ __forceinline__ uint2 ld_stream_u2(const uint32_t* p) {
-    uint2 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-    return v;
-}
-
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
         "{%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait for the phase of the given parity: false after about two seconds.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    const uint32_t addr = smem_u32(bar);
+    uint64_t t0 = 0;
+    for (uint32_t i = 0;; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(addr), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if ((i & 255u) == 0) {
+            const uint64_t t = global_ns();
+            if (i == 0) t0 = t;
+            else if (t - t0 > kWaitLimitNs) return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
 }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -104,13 +177,16 @@ __device__ __forceinline__ void cluster_sync_all() {
 }
 
 __device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t cta) {
-    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(local));
+    const uint32_t a = smem_u32(local);
     uint32_t remote;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(a), "r"(cta));
     float v;
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
     return v;
 }
+
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // Pair p of a word (trits p and p+8) as fp16x2 (B_p + c_lo, B_p + c_hi), c = t + 1.
 // B_p = 16, 4, 64, 16, 4, 64, 16, 4 for p = 0..7. wl = w << 6, wr = w >> 6.
@@ -139,130 +215,44 @@ __device__ __forceinline__ void zero_trit_pattern(int i4, uint32_t& lo, uint32_t
     }
 }
 
-// ------------------------------------------------------------------ the kernel
-template <int NT, bool kResidualPass>
-__global__ void __launch_bounds__(kThreads) gemv_kernel(const GemvArgs a) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    const int M = a.M;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int q = lane & 3, rr = lane >> 2;
-    const int ks = blockIdx.x;
-    const int g_begin = ks * a.gpc;
-    const int ng = max(0, min(a.G, g_begin + a.gpc) - g_begin);
-    const int xs_stride = a.gpc * kGroup;                     // halves per token row in smem
-    __half* xs = reinterpret_cast<__half*>(smem);
-    float* cofs = reinterpret_cast<float*>(smem + size_t(M) * xs_stride * sizeof(__half));
-    float* red = cofs + size_t(a.gpc) * kNegcStride;          // [kRowsPerCta][16]
+// Words 2q and 2q+1 of group gl (0..3) of a row in a 128-byte-swizzled TMA box.
+__device__ __forceinline__ uint2 lds_words(const uint8_t* box, int row, int gl, int q) {
+    const int chunk = 2 * gl + (q >> 1);
+    return *reinterpret_cast<const uint2*>(box + row * 128 + ((chunk ^ (row & 7)) << 4) + 8 * (q & 1));
+}
 
-    // 1. Stage this slice of x, pairing columns (j, j+8) of every 16-column block.
-    {
-        const int blocks16 = ng * kWordsPerGroup;
-        for (int idx = threadIdx.x; idx < M * blocks16; idx += kThreads) {
-            const int m = idx / blocks16, b = idx - m * blocks16;
-            const uint4* src =
-                reinterpret_cast<const uint4*>(a.x + int64_t(m) * a.K + int64_t(g_begin) * kGroup + b * 16);
-            const uint4 lo = __ldg(src), hi = __ldg(src + 1);
-            uint4 o0, o1;
-            o0.x = prmt(lo.x, hi.x, 0x5410u); o0.y = prmt(lo.x, hi.x, 0x7632u);
-            o0.z = prmt(lo.y, hi.y, 0x5410u); o0.w = prmt(lo.y, hi.y, 0x7632u);
-            o1.x = prmt(lo.z, hi.z, 0x5410u); o1.y = prmt(lo.z, hi.z, 0x7632u);
-            o1.z = prmt(lo.w, hi.w, 0x5410u); o1.w = prmt(lo.w, hi.w, 0x7632u);
-            uint4* dst = reinterpret_cast<uint4*>(xs + size_t(m) * xs_stride + b * 16);
-            dst[0] = o0;
-            dst[1] = o1;
-        }
-    }
-    __syncthreads();
-
-    // B fragment of MMA i in group gi for token tile t: pairs (j, j+1) of word 2q + i/4.
-    auto load_b = [&](int gi, int i, int t, uint32_t& b0, uint32_t& b1) {
-        const int n = 8 * t + rr;
-        if (n < M) {
-            const int off = gi * kGroup + 16 * (2 * q + (i >> 2)) + 4 * (i & 3);
-            const uint2 v = *reinterpret_cast<const uint2*>(xs + size_t(n) * xs_stride + off);
-            b0 = v.x;
-            b1 = v.y;
-        } else {
-            b0 = 0u;
-            b1 = 0u;
-        }
-    };
-
-    // 2. C[g][token] = sum_k (B_p(k) + 1) * x[token][k], one MMA chain per group.
-    for (int gi = warp; gi < ng; gi += kWarps) {
-        float c[NT][4];
+// One 16-row strip over the slice: yacc[t][e] += s(row) * (sum_k t * x) over the slice's groups.
+// box(c): smem base of chunk c for this strip (16 rows of 128 B, 128-byte swizzled); sc: the
+// strip's scales [16][kMaxGpc]; xrow[t]: this lane's activation row for token tile t (pairs in
+// word order, or the zero row); cofs: C[g][token]. The lane holds rows rr and rr + 8.
+// Two groups run at once, so their accumulator chains overlap.
+template <int NT, typename BoxFn, typename WaitFn>
+__device__ __forceinline__ void strip_sums(int ng, int q, int rr, const __half* sc, const float* cofs,
+                                           const __half* const (&xrow)[NT], BoxFn box, WaitFn wait_chunk,
+                                           float (&yacc)[NT][4]) {
+    // byte offset of words 2q, 2q+1 of group gl in rows rr and rr+8 (row & 7 == rr & 7):
+    // chunk 2*gl + q/2 of the 128-byte row, swizzled by the row
+    const int qh = q >> 1, r7 = rr & 7, qb = 8 * (q & 1);
+    const int roff_a = rr * 128 + qb, roff_b = (rr + 8) * 128 + qb;
+    for (int g0 = 0; g0 < ng; g0 += 2) {
+        if ((g0 % kChunkGroups) == 0) wait_chunk(g0 / kChunkGroups);
+        const uint8_t* b = box(g0 / kChunkGroups);          // groups g0 and g0 + 1 share a chunk
+        const int ngrp = min(2, ng - g0);
+        float acc[2][NT][4];
 #pragma unroll
-        for (int t = 0; t < NT; ++t) c[t][0] = c[t][1] = c[t][2] = c[t][3] = 0.f;
+        for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            uint32_t A[4];
-            zero_trit_pattern(i & 3, A[0], A[2]);
-            A[1] = A[0];
-            A[3] = A[2];
+            for (int t = 0; t < NT; ++t) acc[u][t][0] = acc[u][t][1] = acc[u][t][2] = acc[u][t][3] = 0.f;
 #pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                uint32_t b0, b1;
-                load_b(gi, i, t, b0, b1);
-                mma_16816(c[t], A, b0, b1);
-            }
-        }
-        if (rr == 0) {
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                cofs[gi * kNegcStride + 8 * t + 2 * q] = c[t][0];
-                cofs[gi * kNegcStride + 8 * t + 2 * q + 1] = c[t][1];
-            }
-        }
-    }
-    __syncthreads();
-
-    // 3. Stream this warp's 16-row strip over the slice.
-    const int64_t block_row0 = int64_t(blockIdx.y) * kRowsPerCta;
-    const int64_t ra = block_row0 + warp * 16 + rr, rb = ra + 8;
-    const bool va = ra < a.rows, vb = rb < a.rows;
-    const int64_t wpr = a.K / kCodesPerWord;
-    const uint32_t* pa = a.plane + (va ? ra : 0) * wpr + int64_t(g_begin) * kWordsPerGroup + 2 * q;
-    const uint32_t* pb = a.plane + (vb ? rb : 0) * wpr + int64_t(g_begin) * kWordsPerGroup + 2 * q;
-    const __half* sa_ptr = a.scale + (va ? ra : 0) * int64_t(a.G) + g_begin;
-    const __half* sb_ptr = a.scale + (vb ? rb : 0) * int64_t(a.G) + g_begin;
-    constexpr uint32_t kZeroCodes = 0x55555555u;                 // code 1 = trit 0 everywhere
-
-    float yacc[NT][4];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) yacc[t][0] = yacc[t][1] = yacc[t][2] = yacc[t][3] = 0.f;
-
-    uint2 bufA[kPrefetch], bufB[kPrefetch];
-    float bsa[kPrefetch], bsb[kPrefetch];
-    auto fetch = [&](int gi, int u) {
-        if (gi < ng) {
-            bufA[u] = va ? ld_stream_u2(pa + gi * kWordsPerGroup) : make_uint2(kZeroCodes, kZeroCodes);
-            bufB[u] = vb ? ld_stream_u2(pb + gi * kWordsPerGroup) : make_uint2(kZeroCodes, kZeroCodes);
-            bsa[u] = va ? __half2float(sa_ptr[gi]) : 0.f;
-            bsb[u] = vb ? __half2float(sb_ptr[gi]) : 0.f;
-        }
-    };
-#pragma unroll
-    for (int u = 0; u < kPrefetch; ++u) fetch(u, u);
-
-    for (int base = 0; base < ng; base += kPrefetch) {
-        uint2 cA[kPrefetch], cB[kPrefetch];
-        float csa[kPrefetch], csb[kPrefetch];
-#pragma unroll
-        for (int u = 0; u < kPrefetch; ++u) {
-            cA[u] = bufA[u]; cB[u] = bufB[u]; csa[u] = bsa[u]; csb[u] = bsb[u];
-        }
-#pragma unroll
-        for (int u = 0; u < kPrefetch; ++u) fetch(base + kPrefetch + u, u);
-#pragma unroll
-        for (int u = 0; u < kPrefetch; ++u) {
-            const int gi = base + u;
-            if (gi >= ng) break;
-            float acc[NT][4];
-#pragma unroll
-            for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+        for (int u = 0; u < 2; ++u) {
+            if (u >= ngrp) break;
+            const int gi = g0 + u, gl = gi % kChunkGroups;
+            const int woff = ((2 * gl + qh) ^ r7) << 4;
+            const uint2 wa2 = *reinterpret_cast<const uint2*>(b + roff_a + woff);
+            const uint2 wb2 = *reinterpret_cast<const uint2*>(b + roff_b + woff);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const uint32_t wa = h ? cA[u].y : cA[u].x, wb = h ? cB[u].y : cB[u].x;
+                const uint32_t wa = h ? wa2.y : wa2.x, wb = h ? wb2.y : wb2.x;
                 const uint32_t wal = wa << 6, war = wa >> 6, wbl = wb << 6, wbr = wb >> 6;
                 uint32_t A[4][4];   // four MMAs per word: pairs (0,1), (2,3), (4,5), (6,7)
                 A[0][0] = decode_pair<0>(wa, wal, war); A[0][1] = decode_pair<0>(wb, wbl, wbr);
@@ -274,71 +264,269 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(const GemvArgs a) {
                 A[3][0] = decode_pair<6>(wa, wal, war); A[3][1] = decode_pair<6>(wb, wbl, wbr);
                 A[3][2] = decode_pair<7>(wa, wal, war); A[3][3] = decode_pair<7>(wb, wbl, wbr);
 #pragma unroll
-                for (int i4 = 0; i4 < 4; ++i4) {
-#pragma unroll
-                    for (int t = 0; t < NT; ++t) {
-                        uint32_t b0, b1;
-                        load_b(gi, 4 * h + i4, t, b0, b1);
-                        mma_16816(acc[t], A[i4], b0, b1);
-                    }
+                for (int t = 0; t < NT; ++t) {
+                    // the B fragments of this word's four MMAs: 32 contiguous bytes of the row
+                    const uint4* xp = reinterpret_cast<const uint4*>(xrow[t] + gi * kGroup + 16 * (2 * q + h));
+                    const uint4 x01 = xp[0], x23 = xp[1];
+                    mma_16816(acc[u][t], A[0], x01.x, x01.y);
+                    mma_16816(acc[u][t], A[1], x01.z, x01.w);
+                    mma_16816(acc[u][t], A[2], x23.x, x23.y);
+                    mma_16816(acc[u][t], A[3], x23.z, x23.w);
                 }
             }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (u >= ngrp) break;
+            const int gi = g0 + u;
+            const float sa = __half2float(sc[rr * kMaxGpc + gi]);
+            const float sb = __half2float(sc[(rr + 8) * kMaxGpc + gi]);
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
-                const float c0 = cofs[gi * kNegcStride + 8 * t + 2 * q];
-                const float c1 = cofs[gi * kNegcStride + 8 * t + 2 * q + 1];
-                yacc[t][0] = fmaf(csa[u], acc[t][0] - c0, yacc[t][0]);
-                yacc[t][1] = fmaf(csa[u], acc[t][1] - c1, yacc[t][1]);
-                yacc[t][2] = fmaf(csb[u], acc[t][2] - c0, yacc[t][2]);
-                yacc[t][3] = fmaf(csb[u], acc[t][3] - c1, yacc[t][3]);
+                const float2 c = *reinterpret_cast<const float2*>(cofs + gi * 16 + 8 * t + 2 * q);
+                yacc[t][0] = fmaf(sa, acc[u][t][0] - c.x, yacc[t][0]);
+                yacc[t][1] = fmaf(sa, acc[u][t][1] - c.y, yacc[t][1]);
+                yacc[t][2] = fmaf(sb, acc[u][t][2] - c.x, yacc[t][2]);
+                yacc[t][3] = fmaf(sb, acc[u][t][3] - c.y, yacc[t][3]);
             }
         }
     }
+}
 
-    // 4. Epilogue: reduce over the cluster's K-slices, then write.
-    auto emit = [&](int64_t row, int tok, float v) {
-        if (row >= a.rows || tok >= M) return;
-        if (kResidualPass) {
-            a.res_out[int64_t(tok) * a.rows + row] = v;
-        } else {
-            if (a.res_slot) {
-                const int32_t s = a.res_slot[row];
-                if (s >= 0 && s < a.r) v += a.res_in[int64_t(tok) * a.r + s];
+// ------------------------------------------------------------------ the kernel
+template <int NT>
+__global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const __grid_constant__ CUtensorMap map1,
+                                                        const __grid_constant__ CUtensorMap map2,
+                                                        const GemvArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* wt1 = smem + Smem::wt1;
+    uint8_t* wt2 = smem + Smem::wt2;
+    uint64_t* mbar1 = reinterpret_cast<uint64_t*>(smem + Smem::bar);
+    uint64_t* mbar2 = mbar1 + kMaxChunks;
+    int* misc = reinterpret_cast<int*>(smem + Smem::misc);
+    __half* sc1 = reinterpret_cast<__half*>(smem + Smem::sc1);
+    __half* sc2 = reinterpret_cast<__half*>(smem + Smem::sc2);
+    int* bslot = reinterpret_cast<int*>(smem + Smem::bslot);
+    float* cofs = reinterpret_cast<float*>(smem + Smem::cofs);
+    __half* xzero = reinterpret_cast<__half*>(smem + Smem::xzero);
+    const int M = a.M;
+    float* red = reinterpret_cast<float*>(smem + Smem::red);                         // [128][M]
+    __half* xs = reinterpret_cast<__half*>(smem + Smem::red + (kRowsPerCta + kMaxResRows) * M * 4);
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int q = lane & 3, rr = lane >> 2;
+    const int ks = blockIdx.x;                        // = rank in the cluster
+    const int g_begin = ks * a.gpc;
+    const int ng = max(0, min(a.G, g_begin + a.gpc) - g_begin);
+    const int nchunks = (ng + kChunkGroups - 1) / kChunkGroups;
+    const int64_t n0 = int64_t(blockIdx.y) * kRowsPerCta;
+    const int xs_stride = a.gpc * kGroup;             // halves per token in smem
+    bool ok = true;
+
+    if (threadIdx.x == 0) {
+        for (int c = 0; c < kMaxChunks; ++c) {
+            mbar_init(&mbar1[c], 1);
+            mbar_init(&mbar2[c], 1);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    __syncthreads();
+
+    int s_lo = 0, nres = 0;
+    // Everything the weight determines, issued at once: TMA of the main tile (thread 0); the
+    // block's residual slots, their TMA and scales (warp 4); the main scales (warps 0-3).
+    auto issue_weight_reads = [&]() {
+        if (threadIdx.x == 0)
+            for (int c = 0; c < nchunks; ++c) {
+                mbar_arrive_expect_tx(&mbar1[c], kMainChunkBytes);
+                tma_load_2d(wt1 + c * kMainChunkBytes, &map1, (g_begin + c * kChunkGroups) * kWordsPerGroup,
+                            int(n0), &mbar1[c]);
             }
-            a.y[int64_t(tok) * a.rows + row] = __float2half_rn(v);
+        if (warp == kMainWarps) {
+            int sl0 = -1, sl1 = -1;
+            if (a.res_slot) {
+                if (n0 + lane < a.N) sl0 = a.res_slot[n0 + lane];
+                if (n0 + 32 + lane < a.N) sl1 = a.res_slot[n0 + 32 + lane];
+            }
+            const bool v0 = sl0 >= 0 && sl0 < a.r, v1 = sl1 >= 0 && sl1 < a.r;
+            const unsigned b0 = __ballot_sync(0xffffffffu, v0);
+            const unsigned b1 = __ballot_sync(0xffffffffu, v1);
+            nres = __popc(b0) + __popc(b1);
+            const int first = b0 ? (__ffs(b0) - 1) : (b1 ? 32 + __ffs(b1) - 1 : 0);
+            s_lo = nres ? __shfl_sync(0xffffffffu, first < 32 ? sl0 : sl1, first & 31) : 0;
+            bslot[lane] = v0 ? sl0 - s_lo : -1;
+            bslot[32 + lane] = v1 ? sl1 - s_lo : -1;
+            if (lane == 0) {
+                misc[0] = s_lo;
+                misc[1] = nres;
+                const int strips = min(kResStrips, (nres + kStrip - 1) / kStrip);
+                for (int c = 0; c < nchunks && strips > 0; ++c) {
+                    mbar_arrive_expect_tx(&mbar2[c], strips * kStripBytes);
+                    for (int j = 0; j < strips; ++j)
+                        tma_load_2d(wt2 + c * kResChunkBytes + j * kStripBytes, &map2,
+                                    (g_begin + c * kChunkGroups) * kWordsPerGroup, s_lo + j * kStrip, &mbar2[c]);
+                }
+            }
+            // residual scales: lane g of each 8-lane quarter loads group g of rows quarter, +4, ...
+            const int g = lane & 7;
+            if (g < ng)
+                for (int row = lane >> 3; row < nres; row += 4)
+                    sc2[row * kMaxGpc + g] = s_lo + row < a.r ? a.scale2[int64_t(s_lo + row) * a.G + g_begin + g]
+                                                              : __float2half(0.f);
+        } else {
+            const int g = threadIdx.x & 7;
+            if (g < ng)
+                for (int row = threadIdx.x >> 3; row < kRowsPerCta; row += kMainWarps * 4) {
+                    const int64_t n = n0 + row;
+                    sc1[row * kMaxGpc + g] = n < a.N ? a.scale1[n * a.G + g_begin + g] : __float2half(0.f);
+                }
         }
     };
 
-    if (a.split == 1) {
+    if (a.static_weights) issue_weight_reads();
+    grid_dependency_wait();           // x (and a non-static weight) may come from the previous kernel
+    if (!a.static_weights) issue_weight_reads();
+
+    // activations of the slice, pairing columns (j, j+8) of every 16-column block; a zero row
+    // stands in for the tokens past M
+    {
+        const int blocks16 = ng * kWordsPerGroup;
+        for (int m = 0; m < M; ++m)
+            for (int b = threadIdx.x; b < blocks16; b += kThreads) {
+                const uint4* src =
+                    reinterpret_cast<const uint4*>(a.x + int64_t(m) * a.K + int64_t(g_begin) * kGroup + b * 16);
+                const uint4 lo = __ldg(src), hi = __ldg(src + 1);
+                uint4 o0, o1;
+                o0.x = prmt(lo.x, hi.x, 0x5410u); o0.y = prmt(lo.x, hi.x, 0x7632u);
+                o0.z = prmt(lo.y, hi.y, 0x5410u); o0.w = prmt(lo.y, hi.y, 0x7632u);
+                o1.x = prmt(lo.z, hi.z, 0x5410u); o1.y = prmt(lo.z, hi.z, 0x7632u);
+                o1.z = prmt(lo.w, hi.w, 0x5410u); o1.w = prmt(lo.w, hi.w, 0x7632u);
+                uint4* dst = reinterpret_cast<uint4*>(xs + size_t(m) * xs_stride + b * 16);
+                dst[0] = o0;
+                dst[1] = o1;
+            }
+        for (int i = threadIdx.x; i < kMaxGpc * kGroup / 8; i += kThreads)
+            reinterpret_cast<uint4*>(xzero)[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncthreads();
+
+    const __half* xrow[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) xrow[t] = (8 * t + rr < M) ? xs + size_t(8 * t + rr) * xs_stride : xzero;
+
+    // C[g][token] = sum_k (B_p(k) + 1) * x[token][k]: one MMA chain per group on the constant
+    // pattern, in the same K order as the main chains, so a zero plane cancels bit for bit
+    for (int gi = warp; gi < ng; gi += kMainWarps + 1) {
+        float c[NT][4];
+#pragma unroll
+        for (int t = 0; t < NT; ++t) c[t][0] = c[t][1] = c[t][2] = c[t][3] = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const uint4* xp = reinterpret_cast<const uint4*>(xrow[t] + gi * kGroup + 16 * (2 * q + h));
+                const uint4 x01 = xp[0], x23 = xp[1];
+                uint32_t Z[4];
+                zero_trit_pattern(0, Z[0], Z[2]); Z[1] = Z[0]; Z[3] = Z[2];
+                mma_16816(c[t], Z, x01.x, x01.y);
+                zero_trit_pattern(1, Z[0], Z[2]); Z[1] = Z[0]; Z[3] = Z[2];
+                mma_16816(c[t], Z, x01.z, x01.w);
+                zero_trit_pattern(2, Z[0], Z[2]); Z[1] = Z[0]; Z[3] = Z[2];
+                mma_16816(c[t], Z, x23.x, x23.y);
+                zero_trit_pattern(3, Z[0], Z[2]); Z[1] = Z[0]; Z[3] = Z[2];
+                mma_16816(c[t], Z, x23.z, x23.w);
+            }
+        }
+        if (rr == 0) {
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+                *reinterpret_cast<float2*>(cofs + gi * 16 + 8 * t + 2 * q) = make_float2(c[t][0], c[t][1]);
+        }
+    }
+    __syncthreads();
+    grid_launch_dependents();
+    s_lo = misc[0];
+    nres = misc[1];
+
+    auto store_red = [&](int lrow_a, float (&yacc)[NT][4]) {
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-            emit(ra, 8 * t + 2 * q, yacc[t][0]);
-            emit(ra, 8 * t + 2 * q + 1, yacc[t][1]);
-            emit(rb, 8 * t + 2 * q, yacc[t][2]);
-            emit(rb, 8 * t + 2 * q + 1, yacc[t][3]);
+            const int t0 = 8 * t + 2 * q;
+            if (t0 < M) {
+                red[lrow_a * M + t0] = yacc[t][0];
+                red[(lrow_a + 8) * M + t0] = yacc[t][2];
+            }
+            if (t0 + 1 < M) {
+                red[lrow_a * M + t0 + 1] = yacc[t][1];
+                red[(lrow_a + 8) * M + t0 + 1] = yacc[t][3];
+            }
         }
-        return;
+    };
+
+    if (warp < kMainWarps) {
+        float yacc[NT][4];
+#pragma unroll
+        for (int t = 0; t < NT; ++t) yacc[t][0] = yacc[t][1] = yacc[t][2] = yacc[t][3] = 0.f;
+        const int strip_row = warp * kStrip;
+        strip_sums<NT>(ng, q, rr, sc1 + strip_row * kMaxGpc, cofs, xrow,
+                       [&](int c) { return wt1 + c * kMainChunkBytes + strip_row * 128; },
+                       [&](int c) { ok = mbar_wait(&mbar1[c], 0) && ok; }, yacc);
+        store_red(strip_row + rr, yacc);
+    } else if (nres > 0) {
+        const int rounds = (nres + kResStrips * kStrip - 1) / (kResStrips * kStrip);
+        for (int round = 0; round < rounds; ++round) {
+            const int strips = min(kResStrips, (nres - round * kResStrips * kStrip + kStrip - 1) / kStrip);
+            if (round > 0) {
+                __syncwarp();                 // every lane is done with the previous round's rows
+                if (lane == 0)
+                    for (int c = 0; c < nchunks; ++c) {
+                        mbar_arrive_expect_tx(&mbar2[c], strips * kStripBytes);
+                        for (int j = 0; j < strips; ++j)
+                            tma_load_2d(wt2 + c * kResChunkBytes + j * kStripBytes, &map2,
+                                        (g_begin + c * kChunkGroups) * kWordsPerGroup,
+                                        s_lo + (round * kResStrips + j) * kStrip, &mbar2[c]);
+                    }
+            }
+            for (int j = 0; j < strips; ++j) {
+                float yacc[NT][4];
+#pragma unroll
+                for (int t = 0; t < NT; ++t) yacc[t][0] = yacc[t][1] = yacc[t][2] = yacc[t][3] = 0.f;
+                const int rrow = (round * kResStrips + j) * kStrip;      // first residual row of the strip
+                strip_sums<NT>(ng, q, rr, sc2 + rrow * kMaxGpc, cofs, xrow,
+                               [&](int c) { return wt2 + c * kResChunkBytes + j * kStripBytes; },
+                               [&](int c) {
+                                   if (j == 0) ok = mbar_wait(&mbar2[c], round & 1) && ok;
+                               },
+                               yacc);
+                store_red(kRowsPerCta + rrow + rr, yacc);
+            }
+        }
     }
 
-    const int lr_a = warp * 16 + rr, lr_b = lr_a + 8;
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-        red[lr_a * 16 + 8 * t + 2 * q] = yacc[t][0];
-        red[lr_a * 16 + 8 * t + 2 * q + 1] = yacc[t][1];
-        red[lr_b * 16 + 8 * t + 2 * q] = yacc[t][2];
-        red[lr_b * 16 + 8 * t + 2 * q + 1] = yacc[t][3];
-    }
+    // Epilogue: fixed-order sum over the cluster's K-slices, residual rows added, one rounding.
     cluster_sync_all();
     const uint32_t me = cluster_rank();
     const int rows_per_rank = (kRowsPerCta + a.split - 1) / a.split;
     const int lr0 = int(me) * rows_per_rank;
-    for (int idx = threadIdx.x; idx < rows_per_rank * M; idx += kThreads) {
-        const int lr = lr0 + idx / M, tok = idx % M;
-        if (lr >= kRowsPerCta) break;
-        float s = 0.f;
-        for (int c = 0; c < a.split; ++c) s += ld_dsmem_f32(red + lr * 16 + tok, uint32_t(c));
-        emit(block_row0 + lr, tok, s);
-    }
+    const int lr_end = min(kRowsPerCta, lr0 + rows_per_rank);
+    for (int tok = 0; tok < M; ++tok)
+        for (int lr = lr0 + threadIdx.x; lr < lr_end; lr += kThreads) {
+            const int64_t n = n0 + lr;
+            if (n >= a.N) break;
+            float s = 0.f;
+            for (int c = 0; c < a.split; ++c) s += ld_dsmem_f32(red + lr * M + tok, uint32_t(c));
+            const int slot = bslot[lr];
+            if (slot >= 0 && slot < nres) {
+                float s2 = 0.f;
+                for (int c = 0; c < a.split; ++c)
+                    s2 += ld_dsmem_f32(red + (kRowsPerCta + slot) * M + tok, uint32_t(c));
+                s += s2;
+            }
+            a.y[int64_t(tok) * a.N + n] = __float2half_rn(s);
+        }
+    if (!ok && a.status) atomicOr(a.status, 1u);
     cluster_sync_all();   // keep this CTA's shared memory alive until every rank has read it
 }
 
@@ -351,32 +539,54 @@ int env_split() {
     return v;
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2D map over an exec plane [rows, K/16] uint32, box 32 words x box_rows, 128-byte swizzle.
+bool plane_map(CUtensorMap* map, const uint32_t* plane, int64_t rows, int64_t K, int box_rows) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cuuint64_t(K / kCodesPerWord), cuuint64_t(rows > 0 ? rows : 1)};
+    const cuuint64_t strides[1] = {cuuint64_t(K / kCodesPerWord) * 4};
+    const cuuint32_t box[2] = {32, cuuint32_t(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(plane), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct Plan {
-    int split, gpc, NT;
-    size_t smem;
+    int split, gpc;
 };
 
-Plan plan_for(int64_t rows, int64_t K, int M) {
-    Plan p;
-    p.NT = M <= 8 ? 1 : 2;
+Plan plan_for(int64_t N, int64_t K) {
     const int G = int(K / kGroup);
-    const int64_t blocks = (rows + kRowsPerCta - 1) / kRowsPerCta;
-    const int gpc_smem = std::max(1, kSmemBudget / (M * kGroup * int(sizeof(__half)) + kNegcStride * 4));
-    const int min_split = (G + gpc_smem - 1) / gpc_smem;
+    const int64_t blocks = (N + kRowsPerCta - 1) / kRowsPerCta;
+    const int min_split = (G + kMaxGpc - 1) / kMaxGpc;
     const int64_t target = 4LL * sm_count();
     const int par = int(std::min<int64_t>(kMaxSplit, (target + blocks - 1) / blocks));
     int split = std::max(min_split, env_split() > 0 ? env_split() : par);
     split = std::max(1, std::min(split, std::min(kMaxSplit, G)));
+    Plan p;
     p.gpc = (G + split - 1) / split;
     p.split = (G + p.gpc - 1) / p.gpc;
-    p.smem = size_t(M) * p.gpc * kGroup * sizeof(__half) + size_t(p.gpc) * kNegcStride * sizeof(float) +
-             size_t(kRowsPerCta) * 16 * sizeof(float);
     return p;
 }
 
-template <int NT, bool kRes>
-tern_status launch_pass(const GemvArgs& args, const Plan& p, int64_t blocks, cudaStream_t stream) {
-    auto kernel = gemv_kernel<NT, kRes>;
+template <int NT>
+tern_status launch(const CUtensorMap& m1, const CUtensorMap& m2, const GemvArgs& args, int64_t blocks, size_t smem,
+                   cudaStream_t stream) {
+    auto kernel = gemv_kernel<NT>;
     static std::mutex mu;
     static bool configured[64] = {false};
     int dev = 0;
@@ -384,74 +594,58 @@ tern_status launch_pass(const GemvArgs& args, const Plan& p, int64_t blocks, cud
     {
         std::lock_guard<std::mutex> lock(mu);
         if (!configured[dev]) {
-            if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
-                    cudaSuccess ||
+            if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024) != cudaSuccess ||
                 cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
                 return TERN_ERR_CUDA;
             configured[dev] = true;
         }
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned(p.split), unsigned(blocks), 1);
+    cfg.gridDim = dim3(unsigned(args.split), unsigned(blocks), 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = p.smem;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = unsigned(p.split);
+    attr[0].val.clusterDim.x = unsigned(args.split);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = p.split > 1 ? 1 : 0;
-    GemvArgs a = args;
-    a.gpc = p.gpc;
-    a.split = p.split;
-    if (cudaLaunchKernelEx(&cfg, kernel, a) != cudaSuccess) return TERN_ERR_CUDA;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, kernel, m1, m2, args) != cudaSuccess) return TERN_ERR_CUDA;
     return TERN_OK;
-}
-
-template <bool kRes>
-tern_status run_pass(const GemvArgs& args, cudaStream_t stream) {
-    const Plan p = plan_for(args.rows, args.K, args.M);
-    if (p.smem > 200 * 1024) return TERN_ERR_SHAPE;
-    const int64_t blocks = (args.rows + kRowsPerCta - 1) / kRowsPerCta;
-    if (blocks > 65535) return TERN_ERR_SHAPE;
-    return p.NT == 1 ? launch_pass<1, kRes>(args, p, blocks, stream) : launch_pass<2, kRes>(args, p, blocks, stream);
 }
 
 }  // namespace
 
-size_t gemv_workspace_bytes(const tern_weight& w, int64_t M) {
-    if (w.r <= 0 || M <= 0) return 0;
-    return size_t(M) * size_t(w.r) * sizeof(float);
-}
+size_t gemv_workspace_bytes(const tern_weight&, int64_t) { return 0; }
 
-tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y, float* res_ws, cudaStream_t stream) {
-    GemvArgs base = {};
-    base.x = x;
-    base.K = w.K;
-    base.G = int32_t(w.K / kGroup);
-    base.M = M;
-    if (w.r > 0) {
-        GemvArgs ra = base;
-        ra.plane = w.plane2;
-        ra.scale = reinterpret_cast<const __half*>(w.scale2);
-        ra.rows = w.r;
-        ra.res_out = res_ws;
-        const tern_status st = run_pass<true>(ra, stream);
-        if (st != TERN_OK) return st;
-    }
-    GemvArgs ma = base;
-    ma.plane = w.plane1;
-    ma.scale = reinterpret_cast<const __half*>(w.scale1);
-    ma.rows = w.N;
-    ma.y = y;
-    if (w.r > 0) {
-        ma.res_in = res_ws;
-        ma.res_slot = w.res_slot;
-        ma.r = w.r;
-    }
-    return run_pass<false>(ma, stream);
+tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y, float*, cudaStream_t stream) {
+    const Plan p = plan_for(w.N, w.K);
+    const int64_t blocks = (w.N + kRowsPerCta - 1) / kRowsPerCta;
+    if (blocks > 65535) return TERN_ERR_SHAPE;
+    CUtensorMap m1, m2;
+    if (!plane_map(&m1, w.plane1, w.N, w.K, kRowsPerCta)) return TERN_ERR_CUDA;
+    if (!plane_map(&m2, w.r > 0 ? w.plane2 : w.plane1, w.r > 0 ? w.r : w.N, w.K, kStrip)) return TERN_ERR_CUDA;
+    GemvArgs a = {};
+    a.scale1 = reinterpret_cast<const __half*>(w.scale1);
+    a.scale2 = reinterpret_cast<const __half*>(w.scale2);
+    a.res_slot = w.r > 0 ? w.res_slot : nullptr;
+    a.x = x;
+    a.y = y;
+    a.status = async_status_word();
+    a.N = w.N;
+    a.r = w.r;
+    a.K = w.K;
+    a.G = int32_t(w.K / kGroup);
+    a.M = M;
+    a.gpc = p.gpc;
+    a.split = p.split;
+    a.static_weights = (w.flags & TERN_WEIGHT_STATIC) ? 1 : 0;
+    const size_t smem = smem_bytes(M);
+    return M <= 8 ? launch<1>(m1, m2, a, blocks, smem, stream) : launch<2>(m1, m2, a, blocks, smem, stream);
 }
 
 }  // namespace tern

@@ -22,6 +22,9 @@ inline cudaStream_t as_cuda(tern_stream s) { return reinterpret_cast<cudaStream_
 // Returns a device pointer to a zeroed slot, or nullptr on a CUDA error.
 unsigned int* acquire_flag_slot(cudaStream_t stream);
 tern_status read_flag_slot(unsigned int* slot, cudaStream_t stream, unsigned int* value);
+// Device address of this device's sticky status word for asynchronous kernels (bounded waits
+// that ran out set it); nullptr on a CUDA error.
+unsigned int* async_status_word();
 
 // Decode GEMV (tern_gemv.cu), M in [1, 16].
 tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y, float* res_ws,

@@ -23,12 +23,26 @@ namespace tern {
 // on different streams or host threads do not share one.
 constexpr int kFlagSlots = 256;
 __device__ unsigned int g_status_words[kFlagSlots];
+__device__ unsigned int g_async_status;            // set by tern_linear kernels whose bounded wait ran out
 
 namespace {
 std::atomic<unsigned int> g_next_slot{0};
 std::mutex g_addr_mu;
 unsigned int* g_slot_base[64] = {nullptr};
 }  // namespace
+
+unsigned int* async_status_word() {
+    static unsigned int* addr[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(g_addr_mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_async_status) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<unsigned int*>(p);
+    }
+    return addr[dev];
+}
 
 unsigned int* acquire_flag_slot(cudaStream_t stream) {
     int dev = 0;
@@ -269,4 +283,19 @@ extern "C" tern_status tern_weight_validate(const tern_weight* w, tern_stream s)
         validate_residual_kernel<<<grid_for(w->N + w->r, 256), 256, 0, st>>>(w->res_rows, w->res_slot, w->N,
                                                                             w->r, f);
     }, TERN_ERR_BAD_CODE);
+}
+
+extern "C" tern_status tern_device_status(tern_stream s) {
+    cudaStream_t st = as_cuda(s);
+    unsigned int* w = async_status_word();
+    if (!w) return TERN_ERR_CUDA;
+    unsigned int v = 0;
+    const tern_status r = read_flag_slot(w, st, &v);
+    if (r != TERN_OK) return r;
+    if (v) {
+        if (cudaMemsetAsync(w, 0, sizeof(unsigned int), st) != cudaSuccess) return TERN_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return TERN_ERR_CUDA;
+        return TERN_ERR_TIMEOUT;
+    }
+    return TERN_OK;
 }

@@ -86,7 +86,7 @@ def test_linear_host_validation(lib):
     """Every check here fails before a launch, so no device is touched."""
     S = _lib.STATUS
     fake = 1 << 20         # an aligned non-null address that is never dereferenced on these paths
-    w = _lib.TernWeightC(64, 256, 128, fake, fake, 0, None, fake, None, None)
+    w = _lib.TernWeightC(64, 256, 128, fake, fake, 0, None, fake, None, None, 0)
     call = lambda w, x, M, y, ws=None, wsb=0: lib.tern_linear(  # noqa: E731
         ctypes.byref(w) if w is not None else None, x, M, y, ws, wsb, None)
     assert call(None, fake, 1, fake) == S["TERN_ERR_NULL"]
@@ -95,23 +95,22 @@ def test_linear_host_validation(lib):
     assert call(w, fake + 2, 1, fake * 4) == S["TERN_ERR_ALIGN"]
     assert call(w, fake, 1, fake) == S["TERN_ERR_SHAPE"]          # x and y overlap
     assert call(w, fake, -1, fake) == S["TERN_ERR_SHAPE"]
-    bad = _lib.TernWeightC(64, 200, 128, fake, fake, 0, None, fake, None, None)
+    bad = _lib.TernWeightC(64, 200, 128, fake, fake, 0, None, fake, None, None, 0)
     assert call(bad, fake, 1, fake * 4) == S["TERN_ERR_SHAPE"]
-    bad = _lib.TernWeightC(64, 256, 64, fake, fake, 0, None, fake, None, None)
+    bad = _lib.TernWeightC(64, 256, 64, fake, fake, 0, None, fake, None, None, 0)
     assert call(bad, fake, 1, fake * 4) == S["TERN_ERR_SHAPE"]
-    bad = _lib.TernWeightC(64, 256, 128, fake, fake, 65, fake, fake, fake, fake)
+    bad = _lib.TernWeightC(64, 256, 128, fake, fake, 65, fake, fake, fake, fake, 0)
     assert call(bad, fake, 1, fake * 4) == S["TERN_ERR_SHAPE"]    # r > N
-    bad = _lib.TernWeightC(64, 256, 128, fake, fake, 4, fake, fake, None, fake)
+    bad = _lib.TernWeightC(64, 256, 128, fake, fake, 4, fake, fake, None, fake, 0)
     assert call(bad, fake, 1, fake * 4) == S["TERN_ERR_NULL"]     # residual plane missing
-    bad = _lib.TernWeightC(64, 256, 128, fake + 4, fake, 0, None, fake, None, None)
+    bad = _lib.TernWeightC(64, 256, 128, fake + 4, fake, 0, None, fake, None, None, 0)
     assert call(bad, fake, 1, fake * 4) == S["TERN_ERR_ALIGN"]
-    # a residual weight needs workspace for the decode path
-    wr = _lib.TernWeightC(64, 256, 128, fake, fake, 4, fake, fake, fake, fake)
-    need = lib.tern_linear_workspace_bytes(ctypes.byref(wr), 3)
-    assert need >= 3 * 4 * 4 and need % 256 == 0
-    assert call(wr, fake, 3, fake * 4) == S["TERN_ERR_WORKSPACE"]
-    assert call(wr, fake, 3, fake * 4, fake * 8, need - 1) == S["TERN_ERR_WORKSPACE"]
-    assert lib.tern_linear_workspace_bytes(ctypes.byref(w), 16) == 0
+    # neither path needs scratch memory
+    wr = _lib.TernWeightC(64, 256, 128, fake, fake, 4, fake, fake, fake, fake, 1)
+    for M in (1, 16, 17, 4096):
+        assert lib.tern_linear_workspace_bytes(ctypes.byref(wr), M) == 0
+    assert call(wr, fake + 2, 3, fake * 4) == S["TERN_ERR_ALIGN"]
+    assert call(wr, fake, 3, fake * 4, fake * 8 + 4, 64) == S["TERN_ERR_ALIGN"]   # misaligned workspace
 
 
 def test_pack_host_validation(lib):

@@ -181,3 +181,41 @@ def test_workspace_and_output_untouched_outside_bounds():
     torch.cuda.synchronize()
     assert (ws[need:] == 0xA5).all() and (yb[M * t.N:] == 7.0).all()
     check(yb[: M * t.N].view(M, t.N).cpu().numpy(), oracle.linear(t.x[:M], t.T1, t.s1, t.res_rows, t.T2, t.s2))
+
+
+@pytest.mark.parametrize("M", [1, 16, 64])
+def test_static_weight_flag_gives_the_same_bits(M):
+    t = next(synth.draw_workload(synth.WORKLOADS[4], only=["o"]))
+    rng = np.random.default_rng(M)
+    x = torch.from_numpy(synth.draw_x(rng, M, t.K)).cuda()
+    w = api.TernWeight.from_numpy(t.T1, t.s1, t.res_rows, t.T2, t.s2)
+    ws = api.TernWeight.from_numpy(t.T1, t.s1, t.res_rows, t.T2, t.s2)
+    ws.static = True
+    y1, y2 = api.linear(x, w), api.linear(x, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+def test_back_to_back_calls_on_one_stream_see_their_inputs():
+    """Consecutive calls overlap under programmatic dependent launch; each must read the x that
+    the previous call wrote (a two-layer chain), and the result must match the oracle's chain."""
+    rng = np.random.default_rng(11)
+    N, K = 1024, 1024
+    ts = [synth.draw_tensor(rng, f"c{i}", N, K, 4, p_zero=0.4, res_pct=15) for i in range(3)]
+    ws = [api.TernWeight.from_numpy(t.T1, t.s1, t.res_rows, t.T2, t.s2) for t in ts]
+    for w in ws:
+        w.static = True
+    x = torch.from_numpy(ts[0].x).cuda()
+    h = x
+    for w in ws:
+        h = api.linear(h, w)
+    torch.cuda.synchronize()
+    ref = ts[0].x.astype(np.float64)
+    for t in ts:
+        ref = oracle.round_fp16(oracle.linear(ref.astype(np.float16), t.T1, t.s1, t.res_rows, t.T2, t.s2))
+    check(h.cpu().numpy(), ref.astype(np.float64), tol=5e-3)
+
+
+def test_device_status_is_clean_after_the_suite():
+    from ternary_weight_only_tern_b200 import _lib
+    assert _lib.load().tern_device_status(api._stream()) == 0
