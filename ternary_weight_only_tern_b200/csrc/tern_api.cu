@@ -73,6 +73,6 @@ extern "C" tern_status tern_linear(const tern_weight* w, const tern_half* x, int
     cudaStream_t st = as_cuda(stream);
     const __half* xh = reinterpret_cast<const __half*>(x);
     __half* yh = reinterpret_cast<__half*>(y);
-    if (M <= kGemvMaxM) return gemv_launch(*w, xh, int(M), yh, static_cast<float*>(workspace), st);
+    if (M <= kGemvMaxM) return gemv_launch(*w, xh, int(M), yh, st);
     return gemm_launch(*w, xh, M, yh, workspace, st);
 }

@@ -7,10 +7,12 @@
 // cores; the weights are never reconstructed in global memory (section 14: native kernels
 // consume the ternary planes directly).
 //
-// One CTA computes a 128 (tokens) x 256 (weight rows) tile with one tcgen05.mma
-// (kind::f16, M = 128, N = 256, K = 16, fp32 accumulator in TMEM) per 16 columns of K:
-//  * warp 0, one thread: TMA loads of the x tile (128 x 64 fp16, 128-byte swizzle) into a
-//    3-stage ring, and TMA loads of the packed codes of the tile's 256 weight rows (16 bytes
+// One CTA computes a 256 (tokens) x 256 (weight rows) tile with two tcgen05.mma (kind::f16,
+// M = 128, N = 256, K = 16, fp32 accumulators in TMEM columns 0-255 and 256-511) per 16
+// columns of K, one per half of the tokens, both reading the same dequantised weight tile: the
+// dequantisation, which bounds this kernel, is done once per 256 x 256 x 64 block of MMA work.
+//  * warp 0, one thread: TMA loads of the x tile (256 x 64 fp16, 128-byte swizzle) into a
+//    2-stage ring, and TMA loads of the packed codes of the tile's 256 weight rows (16 bytes
 //    per row per K block) and of its residual rows into an 8-stage ring that runs ahead;
 //  * warp 1, one thread: issues the MMAs and commits each stage back to the producers;
 //  * warps 2-9 (256 threads, one weight row each): per 64-wide K block, read the row's 16
@@ -21,20 +23,20 @@
 //    ahead. After the K loop the same warps read the accumulator from TMEM and write y.
 //  * every wait is bounded: after about two seconds the kernel records TERN_ERR_TIMEOUT in
 //    a device status word, drains its own copies and MMAs, frees TMEM and returns.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include <mutex>
 
-#include "tern_internal.cuh"
+#include "tern_device.cuh"
 
 namespace tern {
 namespace {
 
-constexpr int BM = 128;
+using namespace dev;
+
+constexpr int BM = 256;                             // tokens per CTA tile
+constexpr int kUmmaM = 128;                         // tokens per MMA (two MMAs per K step)
 constexpr int BN = 256;
 constexpr int BK = 64;
-constexpr int kStages = 3;                          // x tile + dequantised W tile
+constexpr int kStages = 2;                          // x tile + dequantised W tile
 constexpr int kStagesP = 8;                         // packed codes
 constexpr int kDequantThreads = 256;
 constexpr int kThreads = 64 + kDequantThreads;
@@ -42,8 +44,7 @@ constexpr int kABytes = BM * BK * 2;
 constexpr int kBBytes = BN * BK * 2;
 constexpr int kPBytes = BN * 16;                    // 16 bytes (64 trits) of codes per row
 constexpr int kResBox = 32;                         // residual rows per TMA box
-constexpr int kTmemCols = 256;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // bounded waits give up after ~2 s
+constexpr int kTmemCols = 512;                     // two 128 x 256 fp32 accumulators
 constexpr unsigned kTimeoutBit = 1u;
 
 struct GemmArgs {
@@ -74,59 +75,6 @@ constexpr size_t kSmemBytes = SmemLayout::bytes + 1024;                         
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 // ------------------------------------------------------------------ PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ uint64_t global_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Bounded wait for the phase of the given parity: false after about two seconds.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    const uint32_t addr = smem_u32(bar);
-    uint64_t t0 = 0;
-    for (uint32_t i = 0;; ++i) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(addr), "r"(parity)
-            : "memory");
-        if (done) return true;
-        if ((i & 255u) == 0) {
-            const uint64_t t = global_ns();
-            if (i == 0) t0 = t;
-            else if (t - t0 > kWaitLimitNs) return false;
-        }
-    }
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-        "[%4];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-        : "memory");
-}
-
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 bytes apart.
 __device__ __forceinline__ uint64_t umma_desc_sw128(const void* p) {
     const uint64_t addr = smem_u32(p);
@@ -134,8 +82,8 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(const void* p) {
            (2ull << 61);
 }
 
-// Instruction descriptor: kind::f16, A = B = fp16, D = fp32, both K-major, M = BM, N = BN.
-constexpr uint32_t kIdesc = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+// Instruction descriptor: kind::f16, A = B = fp16, D = fp32, both K-major, M = kUmmaM, N = BN.
+constexpr uint32_t kIdesc = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(kUmmaM >> 4) << 24);
 
 __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t a_desc, uint64_t b_desc, uint32_t accumulate) {
     asm volatile(
@@ -168,12 +116,6 @@ __device__ __forceinline__ bool dequant_all(bool pred) {
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
-    uint32_t d;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(magic));
-    return d;
-}
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
@@ -292,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 if (!ok) break;
                 mbar_arrive_expect_tx(&full_a[s], kABytes);
                 tma_load_2d(smem_a + s * kABytes, &tmap_x, kb * BK, int(m0), &full_a[s]);
+                tma_load_2d(smem_a + s * kABytes + kABytes / 2, &tmap_x, kb * BK, int(m0) + kUmmaM, &full_a[s]);
                 issued = kb + 1;
             }
             // drain: every issued copy lands before the CTA may exit
@@ -311,9 +254,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 const uint8_t* as = smem_a + s * kABytes;
                 const uint8_t* bs = smem_b + s * kBBytes;
 #pragma unroll
-                for (int k = 0; k < BK / 16; ++k)
-                    umma_f16(tmem_base, umma_desc_sw128(as + 32 * k), umma_desc_sw128(bs + 32 * k),
-                             (kb > 0 || k > 0) ? 1u : 0u);
+                for (int k = 0; k < BK / 16; ++k) {
+                    const uint64_t bd = umma_desc_sw128(bs + 32 * k);
+                    const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+                    umma_f16(tmem_base, umma_desc_sw128(as + 32 * k), bd, acc);
+                    umma_f16(tmem_base + uint32_t(BN), umma_desc_sw128(as + kABytes / 2 + 32 * k), bd, acc);
+                }
                 umma_commit(&empty[s]);
             }
             umma_commit(tmem_full);          // also on a timeout: every issued MMA retires first
@@ -358,8 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             ok = dequant_all(mbar_wait(&full_p[sp], (kb / kStagesP) & 1) &&
                              (kb < kStages || mbar_wait(&empty[s], ((kb / kStages) - 1) & 1)));
             if (!ok) break;
-            uint8_t* bs = smem_b + s * kBBytes;
-            const uint4 cur = *reinterpret_cast<const uint4*>(smem_p1 + sp * kPBytes + t * 16);
+            const uint32_t bs = smem_u32(smem_b + s * kBBytes);
+            const uint4 cur = lds_u4(smem_u32(smem_p1 + sp * kPBytes + t * 16));
             const __half2 s2 = __half2half2(valid ? sq[0] : __float2half(0.f));
             const uint32_t words[4] = {cur.x, cur.y, cur.z, cur.w};
 #pragma unroll
@@ -372,27 +318,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 o.y = h2_bits(__hmul2(tt[1], s2));
                 o.z = h2_bits(__hmul2(tt[2], s2));
                 o.w = h2_bits(__hmul2(tt[3], s2));
-                *reinterpret_cast<uint4*>(bs + sw128_offset(t, c)) = o;
+                sts_u4(bs + sw128_offset(t, c), o);
             }
             if (n_res > 0) {
                 asm volatile("bar.sync 1, %0;" ::"n"(kDequantThreads) : "memory");
                 for (int i = t; i < n_res * 8; i += kDequantThreads) {
                     const int row = i >> 3, c = i & 7;
                     const int2 e = res_list[row];
-                    const uint32_t w2 =
-                        *reinterpret_cast<const uint32_t*>(smem_p2 + sp * kPBytes + row * 16 + (c >> 1) * 4);
+                    const uint32_t w2 = lds_u32(smem_u32(smem_p2 + sp * kPBytes + row * 16 + (c >> 1) * 4));
                     const __half sc2 = (i == item0) ? rq0[0] : (i == item1) ? rq1[0]
                                                                             : a.scale2[int64_t(e.y) * a.G + g];
                     const __half2 s22 = __half2half2(sc2);
                     __half2 tt[4];
                     decode8((c & 1) ? (w2 >> 16) : (w2 & 0xFFFFu), tt);
-                    uint4* dst = reinterpret_cast<uint4*>(bs + sw128_offset(e.x, c));
-                    uint4 o = *dst;
+                    const uint32_t dst = bs + sw128_offset(e.x, c);
+                    uint4 o = lds_u4(dst);
                     o.x = h2_bits(__hfma2(tt[0], s22, bits_h2(o.x)));
                     o.y = h2_bits(__hfma2(tt[1], s22, bits_h2(o.y)));
                     o.z = h2_bits(__hfma2(tt[2], s22, bits_h2(o.z)));
                     o.w = h2_bits(__hfma2(tt[3], s22, bits_h2(o.w)));
-                    *dst = o;
+                    sts_u4(dst, o);
                 }
             }
             fence_async_smem();
@@ -405,12 +350,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         tc_fence_after();
         if (ok) {
             const int lq = warp & 3;                         // TMEM lanes 32*lq .. 32*lq+31
-            const int col0 = ((warp - 2) >> 2) * (BN / 2);   // columns 0..127 or 128..255
-            const int64_t m = m0 + lq * 32 + lane;
+            const int col0 = ((warp - 2) >> 2) * (BN / 2);   // weight rows 0..127 or 128..255
 #pragma unroll 1
-            for (int cc = 0; cc < BN / 2; cc += 32) {
+            for (int it = 0; it < 2 * (BN / 2) / 32; ++it) {
+                const int half = it / ((BN / 2) / 32), cc = (it % ((BN / 2) / 32)) * 32;
+                const int64_t m = m0 + half * kUmmaM + lq * 32 + lane;
                 uint32_t r[32];
-                const uint32_t taddr = tmem_base + (uint32_t(lq * 32) << 16) + uint32_t(col0 + cc);
+                const uint32_t taddr =
+                    tmem_base + (uint32_t(lq * 32) << 16) + uint32_t(half * BN + col0 + cc);
                 asm volatile(
                     "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
                     "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
@@ -455,19 +402,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
 }  // namespace
 
 size_t gemm_workspace_bytes(const tern_weight&, int64_t) { return 0; }
@@ -481,7 +415,7 @@ tern_status gemm_launch(const tern_weight& w, const __half* x, int64_t M, __half
     CUtensorMap map;
     const cuuint64_t dims[2] = {cuuint64_t(w.K), cuuint64_t(M)};
     const cuuint64_t strides[1] = {cuuint64_t(w.K) * sizeof(__half)};
-    const cuuint32_t box[2] = {BK, BM};
+    const cuuint32_t box[2] = {BK, kUmmaM};
     const cuuint32_t estr[2] = {1, 1};
     if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(x), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

@@ -29,26 +29,28 @@
 //    shift by 6 either way moves the codes of bits 0-3 and 10-15 into mantissa positions,
 //    so a word of 16 trits costs 2 shifts and 8 LOP3. Since c = t + 1, the MMA sums
 //    (B_p + 1 + t) * x from zero, and C = sum (B_p + 1) * x is subtracted once per group. C is
-//    computed once per CTA by the same MMA on the constant pattern B_p + 1 in the same K
-//    order (hidden behind the weight loads), so a zero plane cancels bit for bit. The bases are 4, 16 and 64, so the offsets
+//    computed once per CTA by the same MMA on the constant pattern B_p + 1 in the same K order
+//    and accumulator split (hidden behind the weight loads), so a zero plane cancels bit for bit. The bases are 4, 16 and 64, so the offsets
 //    are small and every partial sum is exact on integer inputs. A non-finite activation
 //    makes every output of its token non-finite (NaN where the dense product has +-inf).
 //  * The contraction order over K is free, so the MMA's K order follows the packed words
-//    (pair j = trits j and j+8 of a word); x is staged in shared memory in that order.
+//    (pair j = trits j and j+8 of a word); x is staged in shared memory in that order, with
+//    the words of a group arranged so that one MMA step's activation fragments are 128
+//    contiguous bytes (no bank conflicts).
 //  * Launches use programmatic dependent launch: a kernel may start while the previous one on
 //    the stream drains; it reads x (and, unless the weight is flagged static, the weight)
 //    only after griddepcontrol.wait, and writes nothing before it.
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <stdlib.h>
 
 #include <algorithm>
 #include <mutex>
 
-#include "tern_internal.cuh"
+#include "tern_device.cuh"
 
 namespace tern {
 namespace {
+
+using namespace dev;
 
 constexpr int kMainWarps = 4;
 constexpr int kThreads = (kMainWarps + 1) * 32;     // + one warp for the residual rows
@@ -63,7 +65,6 @@ constexpr int kMaxSplit = 16;
 constexpr int kMainChunkBytes = kRowsPerCta * 128;  // 8 KB
 constexpr int kStripBytes = kStrip * 128;           // 2 KB
 constexpr int kResChunkBytes = kResStrips * kStripBytes;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // bounded waits give up after ~2 s
 
 struct GemvArgs {
     const __half* scale1;      // [N, G]
@@ -96,182 +97,58 @@ size_t smem_bytes(int M) {
 }
 static_assert(Smem::xzero % 16 == 0 && Smem::red % 16 == 0, "16-byte aligned activation rows");
 
-// ------------------------------------------------------------------ PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
-    uint32_t d;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(magic));   // (a & b) | c
-    return d;
-}
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-    uint32_t d;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-    return d;
-}
-
-__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ uint64_t global_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Bounded wait for the phase of the given parity: false after about two seconds.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    const uint32_t addr = smem_u32(bar);
-    uint64_t t0 = 0;
-    for (uint32_t i = 0;; ++i) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(addr), "r"(parity)
-            : "memory");
-        if (done) return true;
-        if ((i & 255u) == 0) {
-            const uint64_t t = global_ns();
-            if (i == 0) t0 = t;
-            else if (t - t0 > kWaitLimitNs) return false;
-        }
-    }
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-        "[%4];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t cta) {
-    const uint32_t a = smem_u32(local);
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(a), "r"(cta));
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
-// Pair p of a word (trits p and p+8) as fp16x2 (B_p + c_lo, B_p + c_hi), c = t + 1.
-// B_p = 16, 4, 64, 16, 4, 64, 16, 4 for p = 0..7. wl = w << 6, wr = w >> 6.
-template <int P>
-__device__ __forceinline__ uint32_t decode_pair(uint32_t w, uint32_t wl, uint32_t wr) {
-    constexpr uint32_t kMask[3] = {0x00300030u, 0x00C000C0u, 0x03000300u};     // mantissa bits 4-5, 6-7, 8-9
-    constexpr uint32_t kMagic[3] = {0x54005400u, 0x4C004C00u, 0x44004400u};    // 64, 16, 4
-    if (P == 0) return lop3_and_or(wl, kMask[1], kMagic[1]);
-    if (P == 1) return lop3_and_or(wl, kMask[2], kMagic[2]);
-    if (P == 2) return lop3_and_or(w, kMask[0], kMagic[0]);
-    if (P == 3) return lop3_and_or(w, kMask[1], kMagic[1]);
-    if (P == 4) return lop3_and_or(w, kMask[2], kMagic[2]);
-    if (P == 5) return lop3_and_or(wr, kMask[0], kMagic[0]);
-    if (P == 6) return lop3_and_or(wr, kMask[1], kMagic[1]);
-    return lop3_and_or(wr, kMask[2], kMagic[2]);
-}
-
-// B_p + 1 (the decoded value of trit 0) for the pairs of MMA i (pairs 2*(i%4) and 2*(i%4)+1),
-// as fp16x2 bits: 17 = 0x4C40, 5 = 0x4500, 65 = 0x5410.
-__device__ __forceinline__ void zero_trit_pattern(int i4, uint32_t& lo, uint32_t& hi) {
-    switch (i4) {
-        case 0: lo = 0x4C404C40u; hi = 0x45004500u; break;   // pairs 0, 1: bases 16, 4
-        case 1: lo = 0x54105410u; hi = 0x4C404C40u; break;   // pairs 2, 3: bases 64, 16
-        case 2: lo = 0x45004500u; hi = 0x54105410u; break;   // pairs 4, 5: bases 4, 64
-        default: lo = 0x4C404C40u; hi = 0x45004500u; break;  // pairs 6, 7: bases 16, 4
-    }
-}
-
-// Words 2q and 2q+1 of group gl (0..3) of a row in a 128-byte-swizzled TMA box.
-__device__ __forceinline__ uint2 lds_words(const uint8_t* box, int row, int gl, int q) {
-    const int chunk = 2 * gl + (q >> 1);
-    return *reinterpret_cast<const uint2*>(box + row * 128 + ((chunk ^ (row & 7)) << 4) + 8 * (q & 1));
-}
-
 // One 16-row strip over the slice: yacc[t][e] += s(row) * (sum_k t * x) over the slice's groups.
-// box(c): smem base of chunk c for this strip (16 rows of 128 B, 128-byte swizzled); sc: the
-// strip's scales [16][kMaxGpc]; xrow[t]: this lane's activation row for token tile t (pairs in
-// word order, or the zero row); cofs: C[g][token]. The lane holds rows rr and rr + 8.
-// Two groups run at once, so their accumulator chains overlap.
+// All operands are 32-bit shared addresses: box(c) is chunk c of this strip (16 rows of 128 B,
+// 128-byte swizzled), sc the strip's scales [16][kMaxGpc] (fp16), xrow[t] this lane's
+// activation row for token tile t (pairs in word order, or the zero row), cofs C[g][token].
+// The lane holds rows rr and rr + 8. Two groups run at once, each split over two
+// accumulators (the two words of the lane), so four MMA chains are in flight per warp.
 template <int NT, typename BoxFn, typename WaitFn>
-__device__ __forceinline__ void strip_sums(int ng, int q, int rr, const __half* sc, const float* cofs,
-                                           const __half* const (&xrow)[NT], BoxFn box, WaitFn wait_chunk,
+__device__ __forceinline__ void strip_sums(int ng, int q, int rr, uint32_t sc, uint32_t cofs,
+                                           const uint32_t (&xrow)[NT], BoxFn box, WaitFn wait_chunk,
                                            float (&yacc)[NT][4]) {
     // byte offset of words 2q, 2q+1 of group gl in rows rr and rr+8 (row & 7 == rr & 7):
     // chunk 2*gl + q/2 of the 128-byte row, swizzled by the row
     const int qh = q >> 1, r7 = rr & 7, qb = 8 * (q & 1);
-    const int roff_a = rr * 128 + qb, roff_b = (rr + 8) * 128 + qb;
+    const uint32_t roff_a = rr * 128 + qb, roff_b = (rr + 8) * 128 + qb;
+    const uint32_t sc_a = sc + rr * kMaxGpc * 2, sc_b = sc + (rr + 8) * kMaxGpc * 2;
     for (int g0 = 0; g0 < ng; g0 += 2) {
         if ((g0 % kChunkGroups) == 0) wait_chunk(g0 / kChunkGroups);
-        const uint8_t* b = box(g0 / kChunkGroups);          // groups g0 and g0 + 1 share a chunk
+        const uint32_t b = box(g0 / kChunkGroups);          // groups g0 and g0 + 1 share a chunk
         const int ngrp = min(2, ng - g0);
-        float acc[2][NT][4];
+        float acc[2][2][NT][4];                              // [group][word][tile][element]
 #pragma unroll
         for (int u = 0; u < 2; ++u)
 #pragma unroll
-            for (int t = 0; t < NT; ++t) acc[u][t][0] = acc[u][t][1] = acc[u][t][2] = acc[u][t][3] = 0.f;
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int t = 0; t < NT; ++t) acc[u][h][t][0] = acc[u][h][t][1] = acc[u][h][t][2] = acc[u][h][t][3] = 0.f;
+        uint2 wa2[2], wb2[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            if (u >= ngrp) break;
-            const int gi = g0 + u, gl = gi % kChunkGroups;
-            const int woff = ((2 * gl + qh) ^ r7) << 4;
-            const uint2 wa2 = *reinterpret_cast<const uint2*>(b + roff_a + woff);
-            const uint2 wb2 = *reinterpret_cast<const uint2*>(b + roff_b + woff);
+            const int gl = (g0 + u) % kChunkGroups;
+            const uint32_t woff = ((2 * gl + qh) ^ r7) << 4;
+            wa2[u] = lds_u2(b + roff_a + woff);
+            wb2[u] = lds_u2(b + roff_b + woff);
+        }
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint32_t wa = h ? wa2.y : wa2.x, wb = h ? wb2.y : wb2.x;
-                const uint32_t wal = wa << 6, war = wa >> 6, wbl = wb << 6, wbr = wb >> 6;
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                if (u >= ngrp) break;
+                const int gi = g0 + u;
+                const uint32_t wa = h ? wa2[u].y : wa2[u].x, wb = h ? wb2[u].y : wb2[u].x;
                 uint32_t A[4][4];   // four MMAs per word: pairs (0,1), (2,3), (4,5), (6,7)
-                A[0][0] = decode_pair<0>(wa, wal, war); A[0][1] = decode_pair<0>(wb, wbl, wbr);
-                A[0][2] = decode_pair<1>(wa, wal, war); A[0][3] = decode_pair<1>(wb, wbl, wbr);
-                A[1][0] = decode_pair<2>(wa, wal, war); A[1][1] = decode_pair<2>(wb, wbl, wbr);
-                A[1][2] = decode_pair<3>(wa, wal, war); A[1][3] = decode_pair<3>(wb, wbl, wbr);
-                A[2][0] = decode_pair<4>(wa, wal, war); A[2][1] = decode_pair<4>(wb, wbl, wbr);
-                A[2][2] = decode_pair<5>(wa, wal, war); A[2][3] = decode_pair<5>(wb, wbl, wbr);
-                A[3][0] = decode_pair<6>(wa, wal, war); A[3][1] = decode_pair<6>(wb, wbl, wbr);
-                A[3][2] = decode_pair<7>(wa, wal, war); A[3][3] = decode_pair<7>(wb, wbl, wbr);
+                decode_word_pair(wa, wb, A);
 #pragma unroll
                 for (int t = 0; t < NT; ++t) {
                     // the B fragments of this word's four MMAs: 32 contiguous bytes of the row
-                    const uint4* xp = reinterpret_cast<const uint4*>(xrow[t] + gi * kGroup + 16 * (2 * q + h));
-                    const uint4 x01 = xp[0], x23 = xp[1];
-                    mma_16816(acc[u][t], A[0], x01.x, x01.y);
-                    mma_16816(acc[u][t], A[1], x01.z, x01.w);
-                    mma_16816(acc[u][t], A[2], x23.x, x23.y);
-                    mma_16816(acc[u][t], A[3], x23.z, x23.w);
+                    const uint32_t xp = xrow[t] + (gi * kGroup + 16 * (4 * h + q)) * 2;
+                    const uint4 x01 = lds_u4(xp), x23 = lds_u4(xp + 16);
+                    mma_16816(acc[u][h][t], A[0], x01.x, x01.y);
+                    mma_16816(acc[u][h][t], A[1], x01.z, x01.w);
+                    mma_16816(acc[u][h][t], A[2], x23.x, x23.y);
+                    mma_16816(acc[u][h][t], A[3], x23.z, x23.w);
                 }
             }
         }
@@ -279,15 +156,14 @@ __device__ __forceinline__ void strip_sums(int ng, int q, int rr, const __half* 
         for (int u = 0; u < 2; ++u) {
             if (u >= ngrp) break;
             const int gi = g0 + u;
-            const float sa = __half2float(sc[rr * kMaxGpc + gi]);
-            const float sb = __half2float(sc[(rr + 8) * kMaxGpc + gi]);
+            const float sa = lds_h2f(sc_a + gi * 2), sb = lds_h2f(sc_b + gi * 2);
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
-                const float2 c = *reinterpret_cast<const float2*>(cofs + gi * 16 + 8 * t + 2 * q);
-                yacc[t][0] = fmaf(sa, acc[u][t][0] - c.x, yacc[t][0]);
-                yacc[t][1] = fmaf(sa, acc[u][t][1] - c.y, yacc[t][1]);
-                yacc[t][2] = fmaf(sb, acc[u][t][2] - c.x, yacc[t][2]);
-                yacc[t][3] = fmaf(sb, acc[u][t][3] - c.y, yacc[t][3]);
+                const float2 c = lds_f2(cofs + (gi * 16 + 8 * t + 2 * q) * 4);
+                yacc[t][0] = fmaf(sa, (acc[u][0][t][0] + acc[u][1][t][0]) - c.x, yacc[t][0]);
+                yacc[t][1] = fmaf(sa, (acc[u][0][t][1] + acc[u][1][t][1]) - c.y, yacc[t][1]);
+                yacc[t][2] = fmaf(sb, (acc[u][0][t][2] + acc[u][1][t][2]) - c.x, yacc[t][2]);
+                yacc[t][3] = fmaf(sb, (acc[u][0][t][3] + acc[u][1][t][3]) - c.y, yacc[t][3]);
             }
         }
     }
@@ -395,6 +271,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
         const int blocks16 = ng * kWordsPerGroup;
         for (int m = 0; m < M; ++m)
             for (int b = threadIdx.x; b < blocks16; b += kThreads) {
+                // word b of the slice (group b / 8, word w = b % 8 = 2q + h) goes to slot 4h + q of its
+                // group, so the four quad lanes of one MMA step read 128 contiguous bytes
+                const int w = b & 7, slot = (b & ~7) | ((w & 1) << 2) | (w >> 1);
                 const uint4* src =
                     reinterpret_cast<const uint4*>(a.x + int64_t(m) * a.K + int64_t(g_begin) * kGroup + b * 16);
                 const uint4 lo = __ldg(src), hi = __ldg(src + 1);
@@ -403,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
                 o0.z = prmt(lo.y, hi.y, 0x5410u); o0.w = prmt(lo.y, hi.y, 0x7632u);
                 o1.x = prmt(lo.z, hi.z, 0x5410u); o1.y = prmt(lo.z, hi.z, 0x7632u);
                 o1.z = prmt(lo.w, hi.w, 0x5410u); o1.w = prmt(lo.w, hi.w, 0x7632u);
-                uint4* dst = reinterpret_cast<uint4*>(xs + size_t(m) * xs_stride + b * 16);
+                uint4* dst = reinterpret_cast<uint4*>(xs + size_t(m) * xs_stride + slot * 16);
                 dst[0] = o0;
                 dst[1] = o1;
             }
@@ -412,37 +291,41 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
     }
     __syncthreads();
 
-    const __half* xrow[NT];
+    uint32_t xrow[NT];
 #pragma unroll
-    for (int t = 0; t < NT; ++t) xrow[t] = (8 * t + rr < M) ? xs + size_t(8 * t + rr) * xs_stride : xzero;
+    for (int t = 0; t < NT; ++t) xrow[t] = smem_u32((8 * t + rr < M) ? xs + size_t(8 * t + rr) * xs_stride : xzero);
 
-    // C[g][token] = sum_k (B_p(k) + 1) * x[token][k]: one MMA chain per group on the constant
-    // pattern, in the same K order as the main chains, so a zero plane cancels bit for bit
+    // C[g][token] = sum_k (B_p(k) + 1) * x[token][k]: MMA chains on the constant pattern in the
+    // same K order and with the same split into two accumulators (one per word of the lane) as
+    // the main chains, combined by the same single addition, so a zero plane cancels bit for bit
     for (int gi = warp; gi < ng; gi += kMainWarps + 1) {
-        float c[NT][4];
+        float c[2][NT][4];
 #pragma unroll
-        for (int t = 0; t < NT; ++t) c[t][0] = c[t][1] = c[t][2] = c[t][3] = 0.f;
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int t = 0; t < NT; ++t) c[h][t][0] = c[h][t][1] = c[h][t][2] = c[h][t][3] = 0.f;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
-                const uint4* xp = reinterpret_cast<const uint4*>(xrow[t] + gi * kGroup + 16 * (2 * q + h));
-                const uint4 x01 = xp[0], x23 = xp[1];
+                const uint32_t xp = xrow[t] + (gi * kGroup + 16 * (4 * h + q)) * 2;
+                const uint4 x01 = lds_u4(xp), x23 = lds_u4(xp + 16);
                 uint32_t Z[4];
                 zero_trit_pattern(0, Z[0], Z[2]); Z[1] = Z[0]; Z[3] = Z[2];
-                mma_16816(c[t], Z, x01.x, x01.y);
+                mma_16816(c[h][t], Z, x01.x, x01.y);
                 zero_trit_pattern(1, Z[0], Z[2]); Z[1] = Z[0]; Z[3] = Z[2];
-                mma_16816(c[t], Z, x01.z, x01.w);
+                mma_16816(c[h][t], Z, x01.z, x01.w);
                 zero_trit_pattern(2, Z[0], Z[2]); Z[1] = Z[0]; Z[3] = Z[2];
-                mma_16816(c[t], Z, x23.x, x23.y);
+                mma_16816(c[h][t], Z, x23.x, x23.y);
                 zero_trit_pattern(3, Z[0], Z[2]); Z[1] = Z[0]; Z[3] = Z[2];
-                mma_16816(c[t], Z, x23.z, x23.w);
+                mma_16816(c[h][t], Z, x23.z, x23.w);
             }
         }
         if (rr == 0) {
 #pragma unroll
             for (int t = 0; t < NT; ++t)
-                *reinterpret_cast<float2*>(cofs + gi * 16 + 8 * t + 2 * q) = make_float2(c[t][0], c[t][1]);
+                *reinterpret_cast<float2*>(cofs + gi * 16 + 8 * t + 2 * q) =
+                    make_float2(c[0][t][0] + c[1][t][0], c[0][t][1] + c[1][t][1]);
         }
     }
     __syncthreads();
@@ -470,8 +353,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
 #pragma unroll
         for (int t = 0; t < NT; ++t) yacc[t][0] = yacc[t][1] = yacc[t][2] = yacc[t][3] = 0.f;
         const int strip_row = warp * kStrip;
-        strip_sums<NT>(ng, q, rr, sc1 + strip_row * kMaxGpc, cofs, xrow,
-                       [&](int c) { return wt1 + c * kMainChunkBytes + strip_row * 128; },
+        strip_sums<NT>(ng, q, rr, smem_u32(sc1 + strip_row * kMaxGpc), smem_u32(cofs), xrow,
+                       [&](int c) { return smem_u32(wt1 + c * kMainChunkBytes + strip_row * 128); },
                        [&](int c) { ok = mbar_wait(&mbar1[c], 0) && ok; }, yacc);
         store_red(strip_row + rr, yacc);
     } else if (nres > 0) {
@@ -494,8 +377,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
 #pragma unroll
                 for (int t = 0; t < NT; ++t) yacc[t][0] = yacc[t][1] = yacc[t][2] = yacc[t][3] = 0.f;
                 const int rrow = (round * kResStrips + j) * kStrip;      // first residual row of the strip
-                strip_sums<NT>(ng, q, rr, sc2 + rrow * kMaxGpc, cofs, xrow,
-                               [&](int c) { return wt2 + c * kResChunkBytes + j * kStripBytes; },
+                strip_sums<NT>(ng, q, rr, smem_u32(sc2 + rrow * kMaxGpc), smem_u32(cofs), xrow,
+                               [&](int c) { return smem_u32(wt2 + c * kResChunkBytes + j * kStripBytes); },
                                [&](int c) {
                                    if (j == 0) ok = mbar_wait(&mbar2[c], round & 1) && ok;
                                },
@@ -537,32 +420,6 @@ int env_split() {
         return s ? atoi(s) : 0;
     }();
     return v;
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// 2D map over an exec plane [rows, K/16] uint32, box 32 words x box_rows, 128-byte swizzle.
-bool plane_map(CUtensorMap* map, const uint32_t* plane, int64_t rows, int64_t K, int box_rows) {
-    auto enc = encode_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {cuuint64_t(K / kCodesPerWord), cuuint64_t(rows > 0 ? rows : 1)};
-    const cuuint64_t strides[1] = {cuuint64_t(K / kCodesPerWord) * 4};
-    const cuuint32_t box[2] = {32, cuuint32_t(box_rows)};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(plane), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 struct Plan {
@@ -622,13 +479,15 @@ tern_status launch(const CUtensorMap& m1, const CUtensorMap& m2, const GemvArgs&
 
 size_t gemv_workspace_bytes(const tern_weight&, int64_t) { return 0; }
 
-tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y, float*, cudaStream_t stream) {
+tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y, cudaStream_t stream) {
     const Plan p = plan_for(w.N, w.K);
     const int64_t blocks = (w.N + kRowsPerCta - 1) / kRowsPerCta;
     if (blocks > 65535) return TERN_ERR_SHAPE;
     CUtensorMap m1, m2;
-    if (!plane_map(&m1, w.plane1, w.N, w.K, kRowsPerCta)) return TERN_ERR_CUDA;
-    if (!plane_map(&m2, w.r > 0 ? w.plane2 : w.plane1, w.r > 0 ? w.r : w.N, w.K, kStrip)) return TERN_ERR_CUDA;
+    if (!plane_map(&m1, w.plane1, w.N, w.K, 32, kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B)) return TERN_ERR_CUDA;
+    if (!plane_map(&m2, w.r > 0 ? w.plane2 : w.plane1, w.r > 0 ? w.r : w.N, w.K, 32, kStrip,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return TERN_ERR_CUDA;
     GemvArgs a = {};
     a.scale1 = reinterpret_cast<const __half*>(w.scale1);
     a.scale2 = reinterpret_cast<const __half*>(w.scale2);
