@@ -26,6 +26,7 @@ max over ranks.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import subprocess
@@ -36,6 +37,28 @@ import time
 import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
+
+# DRAM bytes (read + write) of one launch of the dominant kernel, from one ncu capture of the
+# `--profile gemv` case (summary and command under profiles/), keyed by a hash of the sources the
+# kernel is built from: when they change, the number no longer describes the kernel and the
+# bench reports null until it is captured again.
+KERNEL_TRAFFIC = {
+    "gemv": {"sources": ["ternary_weight_only_tern_b200/csrc/tern_gemv.cu",
+                         "ternary_weight_only_tern_b200/csrc/tern_device.cuh"],
+             "sha256": "5784ce85cd3d0368a5f86340da309d288e96bc7effb02c2e3c518aa3538d9275",
+             "bytes": 15476480},
+}
+
+
+def measured_traffic(kernel: str):
+    t = KERNEL_TRAFFIC[kernel]
+    if t["sha256"] is None:
+        return None
+    h = hashlib.sha256()
+    for rel in t["sources"]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return t["bytes"] if h.hexdigest() == t["sha256"] else None
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
@@ -364,8 +387,8 @@ def main():
     gate_bytes = (gw + ga) / LAYERS
     achieved = gate_bytes / t_gate / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                "op": "tern_linear gate 12288x4096 (+1843 residual rows) M=1, both passes",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic("gemv"),
+                "op": "tern_linear gate 12288x4096 (+1843 residual rows) M=1",
                 "us_per_call": t_gate * 1e6, "bytes_per_call": gate_bytes, "peak_kind": peak_kind,
                 "frac_of_8000": achieved / 8000.0}
 
@@ -437,10 +460,12 @@ def profile_case(torch, api, shapes, dev, which):
     xs = {n: torch.randn((M, K), device=dev).half() for n, _, K in shapes}
     ys = {n: torch.empty((M, N), dtype=torch.float16, device=dev) for n, N, _ in shapes}
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("tern_calls")   # ncu --nvtx --nvtx-include "tern_calls/" lists these only
     for _ in range(3):
         for layer in pool:
             for n in names:
                 api.linear(xs[n], layer[n], out=ys[n])
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     print(json.dumps({"profile": which, "calls": 3 * len(pool) * len(names)}))
 
