@@ -145,6 +145,14 @@ __device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t cta) 
     return v;
 }
 
+// Store a float at the same shared-memory offset as `local`, in the CTA of cluster rank `cta`.
+__device__ __forceinline__ void st_dsmem_f32(const float* local, uint32_t cta, float v) {
+    const uint32_t a = smem_u32(local);
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(a), "r"(cta));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+}
+
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 

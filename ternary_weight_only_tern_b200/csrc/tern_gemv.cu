@@ -88,12 +88,16 @@ struct Smem {
     static constexpr int sc1 = misc + 16;                                  // half [64][kMaxGpc]
     static constexpr int sc2 = sc1 + kRowsPerCta * kMaxGpc * 2;            // half [64][kMaxGpc]
     static constexpr int bslot = sc2 + kMaxResRows * kMaxGpc * 2;          // int [64]: slot - s_lo, or -1
-    static constexpr int cofs = bslot + kRowsPerCta * 4;                   // float [kMaxGpc][16]
+    static constexpr int srow = bslot + kRowsPerCta * 4;                   // int [64]: residual slot -> row
+    static constexpr int cofs = srow + kMaxResRows * 4;                    // float [kMaxGpc][16]
     static constexpr int xzero = cofs + kMaxGpc * 16 * 4;                  // half [kMaxGpc * 128]: zeros
-    static constexpr int red = xzero + kMaxGpc * kGroup * 2;               // float [128][M], then xs
+    static constexpr int red = xzero + kMaxGpc * kGroup * 2;               // receive buffers, then xs
 };
+// Rows of the block owned by each rank, and the receive buffers: [rank][owned row][token] for the
+// main rows' partial sums and the same for their residual rows', pushed by every rank of the cluster.
+constexpr int kRecvRows = kRowsPerCta + kMaxSplit;                     // >= split * ceil(64 / split)
 size_t smem_bytes(int M) {
-    return size_t(Smem::red) + size_t(kRowsPerCta + kMaxResRows) * M * 4 + size_t(M) * kMaxGpc * kGroup * 2 + 1024;
+    return size_t(Smem::red) + size_t(2 * kRecvRows) * M * 4 + size_t(M) * kMaxGpc * kGroup * 2 + 1024;
 }
 static_assert(Smem::xzero % 16 == 0 && Smem::red % 16 == 0, "16-byte aligned activation rows");
 
@@ -187,8 +191,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
     float* cofs = reinterpret_cast<float*>(smem + Smem::cofs);
     __half* xzero = reinterpret_cast<__half*>(smem + Smem::xzero);
     const int M = a.M;
-    float* red = reinterpret_cast<float*>(smem + Smem::red);                         // [128][M]
-    __half* xs = reinterpret_cast<__half*>(smem + Smem::red + (kRowsPerCta + kMaxResRows) * M * 4);
+    int* srow = reinterpret_cast<int*>(smem + Smem::srow);
+    float* recv = reinterpret_cast<float*>(smem + Smem::red);                        // [split][rows/split][M]
+    float* recv_res = recv + kRecvRows * M;                                          // same, residual rows
+    __half* xs = reinterpret_cast<__half*>(smem + Smem::red + 2 * kRecvRows * M * 4);
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int q = lane & 3, rr = lane >> 2;
@@ -209,6 +215,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     __syncthreads();
+    // this CTA has started; the matching wait comes before the first store into a peer's memory
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    // The next call on the stream may start now: its weight loads overlap this call, and it reads
+    // x (this call's output, possibly) only after griddepcontrol.wait.
+    grid_launch_dependents();
 
     int s_lo = 0, nres = 0;
     // Everything the weight determines, issued at once: TMA of the main tile (thread 0); the
@@ -234,6 +245,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
             s_lo = nres ? __shfl_sync(0xffffffffu, first < 32 ? sl0 : sl1, first & 31) : 0;
             bslot[lane] = v0 ? sl0 - s_lo : -1;
             bslot[32 + lane] = v1 ? sl1 - s_lo : -1;
+            srow[lane] = -1;
+            srow[32 + lane] = -1;
+            __syncwarp();
+            if (v0 && sl0 - s_lo < kMaxResRows) srow[sl0 - s_lo] = lane;
+            if (v1 && sl1 - s_lo < kMaxResRows) srow[sl1 - s_lo] = 32 + lane;
             if (lane == 0) {
                 misc[0] = s_lo;
                 misc[1] = nres;
@@ -329,24 +345,38 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
         }
     }
     __syncthreads();
-    grid_launch_dependents();
     s_lo = misc[0];
     nres = misc[1];
 
-    auto store_red = [&](int lrow_a, float (&yacc)[NT][4]) {
+    // Partial sums go straight to the rank that owns the row: [this rank][row - owner's first][token]
+    // in the owner's receive buffer (buf = recv for main rows, recv_res for residual rows).
+    const uint32_t me = cluster_rank();
+    const int rows_per_rank = (kRowsPerCta + a.split - 1) / a.split;
+    auto push = [&](float* buf, int lrow, int t, float v) {
+        const int owner = lrow / rows_per_rank;
+        st_dsmem_f32(buf + (int(me) * rows_per_rank + (lrow - owner * rows_per_rank)) * M + t, uint32_t(owner), v);
+    };
+    // rows lrow_a and lrow_a + 8 of a strip (local rows of the block, or residual slots), this
+    // lane's tokens
+    auto store_red = [&](bool residual, int lrow_a, float (&yacc)[NT][4]) {
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            const int t0 = 8 * t + 2 * q;
-            if (t0 < M) {
-                red[lrow_a * M + t0] = yacc[t][0];
-                red[(lrow_a + 8) * M + t0] = yacc[t][2];
+        for (int h = 0; h < 2; ++h) {
+            int lrow = lrow_a + 8 * h;
+            if (residual) {
+                if (lrow >= nres || lrow >= kMaxResRows) continue;
+                lrow = srow[lrow];
+                if (lrow < 0 || lrow >= kRowsPerCta) continue;   // only with an inconsistent slot map
             }
-            if (t0 + 1 < M) {
-                red[lrow_a * M + t0 + 1] = yacc[t][1];
-                red[(lrow_a + 8) * M + t0 + 1] = yacc[t][3];
+            float* buf = residual ? recv_res : recv;
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const int t0 = 8 * t + 2 * q;
+                if (t0 < M) push(buf, lrow, t0, yacc[t][2 * h]);
+                if (t0 + 1 < M) push(buf, lrow, t0 + 1, yacc[t][2 * h + 1]);
             }
         }
     };
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");   // every CTA of the cluster has started
 
     if (warp < kMainWarps) {
         float yacc[NT][4];
@@ -356,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
         strip_sums<NT>(ng, q, rr, smem_u32(sc1 + strip_row * kMaxGpc), smem_u32(cofs), xrow,
                        [&](int c) { return smem_u32(wt1 + c * kMainChunkBytes + strip_row * 128); },
                        [&](int c) { ok = mbar_wait(&mbar1[c], 0) && ok; }, yacc);
-        store_red(strip_row + rr, yacc);
+        store_red(false, strip_row + rr, yacc);
     } else if (nres > 0) {
         const int rounds = (nres + kResStrips * kStrip - 1) / (kResStrips * kStrip);
         for (int round = 0; round < rounds; ++round) {
@@ -383,34 +413,34 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
                                    if (j == 0) ok = mbar_wait(&mbar2[c], round & 1) && ok;
                                },
                                yacc);
-                store_red(kRowsPerCta + rrow + rr, yacc);
+                store_red(true, rrow + rr, yacc);
             }
         }
     }
 
-    // Epilogue: fixed-order sum over the cluster's K-slices, residual rows added, one rounding.
-    cluster_sync_all();
-    const uint32_t me = cluster_rank();
-    const int rows_per_rank = (kRowsPerCta + a.split - 1) / a.split;
-    const int lr0 = int(me) * rows_per_rank;
-    const int lr_end = min(kRowsPerCta, lr0 + rows_per_rank);
-    for (int tok = 0; tok < M; ++tok)
-        for (int lr = lr0 + threadIdx.x; lr < lr_end; lr += kThreads) {
+    // Epilogue: the partial sums of this rank's rows arrived from every rank; they are summed in
+    // rank order, the residual rows' sums added, and rounded once. After the barrier no CTA
+    // touches another's memory, so each may exit as soon as it is done.
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    {
+        const int lr0 = int(me) * rows_per_rank;
+        const int nrows = max(0, min(kRowsPerCta, lr0 + rows_per_rank) - lr0);
+        for (int i = threadIdx.x; i < nrows * M; i += kThreads) {
+            const int tok = i / nrows, lo = i - tok * nrows, lr = lr0 + lo;
             const int64_t n = n0 + lr;
-            if (n >= a.N) break;
+            if (n >= a.N) continue;
             float s = 0.f;
-            for (int c = 0; c < a.split; ++c) s += ld_dsmem_f32(red + lr * M + tok, uint32_t(c));
+            for (int c = 0; c < a.split; ++c) s += recv[(c * rows_per_rank + lo) * M + tok];
             const int slot = bslot[lr];
             if (slot >= 0 && slot < nres) {
                 float s2 = 0.f;
-                for (int c = 0; c < a.split; ++c)
-                    s2 += ld_dsmem_f32(red + (kRowsPerCta + slot) * M + tok, uint32_t(c));
+                for (int c = 0; c < a.split; ++c) s2 += recv_res[(c * rows_per_rank + lo) * M + tok];
                 s += s2;
             }
             a.y[int64_t(tok) * a.N + n] = __float2half_rn(s);
         }
+    }
     if (!ok && a.status) atomicOr(a.status, 1u);
-    cluster_sync_all();   // keep this CTA's shared memory alive until every rank has read it
 }
 
 // ------------------------------------------------------------------ host side
