@@ -107,7 +107,8 @@ static_assert(Smem::xzero % 16 == 0 && Smem::red % 16 == 0, "16-byte aligned act
 // activation row for token tile t (pairs in word order, or the zero row), cofs C[g][token].
 // The lane holds rows rr and rr + 8. Two groups run at once, each split over two
 // accumulators (the two words of the lane), so four MMA chains are in flight per warp.
-template <int NT, typename BoxFn, typename WaitFn>
+// kOne: M == 1, so only the first token's elements of the accumulators are kept.
+template <int NT, bool kOne, typename BoxFn, typename WaitFn>
 __device__ __forceinline__ void strip_sums(int ng, int q, int rr, uint32_t sc, uint32_t cofs,
                                            const uint32_t (&xrow)[NT], BoxFn box, WaitFn wait_chunk,
                                            float (&yacc)[NT][4]) {
@@ -165,16 +166,18 @@ __device__ __forceinline__ void strip_sums(int ng, int q, int rr, uint32_t sc, u
             for (int t = 0; t < NT; ++t) {
                 const float2 c = lds_f2(cofs + (gi * 16 + 8 * t + 2 * q) * 4);
                 yacc[t][0] = fmaf(sa, (acc[u][0][t][0] + acc[u][1][t][0]) - c.x, yacc[t][0]);
-                yacc[t][1] = fmaf(sa, (acc[u][0][t][1] + acc[u][1][t][1]) - c.y, yacc[t][1]);
                 yacc[t][2] = fmaf(sb, (acc[u][0][t][2] + acc[u][1][t][2]) - c.x, yacc[t][2]);
-                yacc[t][3] = fmaf(sb, (acc[u][0][t][3] + acc[u][1][t][3]) - c.y, yacc[t][3]);
+                if (!kOne) {
+                    yacc[t][1] = fmaf(sa, (acc[u][0][t][1] + acc[u][1][t][1]) - c.y, yacc[t][1]);
+                    yacc[t][3] = fmaf(sb, (acc[u][0][t][3] + acc[u][1][t][3]) - c.y, yacc[t][3]);
+                }
             }
         }
     }
 }
 
 // ------------------------------------------------------------------ the kernel
-template <int NT>
+template <int NT, bool kOne>
 __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const __grid_constant__ CUtensorMap map1,
                                                         const __grid_constant__ CUtensorMap map2,
                                                         const GemvArgs a) {
@@ -383,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
 #pragma unroll
         for (int t = 0; t < NT; ++t) yacc[t][0] = yacc[t][1] = yacc[t][2] = yacc[t][3] = 0.f;
         const int strip_row = warp * kStrip;
-        strip_sums<NT>(ng, q, rr, smem_u32(sc1 + strip_row * kMaxGpc), smem_u32(cofs), xrow,
+        strip_sums<NT, kOne>(ng, q, rr, smem_u32(sc1 + strip_row * kMaxGpc), smem_u32(cofs), xrow,
                        [&](int c) { return smem_u32(wt1 + c * kMainChunkBytes + strip_row * 128); },
                        [&](int c) { ok = mbar_wait(&mbar1[c], 0) && ok; }, yacc);
         store_red(false, strip_row + rr, yacc);
@@ -407,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
 #pragma unroll
                 for (int t = 0; t < NT; ++t) yacc[t][0] = yacc[t][1] = yacc[t][2] = yacc[t][3] = 0.f;
                 const int rrow = (round * kResStrips + j) * kStrip;      // first residual row of the strip
-                strip_sums<NT>(ng, q, rr, smem_u32(sc2 + rrow * kMaxGpc), smem_u32(cofs), xrow,
+                strip_sums<NT, kOne>(ng, q, rr, smem_u32(sc2 + rrow * kMaxGpc), smem_u32(cofs), xrow,
                                [&](int c) { return smem_u32(wt2 + c * kResChunkBytes + j * kStripBytes); },
                                [&](int c) {
                                    if (j == 0) ok = mbar_wait(&mbar2[c], round & 1) && ok;
@@ -470,10 +473,10 @@ Plan plan_for(int64_t N, int64_t K) {
     return p;
 }
 
-template <int NT>
+template <int NT, bool kOne>
 tern_status launch(const CUtensorMap& m1, const CUtensorMap& m2, const GemvArgs& args, int64_t blocks, size_t smem,
                    cudaStream_t stream) {
-    auto kernel = gemv_kernel<NT>;
+    auto kernel = gemv_kernel<NT, kOne>;
     static std::mutex mu;
     static bool configured[64] = {false};
     int dev = 0;
@@ -534,7 +537,8 @@ tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y,
     a.split = p.split;
     a.static_weights = (w.flags & TERN_WEIGHT_STATIC) ? 1 : 0;
     const size_t smem = smem_bytes(M);
-    return M <= 8 ? launch<1>(m1, m2, a, blocks, smem, stream) : launch<2>(m1, m2, a, blocks, smem, stream);
+    if (M == 1) return launch<1, true>(m1, m2, a, blocks, smem, stream);
+    return M <= 8 ? launch<1, false>(m1, m2, a, blocks, smem, stream) : launch<2, false>(m1, m2, a, blocks, smem, stream);
 }
 
 }  // namespace tern
