@@ -355,12 +355,14 @@ def main():
         return xs, ys
 
     def step_fn(M, xs, ys, only=None):
+        # the calls of a step in order; each also starts bringing the next call's weight into L2
+        calls = [(layer, n) for layer in range(LAYERS) for n in names if only is None or n == only]
+
         def fn():
-            for layer in range(LAYERS):
-                W = pool[layer % POOL_LAYERS]
-                for n in names:
-                    if only is None or n == only:
-                        api.linear(xs[n], W[n], out=ys[layer][n], workspace=ws)
+            for i, (layer, n) in enumerate(calls):
+                nl, nn = calls[(i + 1) % len(calls)]
+                api.linear(xs[n], pool[layer % POOL_LAYERS][n], out=ys[layer][n], workspace=ws,
+                           prefetch=pool[nl % POOL_LAYERS][nn])
         return fn
 
     def step_bytes(M, only=None):

@@ -134,6 +134,16 @@ size_t tern_linear_workspace_bytes(const tern_weight* w, int64_t M);
 tern_status tern_linear(const tern_weight* w, const tern_half* x, int64_t M, tern_half* y,
                         void* workspace, size_t workspace_bytes, tern_stream stream);
 
+/* As tern_linear, and in the same launch starts bringing the planes, scales and slot map of
+ * `next` into the L2 cache: a decode loop passes the weight of its next call, whose loads then
+ * hit the cache while this call's arithmetic runs. A pure cache hint: `next` is read by no
+ * result and may be NULL (then this is tern_linear); its pointers must satisfy the rules of
+ * tern_weight, and a descriptor that fails them is reported as for `w`. The prefill path
+ * (M > 16) ignores it.                                                                  */
+tern_status tern_linear_with_prefetch(const tern_weight* w, const tern_half* x, int64_t M, tern_half* y,
+                                      void* workspace, size_t workspace_bytes, const tern_weight* next,
+                                      tern_stream stream);
+
 /* ---------------------------------------------------------------- bit accounting */
 
 typedef struct {

@@ -27,6 +27,8 @@ EXPORTS = {
     "tern_linear_workspace_bytes": (_c.c_size_t, [_c.c_void_p, _c.c_int64]),
     "tern_linear": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_void_p, _c.c_void_p, _c.c_size_t,
                                _c.c_void_p]),
+    "tern_linear_with_prefetch": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_void_p, _c.c_void_p,
+                                             _c.c_size_t, _c.c_void_p, _c.c_void_p]),
     "tern_bits": (_c.c_int, [_c.c_int64, _c.c_int64, _c.c_int64, _c.c_int32, _c.c_void_p]),
     "tern_device_status": (_c.c_int, [_c.c_void_p]),
     "tern_status_string": (_c.c_char_p, [_c.c_int]),

@@ -152,8 +152,11 @@ def workspace_bytes(w: TernWeight, M: int) -> int:
 
 
 def linear(x: torch.Tensor, w: TernWeight, out: torch.Tensor | None = None,
-           workspace: torch.Tensor | None = None) -> torch.Tensor:
-    """y [M, N] = x [M, K] . W^T (fp16 in, fp32 accumulation, fp16 out)."""
+           workspace: torch.Tensor | None = None, prefetch: TernWeight | None = None) -> torch.Tensor:
+    """y [M, N] = x [M, K] . W^T (fp16 in, fp32 accumulation, fp16 out).
+
+    prefetch: the weight of the next call, whose planes and scales the same launch starts
+    bringing into L2 (a cache hint; the result does not depend on it)."""
     _need(x, torch.float16, "x")
     M, K = x.shape
     if K != w.K:
@@ -168,8 +171,13 @@ def linear(x: torch.Tensor, w: TernWeight, out: torch.Tensor | None = None,
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _lib.check("tern_linear", _lib.load().tern_linear(
-        ctypes.byref(w.c_struct()), _ptr(x), M, _ptr(out), _ptr(workspace), ws_bytes, _stream(x.device)))
+    if prefetch is None:
+        _lib.check("tern_linear", _lib.load().tern_linear(
+            ctypes.byref(w.c_struct()), _ptr(x), M, _ptr(out), _ptr(workspace), ws_bytes, _stream(x.device)))
+    else:
+        _lib.check("tern_linear_with_prefetch", _lib.load().tern_linear_with_prefetch(
+            ctypes.byref(w.c_struct()), _ptr(x), M, _ptr(out), _ptr(workspace), ws_bytes,
+            ctypes.byref(prefetch.c_struct()), _stream(x.device)))
     return out
 
 

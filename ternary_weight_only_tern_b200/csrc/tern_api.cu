@@ -55,10 +55,16 @@ extern "C" size_t tern_linear_workspace_bytes(const tern_weight* w, int64_t M) {
     return (b + 255) & ~size_t(255);
 }
 
-extern "C" tern_status tern_linear(const tern_weight* w, const tern_half* x, int64_t M, tern_half* y,
-                                   void* workspace, size_t workspace_bytes, tern_stream stream) {
+namespace {
+
+tern_status linear(const tern_weight* w, const tern_half* x, int64_t M, tern_half* y, void* workspace,
+                   size_t workspace_bytes, const tern_weight* next, tern_stream stream) {
     const tern_status ws = check_weight(w);
     if (ws != TERN_OK) return ws;
+    if (next) {
+        const tern_status ns = check_weight(next);
+        if (ns != TERN_OK) return ns;
+    }
     if (M < 0 || M > (int64_t(1) << 31)) return TERN_ERR_SHAPE;
     if (M == 0) return TERN_OK;
     if (!x || !y) return TERN_ERR_NULL;
@@ -73,6 +79,19 @@ extern "C" tern_status tern_linear(const tern_weight* w, const tern_half* x, int
     cudaStream_t st = as_cuda(stream);
     const __half* xh = reinterpret_cast<const __half*>(x);
     __half* yh = reinterpret_cast<__half*>(y);
-    if (M <= kGemvMaxM) return gemv_launch(*w, xh, int(M), yh, st);
+    if (M <= kGemvMaxM) return gemv_launch(*w, xh, int(M), yh, next, st);
     return gemm_launch(*w, xh, M, yh, workspace, st);
+}
+
+}  // namespace
+
+extern "C" tern_status tern_linear(const tern_weight* w, const tern_half* x, int64_t M, tern_half* y,
+                                   void* workspace, size_t workspace_bytes, tern_stream stream) {
+    return linear(w, x, M, y, workspace, workspace_bytes, nullptr, stream);
+}
+
+extern "C" tern_status tern_linear_with_prefetch(const tern_weight* w, const tern_half* x, int64_t M, tern_half* y,
+                                                 void* workspace, size_t workspace_bytes, const tern_weight* next,
+                                                 tern_stream stream) {
+    return linear(w, x, M, y, workspace, workspace_bytes, next, stream);
 }

@@ -78,6 +78,10 @@ struct GemvArgs {
     int32_t gpc;               // groups per K-slice
     int32_t split;             // K-slices = cluster size
     int32_t static_weights;    // planes may be read before griddepcontrol.wait
+    // byte ranges of the next call's weight to bring into L2 (16-byte aligned, sizes rounded down
+    // to 16 bytes); every CTA prefetches its share of each
+    const uint8_t* pf_ptr[5];
+    int64_t pf_bytes[5];
 };
 
 struct Smem {
@@ -223,6 +227,15 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
     // The next call on the stream may start now: its weight loads overlap this call, and it reads
     // x (this call's output, possibly) only after griddepcontrol.wait.
     grid_launch_dependents();
+    if (threadIdx.x == kThreads - 1) {
+        // this CTA's share of the next call's weight, into L2
+        const int64_t nctas = int64_t(gridDim.x) * gridDim.y, b = int64_t(blockIdx.y) * gridDim.x + blockIdx.x;
+        for (int i = 0; i < 5; ++i) {
+            const int64_t per = ((a.pf_bytes[i] + nctas - 1) / nctas + 15) / 16 * 16;
+            const int64_t lo = b * per, hi = min(a.pf_bytes[i], lo + per);
+            if (a.pf_ptr[i] != nullptr && lo < hi) prefetch_l2_bulk(a.pf_ptr[i] + lo, uint32_t(hi - lo));
+        }
+    }
 
     int s_lo = 0, nres = 0;
     // Everything the weight determines, issued at once: TMA of the main tile (thread 0); the
@@ -512,7 +525,8 @@ tern_status launch(const CUtensorMap& m1, const CUtensorMap& m2, const GemvArgs&
 
 size_t gemv_workspace_bytes(const tern_weight&, int64_t) { return 0; }
 
-tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y, cudaStream_t stream) {
+tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y, const tern_weight* next,
+                        cudaStream_t stream) {
     const Plan p = plan_for(w.N, w.K);
     const int64_t blocks = (w.N + kRowsPerCta - 1) / kRowsPerCta;
     if (blocks > 65535) return TERN_ERR_SHAPE;
@@ -536,6 +550,17 @@ tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y,
     a.gpc = p.gpc;
     a.split = p.split;
     a.static_weights = (w.flags & TERN_WEIGHT_STATIC) ? 1 : 0;
+    if (next) {
+        const int64_t G = next->K / kGroup, rn = next->r;
+        const void* ptr[5] = {next->plane1, next->scale1, rn > 0 ? next->res_slot : nullptr,
+                              rn > 0 ? next->plane2 : nullptr, rn > 0 ? next->scale2 : nullptr};
+        const int64_t bytes[5] = {next->N * (next->K / 4), next->N * G * 2, next->N * 4, rn * (next->K / 4),
+                                  rn * G * 2};
+        for (int i = 0; i < 5; ++i) {
+            a.pf_ptr[i] = static_cast<const uint8_t*>(ptr[i]);
+            a.pf_bytes[i] = ptr[i] ? bytes[i] / 16 * 16 : 0;
+        }
+    }
     const size_t smem = smem_bytes(M);
     if (M == 1) return launch<1, true>(m1, m2, a, blocks, smem, stream);
     return M <= 8 ? launch<1, false>(m1, m2, a, blocks, smem, stream) : launch<2, false>(m1, m2, a, blocks, smem, stream);

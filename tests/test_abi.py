@@ -30,7 +30,8 @@ def lib():
 def test_header_declares_the_boundary():
     fns = header_functions()
     for name in ["tern_pack_exec", "tern_unpack_exec", "tern_pack_store", "tern_unpack_store",
-                 "tern_linear_workspace_bytes", "tern_linear", "tern_bits", "tern_status_string"]:
+                 "tern_linear_workspace_bytes", "tern_linear", "tern_linear_with_prefetch", "tern_bits",
+                 "tern_status_string"]:
         assert name in fns
     assert set(fns) == set(_lib.EXPORTS), "ctypes declarations and header disagree"
 
@@ -111,6 +112,14 @@ def test_linear_host_validation(lib):
         assert lib.tern_linear_workspace_bytes(ctypes.byref(wr), M) == 0
     assert call(wr, fake + 2, 3, fake * 4) == S["TERN_ERR_ALIGN"]
     assert call(wr, fake, 3, fake * 4, fake * 8 + 4, 64) == S["TERN_ERR_ALIGN"]   # misaligned workspace
+    # the prefetch descriptor is checked like the weight; a good one changes nothing up to the launch
+    pf = lambda nxt, M=1: lib.tern_linear_with_prefetch(  # noqa: E731
+        ctypes.byref(w), fake, M, fake * 4, None, 0, ctypes.byref(nxt) if nxt is not None else None, None)
+    assert pf(_lib.TernWeightC(64, 200, 128, fake, fake, 0, None, fake, None, None, 0)) == S["TERN_ERR_SHAPE"]
+    assert pf(_lib.TernWeightC(64, 256, 128, fake + 4, fake, 0, None, fake, None, None, 0)) == S["TERN_ERR_ALIGN"]
+    assert pf(_lib.TernWeightC(64, 256, 128, fake, fake, 4, fake, fake, None, fake, 0)) == S["TERN_ERR_NULL"]
+    assert pf(w, M=0) == S["TERN_OK"]
+    assert pf(None, M=0) == S["TERN_OK"]
 
 
 def test_pack_host_validation(lib):

@@ -219,3 +219,20 @@ def test_back_to_back_calls_on_one_stream_see_their_inputs():
 def test_device_status_is_clean_after_the_suite():
     from ternary_weight_only_tern_b200 import _lib
     assert _lib.load().tern_device_status(api._stream()) == 0
+
+
+@pytest.mark.parametrize("M", [1, 5, 16, 40])
+def test_prefetch_of_the_next_weight_changes_nothing(M):
+    """tern_linear_with_prefetch gives the same bits as tern_linear; the next weight (here of a
+    different shape, with residual rows) is only a cache hint."""
+    a = next(synth.draw_workload(synth.WORKLOADS[4], only=["q"]))
+    b = next(synth.draw_workload(synth.WORKLOADS[4], only=["down"]))
+    wa = api.TernWeight.from_numpy(a.T1, a.s1, a.res_rows, a.T2, a.s2)
+    wb = api.TernWeight.from_numpy(b.T1, b.s1, b.res_rows, b.T2, b.s2)
+    x = torch.from_numpy(np.ascontiguousarray(np.resize(a.x, (M, a.K)))).cuda()
+    y1 = api.linear(x, wa)
+    y2 = api.linear(x, wa, prefetch=wb)
+    y3 = api.linear(x, wa, prefetch=wa)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    assert torch.equal(y1.view(torch.int16), y3.view(torch.int16))
