@@ -88,7 +88,7 @@ struct Smem {
     static constexpr int wt1 = 0;                                          // [chunk][64 rows][128 B]
     static constexpr int wt2 = wt1 + kMaxChunks * kMainChunkBytes;        // [chunk][2 strips][16][128 B]
     static constexpr int bar = wt2 + kMaxChunks * kResChunkBytes;         // mbar1[chunks], mbar2[chunks]
-    static constexpr int misc = bar + 2 * kMaxChunks * 8;                  // s_lo, nres
+    static constexpr int misc = bar + (2 * kMaxChunks + 2) * 8;            // s_lo, nres (after rbar, pad)
     static constexpr int sc1 = misc + 16;                                  // half [64][kMaxGpc]
     static constexpr int sc2 = sc1 + kRowsPerCta * kMaxGpc * 2;            // half [64][kMaxGpc]
     static constexpr int bslot = sc2 + kMaxResRows * kMaxGpc * 2;          // int [64]: slot - s_lo, or -1
@@ -191,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
     uint8_t* wt2 = smem + Smem::wt2;
     uint64_t* mbar1 = reinterpret_cast<uint64_t*>(smem + Smem::bar);
     uint64_t* mbar2 = mbar1 + kMaxChunks;
+    uint64_t* rbar = mbar2 + kMaxChunks;                 // receive barrier of the partial sums
     int* misc = reinterpret_cast<int*>(smem + Smem::misc);
     __half* sc1 = reinterpret_cast<__half*>(smem + Smem::sc1);
     __half* sc2 = reinterpret_cast<__half*>(smem + Smem::sc2);
@@ -218,6 +219,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
             mbar_init(&mbar1[c], 1);
             mbar_init(&mbar2[c], 1);
         }
+        mbar_init(rbar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -363,14 +365,24 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
     __syncthreads();
     s_lo = misc[0];
     nres = misc[1];
-
-    // Partial sums go straight to the rank that owns the row: [this rank][row - owner's first][token]
-    // in the owner's receive buffer (buf = recv for main rows, recv_res for residual rows).
     const uint32_t me = cluster_rank();
     const int rows_per_rank = (kRowsPerCta + a.split - 1) / a.split;
+    const int lr0 = int(me) * rows_per_rank;
+    const int nrows = max(0, min(kRowsPerCta, lr0 + rows_per_rank) - lr0);
+    if (threadIdx.x == 0) {
+        // every rank sends this rank M sums per owned row, and M more per owned row with a residual
+        int owned_res = 0;
+        for (int lo = 0; lo < nrows; ++lo) owned_res += (bslot[lr0 + lo] >= 0 && bslot[lr0 + lo] < nres) ? 1 : 0;
+        mbar_arrive_expect_tx(rbar, uint32_t(a.split * (nrows + owned_res) * M * 4));
+    }
+
+    // Partial sums go straight to the rank that owns the row: [this rank][row - owner's first][token]
+    // in the owner's receive buffer (buf = recv for main rows, recv_res for residual rows), as
+    // asynchronous stores that complete on the owner's receive barrier.
     auto push = [&](float* buf, int lrow, int t, float v) {
         const int owner = lrow / rows_per_rank;
-        st_dsmem_f32(buf + (int(me) * rows_per_rank + (lrow - owner * rows_per_rank)) * M + t, uint32_t(owner), v);
+        st_async_f32(buf + (int(me) * rows_per_rank + (lrow - owner * rows_per_rank)) * M + t, uint32_t(owner), v,
+                     rbar);
     };
     // rows lrow_a and lrow_a + 8 of a strip (local rows of the block, or residual slots), this
     // lane's tokens
@@ -434,13 +446,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
         }
     }
 
-    // Epilogue: the partial sums of this rank's rows arrived from every rank; they are summed in
-    // rank order, the residual rows' sums added, and rounded once. After the barrier no CTA
-    // touches another's memory, so each may exit as soon as it is done.
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    // Epilogue: once the partial sums of this rank's rows have arrived from every rank (the
+    // receive barrier counts their bytes) they are summed in rank order, the residual rows' sums
+    // added, and rounded once. No CTA reads another's memory, so none waits for its peers to end.
+    if (ok) ok = mbar_wait(rbar, 0);
     {
-        const int lr0 = int(me) * rows_per_rank;
-        const int nrows = max(0, min(kRowsPerCta, lr0 + rows_per_rank) - lr0);
         for (int i = threadIdx.x; i < nrows * M; i += kThreads) {
             const int tok = i / nrows, lo = i - tok * nrows, lr = lr0 + lo;
             const int64_t n = n0 + lr;
