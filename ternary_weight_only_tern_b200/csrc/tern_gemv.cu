@@ -331,7 +331,36 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
 
     // C[g][token] = sum_k (B_p(k) + 1) * x[token][k]: MMA chains on the constant pattern in the
     // same K order and with the same split into two accumulators (one per word of the lane) as
-    // the main chains, combined by the same single addition, so a zero plane cancels bit for bit
+    // the main chains, combined by the same single addition, so a zero plane cancels bit for bit.
+    // With one token the 8 columns of the MMA take 8 groups (column g = group g's activations),
+    // so one warp computes every group's C in a single chain; each column is the same sequence
+    // of operations as the per-group chains below.
+    if (kOne) {
+        if (warp == 0) {
+            float c[2][4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) c[h][0] = c[h][1] = c[h][2] = c[h][3] = 0.f;
+            const uint32_t xg = rr < ng ? smem_u32(xs) + rr * kGroup * 2 : smem_u32(xzero);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t xp = xg + 16 * (4 * h + q) * 2;
+                const uint4 x01 = lds_u4(xp), x23 = lds_u4(xp + 16);
+                uint32_t Z[4];
+                zero_trit_pattern(0, Z[0], Z[2]); Z[1] = Z[0]; Z[3] = Z[2];
+                mma_16816(c[h], Z, x01.x, x01.y);
+                zero_trit_pattern(1, Z[0], Z[2]); Z[1] = Z[0]; Z[3] = Z[2];
+                mma_16816(c[h], Z, x01.z, x01.w);
+                zero_trit_pattern(2, Z[0], Z[2]); Z[1] = Z[0]; Z[3] = Z[2];
+                mma_16816(c[h], Z, x23.x, x23.y);
+                zero_trit_pattern(3, Z[0], Z[2]); Z[1] = Z[0]; Z[3] = Z[2];
+                mma_16816(c[h], Z, x23.z, x23.w);
+            }
+            if (rr == 0) {   // columns 2q and 2q+1: groups 2q and 2q+1, token 0
+                cofs[(2 * q) * 16] = c[0][0] + c[1][0];
+                cofs[(2 * q + 1) * 16] = c[0][1] + c[1][1];
+            }
+        }
+    } else
     for (int gi = warp; gi < ng; gi += kMainWarps + 1) {
         float c[2][NT][4];
 #pragma unroll
