@@ -17,9 +17,14 @@ integers) with numpy, with no blocking, fusion or reordering:
   - the Qwen3-8B scale-up paper (arXiv 2609.09240), its representation
     paragraph: one ternary plane for most weights, a second plane on a
     salience-selected subset, with per-group scales.
-  The row form of the subset (whole output rows carry the second plane) and
-  the absence of the per-group offset are the readings this library builds;
-  the CUDA path follows the same reading.
+  The row form of the subset (whole output rows carry the second plane) is the
+  reading this library builds; the CUDA path follows the same reading.
+* The per-group offset (an optional extension of the layer): E2M-ATQ represents
+  a group's values as {mu - a, mu, mu + a} around an asymmetric offset (4B
+  paper, section 4.3), and the packed format persists scales and offsets (4B
+  paper, section 9.1; 8B paper, its footnote on per-group offsets/scales). Read
+  here as one fp16 offset per (row, 128-wide group), added once to the
+  reconstructed weight: W = mu + s1 T1 (+ s2 T2 on the residual rows).
 * The product: with weights in {-1, 0, +1} the matrix product reduces to adding
   and subtracting activations ("Can Ternary LLMs Hit 1.58 Bits per Weight?",
   promptzone, section "What It Is and How It Works"); the oracle computes it
@@ -164,10 +169,11 @@ def row_bitmap(N: int, res_rows: np.ndarray) -> np.ndarray:
 # Dequantisation and the linear layer
 # --------------------------------------------------------------------------------------
 
-def dequant(T1, s1, res_rows, T2, s2, rows=None) -> np.ndarray:
+def dequant(T1, s1, res_rows, T2, s2, rows=None, mu=None) -> np.ndarray:
     """Dense float64 W [N, K] (or the listed rows of it).
 
-    W[n, k] = s1[n, k // 128] * T1[n, k]
+    W[n, k] = mu[n, k // 128]  (when an offset is given)
+              + s1[n, k // 128] * T1[n, k]
               + [n in R] * s2[rho(n), k // 128] * T2[rho(n), k],
     rho(n) = position of n in the sorted residual-row list R.
     fp16 -> float64 is exact, so W is exact in float64.
@@ -186,12 +192,14 @@ def dequant(T1, s1, res_rows, T2, s2, rows=None) -> np.ndarray:
         if has2.any():
             s2_cols = np.repeat(np.asarray(s2, dtype=np.float64)[rho[has2]], GROUP, axis=1)
             W[has2] += s2_cols * np.asarray(T2)[rho[has2]].astype(np.float64)
+    if mu is not None:
+        W += np.repeat(np.asarray(mu, dtype=np.float64)[rows], GROUP, axis=1)   # mu[n, k // 128]
     return W
 
 
-def linear(x, T1, s1, res_rows, T2, s2, cols=None) -> np.ndarray:
+def linear(x, T1, s1, res_rows, T2, s2, cols=None, mu=None) -> np.ndarray:
     """y_ref [M, N] (or [M, len(cols)]) = x . W^T in float64 (x fp16 -> float64 is exact)."""
-    W = dequant(T1, s1, res_rows, T2, s2, rows=cols)
+    W = dequant(T1, s1, res_rows, T2, s2, rows=cols, mu=mu)
     return np.asarray(x, dtype=np.float64) @ W.T
 
 
@@ -215,7 +223,7 @@ def rel_err(y, y_ref) -> float:
 # Bit accounting
 # --------------------------------------------------------------------------------------
 
-def bits(N: int, K: int, r: int, group: int = GROUP) -> dict:
+def bits(N: int, K: int, r: int, group: int = GROUP, offset: bool = False) -> dict:
     """Bits of one ternarized tensor in its three forms.
 
     info  : log2(3) per plane symbol, (N + r) * K symbols; per weight this is
@@ -223,6 +231,7 @@ def bits(N: int, K: int, r: int, group: int = GROUP) -> dict:
     store : base-3 planes (8 * ceil(K/5) bits per plane row) + fp16 scales per plane row and
             group + the residual-row bitmap (whole bytes) + a 64-byte header.
     exec  : 2-bit planes (2 bits per symbol) + fp16 scales + the int32 slot map [N] + header.
+    offset: the tensor carries a per-group offset: + 16 bits per (row, group) in both forms.
     """
     if K % group:
         raise ValueError("K must be a multiple of the group size")
@@ -232,6 +241,9 @@ def bits(N: int, K: int, r: int, group: int = GROUP) -> dict:
     plane_trits = plane_rows * K
     store_bits = 8 * plane_rows * store_row_bytes(K) + 16 * plane_rows * G + 8 * (-(-N // 8)) + HEADER_BITS
     exec_bits = 2 * plane_trits + 16 * plane_rows * G + 32 * N + HEADER_BITS
+    if offset:
+        store_bits += 16 * N * G
+        exec_bits += 16 * N * G
     return {
         "weights": weights,
         "plane_trits": plane_trits,

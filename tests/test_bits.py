@@ -88,3 +88,13 @@ def test_worked_values(shape, info, store, execb):
 def test_targeted_tensor_count():
     t = GOLD["targeted_linear_tensors"]
     assert t["layers"] * len(t["per_layer"]) == t["value"] == synth.N_LAYERS * len(synth.QWEN3_4B)
+
+
+def test_offset_bits_count_the_serialised_offsets():
+    """The offset adds exactly the bits of an fp16 [N, K/128] array to both forms."""
+    for (N, K, r) in [(13, 384, 5), (4096, 4096, 614), (1, 128, 0)]:
+        a, b = oracle.bits(N, K, r), oracle.bits(N, K, r, offset=True)
+        mu_bits = 8 * np.zeros((N, K // 128), np.float16).nbytes
+        assert b["store_bits"] - a["store_bits"] == mu_bits
+        assert b["exec_bits"] - a["exec_bits"] == mu_bits
+        assert b["bpw_info"] == a["bpw_info"]

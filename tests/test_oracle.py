@@ -123,8 +123,9 @@ def test_exec_roundtrip_and_invalid_trits():
 
 # ----------------------------------------------------------------------------- linear
 
-def brute_linear(x, T1, s1, res_rows, T2, s2):
-    """Exact rational y[m][n] = sum_k x[m,k] * (s1[n,k//128] T1[n,k] + [n in R] s2[rho(n),k//128] T2[rho(n),k])."""
+def brute_linear(x, T1, s1, res_rows, T2, s2, mu=None):
+    """Exact rational y[m][n] = sum_k x[m,k] * (mu[n,k//128] + s1[n,k//128] T1[n,k]
+    + [n in R] s2[rho(n),k//128] T2[rho(n),k]) (mu absent: 0)."""
     M, K = x.shape
     N = T1.shape[0]
     rho = {int(n): i for i, n in enumerate(res_rows)}
@@ -135,6 +136,8 @@ def brute_linear(x, T1, s1, res_rows, T2, s2):
             for k in range(K):
                 g = k // 128
                 w = Fraction(float(s1[n][g])) * int(T1[n][k])
+                if mu is not None:
+                    w += Fraction(float(mu[n][g]))
                 if n in rho:
                     w += Fraction(float(s2[rho[n]][g])) * int(T2[rho[n]][k])
                 acc += Fraction(float(x[m][k])) * w
@@ -311,3 +314,61 @@ def test_round_fp16_is_round_to_nearest_even():
 def test_rel_err():
     assert oracle.rel_err(np.array([1.0, 2.0]), np.array([1.0, 2.0])) == 0.0
     assert math.isclose(oracle.rel_err(np.array([1.0, 2.002]), np.array([1.0, 2.0])), 0.001)
+
+
+# ---------------------------------------------------------------------- per-group offset mu
+def offset_cases():
+    rng = np.random.default_rng(77)
+    out = []
+    for (N, K, M, r) in [(5, 128, 2, 2), (6, 256, 1, 0), (4, 256, 3, 4)]:
+        x = synth.draw_x(rng, M, K)
+        T1 = synth.draw_trits(rng, (N, K), 0.4)
+        s1 = synth.draw_scales(rng, N, K, 0.005, 0.02)
+        rr = np.sort(rng.choice(N, size=r, replace=False)).astype(np.int32)
+        T2 = synth.draw_trits(rng, (r, K), 0.4)
+        s2 = synth.draw_scales(rng, r, K, 0.001, 0.005)
+        mu = (rng.uniform(-0.01, 0.01, size=(N, K // 128))).astype(np.float16)
+        out.append((x, T1, s1, rr, T2, s2, mu))
+    return out
+
+
+@pytest.mark.parametrize("idx", range(3))
+def test_offset_matches_exact_rationals(idx):
+    x, T1, s1, rr, T2, s2, mu = offset_cases()[idx]
+    y = oracle.linear(x, T1, s1, rr, T2, s2, mu=mu)
+    yb = brute_linear(x, T1, s1, rr, T2, s2, mu=mu)
+    for m in range(y.shape[0]):
+        for n in range(y.shape[1]):
+            scale = sum(abs(float(v)) for v in x[m]) * 0.05 + 1e-30
+            assert abs(Fraction(float(y[m, n])) - yb[m][n]) <= Fraction(scale * 1e-14)
+
+
+def test_constant_offset_shifts_every_row_by_the_activation_sum():
+    """mu = c everywhere adds c * sum_k x[m, k] to every output of token m."""
+    x, T1, s1, rr, T2, s2, mu = offset_cases()[2]
+    c = np.float16(0.0078125)
+    y0 = oracle.linear(x, T1, s1, rr, T2, s2)
+    y1 = oracle.linear(x, T1, s1, rr, T2, s2, mu=np.full_like(mu, c))
+    shift = float(c) * x.astype(np.float64).sum(axis=1)
+    np.testing.assert_allclose(y1 - y0, np.repeat(shift[:, None], y0.shape[1], axis=1), rtol=1e-12, atol=1e-15)
+
+
+def test_offset_alone_is_the_scaled_group_sums():
+    """Zero planes: y[m, n] = sum_g mu[n, g] * (sum of x[m] over group g), group sums by Python loops."""
+    x, T1, s1, rr, T2, s2, mu = offset_cases()[0]
+    Z1, Z2 = np.zeros_like(T1), np.zeros_like(T2)
+    y = oracle.linear(x, Z1, s1, rr, Z2, s2, mu=mu)
+    M, K = x.shape
+    for m in range(M):
+        sums = [sum(float(x[m, k]) for k in range(g * 128, (g + 1) * 128)) for g in range(K // 128)]
+        for n in range(mu.shape[0]):
+            assert y[m, n] == pytest.approx(sum(float(mu[n, g]) * sums[g] for g in range(K // 128)), rel=1e-12)
+
+
+def test_planted_offset_mistake_is_caught():
+    """An oracle that adds the offset of the wrong group fails the rational check."""
+    x, T1, s1, rr, T2, s2, mu = offset_cases()[1]
+    bad = oracle.linear(x, T1, s1, rr, T2, s2, mu=np.roll(mu, 1, axis=1))
+    yb = brute_linear(x, T1, s1, rr, T2, s2, mu=mu)
+    assert any(abs(Fraction(float(bad[m, n])) - yb[m][n]) > Fraction(1e-9)
+               for m in range(bad.shape[0]) for n in range(bad.shape[1]))
