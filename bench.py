@@ -26,6 +26,7 @@ max over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -45,8 +46,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 KERNEL_TRAFFIC = {
     "gemv": {"sources": ["ternary_weight_only_tern_b200/csrc/tern_gemv.cu",
                          "ternary_weight_only_tern_b200/csrc/tern_device.cuh"],
-             "sha256": "e7fe425ff5aeb3b356db9f612e59f9ef40e49f9df58d1d2facfdf184715e80f2",
-             "bytes": 15482112},
+             "sha256": "0daddda56f48ec7aee53c14ca90fa7aed5e6fb7bb3b8bf9baea51a55d14a9c84",
+             "bytes": 15496192},
 }
 
 
@@ -354,19 +355,21 @@ def main():
         flat_out[M] = flat
         return xs, ys
 
-    def step_fn(M, xs, ys, only=None):
+    def step_fn(M, xs, ys, only=None, weights=None):
         # the calls of a step in order; each also starts bringing the next call's weight into L2
         calls = [(layer, n) for layer in range(LAYERS) for n in names if only is None or n == only]
+        wp = weights or pool
 
         def fn():
             for i, (layer, n) in enumerate(calls):
                 nl, nn = calls[(i + 1) % len(calls)]
-                api.linear(xs[n], pool[layer % POOL_LAYERS][n], out=ys[layer][n], workspace=ws,
-                           prefetch=pool[nl % POOL_LAYERS][nn])
+                api.linear(xs[n], wp[layer % POOL_LAYERS][n], out=ys[layer][n], workspace=ws,
+                           prefetch=wp[nl % POOL_LAYERS][nn])
         return fn
 
-    def step_bytes(M, only=None):
-        wb = sum(packed_bytes(pool[l % POOL_LAYERS][n]) for l in range(LAYERS) for n in names
+    def step_bytes(M, only=None, weights=None):
+        wp = weights or pool
+        wb = sum(packed_bytes(wp[l % POOL_LAYERS][n]) for l in range(LAYERS) for n in names
                  if only is None or n == only)
         ab = sum(2 * M * (K + N) for l in range(LAYERS) for (n, N, K) in shapes if only is None or n == only)
         return wb, ab
@@ -546,6 +549,36 @@ def extras(torch, api, synth, pool, shapes, names, stream, dev, ws, step_fn, ste
                    "frac_sustained": fl / t / 1e12 / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])}
         del g, x, y, wsg
     out["gemm_m2048"] = gemm
+    # the per-group offset mu (W = mu + s1 T1 + s2 T2): the same pool with an fp16 offset per
+    # (row, group) drawn U[-0.01, 0.01], the M = 1 stack and the gate GEMM at M = 2048
+    gm = torch.Generator(device=dev)
+    gm.manual_seed(17)
+    mpool = [{n: dataclasses.replace(L[n], mu=(torch.rand((L[n].N, L[n].K // 128), generator=gm, device=dev) * 0.02
+                                               - 0.01).half()) for n in names} for L in pool]
+    xs, ys = make_io(1)
+    g = capture(torch, step_fn(1, xs, ys, weights=mpool), stream)
+    t = time_graph(torch, g, 30, stream) / 30
+    wb, ab = step_bytes(1, weights=mpool)
+    off = {"stack_m1": {"us_per_step": t * 1e6, "packed_gbs": wb / t / 1e9, "frac": (wb + ab) / t / 1e9 / hbm,
+                        "packed_bytes_per_step": wb}}
+    del g, xs, ys
+    g = capture(torch, step_fn(1, xs1, ys1, only="gate", weights=mpool), stream)
+    t = time_graph(torch, g, 50, stream) / (50 * LAYERS)
+    wb, ab = step_bytes(1, only="gate", weights=mpool)
+    off["gate_m1"] = {"us": t * 1e6, "frac": (wb + ab) / LAYERS / t / 1e9 / hbm}
+    del g
+    x = torch.randn((2048, 4096), device=dev).half()
+    y = torch.empty((2048, 12288), dtype=torch.float16, device=dev)
+
+    def fn_mu():
+        for i in range(4):
+            api.linear(x, mpool[i]["gate"], out=y)
+    g = capture(torch, fn_mu, stream)
+    t = time_graph(torch, g, 5, stream) / 20
+    fl = 2.0 * 2048 * 12288 * 4096
+    off["gate_m2048"] = {"us": t * 1e6, "tflops": fl / t / 1e12, "frac_burst": fl / t / 1e12 / peaks["bf16_tflops"]}
+    out["offset_mu"] = off
+    del g, x, y, mpool
     # packing throughput on the gate shape
     u = torch.randint(0, 3, (12288, 4096), dtype=torch.int8, device=dev) - 1
     for fn_name, fn in (("pack_exec", api.pack_exec), ("pack_store", api.pack_store)):

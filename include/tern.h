@@ -12,7 +12,8 @@
  *   - R is a salience-selected subset that carries the second plane (4B paper, section 4.4;
  *     the Qwen3-8B scale-up paper, arXiv 2609.09240, representation paragraph). This
  *     library takes the subset as whole output rows; rho(n) is n's index in the sorted R.
- *     The pages' per-group offset is not part of this operation.
+ *   - Optionally a per-group offset mu (fp16 [N, K/128]) adds sum_g mu[n, g] * sum_{k in g}
+ *     x[m, k] to every row, residual or not (see tern_weight.mu).
  *   - x and y stay fp16 (weight-only quantisation, 4B paper section 3.1); the sums are
  *     accumulated in fp32 and rounded to fp16 once.
  *   - With weights in {-1, 0, +1} the product is additions and subtractions of activations
@@ -85,7 +86,14 @@ typedef struct {
     const uint32_t* plane2;      /* [r, K/16]   exec codes of T2                        */
     const tern_half* scale2;     /* [r, K/128]  s2                                      */
     uint32_t flags;              /* 0 or TERN_WEIGHT_STATIC                             */
+    const tern_half* mu;         /* [N, K/128]  per-group offset, or NULL (none)        */
 } tern_weight;
+
+/* With an offset the weight is W[n, k] = mu[n, k/128] + s1[n, k/128] T1[n, k]
+ * (+ s2[rho(n), k/128] T2[rho(n), k] on the residual rows): E2M-ATQ's values {mu - a, mu,
+ * mu + a} around an asymmetric per-group offset ("Post-Training Ternarization of Qwen3-4B",
+ * section 4.3; the packed format keeps scales and offsets, section 9.1). Without one
+ * (mu == NULL) W = s1 T1 (+ s2 T2).                                                     */
 
 /* tern_weight.flags: the planes, scales and slot map are not written by work queued before
  * the call on its stream (model weights). tern_linear may then start reading them while the
@@ -163,6 +171,11 @@ typedef struct {
  * a 64-byte header). 4B paper, sections 3.2, 4.4 and 7.1 (1.641 effective bits against the
  * ideal 1.585); 8B paper, effective-bits equation. Pure host function.                  */
 tern_status tern_bits(int64_t N, int64_t K, int64_t r, int32_t group, tern_bits_report* out);
+
+/* As tern_bits for a tensor that also carries a per-group offset: 16 more bits per
+ * (row, group) in the storage and the execution forms; the information figure counts plane
+ * symbols only and is unchanged.                                                        */
+tern_status tern_bits_offset(int64_t N, int64_t K, int64_t r, int32_t group, tern_bits_report* out);
 
 /* Reports, and clears, the current device's sticky status word for asynchronous work: returns
  * TERN_ERR_TIMEOUT if a tern_linear kernel since the last call gave up a bounded device-side

@@ -30,6 +30,7 @@ EXPORTS = {
     "tern_linear_with_prefetch": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_void_p, _c.c_void_p,
                                              _c.c_size_t, _c.c_void_p, _c.c_void_p]),
     "tern_bits": (_c.c_int, [_c.c_int64, _c.c_int64, _c.c_int64, _c.c_int32, _c.c_void_p]),
+    "tern_bits_offset": (_c.c_int, [_c.c_int64, _c.c_int64, _c.c_int64, _c.c_int32, _c.c_void_p]),
     "tern_device_status": (_c.c_int, [_c.c_void_p]),
     "tern_status_string": (_c.c_char_p, [_c.c_int]),
     "tern_version": (_c.c_int, []),
@@ -43,6 +44,7 @@ class TernWeightC(ctypes.Structure):
         ("plane1", ctypes.c_void_p), ("scale1", ctypes.c_void_p),
         ("r", ctypes.c_int64), ("res_rows", ctypes.c_void_p), ("res_slot", ctypes.c_void_p),
         ("plane2", ctypes.c_void_p), ("scale2", ctypes.c_void_p), ("flags", ctypes.c_uint32),
+        ("mu", ctypes.c_void_p),
     ]
 
 

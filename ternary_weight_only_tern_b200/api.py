@@ -87,6 +87,7 @@ class TernWeight:
     plane2: torch.Tensor     # int32 [r, K/16]
     scale2: torch.Tensor     # float16 [r, K/128]
     static: bool = False     # weights not written by queued work: tern_linear may prefetch them early
+    mu: torch.Tensor | None = None   # float16 [N, K/128] per-group offset: W = mu + s1 T1 (+ s2 T2)
 
     @property
     def r(self) -> int:
@@ -103,19 +104,23 @@ class TernWeight:
                 self.N, self.K, GROUP, self.plane1.data_ptr(), self.scale1.data_ptr(), self.r,
                 self.res_rows.data_ptr() if self.r else None, self.res_slot.data_ptr(),
                 self.plane2.data_ptr() if self.r else None, self.scale2.data_ptr() if self.r else None,
-                _lib.WEIGHT_STATIC if self.static else 0)
+                _lib.WEIGHT_STATIC if self.static else 0, self.mu.data_ptr() if self.mu is not None else None)
             object.__setattr__(self, "_c", c)
         return c
 
     def nbytes(self) -> int:
         """Bytes the decode kernels stream per call: both planes, their scales and the slot map."""
-        return sum(t.numel() * t.element_size() for t in (self.plane1, self.scale1, self.plane2, self.scale2,
-                                                           self.res_slot))
+        ts = (self.plane1, self.scale1, self.plane2, self.scale2, self.res_slot)
+        if self.mu is not None:
+            ts = ts + (self.mu,)
+        return sum(t.numel() * t.element_size() for t in ts)
 
     @classmethod
     def from_trits(cls, T1: torch.Tensor, s1: torch.Tensor, res_rows: torch.Tensor | None = None,
-                   T2: torch.Tensor | None = None, s2: torch.Tensor | None = None) -> "TernWeight":
-        """Packs int8 planes on the device (tern_pack_exec) and builds the residual-row slot map."""
+                   T2: torch.Tensor | None = None, s2: torch.Tensor | None = None,
+                   mu: torch.Tensor | None = None) -> "TernWeight":
+        """Packs int8 planes on the device (tern_pack_exec) and builds the residual-row slot map;
+        mu, if given, is the per-group offset [N, K/128]."""
         _need(T1, torch.int8, "T1")
         _need(s1, torch.float16, "s1")
         N, K = T1.shape
@@ -130,14 +135,20 @@ class TernWeight:
         if r:
             slot[res_rows.long()] = torch.arange(r, dtype=torch.int32, device=dev)
         plane2 = pack_exec(T2) if r else torch.zeros((0, K // 16), dtype=torch.int32, device=dev)
+        if mu is not None:
+            _need(mu, torch.float16, "mu")
+            if tuple(mu.shape) != (N, K // GROUP):
+                raise ValueError(f"mu must have shape {(N, K // GROUP)}")
+            mu = mu.to(dev).contiguous()
         return cls(N, K, pack_exec(T1), s1.contiguous(), res_rows, slot, plane2,
-                   s2.contiguous() if r else torch.zeros((0, K // GROUP), dtype=torch.float16, device=dev))
+                   s2.contiguous() if r else torch.zeros((0, K // GROUP), dtype=torch.float16, device=dev), mu=mu)
 
     @classmethod
-    def from_numpy(cls, T1, s1, res_rows, T2, s2, device="cuda") -> "TernWeight":
+    def from_numpy(cls, T1, s1, res_rows, T2, s2, device="cuda", mu=None) -> "TernWeight":
         t = lambda a, dt: torch.from_numpy(a).to(device=device, dtype=dt).contiguous()  # noqa: E731
         return cls.from_trits(t(T1, torch.int8), t(s1, torch.float16), t(res_rows, torch.int32),
-                              t(T2, torch.int8), t(s2, torch.float16))
+                              t(T2, torch.int8), t(s2, torch.float16),
+                              mu=t(mu, torch.float16) if mu is not None else None)
 
 
 def weight_validate(w: TernWeight) -> None:
@@ -183,7 +194,8 @@ def linear(x: torch.Tensor, w: TernWeight, out: torch.Tensor | None = None,
 
 # ------------------------------------------------------------------------------ bits
 
-def bits(N: int, K: int, r: int, group: int = GROUP) -> dict:
+def bits(N: int, K: int, r: int, group: int = GROUP, offset: bool = False) -> dict:
     rep = _lib.TernBitsReport()
-    _lib.check("tern_bits", _lib.load().tern_bits(N, K, r, group, ctypes.byref(rep)))
+    fn = "tern_bits_offset" if offset else "tern_bits"
+    _lib.check(fn, getattr(_lib.load(), fn)(N, K, r, group, ctypes.byref(rep)))
     return {f: getattr(rep, f) for f, _ in rep._fields_}

@@ -41,6 +41,7 @@ tern_status check_weight(const tern_weight* w) {
     if (!aligned16(w->plane1) || !aligned16(w->scale1)) return TERN_ERR_ALIGN;
     if (w->r > 0 && (!aligned16(w->plane2) || !aligned16(w->scale2) || !aligned16(w->res_slot)))
         return TERN_ERR_ALIGN;
+    if (w->mu && !aligned16(w->mu)) return TERN_ERR_ALIGN;
     return TERN_OK;
 }
 

@@ -33,6 +33,18 @@ extern "C" tern_status tern_bits(int64_t N, int64_t K, int64_t r, int32_t group,
     return TERN_OK;
 }
 
+extern "C" tern_status tern_bits_offset(int64_t N, int64_t K, int64_t r, int32_t group, tern_bits_report* out) {
+    const tern_status st = tern_bits(N, K, r, group, out);
+    if (st != TERN_OK) return st;
+    const uint64_t offset_bits = 16 * static_cast<uint64_t>(N) * static_cast<uint64_t>(K / group);
+    out->store_bits += offset_bits;
+    out->exec_bits += offset_bits;
+    const double w = static_cast<double>(out->weights);
+    out->bpw_store = static_cast<double>(out->store_bits) / w;
+    out->bpw_exec = static_cast<double>(out->exec_bits) / w;
+    return TERN_OK;
+}
+
 extern "C" const char* tern_status_string(tern_status s) {
     switch (s) {
         case TERN_OK: return "ok";

@@ -206,6 +206,8 @@ __device__ __forceinline__ void decode_word_pair(uint32_t wa, uint32_t wb, uint3
     A[3][2] = decode_pair<7>(wa, wal, war); A[3][3] = decode_pair<7>(wb, wbl, wbr);
 }
 
+constexpr uint32_t kHalf2One = 0x3C003C00u;   // the fp16 pair (1, 1)
+
 // B_p + 1 (the decoded value of trit 0) for the pairs of MMA i (pairs 2*(i%4) and 2*(i%4)+1),
 // as fp16x2 bits: 17 = 0x4C40, 5 = 0x4500, 65 = 0x5410.
 __device__ __forceinline__ void zero_trit_pattern(int i4, uint32_t& lo, uint32_t& hi) {

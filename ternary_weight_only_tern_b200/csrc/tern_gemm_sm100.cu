@@ -53,6 +53,7 @@ struct GemmArgs {
     const uint32_t* plane2;
     const __half* scale2;
     const int32_t* res_slot;
+    const __half* mu;          // [N, G] per-group offsets, or nullptr
     int64_t N, K, r, M;
     int32_t G;
     __half* y;
@@ -273,9 +274,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         const __half* srow = a.scale1 + (valid ? n : 0) * int64_t(a.G);
         // scales of this row two groups ahead; residual items (row i = item / 8, chunk item % 8)
         // of this thread: items t and t + 256 carry their scale two groups ahead too
-        __half sq[3];
+        // and the row's offsets, likewise (zero without an offset: the fma is then the product)
+        const __half* mrow = a.mu ? a.mu + (valid ? n : 0) * int64_t(a.G) : nullptr;
+        __half sq[3], mq[3];
 #pragma unroll
-        for (int j = 0; j < 3; ++j) sq[j] = (valid && j < a.G) ? srow[j] : __float2half(0.f);
+        for (int j = 0; j < 3; ++j) {
+            sq[j] = (valid && j < a.G) ? srow[j] : __float2half(0.f);
+            mq[j] = (mrow && valid && j < a.G) ? mrow[j] : __float2half(0.f);
+        }
         const int item0 = t, item1 = t + kDequantThreads;
         const bool has0 = item0 < n_res * 8, has1 = item1 < n_res * 8;
         const __half* s2row0 = has0 ? a.scale2 + int64_t(res_list[item0 >> 3].y) * a.G : a.scale2;
@@ -291,11 +297,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             const int g = kb / 2;
             if ((kb & 1) == 0 && kb > 0) {   // a new group: shift the scale queues, load two ahead
                 sq[0] = sq[1]; sq[1] = sq[2];
+                mq[0] = mq[1]; mq[1] = mq[2];
                 rq0[0] = rq0[1]; rq0[1] = rq0[2];
                 rq1[0] = rq1[1]; rq1[1] = rq1[2];
                 const int g2 = g + 2;
                 if (g2 < a.G) {
                     sq[2] = valid ? srow[g2] : __float2half(0.f);
+                    if (mrow) mq[2] = valid ? mrow[g2] : __float2half(0.f);
                     if (has0) rq0[2] = s2row0[g2];
                     if (has1) rq1[2] = s2row1[g2];
                 }
@@ -307,6 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             const uint32_t bs = smem_u32(smem_b + s * kBBytes);
             const uint4 cur = lds_u4(smem_u32(smem_p1 + sp * kPBytes + t * 16));
             const __half2 s2 = __half2half2(valid ? sq[0] : __float2half(0.f));
+            const __half2 m2 = __half2half2(valid ? mq[0] : __float2half(0.f));
             const uint32_t words[4] = {cur.x, cur.y, cur.z, cur.w};
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -314,10 +323,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 __half2 tt[4];
                 decode8(v, tt);
                 uint4 o;
-                o.x = h2_bits(__hmul2(tt[0], s2));
-                o.y = h2_bits(__hmul2(tt[1], s2));
-                o.z = h2_bits(__hmul2(tt[2], s2));
-                o.w = h2_bits(__hmul2(tt[3], s2));
+                o.x = h2_bits(__hfma2(tt[0], s2, m2));
+                o.y = h2_bits(__hfma2(tt[1], s2, m2));
+                o.z = h2_bits(__hfma2(tt[2], s2, m2));
+                o.w = h2_bits(__hfma2(tt[3], s2, m2));
                 sts_u4(bs + sw128_offset(t, c), o);
             }
             if (n_res > 0) {
@@ -452,6 +461,7 @@ tern_status gemm_launch(const tern_weight& w, const __half* x, int64_t M, __half
     a.plane2 = w.plane2;
     a.scale2 = reinterpret_cast<const __half*>(w.scale2);
     a.res_slot = w.r > 0 ? w.res_slot : nullptr;
+    a.mu = reinterpret_cast<const __half*>(w.mu);
     a.N = w.N;
     a.K = w.K;
     a.r = w.r;

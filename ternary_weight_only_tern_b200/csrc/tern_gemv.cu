@@ -70,6 +70,7 @@ struct GemvArgs {
     const __half* scale1;      // [N, G]
     const __half* scale2;      // [r, G]
     const int32_t* res_slot;   // [N] or nullptr
+    const __half* mu;          // [N, G] per-group offsets, or nullptr
     const __half* x;           // [M, K]
     __half* y;                 // [M, N]
     unsigned int* status;      // sticky timeout word
@@ -80,8 +81,8 @@ struct GemvArgs {
     int32_t static_weights;    // planes may be read before griddepcontrol.wait
     // byte ranges of the next call's weight to bring into L2 (16-byte aligned, sizes rounded down
     // to 16 bytes); every CTA prefetches its share of each
-    const uint8_t* pf_ptr[5];
-    int64_t pf_bytes[5];
+    const uint8_t* pf_ptr[6];
+    int64_t pf_bytes[6];
 };
 
 struct Smem {
@@ -95,7 +96,9 @@ struct Smem {
     static constexpr int srow = bslot + kRowsPerCta * 4;                   // int [64]: residual slot -> row
     static constexpr int cofs = srow + kMaxResRows * 4;                    // float [kMaxGpc][16]
     static constexpr int xzero = cofs + kMaxGpc * 16 * 4;                  // half [kMaxGpc * 128]: zeros
-    static constexpr int red = xzero + kMaxGpc * kGroup * 2;               // receive buffers, then xs
+    static constexpr int smu = xzero + kMaxGpc * kGroup * 2;               // half [64][kMaxGpc]: offsets
+    static constexpr int xsum = smu + kRowsPerCta * kMaxGpc * 2;           // float [kMaxGpc][16]: X_g
+    static constexpr int red = xsum + kMaxGpc * 16 * 4;                    // receive buffers, then xs
 };
 // Rows of the block owned by each rank, and the receive buffers: [rank][owned row][token] for the
 // main rows' partial sums and the same for their residual rows', pushed by every rank of the cluster.
@@ -198,6 +201,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
     int* bslot = reinterpret_cast<int*>(smem + Smem::bslot);
     float* cofs = reinterpret_cast<float*>(smem + Smem::cofs);
     __half* xzero = reinterpret_cast<__half*>(smem + Smem::xzero);
+    __half* smu = reinterpret_cast<__half*>(smem + Smem::smu);
+    float* xsum = reinterpret_cast<float*>(smem + Smem::xsum);
     const int M = a.M;
     int* srow = reinterpret_cast<int*>(smem + Smem::srow);
     float* recv = reinterpret_cast<float*>(smem + Smem::red);                        // [split][rows/split][M]
@@ -232,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
     if (threadIdx.x == kThreads - 1) {
         // this CTA's share of the next call's weight, into L2
         const int64_t nctas = int64_t(gridDim.x) * gridDim.y, b = int64_t(blockIdx.y) * gridDim.x + blockIdx.x;
-        for (int i = 0; i < 5; ++i) {
+        for (int i = 0; i < 6; ++i) {
             const int64_t per = ((a.pf_bytes[i] + nctas - 1) / nctas + 15) / 16 * 16;
             const int64_t lo = b * per, hi = min(a.pf_bytes[i], lo + per);
             if (a.pf_ptr[i] != nullptr && lo < hi) prefetch_l2_bulk(a.pf_ptr[i] + lo, uint32_t(hi - lo));
@@ -291,6 +296,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
                 for (int row = threadIdx.x >> 3; row < kRowsPerCta; row += kMainWarps * 4) {
                     const int64_t n = n0 + row;
                     sc1[row * kMaxGpc + g] = n < a.N ? a.scale1[n * a.G + g_begin + g] : __float2half(0.f);
+                    if (a.mu) smu[row * kMaxGpc + g] = n < a.N ? a.mu[n * a.G + g_begin + g] : __float2half(0.f);
                 }
         }
     };
@@ -359,6 +365,26 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
                 cofs[(2 * q) * 16] = c[0][0] + c[1][0];
                 cofs[(2 * q + 1) * 16] = c[0][1] + c[1][1];
             }
+        } else if (warp == 1 && a.mu) {
+            // X_g = sum of the group's activations: the same chain on an all-ones A
+            float c[2][4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) c[h][0] = c[h][1] = c[h][2] = c[h][3] = 0.f;
+            const uint32_t xg = rr < ng ? smem_u32(xs) + rr * kGroup * 2 : smem_u32(xzero);
+            const uint32_t one[4] = {kHalf2One, kHalf2One, kHalf2One, kHalf2One};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t xp = xg + 16 * (4 * h + q) * 2;
+                const uint4 x01 = lds_u4(xp), x23 = lds_u4(xp + 16);
+                mma_16816(c[h], one, x01.x, x01.y);
+                mma_16816(c[h], one, x01.z, x01.w);
+                mma_16816(c[h], one, x23.x, x23.y);
+                mma_16816(c[h], one, x23.z, x23.w);
+            }
+            if (rr == 0) {
+                xsum[(2 * q) * 16] = c[0][0] + c[1][0];
+                xsum[(2 * q + 1) * 16] = c[0][1] + c[1][1];
+            }
         }
     } else
     for (int gi = warp; gi < ng; gi += kMainWarps + 1) {
@@ -389,6 +415,32 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
             for (int t = 0; t < NT; ++t)
                 *reinterpret_cast<float2*>(cofs + gi * 16 + 8 * t + 2 * q) =
                     make_float2(c[0][t][0] + c[1][t][0], c[0][t][1] + c[1][t][1]);
+        }
+        if (a.mu) {
+            // X_g[token] = sum of the group's activations: the same chain on an all-ones A
+            const uint32_t one[4] = {kHalf2One, kHalf2One, kHalf2One, kHalf2One};
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int t = 0; t < NT; ++t) c[h][t][0] = c[h][t][1] = c[h][t][2] = c[h][t][3] = 0.f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    const uint32_t xp = xrow[t] + (gi * kGroup + 16 * (4 * h + q)) * 2;
+                    const uint4 x01 = lds_u4(xp), x23 = lds_u4(xp + 16);
+                    mma_16816(c[h][t], one, x01.x, x01.y);
+                    mma_16816(c[h][t], one, x01.z, x01.w);
+                    mma_16816(c[h][t], one, x23.x, x23.y);
+                    mma_16816(c[h][t], one, x23.z, x23.w);
+                }
+            }
+            if (rr == 0) {
+#pragma unroll
+                for (int t = 0; t < NT; ++t)
+                    *reinterpret_cast<float2*>(xsum + gi * 16 + 8 * t + 2 * q) =
+                        make_float2(c[0][t][0] + c[1][t][0], c[0][t][1] + c[1][t][1]);
+            }
         }
     }
     __syncthreads();
@@ -443,6 +495,24 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
         strip_sums<NT, kOne>(ng, q, rr, smem_u32(sc1 + strip_row * kMaxGpc), smem_u32(cofs), xrow,
                        [&](int c) { return smem_u32(wt1 + c * kMainChunkBytes + strip_row * 128); },
                        [&](int c) { ok = mbar_wait(&mbar1[c], 0) && ok; }, yacc);
+        if (a.mu) {
+            // the offset's share of the main rows: sum over the slice's groups of mu[row][g] * X_g
+            const __half* ma = smu + (strip_row + rr) * kMaxGpc;
+            const __half* mb = ma + 8 * kMaxGpc;
+            for (int gi = 0; gi < ng; ++gi) {
+                const float fa = __half2float(ma[gi]), fb = __half2float(mb[gi]);
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    const float2 xg = *reinterpret_cast<const float2*>(xsum + gi * 16 + 8 * t + 2 * q);
+                    yacc[t][0] = fmaf(fa, xg.x, yacc[t][0]);
+                    yacc[t][2] = fmaf(fb, xg.x, yacc[t][2]);
+                    if (!kOne) {
+                        yacc[t][1] = fmaf(fa, xg.y, yacc[t][1]);
+                        yacc[t][3] = fmaf(fb, xg.y, yacc[t][3]);
+                    }
+                }
+            }
+        }
         store_red(false, strip_row + rr, yacc);
     } else if (nres > 0) {
         const int rounds = (nres + kResStrips * kStrip - 1) / (kResStrips * kStrip);
@@ -578,6 +648,7 @@ tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y,
     a.scale1 = reinterpret_cast<const __half*>(w.scale1);
     a.scale2 = reinterpret_cast<const __half*>(w.scale2);
     a.res_slot = w.r > 0 ? w.res_slot : nullptr;
+    a.mu = reinterpret_cast<const __half*>(w.mu);
     a.x = x;
     a.y = y;
     a.status = async_status_word();
@@ -591,11 +662,11 @@ tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y,
     a.static_weights = (w.flags & TERN_WEIGHT_STATIC) ? 1 : 0;
     if (next) {
         const int64_t G = next->K / kGroup, rn = next->r;
-        const void* ptr[5] = {next->plane1, next->scale1, rn > 0 ? next->res_slot : nullptr,
-                              rn > 0 ? next->plane2 : nullptr, rn > 0 ? next->scale2 : nullptr};
-        const int64_t bytes[5] = {next->N * (next->K / 4), next->N * G * 2, next->N * 4, rn * (next->K / 4),
-                                  rn * G * 2};
-        for (int i = 0; i < 5; ++i) {
+        const void* ptr[6] = {next->plane1, next->scale1, rn > 0 ? next->res_slot : nullptr,
+                              rn > 0 ? next->plane2 : nullptr, rn > 0 ? next->scale2 : nullptr, next->mu};
+        const int64_t bytes[6] = {next->N * (next->K / 4), next->N * G * 2, next->N * 4, rn * (next->K / 4),
+                                  rn * G * 2, next->N * G * 2};
+        for (int i = 0; i < 6; ++i) {
             a.pf_ptr[i] = static_cast<const uint8_t*>(ptr[i]);
             a.pf_bytes[i] = ptr[i] ? bytes[i] / 16 * 16 : 0;
         }

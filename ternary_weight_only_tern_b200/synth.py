@@ -96,6 +96,19 @@ def draw_scales(rng: np.random.Generator, rows: int, K: int, lo: float, hi: floa
     return rng.uniform(lo, hi, size=(rows, K // GROUP)).astype(np.float16)
 
 
+def draw_offsets(rng: np.random.Generator, rows: int, K: int, bound: float = 0.01) -> np.ndarray:
+    """Per-group offsets, uniform in [-bound, bound] (fp16): of the order of the scales, as an
+    asymmetric group's centre would be."""
+    return rng.uniform(-bound, bound, size=(rows, K // GROUP)).astype(np.float16)
+
+
+def draw_exact_offsets(rng: np.random.Generator, rows: int, K: int) -> np.ndarray:
+    """Offsets for the exact inputs: 0 or +-2^-k, k in 4..6, so mu + s*t stays exact in fp16."""
+    mag = np.ldexp(1.0, -rng.integers(4, 7, size=(rows, K // GROUP)))
+    sign = rng.integers(-1, 2, size=(rows, K // GROUP))
+    return (mag * sign).astype(np.float16)
+
+
 def draw_tensor(rng: np.random.Generator, name: str, N: int, K: int, M: int, *, p_zero: float,
                 res_pct: int, s1_range=(0.005, 0.02), s2_range=(0.001, 0.005)) -> TernTensor:
     x = draw_x(rng, M, K)

@@ -60,6 +60,18 @@ def test_tern_bits_equals_oracle(lib, N, K, r):
         assert getattr(rep, f) == pytest.approx(ref[f], rel=1e-15, abs=0), f
 
 
+@pytest.mark.parametrize("N,K,r", [(4096, 2560, 0), (12288, 4096, 1843), (1, 128, 1)])
+def test_tern_bits_offset_equals_oracle(lib, N, K, r):
+    rep = _lib.TernBitsReport()
+    assert lib.tern_bits_offset(N, K, r, 128, ctypes.byref(rep)) == 0
+    ref = oracle.bits(N, K, r, offset=True)
+    for f in ("weights", "plane_trits", "store_bits", "exec_bits"):
+        assert getattr(rep, f) == ref[f], f
+    for f in ("bpw_info", "bpw_store", "bpw_exec"):
+        assert getattr(rep, f) == pytest.approx(ref[f], rel=1e-15, abs=0), f
+    assert lib.tern_bits_offset(16, 100, 0, 128, ctypes.byref(rep)) == _lib.STATUS["TERN_ERR_SHAPE"]
+
+
 def test_tern_bits_whole_stack(lib):
     # the 252 targeted tensors of the 4B model at 10% residual rows: sum of per-tensor integers
     rep = _lib.TernBitsReport()
@@ -106,6 +118,8 @@ def test_linear_host_validation(lib):
     assert call(bad, fake, 1, fake * 4) == S["TERN_ERR_NULL"]     # residual plane missing
     bad = _lib.TernWeightC(64, 256, 128, fake + 4, fake, 0, None, fake, None, None, 0)
     assert call(bad, fake, 1, fake * 4) == S["TERN_ERR_ALIGN"]
+    bad = _lib.TernWeightC(64, 256, 128, fake, fake, 0, None, fake, None, None, 0, fake + 2)
+    assert call(bad, fake, 1, fake * 4) == S["TERN_ERR_ALIGN"]    # misaligned offset
     # neither path needs scratch memory
     wr = _lib.TernWeightC(64, 256, 128, fake, fake, 4, fake, fake, fake, fake, 1)
     for M in (1, 16, 17, 4096):

@@ -236,3 +236,50 @@ def test_prefetch_of_the_next_weight_changes_nothing(M):
     torch.cuda.synchronize()
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
     assert torch.equal(y1.view(torch.int16), y3.view(torch.int16))
+
+
+# ---------------------------------------------------------------- per-group offset mu
+def run_mu(t: synth.TernTensor, mu: np.ndarray, M: int, weight=None):
+    w = weight or api.TernWeight.from_numpy(t.T1, t.s1, t.res_rows, t.T2, t.s2, mu=mu)
+    return run(t, M, w)
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 9, 16, 17, 300])
+@pytest.mark.parametrize("N,K,pct", [(320, 1152, 10), (1000 + 7, 12288, 15), (64, 128, 100)])
+def test_offset_parity(M, N, K, pct):
+    rng = np.random.default_rng(7 * M + N + K)
+    t = synth.draw_tensor(rng, "mu", N, K, M, p_zero=0.4, res_pct=pct)
+    mu = synth.draw_offsets(rng, N, K)
+    y, _ = run_mu(t, mu, M)
+    check(y, oracle.linear(t.x, t.T1, t.s1, t.res_rows, t.T2, t.s2, mu=mu))
+
+
+@pytest.mark.parametrize("M", [1, 4, 16, 24, 300])
+@pytest.mark.parametrize("N,K,r", [(256, 512, 40), (130, 12288, 13)])
+def test_offset_exact_case_bit_exact(M, N, K, r):
+    rng = np.random.default_rng(M * 17 + N + K)
+    t = synth.draw_exact_tensor(rng, N, K, M, r)
+    mu = synth.draw_exact_offsets(rng, N, K)
+    y, _ = run_mu(t, mu, M)
+    y_ref = oracle.round_fp16(oracle.linear(t.x, t.T1, t.s1, t.res_rows, t.T2, t.s2, mu=mu))
+    assert np.array_equal(y.view(np.uint16), y_ref.view(np.uint16))
+
+
+@pytest.mark.parametrize("M", [1, 5, 16, 40])
+def test_zero_offset_gives_the_bits_of_no_offset(M):
+    rng = np.random.default_rng(300 + M)
+    t = synth.draw_tensor(rng, "mu0", 512, 2560, M, p_zero=0.4, res_pct=10)
+    y0, _ = run(t, M)
+    y1, _ = run_mu(t, np.zeros((t.N, t.K // 128), np.float16), M)
+    assert np.array_equal(y0.view(np.uint16), y1.view(np.uint16))
+
+
+@pytest.mark.parametrize("M", [1, 16, 2048])
+def test_offset_8b_gate_full_size(M):
+    t = next(synth.draw_workload(synth.WORKLOADS[5], only=["gate"]))
+    rng = np.random.default_rng(11)
+    mu = synth.draw_offsets(rng, t.N, t.K)
+    cols = np.unique(np.concatenate([rng.choice(t.N, 40, replace=False), t.res_rows[:24]]))
+    y_ref = oracle.linear(t.x[:M], t.T1, t.s1, t.res_rows, t.T2, t.s2, cols=cols, mu=mu)
+    y, _ = run_mu(t, mu, M)
+    check(y[:, cols], y_ref)
