@@ -25,6 +25,14 @@ integers) with numpy, with no blocking, fusion or reordering:
   paper, section 9.1; 8B paper, its footnote on per-group offsets/scales). Read
   here as one fp16 offset per (row, 128-wide group), added once to the
   reconstructed weight: W = mu + s1 T1 (+ s2 T2 on the residual rows).
+* The element-level second plane (an optional extension of the layer): the
+  8B paper's representation paragraph and the 4B paper's section 4.4 give the
+  second plane to the weights of the two most salient of four disjoint
+  element masks (3.6 % of a recorded projection's weights). Read here as a
+  second ternary plane T2e over all of W that is zero outside the masks, with
+  its own fp16 scale per (row, group): W += s2e[n, k // 128] * T2e[n, k]. It
+  is kept as a list of its nonzero trits per (row, group), defined below by
+  its closed form (the layout is this library's own).
 * The product: with weights in {-1, 0, +1} the matrix product reduces to adding
   and subtracting activations ("Can Ternary LLMs Hit 1.58 Bits per Weight?",
   promptzone, section "What It Is and How It Works"); the oracle computes it
@@ -166,15 +174,90 @@ def row_bitmap(N: int, res_rows: np.ndarray) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------------------
+# Element-level second plane: the nonzero trits of T2e, one byte each,
+#   byte = (k % 128) << 1 | (t < 0),
+# ordered by group g, then row n, then k. ecount[g, n] = number of them in (row n, group g);
+# ebase[g * NB + b] = index of the first byte of (group g, rows 64 b .. 64 b + 63), with
+# NB = ceil(N / 64) and ebase[G * NB] = nnz2.
+# --------------------------------------------------------------------------------------
+ELEM_BLOCK = 64
+
+
+def elem_blocks(N: int) -> int:
+    return -(-N // ELEM_BLOCK)
+
+
+def pack_elem(trits: np.ndarray) -> tuple[np.ndarray, np.ndarray, np.ndarray, int]:
+    """int8 T2e [N, K] -> (ecount uint8 [G, N], ebase int64 [G*NB + 1], eidx uint8 [nnz2], n_invalid).
+
+    An entry outside {-1, 0, +1} is counted invalid and packed as 0 (not listed)."""
+    t = np.asarray(trits, dtype=np.int8)
+    N, K = t.shape
+    if K % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    G, NB = K // GROUP, elem_blocks(N)
+    invalid = (t < -1) | (t > 1)
+    t = np.where(invalid, 0, t)
+    ecount = np.zeros((G, N), dtype=np.uint8)
+    ebase = np.zeros(G * NB + 1, dtype=np.int64)
+    out = []
+    for g in range(G):
+        for b in range(NB):
+            ebase[g * NB + b] = len(out)
+            for n in range(b * ELEM_BLOCK, min(N, (b + 1) * ELEM_BLOCK)):
+                seg = t[n, g * GROUP:(g + 1) * GROUP]
+                ks = np.flatnonzero(seg)                       # ascending k within the group
+                ecount[g, n] = len(ks)
+                out.extend(int(kk) << 1 | int(seg[kk] < 0) for kk in ks)
+    ebase[G * NB] = len(out)
+    return ecount, ebase, np.array(out, dtype=np.uint8), int(invalid.sum())
+
+
+def unpack_elem(ecount, ebase, eidx, N: int, K: int) -> tuple[np.ndarray, int]:
+    """(ecount, ebase, eidx) -> int8 T2e [N, K] and the number of inconsistencies found.
+
+    Inconsistent: a count above 128; a block whose counts do not add up to the gap between its
+    base and the next; ebase[0] != 0 or ebase[-1] != len(eidx); within (row, group) a k that does
+    not increase. The entries that can be placed are placed regardless."""
+    ecount = np.asarray(ecount, dtype=np.int64)
+    ebase = np.asarray(ebase, dtype=np.int64)
+    eidx = np.asarray(eidx, dtype=np.uint8)
+    G, NB = K // GROUP, elem_blocks(N)
+    T = np.zeros((N, K), dtype=np.int8)
+    bad = int(ebase[0] != 0) + int(ebase[G * NB] != len(eidx))
+    for g in range(G):
+        for b in range(NB):
+            i = int(ebase[g * NB + b])
+            rows = range(b * ELEM_BLOCK, min(N, (b + 1) * ELEM_BLOCK))
+            if sum(int(ecount[g, n]) for n in rows) != int(ebase[g * NB + b + 1]) - i:
+                bad += 1
+            for n in rows:
+                c = int(ecount[g, n])
+                if c > GROUP:
+                    bad += 1
+                last = -1
+                for e in range(i, i + c):
+                    if 0 <= e < len(eidx):
+                        kk, neg = int(eidx[e]) >> 1, int(eidx[e]) & 1
+                        if kk <= last:
+                            bad += 1
+                        last = kk
+                        T[n, g * GROUP + kk] = -1 if neg else 1
+                i += c
+    return T, bad
+
+
+# --------------------------------------------------------------------------------------
 # Dequantisation and the linear layer
 # --------------------------------------------------------------------------------------
 
-def dequant(T1, s1, res_rows, T2, s2, rows=None, mu=None) -> np.ndarray:
+def dequant(T1, s1, res_rows, T2, s2, rows=None, mu=None, elem=None) -> np.ndarray:
     """Dense float64 W [N, K] (or the listed rows of it).
 
     W[n, k] = mu[n, k // 128]  (when an offset is given)
               + s1[n, k // 128] * T1[n, k]
-              + [n in R] * s2[rho(n), k // 128] * T2[rho(n), k],
+              + [n in R] * s2[rho(n), k // 128] * T2[rho(n), k]
+              + s2e[n, k // 128] * T2e[n, k]  (when an element plane elem = (T2e, s2e) is given),
     rho(n) = position of n in the sorted residual-row list R.
     fp16 -> float64 is exact, so W is exact in float64.
     """
@@ -194,12 +277,16 @@ def dequant(T1, s1, res_rows, T2, s2, rows=None, mu=None) -> np.ndarray:
             W[has2] += s2_cols * np.asarray(T2)[rho[has2]].astype(np.float64)
     if mu is not None:
         W += np.repeat(np.asarray(mu, dtype=np.float64)[rows], GROUP, axis=1)   # mu[n, k // 128]
+    if elem is not None:
+        T2e, s2e = elem
+        W += np.repeat(np.asarray(s2e, dtype=np.float64)[rows], GROUP, axis=1) * \
+            np.asarray(T2e)[rows].astype(np.float64)
     return W
 
 
-def linear(x, T1, s1, res_rows, T2, s2, cols=None, mu=None) -> np.ndarray:
+def linear(x, T1, s1, res_rows, T2, s2, cols=None, mu=None, elem=None) -> np.ndarray:
     """y_ref [M, N] (or [M, len(cols)]) = x . W^T in float64 (x fp16 -> float64 is exact)."""
-    W = dequant(T1, s1, res_rows, T2, s2, rows=cols, mu=mu)
+    W = dequant(T1, s1, res_rows, T2, s2, rows=cols, mu=mu, elem=elem)
     return np.asarray(x, dtype=np.float64) @ W.T
 
 
@@ -241,6 +328,37 @@ def bits(N: int, K: int, r: int, group: int = GROUP, offset: bool = False) -> di
     plane_trits = plane_rows * K
     store_bits = 8 * plane_rows * store_row_bytes(K) + 16 * plane_rows * G + 8 * (-(-N // 8)) + HEADER_BITS
     exec_bits = 2 * plane_trits + 16 * plane_rows * G + 32 * N + HEADER_BITS
+    if offset:
+        store_bits += 16 * N * G
+        exec_bits += 16 * N * G
+    return {
+        "weights": weights,
+        "plane_trits": plane_trits,
+        "store_bits": store_bits,
+        "exec_bits": exec_bits,
+        "bpw_info": math.log2(3) * plane_trits / weights,
+        "bpw_store": store_bits / weights,
+        "bpw_exec": exec_bits / weights,
+    }
+
+
+def bits_elem(N: int, K: int, masked: int, nnz2: int, group: int = GROUP, offset: bool = False) -> dict:
+    """Bits of a tensor whose second plane is element-level: `masked` weights carry a second
+    symbol (f2 = masked / (N K)), `nnz2` of those symbols are nonzero and listed.
+
+    info  : log2(3) per plane symbol, N K + masked symbols (the pages' accounting, log2(3) (1 + f2)).
+    store : base-3 main plane + fp16 s1 + the element plane (8 bits per ecount entry [G, N],
+            32 per ebase entry [G NB + 1], 8 per listed trit, 16 per s2e entry [N, G]) + header.
+    exec  : the same with the 2-bit main plane.
+    offset: + 16 bits per (row, group) in both forms."""
+    if K % group:
+        raise ValueError("K must be a multiple of the group size")
+    G = K // group
+    weights = N * K
+    plane_trits = weights + masked
+    elem_bits = 8 * G * N + 32 * (G * elem_blocks(N) + 1) + 8 * nnz2 + 16 * N * G
+    store_bits = 8 * N * store_row_bytes(K) + 16 * N * G + elem_bits + HEADER_BITS
+    exec_bits = 2 * weights + 16 * N * G + elem_bits + HEADER_BITS
     if offset:
         store_bits += 16 * N * G
         exec_bits += 16 * N * G

@@ -109,6 +109,17 @@ def draw_exact_offsets(rng: np.random.Generator, rows: int, K: int) -> np.ndarra
     return (mag * sign).astype(np.float16)
 
 
+def draw_elem_plane(rng: np.random.Generator, N: int, K: int, masked_frac: float = 0.036, p_zero: float = 0.4,
+                    s_range=(0.001, 0.005)):
+    """An element-level second plane: each weight is masked with probability masked_frac (the
+    pages' two most salient masks cover 3.6 % of a recorded projection), a masked weight draws a
+    trit like the main plane, an unmasked one is 0; one fp16 scale per (row, group).
+    Returns (T2e int8 [N, K], s2e fp16 [N, K/128], number of masked weights)."""
+    mask = rng.random((N, K), dtype=np.float32) < masked_frac
+    T2e = np.where(mask, draw_trits(rng, (N, K), p_zero), 0).astype(np.int8)
+    return T2e, draw_scales(rng, N, K, *s_range), int(mask.sum())
+
+
 def draw_tensor(rng: np.random.Generator, name: str, N: int, K: int, M: int, *, p_zero: float,
                 res_pct: int, s1_range=(0.005, 0.02), s2_range=(0.001, 0.005)) -> TernTensor:
     x = draw_x(rng, M, K)

@@ -123,9 +123,9 @@ def test_exec_roundtrip_and_invalid_trits():
 
 # ----------------------------------------------------------------------------- linear
 
-def brute_linear(x, T1, s1, res_rows, T2, s2, mu=None):
+def brute_linear(x, T1, s1, res_rows, T2, s2, mu=None, elem=None):
     """Exact rational y[m][n] = sum_k x[m,k] * (mu[n,k//128] + s1[n,k//128] T1[n,k]
-    + [n in R] s2[rho(n),k//128] T2[rho(n),k]) (mu absent: 0)."""
+    + [n in R] s2[rho(n),k//128] T2[rho(n),k] + s2e[n,k//128] T2e[n,k]) (mu, elem absent: 0)."""
     M, K = x.shape
     N = T1.shape[0]
     rho = {int(n): i for i, n in enumerate(res_rows)}
@@ -140,6 +140,8 @@ def brute_linear(x, T1, s1, res_rows, T2, s2, mu=None):
                     w += Fraction(float(mu[n][g]))
                 if n in rho:
                     w += Fraction(float(s2[rho[n]][g])) * int(T2[rho[n]][k])
+                if elem is not None:
+                    w += Fraction(float(elem[1][n][g])) * int(elem[0][n][k])
                 acc += Fraction(float(x[m][k])) * w
             y[m][n] = acc
     return y
@@ -370,5 +372,142 @@ def test_planted_offset_mistake_is_caught():
     x, T1, s1, rr, T2, s2, mu = offset_cases()[1]
     bad = oracle.linear(x, T1, s1, rr, T2, s2, mu=np.roll(mu, 1, axis=1))
     yb = brute_linear(x, T1, s1, rr, T2, s2, mu=mu)
+    assert any(abs(Fraction(float(bad[m, n])) - yb[m][n]) > Fraction(1e-9)
+               for m in range(bad.shape[0]) for n in range(bad.shape[1]))
+
+
+
+# ---------------------------------------------------------------- element-level second plane
+def hand_elem():
+    """N = 2, K = 256. Nonzero T2e: row 0: k=3 -> +1, k=130 -> -1; row 1: k=0 -> -1,
+    k=127 -> +1, k=255 -> +1. Worked by hand: group 0 lists row 0 (3 << 1 = 6), then row 1
+    (0 << 1 | 1 = 1, 127 << 1 = 254); group 1 lists row 0 (2 << 1 | 1 = 5), then row 1
+    (127 << 1 = 254). ecount[g][n] = [[1, 2], [1, 1]]; one 64-row block per group, so
+    ebase = [0, 3, 5]."""
+    T = np.zeros((2, 256), np.int8)
+    T[0, 3], T[0, 130], T[1, 0], T[1, 127], T[1, 255] = 1, -1, -1, 1, 1
+    return T, np.array([[1, 2], [1, 1]], np.uint8), np.array([0, 3, 5]), np.array([6, 1, 254, 5, 254], np.uint8)
+
+
+def test_pack_elem_hand_worked_example():
+    T, cnt, base, idx = hand_elem()
+    c, b, e, bad = oracle.pack_elem(T)
+    assert bad == 0
+    assert np.array_equal(c, cnt) and np.array_equal(b, base) and np.array_equal(e, idx)
+    T2, bad2 = oracle.unpack_elem(cnt, base, idx, 2, 256)
+    assert bad2 == 0 and np.array_equal(T2, T)
+
+
+def _elem_mut_sign(T):
+    c, b, e, _ = oracle.pack_elem(T)
+    return c, b, e ^ np.uint8(1)
+
+
+def _elem_mut_no_shift(T):
+    c, b, e, _ = oracle.pack_elem(T)
+    return c, b, (e >> 1).astype(np.uint8)
+
+
+def _elem_mut_row_major(T):
+    # rows first, then groups: the order of the entries is wrong
+    N, K = T.shape
+    out = [int(kk) << 1 | int(T[n, g * 128 + kk] < 0) for n in range(N) for g in range(K // 128)
+           for kk in np.flatnonzero(T[n, g * 128:(g + 1) * 128])]
+    c, b, _, _ = oracle.pack_elem(T)
+    return c, b, np.array(out, np.uint8)
+
+
+@pytest.mark.parametrize("mutant", [_elem_mut_sign, _elem_mut_no_shift, _elem_mut_row_major])
+def test_planted_elem_packing_mistakes_are_caught(mutant):
+    T, cnt, base, idx = hand_elem()
+    c, b, e = mutant(T)
+    assert not (np.array_equal(c, cnt) and np.array_equal(b, base) and np.array_equal(e, idx))
+
+
+@pytest.mark.parametrize("N,K,density", [(1, 128, 0.05), (63, 256, 0.03), (64, 128, 0.0), (65, 384, 0.03),
+                                         (130, 128, 1.0), (200, 256, 0.2)])
+def test_elem_roundtrip_and_counts(N, K, density):
+    rng = np.random.default_rng(N * K)
+    T = np.where(rng.random((N, K)) < density, rng.choice(np.array([-1, 1], np.int8), (N, K)), 0).astype(np.int8)
+    c, b, e, bad = oracle.pack_elem(T)
+    assert bad == 0 and len(e) == np.count_nonzero(T) and int(b[-1]) == len(e)
+    G, NB = K // 128, oracle.elem_blocks(N)
+    for g in range(G):                      # counts are the nonzeros of each (row, group), by numpy
+        assert np.array_equal(c[g], np.count_nonzero(T[:, g * 128:(g + 1) * 128], axis=1))
+    assert np.all(np.diff(b) >= 0) and b.shape == (G * NB + 1,)
+    T2, bad2 = oracle.unpack_elem(c, b, e, N, K)
+    assert bad2 == 0 and np.array_equal(T2, T)
+
+
+def test_pack_elem_counts_invalid_trits():
+    T = np.zeros((3, 128), np.int8)
+    T[0, 5], T[1, 9], T[2, 0] = 2, -7, 1
+    c, b, e, bad = oracle.pack_elem(T)
+    assert bad == 2 and list(e) == [0] and list(c[0]) == [0, 0, 1]
+
+
+def test_unpack_elem_flags_inconsistent_metadata():
+    T, cnt, base, idx = hand_elem()
+    assert oracle.unpack_elem(cnt, base, idx[[0, 2, 1, 3, 4]], 2, 256)[1] > 0     # k not increasing
+    c2 = cnt.copy(); c2[0, 1] = 1
+    assert oracle.unpack_elem(c2, base, idx, 2, 256)[1] > 0                      # block sum != base gap
+    assert oracle.unpack_elem(cnt, np.array([1, 3, 5]), idx, 2, 256)[1] > 0      # ebase[0] != 0
+    assert oracle.unpack_elem(cnt, base, idx[:4], 2, 256)[1] > 0                 # last base != nnz2
+    c3 = cnt.copy(); c3[0, 0] = 200
+    assert oracle.unpack_elem(c3, base, idx, 2, 256)[1] > 0                      # count above 128
+
+
+def elem_cases():
+    rng = np.random.default_rng(91)
+    out = []
+    for (N, K, M, r) in [(5, 128, 2, 0), (4, 256, 2, 2), (3, 256, 1, 0)]:
+        x = synth.draw_x(rng, M, K)
+        T1 = synth.draw_trits(rng, (N, K), 0.4)
+        s1 = synth.draw_scales(rng, N, K, 0.005, 0.02)
+        rr = np.sort(rng.choice(N, size=r, replace=False)).astype(np.int32)
+        T2 = synth.draw_trits(rng, (r, K), 0.4)
+        s2 = synth.draw_scales(rng, r, K, 0.001, 0.005)
+        T2e = np.where(rng.random((N, K)) < 0.1, synth.draw_trits(rng, (N, K), 0.4), 0).astype(np.int8)
+        s2e = synth.draw_scales(rng, N, K, 0.001, 0.005)
+        out.append((x, T1, s1, rr, T2, s2, (T2e, s2e)))
+    return out
+
+
+@pytest.mark.parametrize("idx", range(3))
+def test_elem_plane_matches_exact_rationals(idx):
+    x, T1, s1, rr, T2, s2, elem = elem_cases()[idx]
+    y = oracle.linear(x, T1, s1, rr, T2, s2, elem=elem)
+    yb = brute_linear(x, T1, s1, rr, T2, s2, elem=elem)
+    for m in range(y.shape[0]):
+        for n in range(y.shape[1]):
+            scale = sum(abs(float(v)) for v in x[m]) * 0.05 + 1e-30
+            assert abs(Fraction(float(y[m, n])) - yb[m][n]) <= Fraction(scale * 1e-14)
+
+
+def test_elem_plane_on_whole_rows_is_the_row_residual():
+    """An element plane that covers whole rows R with T2e[R] = T2 and s2e[R] = s2 is the
+    row-form residual: the two dequantised W are equal element for element."""
+    rng = np.random.default_rng(5)
+    N, K, r = 70, 384, 9
+    T1 = synth.draw_trits(rng, (N, K), 0.4)
+    s1 = synth.draw_scales(rng, N, K, 0.005, 0.02)
+    rr = np.sort(rng.choice(N, size=r, replace=False)).astype(np.int32)
+    T2 = synth.draw_trits(rng, (r, K), 0.4)
+    s2 = synth.draw_scales(rng, r, K, 0.001, 0.005)
+    T2e = np.zeros((N, K), np.int8)
+    T2e[rr] = T2
+    s2e = synth.draw_scales(rng, N, K, 0.001, 0.005)
+    s2e[rr] = s2
+    W_row = oracle.dequant(T1, s1, rr, T2, s2)
+    W_elem = oracle.dequant(T1, s1, np.zeros(0, np.int32), np.zeros((0, K), np.int8),
+                            np.zeros((0, K // 128), np.float16), elem=(T2e, s2e))
+    assert np.array_equal(W_row, W_elem)
+
+
+def test_planted_elem_scale_mistake_is_caught():
+    """An oracle that takes the element plane's scale from the next row fails the rational check."""
+    x, T1, s1, rr, T2, s2, (T2e, s2e) = elem_cases()[0]
+    bad = oracle.linear(x, T1, s1, rr, T2, s2, elem=(T2e, np.roll(s2e, 1, axis=0)))
+    yb = brute_linear(x, T1, s1, rr, T2, s2, elem=(T2e, s2e))
     assert any(abs(Fraction(float(bad[m, n])) - yb[m][n]) > Fraction(1e-9)
                for m in range(bad.shape[0]) for n in range(bad.shape[1]))
