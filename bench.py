@@ -163,11 +163,13 @@ def replica_value(world: int, units_per_rank: float, max_secs: float) -> float:
 
 
 # ------------------------------------------------------------------------------ workload
-def draw_layer_on_device(torch, api, shapes, dev, seed):
+def draw_layer_on_device(torch, api, shapes, dev, seed, elem_frac=None):
     """One layer's projections, drawn on the device with a seeded torch generator (same
     distributions as the host recipe: P(0) = 0.4, P(+-1) = 0.3; s1 ~ U[0.005, 0.02];
     s2 ~ U[0.001, 0.005]; 15% residual rows uniformly without replacement) and packed with
-    tern_pack_exec."""
+    tern_pack_exec. With elem_frac, the second plane is element-level instead: each weight is
+    masked with probability elem_frac and a masked weight draws a trit like the main plane, with
+    s2e ~ U[0.001, 0.005] per (row, group)."""
     from ternary_weight_only_tern_b200.synth import residual_count
     g = torch.Generator(device=dev)
     g.manual_seed(seed)
@@ -181,6 +183,15 @@ def draw_layer_on_device(torch, api, shapes, dev, seed):
 
         T1 = trits(N)
         s1 = (torch.rand((N, G), generator=g, device=dev) * 0.015 + 0.005).half()
+        if elem_frac is not None:
+            mask = torch.rand((N, K), generator=g, device=dev) < elem_frac
+            T2e = trits(N) * mask.to(torch.int8)
+            s2e = (torch.rand((N, G), generator=g, device=dev) * 0.004 + 0.001).half()
+            w = api.TernWeight.from_trits(T1, s1, T2e=T2e, s2e=s2e)
+            w.static = True
+            out[name] = w
+            del T1, T2e, mask
+            continue
         r = residual_count(N, RES_PCT)
         rows = torch.randperm(N, generator=g, device=dev)[:r].sort().values.to(torch.int32)
         T2 = trits(r)
@@ -579,6 +590,35 @@ def extras(torch, api, synth, pool, shapes, names, stream, dev, ws, step_fn, ste
     off["gate_m2048"] = {"us": t * 1e6, "tflops": fl / t / 1e12, "frac_burst": fl / t / 1e12 / peaks["bf16_tflops"]}
     out["offset_mu"] = off
     del g, x, y, mpool
+    # the element-level second plane: 3.6 % of the weights masked (the pages' two most salient
+    # masks) instead of 15 % of the rows, the M = 1 stack and the gate GEMM at M = 2048
+    epool = [draw_layer_on_device(torch, api, shapes, dev, seed=2000 + i, elem_frac=0.036) for i in range(POOL_LAYERS)]
+    torch.cuda.synchronize()
+    xs, ys = make_io(1)
+    g = capture(torch, step_fn(1, xs, ys, weights=epool), stream)
+    t = time_graph(torch, g, 30, stream) / 30
+    wb, ab = step_bytes(1, weights=epool)
+    el = {"stack_m1": {"us_per_step": t * 1e6, "packed_gbs": wb / t / 1e9, "frac": (wb + ab) / t / 1e9 / hbm,
+                       "packed_bytes_per_step": wb,
+                       "nnz2_per_weight": float(np.mean([L[n].elem.nnz2 / (L[n].N * L[n].K) for L in epool
+                                                          for n in names]))}}
+    del g, xs, ys
+    g = capture(torch, step_fn(1, xs1, ys1, only="gate", weights=epool), stream)
+    t = time_graph(torch, g, 50, stream) / (50 * LAYERS)
+    wb, ab = step_bytes(1, only="gate", weights=epool)
+    el["gate_m1"] = {"us": t * 1e6, "frac": (wb + ab) / LAYERS / t / 1e9 / hbm}
+    del g
+    x = torch.randn((2048, 4096), device=dev).half()
+    y = torch.empty((2048, 12288), dtype=torch.float16, device=dev)
+
+    def fn_elem():
+        for i in range(4):
+            api.linear(x, epool[i]["gate"], out=y)
+    g = capture(torch, fn_elem, stream)
+    t = time_graph(torch, g, 5, stream) / 20
+    el["gate_m2048"] = {"us": t * 1e6, "tflops": fl / t / 1e12, "frac_burst": fl / t / 1e12 / peaks["bf16_tflops"]}
+    out["elem_plane"] = el
+    del g, x, y, epool
     # packing throughput on the gate shape
     u = torch.randint(0, 3, (12288, 4096), dtype=torch.int8, device=dev) - 1
     for fn_name, fn in (("pack_exec", api.pack_exec), ("pack_store", api.pack_store)):
@@ -601,6 +641,17 @@ def extras(torch, api, synth, pool, shapes, names, stream, dev, ws, step_fn, ste
                             "bpw_store": tot["store_bits"] / tot["weights"],
                             "bpw_exec": tot["exec_bits"] / tot["weights"],
                             "store_gib": tot["store_bits"] / 8 / 2 ** 30}
+    # the same stack with the element-level second plane at the pages' 3.6 % (P(t2 != 0) = 0.6 of it)
+    tot = {"weights": 0, "store_bits": 0, "exec_bits": 0, "plane_trits": 0}
+    for (n, N, K) in shapes:
+        masked = round(0.036 * N * K)
+        b = api.bits_elem(N, K, masked, round(0.6 * masked))
+        for k in tot:
+            tot[k] += LAYERS * b[k]
+    out["bits_8b_stack_elem"] = {"bpw_info": 1.584962500721156 * tot["plane_trits"] / tot["weights"],
+                                 "bpw_store": tot["store_bits"] / tot["weights"],
+                                 "bpw_exec": tot["exec_bits"] / tot["weights"],
+                                 "store_gib": tot["store_bits"] / 8 / 2 ** 30}
     # dense fp16 cuBLAS on the gate shape (context, as in the pages' comparison)
     Wd = [torch.randn((12288, 4096), device=dev).half() for _ in range(4)]
     x1 = torch.randn((1, 4096), device=dev).half()

@@ -14,6 +14,10 @@
  *     library takes the subset as whole output rows; rho(n) is n's index in the sorted R.
  *   - Optionally a per-group offset mu (fp16 [N, K/128]) adds sum_g mu[n, g] * sum_{k in g}
  *     x[m, k] to every row, residual or not (see tern_weight.mu).
+ *   - Optionally the second plane is element-level instead of row-level: a plane T2e over all
+ *     of W, nonzero only on salience-selected weights, with its own fp16 scale per (row,
+ *     group), adds sum_g s2e[n, g] * sum_{k in g} T2e[n, k] * x[m, k] (see "element plane"
+ *     below).
  *   - x and y stay fp16 (weight-only quantisation, 4B paper section 3.1); the sums are
  *     accumulated in fp32 and rounded to fp16 once.
  *   - With weights in {-1, 0, +1} the product is additions and subtractions of activations
@@ -69,7 +73,9 @@ typedef enum {
                                 or inconsistent with the slot map */
     TERN_ERR_WORKSPACE = 7,  /* workspace smaller than tern_linear_workspace_bytes() or NULL */
     TERN_ERR_CUDA = 8,       /* a CUDA runtime call failed (launch error, no device, ...) */
-    TERN_ERR_TIMEOUT = 9     /* a bounded device-side wait ran out (see tern_device_status) */
+    TERN_ERR_TIMEOUT = 9,    /* a bounded device-side wait ran out (see tern_device_status) */
+    TERN_ERR_ELEM = 10       /* unpack_elem / validate: element-plane counts, bases or order
+                                inconsistent */
 } tern_status;
 
 /* A ternarized weight W [N, K] in execution form. Every pointer is device memory,
@@ -87,6 +93,13 @@ typedef struct {
     const tern_half* scale2;     /* [r, K/128]  s2                                      */
     uint32_t flags;              /* 0 or TERN_WEIGHT_STATIC                             */
     const tern_half* mu;         /* [N, K/128]  per-group offset, or NULL (none)        */
+    /* element plane (NULL ecount = none; needs r == 0), layout below                    */
+    const uint8_t* ecount;       /* [K/128, N]  listed trits of (group g, row n)         */
+    const int32_t* ebase;        /* [K/128 * ceil(N/64) + 1] first listed trit of each
+                                    (group, 64-row block); the last entry is nnz2        */
+    const uint8_t* eidx;         /* [nnz2] listed trits, allocated to a multiple of 16 bytes */
+    const tern_half* escale;     /* [N, K/128]  s2e                                     */
+    int64_t nnz2;                /* number of listed trits                              */
 } tern_weight;
 
 /* With an offset the weight is W[n, k] = mu[n, k/128] + s1[n, k/128] T1[n, k]
@@ -94,6 +107,17 @@ typedef struct {
  * mu + a} around an asymmetric per-group offset ("Post-Training Ternarization of Qwen3-4B",
  * section 4.3; the packed format keeps scales and offsets, section 9.1). Without one
  * (mu == NULL) W = s1 T1 (+ s2 T2).                                                     */
+
+/* Element plane. The pages give a second ternary plane to the weights of the two most salient
+ * of four disjoint element masks (3.6 % of a recorded projection's weights: the Qwen3-8B
+ * scale-up paper, representation paragraph; "Post-Training Ternarization of Qwen3-4B",
+ * section 4.4). Here that plane is T2e [N, K], zero outside the masks, with one fp16 scale per
+ * (row, group): W += s2e[n, k/128] T2e[n, k]. It is kept as the list of its nonzero trits,
+ * one byte each, (k % 128) << 1 | (t < 0), ordered by group, then row, then k; ecount[g, n] is
+ * the number listed for (row n, group g), and ebase[g * ceil(N/64) + b] the index of the first
+ * one of rows 64b .. 64b+63 in group g, so that the trits of one group of 64 consecutive rows
+ * are contiguous. A row may carry a row-level second plane (r > 0) or an element plane, not
+ * both; an element plane may carry an offset. Every pointer 16-byte aligned.             */
 
 /* tern_weight.flags: the planes, scales and slot map are not written by work queued before
  * the call on its stream (model weights). tern_linear may then start reading them while the
@@ -121,9 +145,26 @@ tern_status tern_pack_store(const int8_t* t, int64_t rows, int64_t K, uint8_t* o
  * return TERN_ERR_BAD_CODE. Synchronous on `stream`.                                    */
 tern_status tern_unpack_store(const uint8_t* b, int64_t rows, int64_t K, int8_t* out, tern_stream stream);
 
+/* int8 T2e [N, K] (device) -> element plane: ecount [K/128, N], ebase [K/128 * ceil(N/64) + 1]
+ * and, when eidx is not NULL, the listed trits eidx (device), of which there are *nnz2.
+ * K % 128 == 0. Call once with eidx == NULL to learn *nnz2 (ecount and ebase are written),
+ * then with eidx of eidx_bytes >= nnz2 rounded up to 16 (the padding is zeroed); a smaller
+ * eidx returns TERN_ERR_WORKSPACE and leaves eidx untouched. An input outside {-1,0,+1} is
+ * listed as 0 (not at all) and the call returns TERN_ERR_BAD_TRIT. Synchronous on `stream`. */
+tern_status tern_pack_elem(const int8_t* t, int64_t N, int64_t K, uint8_t* ecount, int32_t* ebase, uint8_t* eidx,
+                           int64_t eidx_bytes, int64_t* nnz2, tern_stream stream);
+
+/* Element plane (device) -> int8 T2e out [N, K] (device). Inconsistent input (a count above
+ * 128, a block whose counts do not add up to the gap between its base and the next, ebase[0]
+ * != 0 or the last base != nnz2, a k that does not increase within a (row, group)) returns
+ * TERN_ERR_ELEM; every trit whose index lies in [0, nnz2) is still placed. Synchronous.   */
+tern_status tern_unpack_elem(const uint8_t* ecount, const int32_t* ebase, const uint8_t* eidx, int64_t nnz2,
+                             int64_t N, int64_t K, int8_t* out, tern_stream stream);
+
 /* Checks a weight descriptor's device data: every code of plane1/plane2 is in {0,1,2},
  * res_rows is strictly increasing in [0, N), and res_slot[n] == i exactly when
- * res_rows[i] == n (else -1). Returns TERN_OK, TERN_ERR_BAD_CODE or TERN_ERR_RESIDUAL.
+ * res_rows[i] == n (else -1); an element plane is checked as by tern_unpack_elem.
+ * Returns TERN_OK, TERN_ERR_BAD_CODE, TERN_ERR_RESIDUAL or TERN_ERR_ELEM.
  * Synchronous on `stream`. tern_linear does not repeat these checks; it only keeps its
  * own memory accesses in bounds when a slot is out of range.                            */
 tern_status tern_weight_validate(const tern_weight* w, tern_stream stream);
@@ -176,6 +217,14 @@ tern_status tern_bits(int64_t N, int64_t K, int64_t r, int32_t group, tern_bits_
  * (row, group) in the storage and the execution forms; the information figure counts plane
  * symbols only and is unchanged.                                                        */
 tern_status tern_bits_offset(int64_t N, int64_t K, int64_t r, int32_t group, tern_bits_report* out);
+
+/* Bits of a tensor whose second plane is element-level: `masked` weights carry a second
+ * symbol (the information rate is log2(3) (1 + masked / (N K)), the pages' f2 accounting) and
+ * nnz2 of them are listed. store and exec add to the main plane and s1 the element plane's
+ * bytes: 8 bits per ecount entry, 32 per ebase entry, 8 per listed trit, 16 per s2e entry;
+ * offset != 0 adds 16 bits per (row, group). plane_trits = N K + masked. Host only.      */
+tern_status tern_bits_elem(int64_t N, int64_t K, int64_t masked, int64_t nnz2, int32_t group, int32_t offset,
+                           tern_bits_report* out);
 
 /* Reports, and clears, the current device's sticky status word for asynchronous work: returns
  * TERN_ERR_TIMEOUT if a tern_linear kernel since the last call gave up a bounded device-side

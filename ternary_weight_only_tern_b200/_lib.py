@@ -12,7 +12,7 @@ TERN_OK = 0
 STATUS_NAMES = {
     0: "TERN_OK", 1: "TERN_ERR_NULL", 2: "TERN_ERR_SHAPE", 3: "TERN_ERR_ALIGN", 4: "TERN_ERR_BAD_TRIT",
     5: "TERN_ERR_BAD_CODE", 6: "TERN_ERR_RESIDUAL", 7: "TERN_ERR_WORKSPACE", 8: "TERN_ERR_CUDA",
-    9: "TERN_ERR_TIMEOUT",
+    9: "TERN_ERR_TIMEOUT", 10: "TERN_ERR_ELEM",
 }
 STATUS = {v: k for k, v in STATUS_NAMES.items()}
 
@@ -31,6 +31,12 @@ EXPORTS = {
                                              _c.c_size_t, _c.c_void_p, _c.c_void_p]),
     "tern_bits": (_c.c_int, [_c.c_int64, _c.c_int64, _c.c_int64, _c.c_int32, _c.c_void_p]),
     "tern_bits_offset": (_c.c_int, [_c.c_int64, _c.c_int64, _c.c_int64, _c.c_int32, _c.c_void_p]),
+    "tern_bits_elem": (_c.c_int, [_c.c_int64, _c.c_int64, _c.c_int64, _c.c_int64, _c.c_int32, _c.c_int32,
+                                  _c.c_void_p]),
+    "tern_pack_elem": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_int64, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                  _c.c_int64, _c.c_void_p, _c.c_void_p]),
+    "tern_unpack_elem": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_int64,
+                                    _c.c_void_p, _c.c_void_p]),
     "tern_device_status": (_c.c_int, [_c.c_void_p]),
     "tern_status_string": (_c.c_char_p, [_c.c_int]),
     "tern_version": (_c.c_int, []),
@@ -45,6 +51,8 @@ class TernWeightC(ctypes.Structure):
         ("r", ctypes.c_int64), ("res_rows", ctypes.c_void_p), ("res_slot", ctypes.c_void_p),
         ("plane2", ctypes.c_void_p), ("scale2", ctypes.c_void_p), ("flags", ctypes.c_uint32),
         ("mu", ctypes.c_void_p),
+        ("ecount", ctypes.c_void_p), ("ebase", ctypes.c_void_p), ("eidx", ctypes.c_void_p),
+        ("escale", ctypes.c_void_p), ("nnz2", ctypes.c_int64),
     ]
 
 

@@ -73,6 +73,44 @@ def unpack_store(data: torch.Tensor, K: int) -> torch.Tensor:
     return out
 
 
+@dataclass
+class ElemPlane:
+    """An element-level second plane in its listed form (tern_pack_elem): the nonzero trits of
+    T2e, one byte each, with per-(group, row) counts and per-(group, 64-row block) bases."""
+    N: int
+    K: int
+    ecount: torch.Tensor     # uint8 [K/128, N]
+    ebase: torch.Tensor      # int32 [K/128 * ceil(N/64) + 1]
+    eidx: torch.Tensor       # uint8 [nnz2 rounded up to 16]
+    nnz2: int
+
+
+def pack_elem(T2e: torch.Tensor) -> ElemPlane:
+    """int8 T2e [N, K] -> its listed form (two calls: the count, then the fill)."""
+    _need(T2e, torch.int8, "T2e")
+    N, K = T2e.shape
+    if K % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    dev = T2e.device
+    ecount = torch.empty((K // GROUP, N), dtype=torch.uint8, device=dev)
+    ebase = torch.empty(K // GROUP * (-(-N // 64)) + 1, dtype=torch.int32, device=dev)
+    nnz = ctypes.c_int64(0)
+    lib = _lib.load()
+    _lib.check("tern_pack_elem", lib.tern_pack_elem(_ptr(T2e), N, K, _ptr(ecount), _ptr(ebase), None, 0,
+                                                    ctypes.byref(nnz), _stream(dev)))
+    eidx = torch.empty(max(16, -(-nnz.value // 16) * 16), dtype=torch.uint8, device=dev)
+    _lib.check("tern_pack_elem", lib.tern_pack_elem(_ptr(T2e), N, K, _ptr(ecount), _ptr(ebase), _ptr(eidx),
+                                                    eidx.numel(), ctypes.byref(nnz), _stream(dev)))
+    return ElemPlane(N, K, ecount, ebase, eidx, int(nnz.value))
+
+
+def unpack_elem(e: ElemPlane) -> torch.Tensor:
+    out = torch.empty((e.N, e.K), dtype=torch.int8, device=e.ecount.device)
+    _lib.check("tern_unpack_elem", _lib.load().tern_unpack_elem(_ptr(e.ecount), _ptr(e.ebase), _ptr(e.eidx), e.nnz2,
+                                                                e.N, e.K, _ptr(out), _stream(out.device)))
+    return out
+
+
 # ------------------------------------------------------------------------------ weights
 
 @dataclass
@@ -88,6 +126,8 @@ class TernWeight:
     scale2: torch.Tensor     # float16 [r, K/128]
     static: bool = False     # weights not written by queued work: tern_linear may prefetch them early
     mu: torch.Tensor | None = None   # float16 [N, K/128] per-group offset: W = mu + s1 T1 (+ s2 T2)
+    elem: ElemPlane | None = None    # element-level second plane (then r == 0)
+    escale: torch.Tensor | None = None   # float16 [N, K/128] its scales s2e
 
     @property
     def r(self) -> int:
@@ -104,23 +144,37 @@ class TernWeight:
                 self.N, self.K, GROUP, self.plane1.data_ptr(), self.scale1.data_ptr(), self.r,
                 self.res_rows.data_ptr() if self.r else None, self.res_slot.data_ptr(),
                 self.plane2.data_ptr() if self.r else None, self.scale2.data_ptr() if self.r else None,
-                _lib.WEIGHT_STATIC if self.static else 0, self.mu.data_ptr() if self.mu is not None else None)
+                _lib.WEIGHT_STATIC if self.static else 0, self.mu.data_ptr() if self.mu is not None else None,
+                *self._elem_fields())
             object.__setattr__(self, "_c", c)
         return c
 
+    def _elem_fields(self):
+        e = self.elem
+        if e is None:
+            return (None, None, None, None, 0)
+        return (e.ecount.data_ptr(), e.ebase.data_ptr(), e.eidx.data_ptr(), self.escale.data_ptr(), e.nnz2)
+
     def nbytes(self) -> int:
-        """Bytes the decode kernels stream per call: both planes, their scales and the slot map."""
+        """Bytes the decode kernels stream per call: the planes, their scales, the slot map, the
+        offset and the element plane's counts, bases, listed trits and scales."""
         ts = (self.plane1, self.scale1, self.plane2, self.scale2, self.res_slot)
         if self.mu is not None:
             ts = ts + (self.mu,)
-        return sum(t.numel() * t.element_size() for t in ts)
+        n = sum(t.numel() * t.element_size() for t in ts)
+        if self.elem is not None:
+            e = self.elem
+            n += e.ecount.numel() + 4 * e.ebase.numel() + e.nnz2 + 2 * self.escale.numel()
+        return n
 
     @classmethod
     def from_trits(cls, T1: torch.Tensor, s1: torch.Tensor, res_rows: torch.Tensor | None = None,
                    T2: torch.Tensor | None = None, s2: torch.Tensor | None = None,
-                   mu: torch.Tensor | None = None) -> "TernWeight":
+                   mu: torch.Tensor | None = None, T2e: torch.Tensor | None = None,
+                   s2e: torch.Tensor | None = None) -> "TernWeight":
         """Packs int8 planes on the device (tern_pack_exec) and builds the residual-row slot map;
-        mu, if given, is the per-group offset [N, K/128]."""
+        mu, if given, is the per-group offset [N, K/128]; T2e and s2e, if given, an element-level
+        second plane (tern_pack_elem) and its scales, in place of residual rows."""
         _need(T1, torch.int8, "T1")
         _need(s1, torch.float16, "s1")
         N, K = T1.shape
@@ -140,15 +194,29 @@ class TernWeight:
             if tuple(mu.shape) != (N, K // GROUP):
                 raise ValueError(f"mu must have shape {(N, K // GROUP)}")
             mu = mu.to(dev).contiguous()
+        elem = None
+        if T2e is not None:
+            if r:
+                raise ValueError("a weight carries residual rows or an element plane, not both")
+            if tuple(T2e.shape) != (N, K):
+                raise ValueError(f"T2e must have shape {(N, K)}")
+            _need(s2e, torch.float16, "s2e")
+            if tuple(s2e.shape) != (N, K // GROUP):
+                raise ValueError(f"s2e must have shape {(N, K // GROUP)}")
+            elem = pack_elem(T2e.to(dev).contiguous())
+            s2e = s2e.to(dev).contiguous()
         return cls(N, K, pack_exec(T1), s1.contiguous(), res_rows, slot, plane2,
-                   s2.contiguous() if r else torch.zeros((0, K // GROUP), dtype=torch.float16, device=dev), mu=mu)
+                   s2.contiguous() if r else torch.zeros((0, K // GROUP), dtype=torch.float16, device=dev), mu=mu,
+                   elem=elem, escale=s2e if elem is not None else None)
 
     @classmethod
-    def from_numpy(cls, T1, s1, res_rows, T2, s2, device="cuda", mu=None) -> "TernWeight":
+    def from_numpy(cls, T1, s1, res_rows, T2, s2, device="cuda", mu=None, T2e=None, s2e=None) -> "TernWeight":
         t = lambda a, dt: torch.from_numpy(a).to(device=device, dtype=dt).contiguous()  # noqa: E731
         return cls.from_trits(t(T1, torch.int8), t(s1, torch.float16), t(res_rows, torch.int32),
                               t(T2, torch.int8), t(s2, torch.float16),
-                              mu=t(mu, torch.float16) if mu is not None else None)
+                              mu=t(mu, torch.float16) if mu is not None else None,
+                              T2e=t(T2e, torch.int8) if T2e is not None else None,
+                              s2e=t(s2e, torch.float16) if s2e is not None else None)
 
 
 def weight_validate(w: TernWeight) -> None:
@@ -193,6 +261,13 @@ def linear(x: torch.Tensor, w: TernWeight, out: torch.Tensor | None = None,
 
 
 # ------------------------------------------------------------------------------ bits
+
+def bits_elem(N: int, K: int, masked: int, nnz2: int, group: int = GROUP, offset: bool = False) -> dict:
+    rep = _lib.TernBitsReport()
+    _lib.check("tern_bits_elem", _lib.load().tern_bits_elem(N, K, masked, nnz2, group, int(offset),
+                                                            ctypes.byref(rep)))
+    return {f: getattr(rep, f) for f, _ in rep._fields_}
+
 
 def bits(N: int, K: int, r: int, group: int = GROUP, offset: bool = False) -> dict:
     rep = _lib.TernBitsReport()

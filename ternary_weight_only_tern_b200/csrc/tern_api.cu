@@ -42,6 +42,12 @@ tern_status check_weight(const tern_weight* w) {
     if (w->r > 0 && (!aligned16(w->plane2) || !aligned16(w->scale2) || !aligned16(w->res_slot)))
         return TERN_ERR_ALIGN;
     if (w->mu && !aligned16(w->mu)) return TERN_ERR_ALIGN;
+    if (w->ecount) {
+        if (w->r > 0 || w->nnz2 < 0 || w->nnz2 > 0x7fffffff || w->K / kGroup > 65535) return TERN_ERR_SHAPE;
+        if (!w->ebase || !w->escale || (w->nnz2 > 0 && !w->eidx)) return TERN_ERR_NULL;
+        if (!aligned16(w->ecount) || !aligned16(w->ebase) || !aligned16(w->escale) || (w->eidx && !aligned16(w->eidx)))
+            return TERN_ERR_ALIGN;
+    }
     return TERN_OK;
 }
 

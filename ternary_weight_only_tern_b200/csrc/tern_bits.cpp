@@ -6,7 +6,7 @@
 // planes (1.641 bits per weight measured, against log2 3 = 1.585 for one plane),
 // which counts log2 3 per plane symbol with a fraction f2 of weights carrying a second
 // plane; and what a file or an execution buffer actually holds. This function reports
-// all three for the row-subset form this library builds.
+// all three for the row-subset form and for the element-level second plane.
 #include <math.h>
 
 #include "../../include/tern.h"
@@ -45,6 +45,33 @@ extern "C" tern_status tern_bits_offset(int64_t N, int64_t K, int64_t r, int32_t
     return TERN_OK;
 }
 
+extern "C" tern_status tern_bits_elem(int64_t N, int64_t K, int64_t masked, int64_t nnz2, int32_t group,
+                                      int32_t offset, tern_bits_report* out) {
+    if (!out) return TERN_ERR_NULL;
+    if (N <= 0 || K <= 0 || group != 128 || K % group) return TERN_ERR_SHAPE;
+    if (N > (int64_t(1) << 40) || K > (int64_t(1) << 20) || N > (int64_t(1) << 62) / K) return TERN_ERR_SHAPE;
+    if (masked < 0 || masked > N * K || nnz2 < 0 || nnz2 > masked) return TERN_ERR_SHAPE;
+    const uint64_t n = static_cast<uint64_t>(N), k = static_cast<uint64_t>(K);
+    const uint64_t G = k / static_cast<uint64_t>(group);
+    const uint64_t blocks = (n + 63) / 64;             // ebase: one entry per (group, 64-row block), + 1
+    const uint64_t header_bits = 512;
+    const uint64_t store_row_bytes = (k + 4) / 5;
+    const uint64_t elem_bits = 8 * G * n + 32 * (G * blocks + 1) + 8 * static_cast<uint64_t>(nnz2) + 16 * n * G;
+    out->weights = n * k;
+    out->plane_trits = n * k + static_cast<uint64_t>(masked);
+    out->store_bits = 8 * n * store_row_bytes + 16 * n * G + elem_bits + header_bits;
+    out->exec_bits = 2 * n * k + 16 * n * G + elem_bits + header_bits;
+    if (offset) {
+        out->store_bits += 16 * n * G;
+        out->exec_bits += 16 * n * G;
+    }
+    const double w = static_cast<double>(out->weights);
+    out->bpw_info = log2(3.0) * static_cast<double>(out->plane_trits) / w;
+    out->bpw_store = static_cast<double>(out->store_bits) / w;
+    out->bpw_exec = static_cast<double>(out->exec_bits) / w;
+    return TERN_OK;
+}
+
 extern "C" const char* tern_status_string(tern_status s) {
     switch (s) {
         case TERN_OK: return "ok";
@@ -57,6 +84,7 @@ extern "C" const char* tern_status_string(tern_status s) {
         case TERN_ERR_WORKSPACE: return "workspace too small";
         case TERN_ERR_CUDA: return "CUDA error";
         case TERN_ERR_TIMEOUT: return "device wait timed out";
+        case TERN_ERR_ELEM: return "inconsistent element-plane metadata";
     }
     return "unknown status";
 }

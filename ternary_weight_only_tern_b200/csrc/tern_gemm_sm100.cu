@@ -3,9 +3,10 @@
 //
 // The operation is that of "Post-Training Ternarization of Qwen3-4B" (arXiv 2609.01962v1),
 // sections 4.3-4.5: W = s1 (.) T1, plus s2 (.) T2 on the residual rows, fp16 activations
-// (section 3.1). At M in the thousands it is a dense contraction, so it runs on the tensor
-// cores; the weights are never reconstructed in global memory (section 14: native kernels
-// consume the ternary planes directly).
+// (section 3.1); optionally a per-group offset (W = mu + ...) and an element-level second
+// plane (W += s2e T2e on its listed trits; section 4.4). At M in the thousands it is a dense
+// contraction, so it runs on the tensor cores; the weights are never reconstructed in global
+// memory (section 14: native kernels consume the ternary planes directly).
 //
 // One CTA computes a 256 (tokens) x 256 (weight rows) tile with two tcgen05.mma (kind::f16,
 // M = 128, N = 256, K = 16, fp32 accumulators in TMEM columns 0-255 and 256-511) per 16
@@ -54,6 +55,12 @@ struct GemmArgs {
     const __half* scale2;
     const int32_t* res_slot;
     const __half* mu;          // [N, G] per-group offsets, or nullptr
+    const uint8_t* ecount;     // element plane: [G, N] listed trits per (group, row), or nullptr
+    const int32_t* ebase;      // [G * nb + 1]
+    const uint8_t* eidx;       // [nnz2] (k % 128) << 1 | (t < 0)
+    const __half* escale;      // [N, G]
+    int64_t nnz2;
+    int64_t nb;                // ceil(N / 64)
     int64_t N, K, r, M;
     int32_t G;
     __half* y;
@@ -292,22 +299,63 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             rq0[j] = (has0 && j < a.G) ? s2row0[j] : __float2half(0.f);
             rq1[j] = (has1 && j < a.G) ? s2row1[j] : __float2half(0.f);
         }
+        // Element plane: this row's listed trits of a group start at ebase[g, its 64-row block]
+        // + the counts of the rows before it in that block (a scan over the warp, plus the
+        // previous warp's total for the second warp of the block). Its count, the previous
+        // warp's count at the same lane, the block base and s2e are queued two groups ahead.
+        const bool elem = a.ecount != nullptr;
+        const bool odd = ((t >> 5) & 1) != 0;
+        const int64_t eblk = (n0 + t) / kElemBlock;
+        int eq_c[3] = {0, 0, 0}, eq_p[3] = {0, 0, 0}, eq_b[3] = {0, 0, 0};
+        __half eq_s[3] = {__float2half(0.f), __float2half(0.f), __float2half(0.f)};
+        auto elem_load = [&](int j, int g) {
+            if (!elem || g >= a.G) return;
+            eq_c[j] = valid ? int(__ldg(a.ecount + int64_t(g) * a.N + n)) : 0;
+            eq_p[j] = (odd && n - 32 < a.N) ? int(__ldg(a.ecount + int64_t(g) * a.N + n - 32)) : 0;
+            eq_b[j] = eblk < a.nb ? __ldg(a.ebase + int64_t(g) * a.nb + eblk) : 0;   // (rows past N: none)
+            eq_s[j] = valid ? a.escale[n * int64_t(a.G) + g] : __float2half(0.f);
+        };
+#pragma unroll
+        for (int j = 0; j < 3; ++j) elem_load(j, j);
+        int64_t e_pos = 0, e_end = 0;   // this row's listed trits of the current group
         for (int kb = 0; kb < num_kb; ++kb) {
             const int s = kb % kStages, sp = kb % kStagesP;
             const int g = kb / 2;
             if ((kb & 1) == 0 && kb > 0) {   // a new group: shift the scale queues, load two ahead
                 sq[0] = sq[1]; sq[1] = sq[2];
                 mq[0] = mq[1]; mq[1] = mq[2];
+                eq_c[0] = eq_c[1]; eq_c[1] = eq_c[2];
+                eq_p[0] = eq_p[1]; eq_p[1] = eq_p[2];
+                eq_b[0] = eq_b[1]; eq_b[1] = eq_b[2];
+                eq_s[0] = eq_s[1]; eq_s[1] = eq_s[2];
                 rq0[0] = rq0[1]; rq0[1] = rq0[2];
                 rq1[0] = rq1[1]; rq1[1] = rq1[2];
                 const int g2 = g + 2;
                 if (g2 < a.G) {
                     sq[2] = valid ? srow[g2] : __float2half(0.f);
                     if (mrow) mq[2] = valid ? mrow[g2] : __float2half(0.f);
+                    elem_load(2, g2);
                     if (has0) rq0[2] = s2row0[g2];
                     if (has1) rq1[2] = s2row1[g2];
                 }
             }
+            if (elem && (kb & 1) == 0) {
+                // the row's run of this group: every lane of the warp takes part in the scans
+                const int c = min(eq_c[0], kGroup);
+                int incl = c, prev = min(eq_p[0], kGroup);
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+                    if ((t & 31) >= o) incl += u;
+                    prev += __shfl_xor_sync(0xffffffffu, prev, o);
+                }
+                e_pos = min(max(int64_t(eq_b[0]) + (odd ? prev : 0) + incl - c, int64_t(0)), a.nnz2);
+                e_end = min(e_pos + c, a.nnz2);
+            }
+            // the first listed trits of this half, fetched before the wait
+            uint32_t ev[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) ev[j] = (elem && e_pos + j < e_end) ? uint32_t(__ldg(a.eidx + e_pos + j)) : 0xffffu;
             // every dequantising thread takes the same decision, so the named barriers below match
             ok = dequant_all(mbar_wait(&full_p[sp], (kb / kStagesP) & 1) &&
                              (kb < kStages || mbar_wait(&empty[s], ((kb / kStages) - 1) & 1)));
@@ -328,6 +376,33 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 o.z = h2_bits(__hfma2(tt[2], s2, m2));
                 o.w = h2_bits(__hfma2(tt[3], s2, m2));
                 sts_u4(bs + sw128_offset(t, c), o);
+            }
+            if (elem && e_pos < e_end) {
+                // RN(w + s2e t2e) for this row's listed trits in this half (k % 128 in [64 h, 64 h + 64))
+                const __half se = eq_s[0];
+                const uint32_t lim = 64u * uint32_t((kb & 1) + 1);
+                auto apply = [&](uint32_t v) {
+                    const uint32_t kk = (v >> 1) & 63u;
+                    const uint32_t addr = bs + sw128_offset(t, int(kk >> 3)) + (kk & 7u) * 2u;
+                    unsigned short h;
+                    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(h) : "r"(addr));
+                    const __half w = __ushort_as_half(h);
+                    const __half r = (v & 1u) ? __hsub(w, se) : __hadd(w, se);
+                    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(__half_as_ushort(r)) : "memory");
+                };
+                int j = 0;
+                for (; j < 4 && e_pos < e_end; ++j) {
+                    if ((ev[j] >> 1) >= lim) break;
+                    apply(ev[j]);
+                    ++e_pos;
+                }
+                if (j == 4)
+                    while (e_pos < e_end) {
+                        const uint32_t v = __ldg(a.eidx + e_pos);
+                        if ((v >> 1) >= lim) break;
+                        apply(v);
+                        ++e_pos;
+                    }
             }
             if (n_res > 0) {
                 asm volatile("bar.sync 1, %0;" ::"n"(kDequantThreads) : "memory");
@@ -462,6 +537,12 @@ tern_status gemm_launch(const tern_weight& w, const __half* x, int64_t M, __half
     a.scale2 = reinterpret_cast<const __half*>(w.scale2);
     a.res_slot = w.r > 0 ? w.res_slot : nullptr;
     a.mu = reinterpret_cast<const __half*>(w.mu);
+    a.ecount = w.ecount;
+    a.ebase = w.ebase;
+    a.eidx = w.eidx;
+    a.escale = reinterpret_cast<const __half*>(w.escale);
+    a.nnz2 = w.ecount ? w.nnz2 : 0;
+    a.nb = (w.N + kElemBlock - 1) / kElemBlock;
     a.N = w.N;
     a.K = w.K;
     a.r = w.r;

@@ -65,12 +65,24 @@ constexpr int kMaxSplit = 16;
 constexpr int kMainChunkBytes = kRowsPerCta * 128;  // 8 KB
 constexpr int kStripBytes = kStrip * 128;           // 2 KB
 constexpr int kResChunkBytes = kResStrips * kStripBytes;
+// element plane: its staged runs and per-row starts live in the residual tile's space, which
+// that form does not use
+constexpr int kEStageBytes = kMaxChunks * kResChunkBytes - kMaxGpc * kRowsPerCta * 4;
+static_assert(kRowsPerCta == kElemBlock, "one element-plane block per CTA");
+
+constexpr int kPrefetchRanges = 9;
 
 struct GemvArgs {
     const __half* scale1;      // [N, G]
     const __half* scale2;      // [r, G]
     const int32_t* res_slot;   // [N] or nullptr
     const __half* mu;          // [N, G] per-group offsets, or nullptr
+    const uint8_t* ecount;     // element plane: [G, N] listed trits per (group, row), or nullptr
+    const int32_t* ebase;      // [G * nb + 1] first listed trit of each (group, 64-row block)
+    const uint8_t* eidx;       // [nnz2, padded to 16] (k % 128) << 1 | (t < 0)
+    const __half* escale;      // [N, G]
+    int64_t nnz2;
+    int32_t nb;                // ceil(N / 64)
     const __half* x;           // [M, K]
     __half* y;                 // [M, N]
     unsigned int* status;      // sticky timeout word
@@ -81,8 +93,8 @@ struct GemvArgs {
     int32_t static_weights;    // planes may be read before griddepcontrol.wait
     // byte ranges of the next call's weight to bring into L2 (16-byte aligned, sizes rounded down
     // to 16 bytes); every CTA prefetches its share of each
-    const uint8_t* pf_ptr[6];
-    int64_t pf_bytes[6];
+    const uint8_t* pf_ptr[kPrefetchRanges];
+    int64_t pf_bytes[kPrefetchRanges];
 };
 
 struct Smem {
@@ -237,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
     if (threadIdx.x == kThreads - 1) {
         // this CTA's share of the next call's weight, into L2
         const int64_t nctas = int64_t(gridDim.x) * gridDim.y, b = int64_t(blockIdx.y) * gridDim.x + blockIdx.x;
-        for (int i = 0; i < 6; ++i) {
+        for (int i = 0; i < kPrefetchRanges; ++i) {
             const int64_t per = ((a.pf_bytes[i] + nctas - 1) / nctas + 15) / 16 * 16;
             const int64_t lo = b * per, hi = min(a.pf_bytes[i], lo + per);
             if (a.pf_ptr[i] != nullptr && lo < hi) prefetch_l2_bulk(a.pf_ptr[i] + lo, uint32_t(hi - lo));
@@ -454,6 +466,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
         // every rank sends this rank M sums per owned row, and M more per owned row with a residual
         int owned_res = 0;
         for (int lo = 0; lo < nrows; ++lo) owned_res += (bslot[lr0 + lo] >= 0 && bslot[lr0 + lo] < nres) ? 1 : 0;
+        if (a.ecount) owned_res = nrows;     // the element plane sends a sum for every row
         mbar_arrive_expect_tx(rbar, uint32_t(a.split * (nrows + owned_res) * M * 4));
     }
 
@@ -543,6 +556,143 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
                 store_red(true, rrow + rr, yacc);
             }
         }
+    } else if (a.ecount) {
+        // Element plane of this block's 64 rows over the slice. Lane gi reads group gi's run
+        // bounds, the warp copies the runs (16-byte aligned spans) into shared memory, each lane
+        // finds the start of rows lane and lane + 32 in them (scan of the counts), then sums
+        // +-x over its rows' listed trits per group and scales by s2e.
+        constexpr int kTok = kOne ? 1 : 8 * NT;
+        const int64_t blk = blockIdx.y;
+        uint8_t* ebuf = wt2;
+        int* estart = reinterpret_cast<int*>(wt2 + kEStageBytes);      // [kMaxGpc][64]
+        int64_t b0 = 0, b1 = 0;
+        if (lane < ng) {
+            const int64_t cell = int64_t(g_begin + lane) * a.nb + blk;
+            b0 = min(max(int64_t(__ldg(a.ebase + cell)), int64_t(0)), a.nnz2);
+            b1 = min(max(int64_t(__ldg(a.ebase + cell + 1)), b0), a.nnz2);
+        }
+        uint32_t cpk[2][2] = {{0u, 0u}, {0u, 0u}};   // counts of rows lane, lane + 32: 8 bits per group
+        uint32_t spk[2][kMaxGpc / 2];                 // their scales s2e, fp16 pairs
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int64_t n = n0 + lane + 32 * h;
+#pragma unroll
+            for (int gi = 0; gi < kMaxGpc; gi += 2) {
+                uint32_t s01 = 0u;
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    if (gi + u < ng && n < a.N) {
+                        const uint32_t c = __ldg(a.ecount + int64_t(g_begin + gi + u) * a.N + n);
+                        cpk[h][(gi + u) >> 2] |= min(c, uint32_t(kGroup)) << (8 * ((gi + u) & 3));
+                        s01 |= uint32_t(__half_as_ushort(a.escale[n * a.G + g_begin + gi + u])) << (16 * u);
+                    }
+                }
+                spk[h][gi >> 1] = s01;
+            }
+        }
+        const int64_t a0 = b0 & ~int64_t(15), a1 = (b1 + 15) & ~int64_t(15);
+        const int nchunk = lane < ng ? int((a1 - a0) >> 4) : 0;
+        int coff = nchunk;                             // inclusive scan of the chunk counts
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, coff, o);
+            if (lane >= o) coff += u;
+        }
+        const int total = __shfl_sync(0xffffffffu, coff, 31);
+        coff -= nchunk;
+        const bool staged = total * 16 <= kEStageBytes;
+        if (staged) {
+            // chunk j of the copy belongs to the last group whose first chunk is <= j
+            int cof[kMaxGpc], src0[kMaxGpc];
+#pragma unroll
+            for (int gi = 0; gi < kMaxGpc; ++gi) {
+                cof[gi] = __shfl_sync(0xffffffffu, coff, gi);
+                src0[gi] = int(__shfl_sync(0xffffffffu, a0, gi) >> 4);
+            }
+            const uint4* gsrc = reinterpret_cast<const uint4*>(a.eidx);
+            uint4* sdst = reinterpret_cast<uint4*>(ebuf);
+            for (int j0 = 0; j0 < total; j0 += 64) {
+                uint4 v[2];
+                int dj[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int j = j0 + 32 * u + lane;
+                    dj[u] = -1;
+                    if (j < total) {
+                        int from = src0[0] + j - cof[0];
+#pragma unroll
+                        for (int q2 = 1; q2 < kMaxGpc; ++q2)
+                            if (q2 < ng && cof[q2] <= j) from = src0[q2] + j - cof[q2];
+                        v[u] = __ldg(gsrc + from);
+                        dj[u] = j;
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+                    if (dj[u] >= 0) sdst[dj[u]] = v[u];
+            }
+        }
+        // run base of each group in the source: the staged copy or the global list
+        const int64_t rbase = staged ? int64_t(coff) * 16 + (b0 - a0) : b0;
+        const int64_t rend = rbase + (b1 - b0);
+#pragma unroll
+        for (int gi = 0; gi < kMaxGpc; ++gi) {
+            if (gi >= ng) break;
+            const int c0 = (cpk[0][gi >> 2] >> (8 * (gi & 3))) & 0xff, c1 = (cpk[1][gi >> 2] >> (8 * (gi & 3))) & 0xff;
+            int i0 = c0, i1 = c1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u0 = __shfl_up_sync(0xffffffffu, i0, o), u1 = __shfl_up_sync(0xffffffffu, i1, o);
+                if (lane >= o) {
+                    i0 += u0;
+                    i1 += u1;
+                }
+            }
+            const int tot0 = __shfl_sync(0xffffffffu, i0, 31);
+            const int base = int(__shfl_sync(0xffffffffu, rbase, gi));
+            estart[gi * kRowsPerCta + lane] = base + i0 - c0;
+            estart[gi * kRowsPerCta + 32 + lane] = base + tot0 + i1 - c1;
+        }
+        __syncwarp();
+        const uint8_t* src = staged ? ebuf : a.eidx;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int lr = lane + 32 * h;
+            float acc[kTok];
+#pragma unroll
+            for (int t = 0; t < kTok; ++t) acc[t] = 0.f;
+#pragma unroll
+            for (int gi = 0; gi < kMaxGpc; ++gi) {
+                if (gi >= ng) break;
+                const int c = (cpk[h][gi >> 2] >> (8 * (gi & 3))) & 0xff;
+                const int64_t end = __shfl_sync(0xffffffffu, rend, gi);
+                if (c == 0) continue;
+                const int st = estart[gi * kRowsPerCta + lr];
+                float gs[kTok];
+#pragma unroll
+                for (int t = 0; t < kTok; ++t) gs[t] = 0.f;
+                for (int e = 0; e < c; ++e) {
+                    if (st + e >= end) break;       // only with inconsistent counts
+                    const uint32_t v = src[st + e];
+                    const uint32_t kk = v >> 1, w = kk >> 4, j = kk & 15;
+                    const int off = gi * kGroup + int((((w & 1) << 2) | (w >> 1)) * 16 + (((j & 7) << 1) | (j >> 3)));
+#pragma unroll
+                    for (int t = 0; t < kTok; ++t) {
+                        if (t < M) {
+                            const float xv = __half2float(xs[size_t(t) * xs_stride + off]);
+                            gs[t] += (v & 1) ? -xv : xv;
+                        }
+                    }
+                }
+                const uint32_t sp = spk[h][gi >> 1] >> (16 * (gi & 1));
+                const float sc = __half2float(__ushort_as_half(static_cast<unsigned short>(sp & 0xffffu)));
+#pragma unroll
+                for (int t = 0; t < kTok; ++t) acc[t] = fmaf(sc, gs[t], acc[t]);
+            }
+#pragma unroll
+            for (int t = 0; t < kTok; ++t)
+                if (t < M) push(recv_res, lr, t, acc[t]);
+        }
     }
 
     // Epilogue: once the partial sums of this rank's rows have arrived from every rank (the
@@ -557,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
             float s = 0.f;
             for (int c = 0; c < a.split; ++c) s += recv[(c * rows_per_rank + lo) * M + tok];
             const int slot = bslot[lr];
-            if (slot >= 0 && slot < nres) {
+            if (a.ecount || (slot >= 0 && slot < nres)) {
                 float s2 = 0.f;
                 for (int c = 0; c < a.split; ++c) s2 += recv_res[(c * rows_per_rank + lo) * M + tok];
                 s += s2;
@@ -649,6 +799,14 @@ tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y,
     a.scale2 = reinterpret_cast<const __half*>(w.scale2);
     a.res_slot = w.r > 0 ? w.res_slot : nullptr;
     a.mu = reinterpret_cast<const __half*>(w.mu);
+    if (w.ecount) {
+        a.ecount = w.ecount;
+        a.ebase = w.ebase;
+        a.eidx = w.eidx;
+        a.escale = reinterpret_cast<const __half*>(w.escale);
+        a.nnz2 = w.nnz2;
+    }
+    a.nb = int32_t((w.N + kRowsPerCta - 1) / kRowsPerCta);
     a.x = x;
     a.y = y;
     a.status = async_status_word();
@@ -662,11 +820,15 @@ tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y,
     a.static_weights = (w.flags & TERN_WEIGHT_STATIC) ? 1 : 0;
     if (next) {
         const int64_t G = next->K / kGroup, rn = next->r;
-        const void* ptr[6] = {next->plane1, next->scale1, rn > 0 ? next->res_slot : nullptr,
-                              rn > 0 ? next->plane2 : nullptr, rn > 0 ? next->scale2 : nullptr, next->mu};
-        const int64_t bytes[6] = {next->N * (next->K / 4), next->N * G * 2, next->N * 4, rn * (next->K / 4),
-                                  rn * G * 2, next->N * G * 2};
-        for (int i = 0; i < 6; ++i) {
+        const bool ne = next->ecount != nullptr;
+        const void* ptr[kPrefetchRanges] = {next->plane1, next->scale1, rn > 0 ? next->res_slot : nullptr,
+                                            rn > 0 ? next->plane2 : nullptr, rn > 0 ? next->scale2 : nullptr,
+                                            next->mu, ne ? next->ecount : nullptr, ne ? next->eidx : nullptr,
+                                            ne ? next->escale : nullptr};
+        const int64_t bytes[kPrefetchRanges] = {next->N * (next->K / 4), next->N * G * 2, next->N * 4,
+                                                rn * (next->K / 4), rn * G * 2, next->N * G * 2, next->N * G,
+                                                ne ? next->nnz2 : 0, next->N * G * 2};
+        for (int i = 0; i < kPrefetchRanges; ++i) {
             a.pf_ptr[i] = static_cast<const uint8_t*>(ptr[i]);
             a.pf_bytes[i] = ptr[i] ? bytes[i] / 16 * 16 : 0;
         }

@@ -37,6 +37,11 @@ tern_status gemm_launch(const tern_weight& w, const __half* x, int64_t M, __half
                         cudaStream_t stream);
 size_t gemm_workspace_bytes(const tern_weight& w, int64_t M);
 
+// Consistency of a descriptor's element plane (tern_elem.cu): TERN_OK or TERN_ERR_ELEM.
+tern_status elem_check(const tern_weight& w, cudaStream_t stream);
+
+constexpr int kElemBlock = 64;       // rows per ebase entry of the element plane
+
 int sm_count();   // of the current device, cached per device
 
 }  // namespace tern

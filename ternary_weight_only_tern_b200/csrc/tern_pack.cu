@@ -277,12 +277,16 @@ extern "C" tern_status tern_weight_validate(const tern_weight* w, tern_stream s)
     cudaStream_t st = as_cuda(s);
     const int64_t n1 = w->N * (w->K / kCodesPerWord);
     const int64_t n2 = w->r * (w->K / kCodesPerWord);
-    return run_checked(st, [&](unsigned int* f) {
+    if (w->ecount && (w->r > 0 || !w->ebase || !w->escale || (w->nnz2 > 0 && !w->eidx))) return TERN_ERR_NULL;
+    if (w->ecount && (w->nnz2 < 0 || w->nnz2 > 0x7fffffff)) return TERN_ERR_SHAPE;
+    const tern_status cs = run_checked(st, [&](unsigned int* f) {
         validate_codes_kernel<<<grid_for(n1, 256), 256, 0, st>>>(w->plane1, n1, f);
         if (n2) validate_codes_kernel<<<grid_for(n2, 256), 256, 0, st>>>(w->plane2, n2, f);
         validate_residual_kernel<<<grid_for(w->N + w->r, 256), 256, 0, st>>>(w->res_rows, w->res_slot, w->N,
                                                                             w->r, f);
     }, TERN_ERR_BAD_CODE);
+    if (cs != TERN_OK || !w->ecount) return cs;
+    return elem_check(*w, st);
 }
 
 extern "C" tern_status tern_device_status(tern_stream s) {

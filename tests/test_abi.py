@@ -120,6 +120,18 @@ def test_linear_host_validation(lib):
     assert call(bad, fake, 1, fake * 4) == S["TERN_ERR_ALIGN"]
     bad = _lib.TernWeightC(64, 256, 128, fake, fake, 0, None, fake, None, None, 0, fake + 2)
     assert call(bad, fake, 1, fake * 4) == S["TERN_ERR_ALIGN"]    # misaligned offset
+    # element plane: exclusive with residual rows, its arrays non-null and aligned
+    E = lambda r=0, ec=fake, eb=fake, ei=fake, es=fake, nnz=5: _lib.TernWeightC(  # noqa: E731
+        64, 256, 128, fake, fake, r, fake if r else None, fake, fake if r else None, fake if r else None, 0, None,
+        ec, eb, ei, es, nnz)
+    assert call(E(r=4), fake, 1, fake * 4) == S["TERN_ERR_SHAPE"]
+    assert call(E(nnz=-1), fake, 1, fake * 4) == S["TERN_ERR_SHAPE"]
+    assert call(E(eb=None), fake, 1, fake * 4) == S["TERN_ERR_NULL"]
+    assert call(E(es=None), fake, 1, fake * 4) == S["TERN_ERR_NULL"]
+    assert call(E(ei=None), fake, 1, fake * 4) == S["TERN_ERR_NULL"]
+    assert call(E(ec=fake + 1), fake, 1, fake * 4) == S["TERN_ERR_ALIGN"]
+    assert call(E(ei=fake + 8), fake, 1, fake * 4) == S["TERN_ERR_ALIGN"]
+    assert call(E(), fake, 0, fake) == S["TERN_OK"]
     # neither path needs scratch memory
     wr = _lib.TernWeightC(64, 256, 128, fake, fake, 4, fake, fake, fake, fake, 1)
     for M in (1, 16, 17, 4096):
@@ -134,6 +146,42 @@ def test_linear_host_validation(lib):
     assert pf(_lib.TernWeightC(64, 256, 128, fake, fake, 4, fake, fake, None, fake, 0)) == S["TERN_ERR_NULL"]
     assert pf(w, M=0) == S["TERN_OK"]
     assert pf(None, M=0) == S["TERN_OK"]
+
+
+@pytest.mark.parametrize("N,K,masked,nnz2,offset", [(4096, 2560, 377487, 226492, 0), (13, 384, 250, 140, 1),
+                                                     (12288, 4096, 0, 0, 0)])
+def test_tern_bits_elem_equals_oracle(lib, N, K, masked, nnz2, offset):
+    rep = _lib.TernBitsReport()
+    assert lib.tern_bits_elem(N, K, masked, nnz2, 128, offset, ctypes.byref(rep)) == 0
+    ref = oracle.bits_elem(N, K, masked, nnz2, offset=bool(offset))
+    for f in ("weights", "plane_trits", "store_bits", "exec_bits"):
+        assert getattr(rep, f) == ref[f], f
+    for f in ("bpw_info", "bpw_store", "bpw_exec"):
+        assert getattr(rep, f) == pytest.approx(ref[f], rel=1e-15, abs=0), f
+    S = _lib.STATUS
+    assert lib.tern_bits_elem(N, K, masked, masked + 1, 128, 0, ctypes.byref(rep)) == S["TERN_ERR_SHAPE"]
+    assert lib.tern_bits_elem(N, K, N * K + 1, 0, 128, 0, ctypes.byref(rep)) == S["TERN_ERR_SHAPE"]
+    assert lib.tern_bits_elem(N, K, masked, nnz2, 128, 0, None) == S["TERN_ERR_NULL"]
+
+
+def test_elem_pack_host_validation(lib):
+    """Checks that fail before any launch."""
+    S = _lib.STATUS
+    fake = 1 << 20
+    nnz = ctypes.c_int64(7)
+    assert lib.tern_pack_elem(fake, 4, 128, fake, fake, None, 0, None, None) == S["TERN_ERR_NULL"]
+    assert lib.tern_pack_elem(fake, 4, 100, fake, fake, None, 0, ctypes.byref(nnz), None) == S["TERN_ERR_SHAPE"]
+    assert nnz.value == 0
+    assert lib.tern_pack_elem(fake, -1, 128, fake, fake, None, 0, ctypes.byref(nnz), None) == S["TERN_ERR_SHAPE"]
+    assert lib.tern_pack_elem(fake, 4, 128, fake, None, None, 0, ctypes.byref(nnz), None) == S["TERN_ERR_NULL"]
+    assert lib.tern_pack_elem(fake, 4, 128, fake, fake + 4, None, 0, ctypes.byref(nnz), None) == S["TERN_ERR_ALIGN"]
+    assert lib.tern_pack_elem(None, 4, 128, fake, fake, None, 0, ctypes.byref(nnz), None) == S["TERN_ERR_NULL"]
+    assert lib.tern_pack_elem(fake + 1, 4, 128, fake, fake, None, 0, ctypes.byref(nnz), None) == S["TERN_ERR_ALIGN"]
+    assert lib.tern_unpack_elem(fake, fake, fake, 3, 4, 100, fake, None) == S["TERN_ERR_SHAPE"]
+    assert lib.tern_unpack_elem(fake, fake, fake, -1, 4, 128, fake, None) == S["TERN_ERR_SHAPE"]
+    assert lib.tern_unpack_elem(fake, fake, None, 3, 4, 128, fake, None) == S["TERN_ERR_NULL"]
+    assert lib.tern_unpack_elem(fake, fake + 4, fake, 3, 4, 128, fake, None) == S["TERN_ERR_ALIGN"]
+    assert lib.tern_unpack_elem(fake, fake, fake, 3, 0, 128, fake, None) == S["TERN_OK"]
 
 
 def test_pack_host_validation(lib):
