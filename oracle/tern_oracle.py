@@ -33,6 +33,15 @@ integers) with numpy, with no blocking, fusion or reordering:
   its own fp16 scale per (row, group): W += s2e[n, k // 128] * T2e[n, k]. It
   is kept as a list of its nonzero trits per (row, group), defined below by
   its closed form (the layout is this library's own).
+* The activation-side rotation (an optional step before the layer): the pages'
+  KOTMS rotation puts the weights into a ternary-friendly basis with structured
+  orthogonal matrices, and inference applies the equivalent rotation to the
+  activations before the quantized linear operation (4B paper, section 4.2;
+  the measured path adds that activation-side matrix operation, section 10.1).
+  The structure is not on the pages; read here as block-diagonal with one
+  128 x 128 block per 128-wide K group (the method's group size):
+  x' = x . blockdiag(R_0, ..., R_{G-1}), so that x' . (W R)^T = x . W^T for
+  orthogonal R.
 * The product: with weights in {-1, 0, +1} the matrix product reduces to adding
   and subtracting activations ("Can Ternary LLMs Hit 1.58 Bits per Weight?",
   promptzone, section "What It Is and How It Works"); the oracle computes it
@@ -371,3 +380,22 @@ def bits_elem(N: int, K: int, masked: int, nnz2: int, group: int = GROUP, offset
         "bpw_store": store_bits / weights,
         "bpw_exec": exec_bits / weights,
     }
+
+
+# --------------------------------------------------------------------------------------
+# Activation-side rotation: y[:, 128 g + j] = sum_i x[:, 128 g + i] R[g, i, j]
+# --------------------------------------------------------------------------------------
+
+def rotate(x, R) -> np.ndarray:
+    """x [M, K] (fp16 -> float64) times the block-diagonal matrix with blocks R [K/128, 128, 128]."""
+    x = np.asarray(x, dtype=np.float64)
+    R = np.asarray(R, dtype=np.float64)
+    M, K = x.shape
+    G = K // GROUP
+    if K % GROUP or R.shape != (G, GROUP, GROUP):
+        raise ValueError("R must hold one 128 x 128 block per 128-wide group of K")
+    y = np.empty((M, K), dtype=np.float64)
+    for g in range(G):
+        cols = slice(g * GROUP, (g + 1) * GROUP)
+        y[:, cols] = x[:, cols] @ R[g]
+    return y

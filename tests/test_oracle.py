@@ -511,3 +511,63 @@ def test_planted_elem_scale_mistake_is_caught():
     yb = brute_linear(x, T1, s1, rr, T2, s2, elem=(T2e, s2e))
     assert any(abs(Fraction(float(bad[m, n])) - yb[m][n]) > Fraction(1e-9)
                for m in range(bad.shape[0]) for n in range(bad.shape[1]))
+
+
+
+# ---------------------------------------------------------------- activation-side rotation
+def _orthogonal_blocks(rng, G):
+    """G random 128 x 128 orthogonal blocks (float64, QR of a Gaussian), not symmetric."""
+    out = np.empty((G, 128, 128))
+    for g in range(G):
+        q, r = np.linalg.qr(rng.standard_normal((128, 128)))
+        out[g] = q * np.sign(np.diag(r))
+    return out
+
+
+def test_rotate_by_identity_and_signed_permutations_is_exact():
+    rng = np.random.default_rng(8)
+    x = synth.draw_x(rng, 3, 384)
+    eye = np.stack([np.eye(128)] * 3)
+    assert np.array_equal(oracle.rotate(x, eye), x.astype(np.float64))
+    # block g sends input i to output perm[g][i] with sign sgn[g][i]
+    perm = [rng.permutation(128) for _ in range(3)]
+    sgn = [rng.choice([-1.0, 1.0], 128) for _ in range(3)]
+    R = np.zeros((3, 128, 128))
+    for g in range(3):
+        for i in range(128):
+            R[g, i, perm[g][i]] = sgn[g][i]
+    y = oracle.rotate(x, R)
+    for m in range(3):
+        for g in range(3):
+            for i in range(128):
+                assert y[m, g * 128 + perm[g][i]] == sgn[g][i] * float(x[m, g * 128 + i])
+
+
+def test_rotate_matches_exact_rationals():
+    rng = np.random.default_rng(9)
+    x = synth.draw_x(rng, 2, 256)
+    R = rng.integers(-3, 4, size=(2, 128, 128)).astype(np.float64) / 8
+    y = oracle.rotate(x, R)
+    for m in range(2):
+        for g in range(2):
+            for j in range(0, 128, 17):
+                exact = sum(Fraction(float(x[m, g * 128 + i])) * Fraction(R[g, i, j]) for i in range(128))
+                assert Fraction(float(y[m, g * 128 + j])) == exact
+
+
+def test_rotated_activations_with_rotated_weights_give_the_layer():
+    """x' = x R and W' = W R (R orthogonal, block-diagonal) give x' W'^T = x W^T: the rotation
+    the pages apply to activations is the one that undoes the weights' basis change."""
+    from scipy.linalg import block_diag
+    rng = np.random.default_rng(10)
+    N, K, M = 7, 384, 3
+    x = synth.draw_x(rng, M, K)
+    W = oracle.dequant(synth.draw_trits(rng, (N, K), 0.4), synth.draw_scales(rng, N, K, 0.005, 0.02),
+                       np.zeros(0, np.int32), np.zeros((0, K), np.int8), np.zeros((0, 3), np.float16))
+    blocks = _orthogonal_blocks(rng, 3)
+    Rfull = block_diag(*blocks)
+    y = oracle.rotate(x, blocks) @ (W @ Rfull).T
+    np.testing.assert_allclose(y, x.astype(np.float64) @ W.T, rtol=0, atol=1e-12 * np.abs(W).sum())
+    # planted mistake: the transposed blocks do not undo the basis change
+    bad = oracle.rotate(x, np.transpose(blocks, (0, 2, 1))) @ (W @ Rfull).T
+    assert np.abs(bad - x.astype(np.float64) @ W.T).max() > 1e-3
