@@ -39,15 +39,15 @@ import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 
-# DRAM bytes (read + write) of one launch of the dominant kernel, from one ncu capture of the
-# `--profile gemv` case (summary and command under profiles/), keyed by a hash of the sources the
+# DRAM bytes (read + write) of one launch of the dominant kernel (the gate + up launch), from one
+# ncu capture of the `--profile gemv` case (summary and command under profiles/), keyed by a hash of the sources the
 # kernel is built from: when they change, the number no longer describes the kernel and the
 # bench reports null until it is captured again.
 KERNEL_TRAFFIC = {
     "gemv": {"sources": ["ternary_weight_only_tern_b200/csrc/tern_gemv.cu",
                          "ternary_weight_only_tern_b200/csrc/tern_device.cuh"],
-             "sha256": "0daddda56f48ec7aee53c14ca90fa7aed5e6fb7bb3b8bf9baea51a55d14a9c84",
-             "bytes": 15496192},
+             "sha256": "999783d04b7d19b94ad4c7def044890540992f9fdf51ae8fd7ef32301bb3d1f8",
+             "bytes": 30935808},
 }
 
 
@@ -68,6 +68,8 @@ WORKLOAD = "qwen3-8b-decode-stack-m1"
 RES_PCT = 15
 POOL_LAYERS = 8
 LAYERS = 36
+# projections that read the same activation run as one tern_linear_group launch
+GROUPS = [("qkv", ("q", "k", "v")), ("o", ("o",)), ("gateup", ("gate", "up")), ("down", ("down",))]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -303,7 +305,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="skip the extra measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline")
-    ap.add_argument("--profile", choices=["gemv", "gemm"], default=None,
+    ap.add_argument("--profile", choices=["gemv", "gemv_elem", "gemm"], default=None,
                     help="run a few calls of one op on one pool layer and exit (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -351,10 +353,13 @@ def main():
 
     flat_out = {}
 
+    kdim = {n: K for n, _, K in shapes}
+    ndim = {n: N for n, N, _ in shapes}
+
     def make_io(M):
-        # the 252 outputs of a step are views of one buffer, so a step's results leave the device
-        # in one copy
-        xs = {n: torch.randn((M, K), generator=gen, device=dev).half() for n, _, K in shapes}
+        # one input per group of projections that share it; the 252 outputs of a step are views of
+        # one buffer, so a step's results leave the device in one copy
+        xs = {gname: torch.randn((M, kdim[members[0]]), generator=gen, device=dev).half() for gname, members in GROUPS}
         flat = torch.empty(LAYERS * M * sum(N for _, N, _ in shapes), dtype=torch.float16, device=dev)
         ys, off = [], 0
         for _ in range(LAYERS):
@@ -366,30 +371,45 @@ def main():
         flat_out[M] = flat
         return xs, ys
 
-    def step_fn(M, xs, ys, only=None, weights=None):
-        # the calls of a step in order; each also starts bringing the next call's weight into L2
-        calls = [(layer, n) for layer in range(LAYERS) for n in names if only is None or n == only]
+    def calls_of(only=None, grouped=True):
+        # (layer, input, projections) of a step in order: a group per call, or (grouped=False)
+        # one projection per call; `only` keeps one group or one projection
+        out = []
+        for layer in range(LAYERS):
+            for gname, members in GROUPS:
+                if grouped:
+                    if only is None or only == gname:
+                        out.append((layer, gname, members))
+                else:
+                    out += [(layer, gname, (n,)) for n in members if only is None or only == n]
+        return out
+
+    def step_fn(M, xs, ys, only=None, weights=None, grouped=True):
+        # the calls of a step in order; each also starts bringing the next call's weights into L2
+        calls = calls_of(only, grouped)
         wp = weights or pool
 
         def fn():
-            for i, (layer, n) in enumerate(calls):
-                nl, nn = calls[(i + 1) % len(calls)]
-                api.linear(xs[n], wp[layer % POOL_LAYERS][n], out=ys[layer][n], workspace=ws,
-                           prefetch=wp[nl % POOL_LAYERS][nn])
+            for i, (layer, gname, members) in enumerate(calls):
+                nl, _, nm = calls[(i + 1) % len(calls)]
+                api.linear_group(xs[gname], [wp[layer % POOL_LAYERS][n] for n in members],
+                                 outs=[ys[layer][n] for n in members], workspace=ws,
+                                 prefetch=[wp[nl % POOL_LAYERS][n] for n in nm])
         return fn
 
-    def step_bytes(M, only=None, weights=None):
+    def step_bytes(M, only=None, weights=None, grouped=True):
+        # weights streamed, and activations: each call reads its input once and writes its outputs
         wp = weights or pool
-        wb = sum(packed_bytes(wp[l % POOL_LAYERS][n]) for l in range(LAYERS) for n in names
-                 if only is None or n == only)
-        ab = sum(2 * M * (K + N) for l in range(LAYERS) for (n, N, K) in shapes if only is None or n == only)
+        calls = calls_of(only, grouped)
+        wb = sum(packed_bytes(wp[layer % POOL_LAYERS][n]) for layer, _, members in calls for n in members)
+        ab = sum(2 * M * (kdim[members[0]] + sum(ndim[n] for n in members)) for _, _, members in calls)
         return wb, ab
 
     # ---------------- the timed region: K graph replays of the full M = 1 step
     xs1, ys1 = make_io(1)
     flat1 = flat_out[1]                 # the buffer behind ys1
     g_step = capture(torch, step_fn(1, xs1, ys1), stream)
-    launches_per_step = LAYERS * len(names) * launches_per_call
+    launches_per_step = len(calls_of()) * launches_per_call
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             g_step.replay()
@@ -405,19 +425,19 @@ def main():
     value = replica_value(world, wb * args.steps, secs) / 1e9
     ms_per_step = secs / args.steps * 1e3
 
-    # ---------------- the dominant op: the gate projection's tern_linear at M = 1
-    g_gate = capture(torch, step_fn(1, xs1, ys1, only="gate"), stream)
+    # ---------------- the dominant op: the gate + up launch (tern_linear_group) at M = 1
+    g_gate = capture(torch, step_fn(1, xs1, ys1, only="gateup"), stream)
     with torch.cuda.stream(stream):
         for _ in range(5):
             g_gate.replay()
     reps = max(20, min(400, args.steps // 10))
     t_gate = time_graph(torch, g_gate, reps, stream) / (reps * LAYERS)
-    gw, ga = step_bytes(1, only="gate")
+    gw, ga = step_bytes(1, only="gateup")
     gate_bytes = (gw + ga) / LAYERS
     achieved = gate_bytes / t_gate / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic("gemv"),
-                "op": "tern_linear gate 12288x4096 (+1843 residual rows) M=1",
+                "op": "tern_linear_group gate+up 2 x 12288x4096 (+1843 residual rows each) M=1",
                 "us_per_call": t_gate * 1e6, "bytes_per_call": gate_bytes, "peak_kind": peak_kind,
                 "frac_of_8000": achieved / 8000.0}
 
@@ -428,14 +448,14 @@ def main():
 
     # ---------------- e2e through the Python API with host buffers
     e2e_steps = max(3, min(20, args.steps // 100))
-    xh = {n: torch.randn((1, K)).half().pin_memory() for n, _, K in shapes}
+    xh = {gname: torch.randn((1, kdim[members[0]])).half().pin_memory() for gname, members in GROUPS}
     yh = torch.empty(flat1.numel(), dtype=torch.float16).pin_memory()
-    h2d = sum(2 * K for _, _, K in shapes)
+    h2d = sum(2 * kdim[members[0]] for _, members in GROUPS)
     d2h = LAYERS * sum(2 * N for _, N, _ in shapes)
 
     def copies_and_calls():
-        for n in names:
-            xs1[n].copy_(xh[n], non_blocking=True)
+        for gname, _ in GROUPS:
+            xs1[gname].copy_(xh[gname], non_blocking=True)
         step_fn(1, xs1, ys1)()
         yh.copy_(flat1, non_blocking=True)
 
@@ -468,8 +488,8 @@ def main():
     e2e = {"value": world * wb * e2e_steps / e2e_secs / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "steps": e2e_steps,
            "eager_value": world * wb * e2e_steps / eager_secs / 1e9,
-           "note": "252 api.linear calls per step with the step's activations copied in from pinned host memory "
-                   "and all 252 outputs (one buffer) copied back, captured once into a CUDA graph and replayed (wall clock "
+           "note": "144 api.linear_group calls per step (q+k+v, o, gate+up, down per layer) with the step's 4 "
+                   "inputs copied in from pinned host memory and all 252 outputs (one buffer) copied back, captured once into a CUDA graph and replayed (wall clock "
                    "around replay + synchronize); eager_value: the same calls issued from Python each step"}
 
     cpu = None
@@ -488,6 +508,7 @@ def main():
         "vs_baseline": None, "dtype": "f16",
         "data": "synthetic: trits P(0)=0.4, P(+-1)=0.3, fp16 group-128 scales, seeded torch generator per pool layer",
         "config": {"workload": WORKLOAD, "layers": LAYERS, "projections": names, "M": 1, "residual_pct": RES_PCT,
+                   "launches_per_layer": "q+k+v, o, gate+up, down (tern_linear_group on a shared input)",
                    "pool_layers": POOL_LAYERS, "packed_bytes_per_step": wb, "activation_bytes_per_step": ab,
                    "l2": f"inputs larger than L2: {POOL_LAYERS}-layer weight pool of "
                          f"{sum(packed_bytes(w) for L in pool for w in L.values()) / 1e6:.0f} MB rotated through",
@@ -500,38 +521,56 @@ def main():
 
 
 def profile_case(torch, api, shapes, dev, which):
-    """A minimal run for ncu: the 7 projections of two layers at M = 1 (gemv), or gate, up and
-    down at M = 2048 (gemm), each called three times in the order q, k, v, o, gate, up, down."""
-    pool = [draw_layer_on_device(torch, api, shapes, dev, seed=1000 + i) for i in range(2)]
-    names = ["q", "k", "v", "o", "gate", "up", "down"] if which == "gemv" else ["gate", "up", "down"]
-    M = 1 if which == "gemv" else 2048
-    xs = {n: torch.randn((M, K), device=dev).half() for n, _, K in shapes}
+    """A minimal run for ncu, three repetitions over two layers: at M = 1 (gemv) the bench's four
+    launches per layer (q+k+v, o, gate+up, down), or (gemv_elem) the same with element planes
+    (3.6 % masked) in place of residual rows; at M = 2048 (gemm) gate, up and down."""
+    elem = 0.036 if which == "gemv_elem" else None
+    pool = [draw_layer_on_device(torch, api, shapes, dev, seed=1000 + i, elem_frac=elem) for i in range(2)]
+    kdim = {n: K for n, _, K in shapes}
+    groups = GROUPS if which != "gemm" else [("gate", ("gate",)), ("up", ("up",)), ("down", ("down",))]
+    M = 2048 if which == "gemm" else 1
+    xs = {g: torch.randn((M, kdim[m[0]]), device=dev).half() for g, m in groups}
     ys = {n: torch.empty((M, N), dtype=torch.float16, device=dev) for n, N, _ in shapes}
     torch.cuda.synchronize()
     torch.cuda.nvtx.range_push("tern_calls")   # ncu --nvtx --nvtx-include "tern_calls/" lists these only
     for _ in range(3):
         for layer in pool:
-            for n in names:
-                api.linear(xs[n], layer[n], out=ys[n])
+            for g, members in groups:
+                api.linear_group(xs[g], [layer[n] for n in members], outs=[ys[n] for n in members])
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
-    print(json.dumps({"profile": which, "calls": 3 * len(pool) * len(names)}))
+    print(json.dumps({"profile": which, "calls": 3 * len(pool) * len(groups)}))
 
 
 def extras(torch, api, synth, pool, shapes, names, stream, dev, ws, step_fn, step_bytes, make_io, peaks,
            time_graph, capture):
     out = {}
     hbm = peaks["hbm_gbs"]
-    # per projection at M = 1
+    # per projection at M = 1 (one launch per projection), and per group (one launch per group)
     xs1, ys1 = make_io(1)
     per = {}
     for n in names:
-        g = capture(torch, step_fn(1, xs1, ys1, only=n), stream)
+        g = capture(torch, step_fn(1, xs1, ys1, only=n, grouped=False), stream)
         t = time_graph(torch, g, 50, stream) / (50 * LAYERS)
-        wb, ab = step_bytes(1, only=n)
+        wb, ab = step_bytes(1, only=n, grouped=False)
         per[n] = {"us": t * 1e6, "packed_gbs": wb / LAYERS / t / 1e9, "frac": (wb + ab) / LAYERS / t / 1e9 / hbm}
         del g
     out["per_projection_m1"] = per
+    per = {}
+    for gname, _ in GROUPS:
+        g = capture(torch, step_fn(1, xs1, ys1, only=gname), stream)
+        t = time_graph(torch, g, 50, stream) / (50 * LAYERS)
+        wb, ab = step_bytes(1, only=gname)
+        per[gname] = {"us": t * 1e6, "packed_gbs": wb / LAYERS / t / 1e9, "frac": (wb + ab) / LAYERS / t / 1e9 / hbm}
+        del g
+    out["per_group_m1"] = per
+    # the whole stack with one launch per projection (252 per step), for comparison
+    g = capture(torch, step_fn(1, xs1, ys1, grouped=False), stream)
+    t = time_graph(torch, g, 30, stream) / 30
+    wb, ab = step_bytes(1, grouped=False)
+    out["stack_m1_one_launch_per_projection"] = {"us_per_step": t * 1e6, "packed_gbs": wb / t / 1e9,
+                                                 "frac": (wb + ab) / t / 1e9 / hbm}
+    del g
     # per M over the whole stack
     perm = {}
     for M in (1, 4, 8, 16):
@@ -573,10 +612,10 @@ def extras(torch, api, synth, pool, shapes, names, stream, dev, ws, step_fn, ste
     off = {"stack_m1": {"us_per_step": t * 1e6, "packed_gbs": wb / t / 1e9, "frac": (wb + ab) / t / 1e9 / hbm,
                         "packed_bytes_per_step": wb}}
     del g, xs, ys
-    g = capture(torch, step_fn(1, xs1, ys1, only="gate", weights=mpool), stream)
+    g = capture(torch, step_fn(1, xs1, ys1, only="gateup", weights=mpool), stream)
     t = time_graph(torch, g, 50, stream) / (50 * LAYERS)
-    wb, ab = step_bytes(1, only="gate", weights=mpool)
-    off["gate_m1"] = {"us": t * 1e6, "frac": (wb + ab) / LAYERS / t / 1e9 / hbm}
+    wb, ab = step_bytes(1, only="gateup", weights=mpool)
+    off["gateup_m1"] = {"us": t * 1e6, "frac": (wb + ab) / LAYERS / t / 1e9 / hbm}
     del g
     x = torch.randn((2048, 4096), device=dev).half()
     y = torch.empty((2048, 12288), dtype=torch.float16, device=dev)
@@ -603,10 +642,10 @@ def extras(torch, api, synth, pool, shapes, names, stream, dev, ws, step_fn, ste
                        "nnz2_per_weight": float(np.mean([L[n].elem.nnz2 / (L[n].N * L[n].K) for L in epool
                                                           for n in names]))}}
     del g, xs, ys
-    g = capture(torch, step_fn(1, xs1, ys1, only="gate", weights=epool), stream)
+    g = capture(torch, step_fn(1, xs1, ys1, only="gateup", weights=epool), stream)
     t = time_graph(torch, g, 50, stream) / (50 * LAYERS)
-    wb, ab = step_bytes(1, only="gate", weights=epool)
-    el["gate_m1"] = {"us": t * 1e6, "frac": (wb + ab) / LAYERS / t / 1e9 / hbm}
+    wb, ab = step_bytes(1, only="gateup", weights=epool)
+    el["gateup_m1"] = {"us": t * 1e6, "frac": (wb + ab) / LAYERS / t / 1e9 / hbm}
     del g
     x = torch.randn((2048, 4096), device=dev).half()
     y = torch.empty((2048, 12288), dtype=torch.float16, device=dev)

@@ -193,6 +193,19 @@ tern_status tern_linear_with_prefetch(const tern_weight* w, const tern_half* x, 
                                       void* workspace, size_t workspace_bytes, const tern_weight* next,
                                       tern_stream stream);
 
+/* y[i] [M, N_i] = x [M, K] . W_i^T for n weights that share one input x (1 <= n <= 4, every
+ * W_i with the same K, and either all or none with an element plane): the projections of one
+ * activation, such as q, k and v, or gate and up.
+ * M <= 16 runs them as one decode-GEMV launch (each weight's 64-row blocks are blocks of the
+ * same grid), so the per-launch latency is paid once; larger M runs the GEMM once per weight.
+ * `next` (n_next <= 4 weights, or NULL) is prefetched into L2 as by tern_linear_with_prefetch.
+ * No y[i] may overlap x or another y[j]. The workspace rule of tern_linear holds for each W_i.
+ * Asynchronous on `stream`; capturable in a CUDA graph. w, y and next are host arrays of
+ * device descriptors and device pointers.                                                  */
+tern_status tern_linear_group(const tern_weight* const* w, int32_t n, const tern_half* x, int64_t M,
+                              tern_half* const* y, void* workspace, size_t workspace_bytes,
+                              const tern_weight* const* next, int32_t n_next, tern_stream stream);
+
 /* ---------------------------------------------------------------- bit accounting */
 
 typedef struct {

@@ -260,6 +260,36 @@ def linear(x: torch.Tensor, w: TernWeight, out: torch.Tensor | None = None,
     return out
 
 
+def linear_group(x: torch.Tensor, ws: list, outs: list | None = None, workspace: torch.Tensor | None = None,
+                 prefetch: list | None = None) -> list:
+    """[x . W_i^T for W_i in ws]: weights that share the input x (same K), one decode launch for
+    M <= 16. prefetch: the weights of the next call (a cache hint)."""
+    _need(x, torch.float16, "x")
+    M, K = x.shape
+    if not 1 <= len(ws) <= 4 or any(w.K != K for w in ws):
+        raise ValueError("linear_group takes 1 to 4 weights with the input's K")
+    if outs is None:
+        outs = [torch.empty((M, w.N), dtype=torch.float16, device=x.device) for w in ws]
+    for o, w in zip(outs, ws):
+        _need(o, torch.float16, "out")
+        if tuple(o.shape) != (M, w.N):
+            raise ValueError(f"out must have shape {(M, w.N)}, got {tuple(o.shape)}")
+    need = max(workspace_bytes(w, M) for w in ws)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    structs = [w.c_struct() for w in ws]
+    warr = (ctypes.c_void_p * len(ws))(*[ctypes.addressof(c) for c in structs])
+    yarr = (ctypes.c_void_p * len(ws))(*[o.data_ptr() for o in outs])
+    pf = list(prefetch or [])
+    pstructs = [w.c_struct() for w in pf]
+    parr = (ctypes.c_void_p * max(1, len(pf)))(*[ctypes.addressof(c) for c in pstructs])
+    _lib.check("tern_linear_group", _lib.load().tern_linear_group(
+        warr, len(ws), _ptr(x), M, yarr, _ptr(workspace), ws_bytes, parr if pf else None, len(pf),
+        _stream(x.device)))
+    return outs
+
+
 # ------------------------------------------------------------------------------ bits
 
 def bits_elem(N: int, K: int, masked: int, nnz2: int, group: int = GROUP, offset: bool = False) -> dict:

@@ -64,41 +64,76 @@ extern "C" size_t tern_linear_workspace_bytes(const tern_weight* w, int64_t M) {
 
 namespace {
 
-tern_status linear(const tern_weight* w, const tern_half* x, int64_t M, tern_half* y, void* workspace,
-                   size_t workspace_bytes, const tern_weight* next, tern_stream stream) {
-    const tern_status ws = check_weight(w);
-    if (ws != TERN_OK) return ws;
-    if (next) {
-        const tern_status ns = check_weight(next);
+bool overlap(const void* a, size_t abytes, const void* b, size_t bbytes) {
+    const uintptr_t ab = reinterpret_cast<uintptr_t>(a), bb = reinterpret_cast<uintptr_t>(b);
+    return ab < bb + bbytes && bb < ab + abytes;
+}
+
+tern_status linear_group(const tern_weight* const* w, int n, const tern_half* x, int64_t M, tern_half* const* y,
+                         void* workspace, size_t workspace_bytes, const tern_weight* const* next, int nnext,
+                         tern_stream stream) {
+    if (n < 1 || n > kMaxGemvGroup || nnext < 0 || nnext > kMaxGemvGroup) return TERN_ERR_SHAPE;
+    if (!w || !y || (nnext > 0 && !next)) return TERN_ERR_NULL;
+    for (int i = 0; i < n; ++i) {
+        const tern_status ws = check_weight(w[i]);
+        if (ws != TERN_OK) return ws;
+        if (w[i]->K != w[0]->K) return TERN_ERR_SHAPE;
+        if ((w[i]->ecount != nullptr) != (w[0]->ecount != nullptr)) return TERN_ERR_SHAPE;
+    }
+    for (int j = 0; j < nnext; ++j) {
+        const tern_status ns = check_weight(next[j]);
         if (ns != TERN_OK) return ns;
     }
     if (M < 0 || M > (int64_t(1) << 31)) return TERN_ERR_SHAPE;
     if (M == 0) return TERN_OK;
-    if (!x || !y) return TERN_ERR_NULL;
-    if (!aligned16(x) || !aligned16(y)) return TERN_ERR_ALIGN;
-    const size_t need = tern_linear_workspace_bytes(w, M);
+    if (!x) return TERN_ERR_NULL;
+    if (!aligned16(x)) return TERN_ERR_ALIGN;
+    size_t need = 0;
+    for (int i = 0; i < n; ++i) {
+        if (!y[i]) return TERN_ERR_NULL;
+        if (!aligned16(y[i])) return TERN_ERR_ALIGN;
+        const size_t b = tern_linear_workspace_bytes(w[i], M);
+        need = b > need ? b : need;
+    }
     if (need && (!workspace || workspace_bytes < need)) return TERN_ERR_WORKSPACE;
     if (workspace && !aligned16(workspace)) return TERN_ERR_ALIGN;
-    // x and y must not overlap
-    const uintptr_t xb = reinterpret_cast<uintptr_t>(x), yb = reinterpret_cast<uintptr_t>(y);
-    const uintptr_t xe = xb + size_t(M) * size_t(w->K) * 2, ye = yb + size_t(M) * size_t(w->N) * 2;
-    if (xb < ye && yb < xe) return TERN_ERR_SHAPE;
+    // no output overlaps x or another output
+    const size_t xbytes = size_t(M) * size_t(w[0]->K) * 2;
+    for (int i = 0; i < n; ++i) {
+        const size_t yi = size_t(M) * size_t(w[i]->N) * 2;
+        if (overlap(x, xbytes, y[i], yi)) return TERN_ERR_SHAPE;
+        for (int j = 0; j < i; ++j)
+            if (overlap(y[j], size_t(M) * size_t(w[j]->N) * 2, y[i], yi)) return TERN_ERR_SHAPE;
+    }
     cudaStream_t st = as_cuda(stream);
     const __half* xh = reinterpret_cast<const __half*>(x);
-    __half* yh = reinterpret_cast<__half*>(y);
-    if (M <= kGemvMaxM) return gemv_launch(*w, xh, int(M), yh, next, st);
-    return gemm_launch(*w, xh, M, yh, workspace, st);
+    __half* yh[kMaxGemvGroup];
+    for (int i = 0; i < n; ++i) yh[i] = reinterpret_cast<__half*>(y[i]);
+    if (M <= kGemvMaxM) return gemv_launch_group(w, n, xh, int(M), yh, next, nnext, st);
+    for (int i = 0; i < n; ++i) {
+        const tern_status s = gemm_launch(*w[i], xh, M, yh[i], workspace, st);
+        if (s != TERN_OK) return s;
+    }
+    return TERN_OK;
 }
 
 }  // namespace
 
+extern "C" tern_status tern_linear_group(const tern_weight* const* w, int32_t n, const tern_half* x, int64_t M,
+                                         tern_half* const* y, void* workspace, size_t workspace_bytes,
+                                         const tern_weight* const* next, int32_t n_next, tern_stream stream) {
+    return linear_group(w, n, x, M, y, workspace, workspace_bytes, next, n_next, stream);
+}
+
 extern "C" tern_status tern_linear(const tern_weight* w, const tern_half* x, int64_t M, tern_half* y,
                                    void* workspace, size_t workspace_bytes, tern_stream stream) {
-    return linear(w, x, M, y, workspace, workspace_bytes, nullptr, stream);
+    if (!w) return TERN_ERR_NULL;
+    return linear_group(&w, 1, x, M, &y, workspace, workspace_bytes, nullptr, 0, stream);
 }
 
 extern "C" tern_status tern_linear_with_prefetch(const tern_weight* w, const tern_half* x, int64_t M, tern_half* y,
                                                  void* workspace, size_t workspace_bytes, const tern_weight* next,
                                                  tern_stream stream) {
-    return linear(w, x, M, y, workspace, workspace_bytes, next, stream);
+    if (!w) return TERN_ERR_NULL;
+    return linear_group(&w, 1, x, M, &y, workspace, workspace_bytes, next ? &next : nullptr, next ? 1 : 0, stream);
 }

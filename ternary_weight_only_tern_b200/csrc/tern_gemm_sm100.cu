@@ -145,6 +145,9 @@ __device__ __forceinline__ uint32_t sw128_offset(int n, int c) {
     return uint32_t(n) * 128u + uint32_t((c ^ (n & 7)) << 4);
 }
 
+// kElem: the weight carries an element plane (a separate instantiation, so that the plain path
+// keeps its instruction stream and registers)
+template <bool kElem>
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                            const __grid_constant__ CUtensorMap tmap_p1,
                                                            const __grid_constant__ CUtensorMap tmap_p2,
@@ -303,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         // + the counts of the rows before it in that block (a scan over the warp, plus the
         // previous warp's total for the second warp of the block). Its count, the previous
         // warp's count at the same lane, the block base and s2e are queued two groups ahead.
-        const bool elem = a.ecount != nullptr;
+        constexpr bool elem = kElem;
         const bool odd = ((t >> 5) & 1) != 0;
         const int64_t eblk = (n0 + t) / kElemBlock;
         int eq_c[3] = {0, 0, 0}, eq_p[3] = {0, 0, 0}, eq_b[3] = {0, 0, 0};
@@ -524,8 +527,10 @@ tern_status gemm_launch(const tern_weight& w, const __half* x, int64_t M, __half
     {
         std::lock_guard<std::mutex> lock(mu);
         if (!configured[dev]) {
-            if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes)) !=
-                cudaSuccess)
+            if (cudaFuncSetAttribute(gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     int(kSmemBytes)) != cudaSuccess ||
+                cudaFuncSetAttribute(gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     int(kSmemBytes)) != cudaSuccess)
                 return TERN_ERR_CUDA;
             configured[dev] = true;
         }
@@ -550,7 +555,11 @@ tern_status gemm_launch(const tern_weight& w, const __half* x, int64_t M, __half
     a.G = int32_t(w.K / kGroup);
     a.y = y;
     a.status = async_status_word();
-    gemm_kernel<<<dim3(unsigned(n_tiles), unsigned(m_tiles)), kThreads, kSmemBytes, stream>>>(map, map_p1, map_p2, a);
+    const dim3 grid{unsigned(n_tiles), unsigned(m_tiles), 1u};
+    if (w.ecount)
+        gemm_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(map, map_p1, map_p2, a);
+    else
+        gemm_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(map, map_p1, map_p2, a);
     return cudaGetLastError() == cudaSuccess ? TERN_OK : TERN_ERR_CUDA;
 }
 

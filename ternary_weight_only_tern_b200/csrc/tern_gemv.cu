@@ -70,9 +70,12 @@ constexpr int kResChunkBytes = kResStrips * kStripBytes;
 constexpr int kEStageBytes = kMaxChunks * kResChunkBytes - kMaxGpc * kRowsPerCta * 4;
 static_assert(kRowsPerCta == kElemBlock, "one element-plane block per CTA");
 
-constexpr int kPrefetchRanges = 9;
+constexpr int kMaxGroup = kMaxGemvGroup;            // weights sharing x in one launch
+constexpr int kPrefetchPerWeight = 9;
+constexpr int kPrefetchRanges = kPrefetchPerWeight * kMaxGroup;
 
-struct GemvArgs {
+// One weight of the launch; its 64-row blocks are blockIdx.y in [block0, block0 + nb).
+struct GemvWeight {
     const __half* scale1;      // [N, G]
     const __half* scale2;      // [r, G]
     const int32_t* res_slot;   // [N] or nullptr
@@ -82,19 +85,34 @@ struct GemvArgs {
     const uint8_t* eidx;       // [nnz2, padded to 16] (k % 128) << 1 | (t < 0)
     const __half* escale;      // [N, G]
     int64_t nnz2;
-    int32_t nb;                // ceil(N / 64)
-    const __half* x;           // [M, K]
     __half* y;                 // [M, N]
+    int64_t N, r;
+    int32_t nb;                // ceil(N / 64)
+    int32_t block0;
+};
+
+struct GemvMaps {
+    CUtensorMap m1[kMaxGroup];     // main planes: boxes of 64 rows x 128 bytes
+    CUtensorMap m2[kMaxGroup];     // residual planes: boxes of 16 rows x 128 bytes
+};
+
+struct GemvArgs {
+    GemvWeight w[kMaxGroup];
+    int32_t nw;
+    const __half* x;           // [M, K], shared by the weights
     unsigned int* status;      // sticky timeout word
-    int64_t N, r, K;
+    int64_t K;
     int32_t G, M;
     int32_t gpc;               // groups per K-slice
     int32_t split;             // K-slices = cluster size
     int32_t static_weights;    // planes may be read before griddepcontrol.wait
     // byte ranges of the next call's weight to bring into L2 (16-byte aligned, sizes rounded down
     // to 16 bytes); every CTA prefetches its share of each
+    // (the first npf entries; each CTA takes pf_per bytes at pf_per * its linear index)
     const uint8_t* pf_ptr[kPrefetchRanges];
     int64_t pf_bytes[kPrefetchRanges];
+    int64_t pf_per[kPrefetchRanges];
+    int32_t npf;
 };
 
 struct Smem {
@@ -110,7 +128,8 @@ struct Smem {
     static constexpr int xzero = cofs + kMaxGpc * 16 * 4;                  // half [kMaxGpc * 128]: zeros
     static constexpr int smu = xzero + kMaxGpc * kGroup * 2;               // half [64][kMaxGpc]: offsets
     static constexpr int xsum = smu + kRowsPerCta * kMaxGpc * 2;           // float [kMaxGpc][16]: X_g
-    static constexpr int red = xsum + kMaxGpc * 16 * 4;                    // receive buffers, then xs
+    static constexpr int wdesc = xsum + kMaxGpc * 16 * 4;                  // this CTA's GemvWeight
+    static constexpr int red = wdesc + 128;                                // receive buffers, then xs
 };
 // Rows of the block owned by each rank, and the receive buffers: [rank][owned row][token] for the
 // main rows' partial sums and the same for their residual rows', pushed by every rank of the cluster.
@@ -196,12 +215,30 @@ __device__ __forceinline__ void strip_sums(int ng, int q, int rr, uint32_t sc, u
 }
 
 // ------------------------------------------------------------------ the kernel
-template <int NT, bool kOne>
-__global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const __grid_constant__ CUtensorMap map1,
-                                                        const __grid_constant__ CUtensorMap map2,
-                                                        const GemvArgs a) {
+// kElem: the weight carries an element plane (a separate instantiation; warp 4 then sums it)
+template <int NT, bool kOne, bool kElem>
+__global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const __grid_constant__ GemvMaps maps,
+                                                                      const __grid_constant__ GemvArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // this CTA's weight: the last whose first block is at or below blockIdx.y. Its descriptor is
+    // read from a copy in shared memory (loads that may be repeated after each barrier), not
+    // kept in registers for the whole kernel.
+    int wi = 0;
+#pragma unroll
+    for (int i = 1; i < kMaxGroup; ++i)
+        if (i < a.nw && int(blockIdx.y) >= a.w[i].block0) wi = i;
+    static_assert(sizeof(GemvWeight) <= 120 && sizeof(GemvWeight) % 8 == 0, "descriptor slot");
+    int* wsel = reinterpret_cast<int*>(smem + Smem::wdesc + 120);   // wi, for the tensor maps
+    if (threadIdx.x < sizeof(GemvWeight) / 8)
+        reinterpret_cast<uint64_t*>(smem + Smem::wdesc)[threadIdx.x] =
+            reinterpret_cast<const uint64_t*>(&a.w[wi])[threadIdx.x];
+    if (threadIdx.x == 0) *wsel = wi;
+    const GemvWeight& W = *reinterpret_cast<const GemvWeight*>(smem + Smem::wdesc);
+    // (the map addresses are formed where a copy is issued, from wi in shared memory)
+    auto map1 = [&]() { return &maps.m1[*wsel]; };
+    auto map2 = [&]() { return &maps.m2[*wsel]; };
+    const int blk = int(blockIdx.y) - a.w[wi].block0;    // 64-row block within the weight
     uint8_t* wt1 = smem + Smem::wt1;
     uint8_t* wt2 = smem + Smem::wt2;
     uint64_t* mbar1 = reinterpret_cast<uint64_t*>(smem + Smem::bar);
@@ -227,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
     const int g_begin = ks * a.gpc;
     const int ng = max(0, min(a.G, g_begin + a.gpc) - g_begin);
     const int nchunks = (ng + kChunkGroups - 1) / kChunkGroups;
-    const int64_t n0 = int64_t(blockIdx.y) * kRowsPerCta;
+    const int64_t n0 = int64_t(blk) * kRowsPerCta;
     const int xs_stride = a.gpc * kGroup;             // halves per token in smem
     bool ok = true;
 
@@ -246,15 +283,6 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
     // The next call on the stream may start now: its weight loads overlap this call, and it reads
     // x (this call's output, possibly) only after griddepcontrol.wait.
     grid_launch_dependents();
-    if (threadIdx.x == kThreads - 1) {
-        // this CTA's share of the next call's weight, into L2
-        const int64_t nctas = int64_t(gridDim.x) * gridDim.y, b = int64_t(blockIdx.y) * gridDim.x + blockIdx.x;
-        for (int i = 0; i < kPrefetchRanges; ++i) {
-            const int64_t per = ((a.pf_bytes[i] + nctas - 1) / nctas + 15) / 16 * 16;
-            const int64_t lo = b * per, hi = min(a.pf_bytes[i], lo + per);
-            if (a.pf_ptr[i] != nullptr && lo < hi) prefetch_l2_bulk(a.pf_ptr[i] + lo, uint32_t(hi - lo));
-        }
-    }
 
     int s_lo = 0, nres = 0;
     // Everything the weight determines, issued at once: TMA of the main tile (thread 0); the
@@ -263,16 +291,16 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
         if (threadIdx.x == 0)
             for (int c = 0; c < nchunks; ++c) {
                 mbar_arrive_expect_tx(&mbar1[c], kMainChunkBytes);
-                tma_load_2d(wt1 + c * kMainChunkBytes, &map1, (g_begin + c * kChunkGroups) * kWordsPerGroup,
+                tma_load_2d(wt1 + c * kMainChunkBytes, map1(), (g_begin + c * kChunkGroups) * kWordsPerGroup,
                             int(n0), &mbar1[c]);
             }
         if (warp == kMainWarps) {
             int sl0 = -1, sl1 = -1;
-            if (a.res_slot) {
-                if (n0 + lane < a.N) sl0 = a.res_slot[n0 + lane];
-                if (n0 + 32 + lane < a.N) sl1 = a.res_slot[n0 + 32 + lane];
+            if (W.res_slot) {
+                if (n0 + lane < W.N) sl0 = W.res_slot[n0 + lane];
+                if (n0 + 32 + lane < W.N) sl1 = W.res_slot[n0 + 32 + lane];
             }
-            const bool v0 = sl0 >= 0 && sl0 < a.r, v1 = sl1 >= 0 && sl1 < a.r;
+            const bool v0 = sl0 >= 0 && sl0 < W.r, v1 = sl1 >= 0 && sl1 < W.r;
             const unsigned b0 = __ballot_sync(0xffffffffu, v0);
             const unsigned b1 = __ballot_sync(0xffffffffu, v1);
             nres = __popc(b0) + __popc(b1);
@@ -292,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
                 for (int c = 0; c < nchunks && strips > 0; ++c) {
                     mbar_arrive_expect_tx(&mbar2[c], strips * kStripBytes);
                     for (int j = 0; j < strips; ++j)
-                        tma_load_2d(wt2 + c * kResChunkBytes + j * kStripBytes, &map2,
+                        tma_load_2d(wt2 + c * kResChunkBytes + j * kStripBytes, map2(),
                                     (g_begin + c * kChunkGroups) * kWordsPerGroup, s_lo + j * kStrip, &mbar2[c]);
                 }
             }
@@ -300,20 +328,28 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
             const int g = lane & 7;
             if (g < ng)
                 for (int row = lane >> 3; row < nres; row += 4)
-                    sc2[row * kMaxGpc + g] = s_lo + row < a.r ? a.scale2[int64_t(s_lo + row) * a.G + g_begin + g]
+                    sc2[row * kMaxGpc + g] = s_lo + row < W.r ? W.scale2[int64_t(s_lo + row) * a.G + g_begin + g]
                                                               : __float2half(0.f);
         } else {
             const int g = threadIdx.x & 7;
             if (g < ng)
                 for (int row = threadIdx.x >> 3; row < kRowsPerCta; row += kMainWarps * 4) {
                     const int64_t n = n0 + row;
-                    sc1[row * kMaxGpc + g] = n < a.N ? a.scale1[n * a.G + g_begin + g] : __float2half(0.f);
-                    if (a.mu) smu[row * kMaxGpc + g] = n < a.N ? a.mu[n * a.G + g_begin + g] : __float2half(0.f);
+                    sc1[row * kMaxGpc + g] = n < W.N ? W.scale1[n * a.G + g_begin + g] : __float2half(0.f);
+                    if (W.mu) smu[row * kMaxGpc + g] = n < W.N ? W.mu[n * a.G + g_begin + g] : __float2half(0.f);
                 }
         }
     };
 
     if (a.static_weights) issue_weight_reads();
+    if (threadIdx.x == kThreads - 1) {
+        // this CTA's share of the next call's weights, into L2
+        const int64_t b = int64_t(blockIdx.y) * gridDim.x + blockIdx.x;
+        for (int i = 0; i < a.npf; ++i) {
+            const int64_t lo = b * a.pf_per[i], hi = min(a.pf_bytes[i], lo + a.pf_per[i]);
+            if (lo < hi) prefetch_l2_bulk(a.pf_ptr[i] + lo, uint32_t(hi - lo));
+        }
+    }
     grid_dependency_wait();           // x (and a non-static weight) may come from the previous kernel
     if (!a.static_weights) issue_weight_reads();
 
@@ -377,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
                 cofs[(2 * q) * 16] = c[0][0] + c[1][0];
                 cofs[(2 * q + 1) * 16] = c[0][1] + c[1][1];
             }
-        } else if (warp == 1 && a.mu) {
+        } else if (warp == 1 && W.mu) {
             // X_g = sum of the group's activations: the same chain on an all-ones A
             float c[2][4];
 #pragma unroll
@@ -428,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
                 *reinterpret_cast<float2*>(cofs + gi * 16 + 8 * t + 2 * q) =
                     make_float2(c[0][t][0] + c[1][t][0], c[0][t][1] + c[1][t][1]);
         }
-        if (a.mu) {
+        if (W.mu) {
             // X_g[token] = sum of the group's activations: the same chain on an all-ones A
             const uint32_t one[4] = {kHalf2One, kHalf2One, kHalf2One, kHalf2One};
 #pragma unroll
@@ -466,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
         // every rank sends this rank M sums per owned row, and M more per owned row with a residual
         int owned_res = 0;
         for (int lo = 0; lo < nrows; ++lo) owned_res += (bslot[lr0 + lo] >= 0 && bslot[lr0 + lo] < nres) ? 1 : 0;
-        if (a.ecount) owned_res = nrows;     // the element plane sends a sum for every row
+        if (kElem) owned_res = nrows;        // the element plane sends a sum for every row
         mbar_arrive_expect_tx(rbar, uint32_t(a.split * (nrows + owned_res) * M * 4));
     }
 
@@ -508,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
         strip_sums<NT, kOne>(ng, q, rr, smem_u32(sc1 + strip_row * kMaxGpc), smem_u32(cofs), xrow,
                        [&](int c) { return smem_u32(wt1 + c * kMainChunkBytes + strip_row * 128); },
                        [&](int c) { ok = mbar_wait(&mbar1[c], 0) && ok; }, yacc);
-        if (a.mu) {
+        if (W.mu) {
             // the offset's share of the main rows: sum over the slice's groups of mu[row][g] * X_g
             const __half* ma = smu + (strip_row + rr) * kMaxGpc;
             const __half* mb = ma + 8 * kMaxGpc;
@@ -537,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
                     for (int c = 0; c < nchunks; ++c) {
                         mbar_arrive_expect_tx(&mbar2[c], strips * kStripBytes);
                         for (int j = 0; j < strips; ++j)
-                            tma_load_2d(wt2 + c * kResChunkBytes + j * kStripBytes, &map2,
+                            tma_load_2d(wt2 + c * kResChunkBytes + j * kStripBytes, map2(),
                                         (g_begin + c * kChunkGroups) * kWordsPerGroup,
                                         s_lo + (round * kResStrips + j) * kStrip, &mbar2[c]);
                     }
@@ -556,20 +592,19 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
                 store_red(true, rrow + rr, yacc);
             }
         }
-    } else if (a.ecount) {
+    } else if (kElem) {
         // Element plane of this block's 64 rows over the slice. Lane gi reads group gi's run
         // bounds, the warp copies the runs (16-byte aligned spans) into shared memory, each lane
         // finds the start of rows lane and lane + 32 in them (scan of the counts), then sums
         // +-x over its rows' listed trits per group and scales by s2e.
         constexpr int kTok = kOne ? 1 : 8 * NT;
-        const int64_t blk = blockIdx.y;
         uint8_t* ebuf = wt2;
         int* estart = reinterpret_cast<int*>(wt2 + kEStageBytes);      // [kMaxGpc][64]
         int64_t b0 = 0, b1 = 0;
         if (lane < ng) {
-            const int64_t cell = int64_t(g_begin + lane) * a.nb + blk;
-            b0 = min(max(int64_t(__ldg(a.ebase + cell)), int64_t(0)), a.nnz2);
-            b1 = min(max(int64_t(__ldg(a.ebase + cell + 1)), b0), a.nnz2);
+            const int64_t cell = int64_t(g_begin + lane) * W.nb + blk;
+            b0 = min(max(int64_t(__ldg(W.ebase + cell)), int64_t(0)), W.nnz2);
+            b1 = min(max(int64_t(__ldg(W.ebase + cell + 1)), b0), W.nnz2);
         }
         uint32_t cpk[2][2] = {{0u, 0u}, {0u, 0u}};   // counts of rows lane, lane + 32: 8 bits per group
         uint32_t spk[2][kMaxGpc / 2];                 // their scales s2e, fp16 pairs
@@ -581,10 +616,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
                 uint32_t s01 = 0u;
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
-                    if (gi + u < ng && n < a.N) {
-                        const uint32_t c = __ldg(a.ecount + int64_t(g_begin + gi + u) * a.N + n);
+                    if (gi + u < ng && n < W.N) {
+                        const uint32_t c = __ldg(W.ecount + int64_t(g_begin + gi + u) * W.N + n);
                         cpk[h][(gi + u) >> 2] |= min(c, uint32_t(kGroup)) << (8 * ((gi + u) & 3));
-                        s01 |= uint32_t(__half_as_ushort(a.escale[n * a.G + g_begin + gi + u])) << (16 * u);
+                        s01 |= uint32_t(__half_as_ushort(W.escale[n * a.G + g_begin + gi + u])) << (16 * u);
                     }
                 }
                 spk[h][gi >> 1] = s01;
@@ -609,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
                 cof[gi] = __shfl_sync(0xffffffffu, coff, gi);
                 src0[gi] = int(__shfl_sync(0xffffffffu, a0, gi) >> 4);
             }
-            const uint4* gsrc = reinterpret_cast<const uint4*>(a.eidx);
+            const uint4* gsrc = reinterpret_cast<const uint4*>(W.eidx);
             uint4* sdst = reinterpret_cast<uint4*>(ebuf);
             for (int j0 = 0; j0 < total; j0 += 64) {
                 uint4 v[2];
@@ -654,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
             estart[gi * kRowsPerCta + 32 + lane] = base + tot0 + i1 - c1;
         }
         __syncwarp();
-        const uint8_t* src = staged ? ebuf : a.eidx;
+        const uint8_t* src = staged ? ebuf : W.eidx;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int lr = lane + 32 * h;
@@ -703,16 +738,16 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
         for (int i = threadIdx.x; i < nrows * M; i += kThreads) {
             const int tok = i / nrows, lo = i - tok * nrows, lr = lr0 + lo;
             const int64_t n = n0 + lr;
-            if (n >= a.N) continue;
+            if (n >= W.N) continue;
             float s = 0.f;
             for (int c = 0; c < a.split; ++c) s += recv[(c * rows_per_rank + lo) * M + tok];
             const int slot = bslot[lr];
-            if (a.ecount || (slot >= 0 && slot < nres)) {
+            if (kElem || (slot >= 0 && slot < nres)) {
                 float s2 = 0.f;
                 for (int c = 0; c < a.split; ++c) s2 += recv_res[(c * rows_per_rank + lo) * M + tok];
                 s += s2;
             }
-            a.y[int64_t(tok) * a.N + n] = __float2half_rn(s);
+            W.y[int64_t(tok) * W.N + n] = __float2half_rn(s);
         }
     }
     if (!ok && a.status) atomicOr(a.status, 1u);
@@ -731,9 +766,8 @@ struct Plan {
     int split, gpc;
 };
 
-Plan plan_for(int64_t N, int64_t K) {
+Plan plan_for(int64_t blocks, int64_t K) {
     const int G = int(K / kGroup);
-    const int64_t blocks = (N + kRowsPerCta - 1) / kRowsPerCta;
     const int min_split = (G + kMaxGpc - 1) / kMaxGpc;
     const int64_t target = 4LL * sm_count();
     const int par = int(std::min<int64_t>(kMaxSplit, (target + blocks - 1) / blocks));
@@ -745,10 +779,9 @@ Plan plan_for(int64_t N, int64_t K) {
     return p;
 }
 
-template <int NT, bool kOne>
-tern_status launch(const CUtensorMap& m1, const CUtensorMap& m2, const GemvArgs& args, int64_t blocks, size_t smem,
-                   cudaStream_t stream) {
-    auto kernel = gemv_kernel<NT, kOne>;
+template <int NT, bool kOne, bool kElem>
+tern_status launch(const GemvMaps& maps, const GemvArgs& args, int64_t blocks, size_t smem, cudaStream_t stream) {
+    auto kernel = gemv_kernel<NT, kOne, kElem>;
     static std::mutex mu;
     static bool configured[64] = {false};
     int dev = 0;
@@ -776,7 +809,7 @@ tern_status launch(const CUtensorMap& m1, const CUtensorMap& m2, const GemvArgs&
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, kernel, m1, m2, args) != cudaSuccess) return TERN_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kernel, maps, args) != cudaSuccess) return TERN_ERR_CUDA;
     return TERN_OK;
 }
 
@@ -784,58 +817,83 @@ tern_status launch(const CUtensorMap& m1, const CUtensorMap& m2, const GemvArgs&
 
 size_t gemv_workspace_bytes(const tern_weight&, int64_t) { return 0; }
 
-tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y, const tern_weight* next,
-                        cudaStream_t stream) {
-    const Plan p = plan_for(w.N, w.K);
-    const int64_t blocks = (w.N + kRowsPerCta - 1) / kRowsPerCta;
-    if (blocks > 65535) return TERN_ERR_SHAPE;
-    CUtensorMap m1, m2;
-    if (!plane_map(&m1, w.plane1, w.N, w.K, 32, kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B)) return TERN_ERR_CUDA;
-    if (!plane_map(&m2, w.r > 0 ? w.plane2 : w.plane1, w.r > 0 ? w.r : w.N, w.K, 32, kStrip,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
-        return TERN_ERR_CUDA;
+tern_status gemv_launch_group(const tern_weight* const* ws, int nw, const __half* x, int M, __half* const* ys,
+                              const tern_weight* const* next, int nnext, cudaStream_t stream) {
+    if (nw < 1 || nw > kMaxGroup || nnext < 0 || nnext > kMaxGroup) return TERN_ERR_SHAPE;
+    GemvMaps maps;
     GemvArgs a = {};
-    a.scale1 = reinterpret_cast<const __half*>(w.scale1);
-    a.scale2 = reinterpret_cast<const __half*>(w.scale2);
-    a.res_slot = w.r > 0 ? w.res_slot : nullptr;
-    a.mu = reinterpret_cast<const __half*>(w.mu);
-    if (w.ecount) {
-        a.ecount = w.ecount;
-        a.ebase = w.ebase;
-        a.eidx = w.eidx;
-        a.escale = reinterpret_cast<const __half*>(w.escale);
-        a.nnz2 = w.nnz2;
+    int64_t blocks = 0;
+    bool elem = false, all_static = true;
+    for (int i = 0; i < nw; ++i) {
+        const tern_weight& w = *ws[i];
+        if (w.K != ws[0]->K) return TERN_ERR_SHAPE;
+        if (!plane_map(&maps.m1[i], w.plane1, w.N, w.K, 32, kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B))
+            return TERN_ERR_CUDA;
+        if (!plane_map(&maps.m2[i], w.r > 0 ? w.plane2 : w.plane1, w.r > 0 ? w.r : w.N, w.K, 32, kStrip,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+            return TERN_ERR_CUDA;
+        GemvWeight& g = a.w[i];
+        g.scale1 = reinterpret_cast<const __half*>(w.scale1);
+        g.scale2 = reinterpret_cast<const __half*>(w.scale2);
+        g.res_slot = w.r > 0 ? w.res_slot : nullptr;
+        g.mu = reinterpret_cast<const __half*>(w.mu);
+        if (w.ecount) {
+            g.ecount = w.ecount;
+            g.ebase = w.ebase;
+            g.eidx = w.eidx;
+            g.escale = reinterpret_cast<const __half*>(w.escale);
+            g.nnz2 = w.nnz2;
+            elem = true;
+        }
+        g.y = ys[i];
+        g.N = w.N;
+        g.r = w.r;
+        g.nb = int32_t((w.N + kRowsPerCta - 1) / kRowsPerCta);
+        g.block0 = int32_t(blocks);
+        blocks += g.nb;
+        all_static = all_static && (w.flags & TERN_WEIGHT_STATIC);
     }
-    a.nb = int32_t((w.N + kRowsPerCta - 1) / kRowsPerCta);
+    if (blocks > 65535) return TERN_ERR_SHAPE;
+    const Plan p = plan_for(blocks, ws[0]->K);
+    a.nw = nw;
     a.x = x;
-    a.y = y;
     a.status = async_status_word();
-    a.N = w.N;
-    a.r = w.r;
-    a.K = w.K;
-    a.G = int32_t(w.K / kGroup);
+    a.K = ws[0]->K;
+    a.G = int32_t(ws[0]->K / kGroup);
     a.M = M;
     a.gpc = p.gpc;
     a.split = p.split;
-    a.static_weights = (w.flags & TERN_WEIGHT_STATIC) ? 1 : 0;
-    if (next) {
-        const int64_t G = next->K / kGroup, rn = next->r;
-        const bool ne = next->ecount != nullptr;
-        const void* ptr[kPrefetchRanges] = {next->plane1, next->scale1, rn > 0 ? next->res_slot : nullptr,
-                                            rn > 0 ? next->plane2 : nullptr, rn > 0 ? next->scale2 : nullptr,
-                                            next->mu, ne ? next->ecount : nullptr, ne ? next->eidx : nullptr,
-                                            ne ? next->escale : nullptr};
-        const int64_t bytes[kPrefetchRanges] = {next->N * (next->K / 4), next->N * G * 2, next->N * 4,
-                                                rn * (next->K / 4), rn * G * 2, next->N * G * 2, next->N * G,
-                                                ne ? next->nnz2 : 0, next->N * G * 2};
-        for (int i = 0; i < kPrefetchRanges; ++i) {
-            a.pf_ptr[i] = static_cast<const uint8_t*>(ptr[i]);
-            a.pf_bytes[i] = ptr[i] ? bytes[i] / 16 * 16 : 0;
+    a.static_weights = all_static ? 1 : 0;
+    for (int j = 0; j < nnext; ++j) {
+        const tern_weight* nx = next[j];
+        const int64_t G = nx->K / kGroup, rn = nx->r;
+        const bool ne = nx->ecount != nullptr;
+        const void* ptr[kPrefetchPerWeight] = {nx->plane1, nx->scale1, rn > 0 ? nx->res_slot : nullptr,
+                                               rn > 0 ? nx->plane2 : nullptr, rn > 0 ? nx->scale2 : nullptr,
+                                               nx->mu, ne ? nx->ecount : nullptr, ne ? nx->eidx : nullptr,
+                                               ne ? nx->escale : nullptr};
+        const int64_t bytes[kPrefetchPerWeight] = {nx->N * (nx->K / 4), nx->N * G * 2, nx->N * 4, rn * (nx->K / 4),
+                                                   rn * G * 2, nx->N * G * 2, nx->N * G, ne ? nx->nnz2 : 0,
+                                                   nx->N * G * 2};
+        for (int i = 0; i < kPrefetchPerWeight; ++i) {
+            const int64_t b16 = bytes[i] / 16 * 16;
+            if (!ptr[i] || b16 <= 0) continue;
+            a.pf_ptr[a.npf] = static_cast<const uint8_t*>(ptr[i]);
+            a.pf_bytes[a.npf] = b16;
+            ++a.npf;
         }
     }
+    const int64_t nctas = int64_t(p.split) * blocks;
+    for (int i = 0; i < a.npf; ++i) a.pf_per[i] = ((a.pf_bytes[i] + nctas - 1) / nctas + 15) / 16 * 16;
     const size_t smem = smem_bytes(M);
-    if (M == 1) return launch<1, true>(m1, m2, a, blocks, smem, stream);
-    return M <= 8 ? launch<1, false>(m1, m2, a, blocks, smem, stream) : launch<2, false>(m1, m2, a, blocks, smem, stream);
+    if (elem) {
+        if (M == 1) return launch<1, true, true>(maps, a, blocks, smem, stream);
+        return M <= 8 ? launch<1, false, true>(maps, a, blocks, smem, stream)
+                      : launch<2, false, true>(maps, a, blocks, smem, stream);
+    }
+    if (M == 1) return launch<1, true, false>(maps, a, blocks, smem, stream);
+    return M <= 8 ? launch<1, false, false>(maps, a, blocks, smem, stream)
+                  : launch<2, false, false>(maps, a, blocks, smem, stream);
 }
 
 }  // namespace tern

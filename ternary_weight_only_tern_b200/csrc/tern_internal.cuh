@@ -26,10 +26,12 @@ tern_status read_flag_slot(unsigned int* slot, cudaStream_t stream, unsigned int
 // that ran out set it); nullptr on a CUDA error.
 unsigned int* async_status_word();
 
-// Decode GEMV on a thread-block cluster per 64-row block (tern_gemv.cu), M in [1, 16]. When
-// `next` is not null the launch also prefetches its planes, scales and slot map into L2.
-tern_status gemv_launch(const tern_weight& w, const __half* x, int M, __half* y, const tern_weight* next,
-                        cudaStream_t stream);
+// Decode GEMV on a thread-block cluster per 64-row block (tern_gemv.cu), M in [1, 16], for
+// 1..kMaxGemvGroup weights of the same K that share x (one launch; output i is ys[i]). The
+// launch also prefetches the planes, scales and slot maps of the `nnext` weights `next` into L2.
+constexpr int kMaxGemvGroup = 4;
+tern_status gemv_launch_group(const tern_weight* const* ws, int nw, const __half* x, int M, __half* const* ys,
+                              const tern_weight* const* next, int nnext, cudaStream_t stream);
 size_t gemv_workspace_bytes(const tern_weight& w, int64_t M);
 
 // Prefill GEMM on tcgen05 (tern_gemm_sm100.cu), M > 16.

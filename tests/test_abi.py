@@ -184,6 +184,33 @@ def test_elem_pack_host_validation(lib):
     assert lib.tern_unpack_elem(fake, fake, fake, 3, 0, 128, fake, None) == S["TERN_OK"]
 
 
+def test_linear_group_host_validation(lib):
+    """Checks of tern_linear_group that fail before a launch."""
+    S = _lib.STATUS
+    fake = 1 << 20
+    mk = lambda N=64, K=256, ec=None: _lib.TernWeightC(64 if N is None else N, K, 128, fake, fake, 0, None, fake,  # noqa
+                                                        None, None, 0, None, ec, fake if ec else None,
+                                                        fake if ec else None, fake if ec else None, 0)
+    w1, w2 = mk(), mk(N=32)
+    arr = lambda *ws: (ctypes.c_void_p * len(ws))(*[ctypes.addressof(w) for w in ws])  # noqa: E731
+    ys = lambda *ps: (ctypes.c_void_p * len(ps))(*ps)  # noqa: E731
+    g = lambda w, n, M, y, x=fake: lib.tern_linear_group(w, n, x, M, y, None, 0, None, 0, None)  # noqa: E731
+    Y = ys(fake * 4, fake * 8)
+    assert g(arr(w1, w2), 0, 1, Y) == S["TERN_ERR_SHAPE"]
+    assert g(arr(w1, w2, w1, w2, w1), 5, 1, ys(*[fake * 4] * 5)) == S["TERN_ERR_SHAPE"]
+    assert g(None, 2, 1, Y) == S["TERN_ERR_NULL"]
+    assert g(arr(w1, w2), 2, 1, None) == S["TERN_ERR_NULL"]
+    assert g(arr(w1, mk(K=384)), 2, 1, Y) == S["TERN_ERR_SHAPE"]                  # K differs
+    assert g(arr(w1, mk(ec=fake)), 2, 1, Y) == S["TERN_ERR_SHAPE"]                # element plane on one only
+    assert g(arr(w1, w2), 2, 1, ys(fake * 4, fake * 4 + 64)) == S["TERN_ERR_SHAPE"]   # outputs overlap
+    assert g(arr(w1, w2), 2, 1, ys(fake * 4, fake)) == S["TERN_ERR_SHAPE"]        # an output overlaps x
+    assert g(arr(w1, w2), 2, 1, ys(fake * 4, fake * 8 + 2)) == S["TERN_ERR_ALIGN"]
+    assert g(arr(w1, w2), 2, 1, ys(fake * 4, None)) == S["TERN_ERR_NULL"]
+    assert g(arr(w1, w2), 2, 0, Y) == S["TERN_OK"]                                # M == 0 is a no-op
+    assert lib.tern_linear_group(arr(w1, w2), 2, fake, 1, Y, None, 0, None, 1, None) == S["TERN_ERR_NULL"]
+    assert lib.tern_linear_group(arr(w1, w2), 2, fake, 1, Y, None, 0, arr(mk(K=100)), 1, None) == S["TERN_ERR_SHAPE"]
+
+
 def test_pack_host_validation(lib):
     S = _lib.STATUS
     fake = 1 << 20

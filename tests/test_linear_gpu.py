@@ -283,3 +283,72 @@ def test_offset_8b_gate_full_size(M):
     y_ref = oracle.linear(t.x[:M], t.T1, t.s1, t.res_rows, t.T2, t.s2, cols=cols, mu=mu)
     y, _ = run_mu(t, mu, M)
     check(y[:, cols], y_ref)
+
+
+# ---------------------------------------------------------------- weights sharing one input
+def _group_tensors(rng, shapes, M, res_pct=10):
+    x = synth.draw_x(rng, M, shapes[0][1])
+    out = []
+    for N, K in shapes:
+        t = synth.draw_tensor(rng, "g", N, K, 1, p_zero=0.4, res_pct=res_pct)
+        out.append(synth.TernTensor("g", N, K, x, t.T1, t.s1, t.res_rows, t.T2, t.s2))
+    return x, out
+
+
+@pytest.mark.parametrize("M", [1, 3, 8, 16, 17, 40])
+@pytest.mark.parametrize("which", ["qkv", "gateup"])
+def test_group_matches_oracle(M, which):
+    names = ["q", "k", "v"] if which == "qkv" else ["gate", "up"]
+    rng = np.random.default_rng(M + len(which))
+    x, ts = _group_tensors(rng, [synth.QWEN3_8B[n] for n in names], M, res_pct=15)
+    ws = [api.TernWeight.from_numpy(t.T1, t.s1, t.res_rows, t.T2, t.s2) for t in ts]
+    ys = api.linear_group(torch.from_numpy(x).cuda(), ws)
+    torch.cuda.synchronize()
+    for y, t in zip(ys, ts):
+        check(y.cpu().numpy(), oracle.linear(x, t.T1, t.s1, t.res_rows, t.T2, t.s2))
+
+
+@pytest.mark.parametrize("M", [1, 4, 16, 24])
+def test_group_exact_case_bit_exact(M):
+    rng = np.random.default_rng(900 + M)
+    ts = [synth.draw_exact_tensor(rng, N, 1536, M, r) for N, r in [(300, 17), (64, 0), (1000 + 7, 100), (130, 130)]]
+    x = ts[0].x
+    ws = [api.TernWeight.from_numpy(t.T1, t.s1, t.res_rows, t.T2, t.s2) for t in ts]
+    ys = api.linear_group(torch.from_numpy(x).cuda(), ws)
+    torch.cuda.synchronize()
+    for y, t in zip(ys, ts):
+        y_ref = oracle.round_fp16(oracle.linear(x, t.T1, t.s1, t.res_rows, t.T2, t.s2))
+        assert np.array_equal(y.cpu().numpy().view(np.uint16), y_ref.view(np.uint16))
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+def test_group_of_one_is_tern_linear_and_prefetch_changes_nothing(M):
+    rng = np.random.default_rng(70 + M)
+    t = synth.draw_tensor(rng, "g1", 1000 + 7, 2560, M, p_zero=0.4, res_pct=10)
+    w = api.TernWeight.from_numpy(t.T1, t.s1, t.res_rows, t.T2, t.s2)
+    x = torch.from_numpy(t.x).cuda()
+    y0 = api.linear(x, w)
+    (y1,) = api.linear_group(x, [w])
+    (y2,) = api.linear_group(x, [w], prefetch=[w, w, w])
+    torch.cuda.synchronize()
+    assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
+    assert torch.equal(y0.view(torch.int16), y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("M", [1, 9, 300])
+def test_group_with_offsets_and_element_planes(M):
+    rng = np.random.default_rng(55 + M)
+    x = synth.draw_x(rng, M, 2560)
+    refs, ws = [], []
+    for N in (512, 130, 1000 + 7):
+        T1 = synth.draw_trits(rng, (N, 2560), 0.4)
+        s1 = synth.draw_scales(rng, N, 2560, 0.005, 0.02)
+        T2e, s2e, _ = synth.draw_elem_plane(rng, N, 2560)
+        mu = synth.draw_offsets(rng, N, 2560)
+        none = (np.zeros(0, np.int32), np.zeros((0, 2560), np.int8), np.zeros((0, 20), np.float16))
+        ws.append(api.TernWeight.from_numpy(T1, s1, *none, mu=mu, T2e=T2e, s2e=s2e))
+        refs.append(oracle.linear(x, T1, s1, *none, mu=mu, elem=(T2e, s2e)))
+    ys = api.linear_group(torch.from_numpy(x).cuda(), ws)
+    torch.cuda.synchronize()
+    for y, y_ref in zip(ys, refs):
+        check(y.cpu().numpy(), y_ref)
