@@ -305,7 +305,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="skip the extra measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline")
-    ap.add_argument("--profile", choices=["gemv", "gemv_elem", "gemm"], default=None,
+    ap.add_argument("--profile", choices=["gemv", "gemv_elem", "gemm", "rotate"], default=None,
                     help="run a few calls of one op on one pool layer and exit (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -384,15 +384,19 @@ def main():
                     out += [(layer, gname, (n,)) for n in members if only is None or only == n]
         return out
 
-    def step_fn(M, xs, ys, only=None, weights=None, grouped=True):
-        # the calls of a step in order; each also starts bringing the next call's weights into L2
+    def step_fn(M, xs, ys, only=None, weights=None, grouped=True, rot=None):
+        # the calls of a step in order; each also starts bringing the next call's weights into L2.
+        # rot: per layer {input: (R, buffer)}: each call's input is first rotated (tern_rotate)
         calls = calls_of(only, grouped)
         wp = weights or pool
 
         def fn():
             for i, (layer, gname, members) in enumerate(calls):
                 nl, _, nm = calls[(i + 1) % len(calls)]
-                api.linear_group(xs[gname], [wp[layer % POOL_LAYERS][n] for n in members],
+                x_in = xs[gname]
+                if rot is not None:
+                    x_in = api.rotate(x_in, rot[layer][gname][0], out=rot[layer][gname][1])
+                api.linear_group(x_in, [wp[layer % POOL_LAYERS][n] for n in members],
                                  outs=[ys[layer][n] for n in members], workspace=ws,
                                  prefetch=[wp[nl % POOL_LAYERS][n] for n in nm])
         return fn
@@ -524,6 +528,20 @@ def profile_case(torch, api, shapes, dev, which):
     """A minimal run for ncu, three repetitions over two layers: at M = 1 (gemv) the bench's four
     launches per layer (q+k+v, o, gate+up, down), or (gemv_elem) the same with element planes
     (3.6 % masked) in place of residual rows; at M = 2048 (gemm) gate, up and down."""
+    if which == "rotate":
+        # tern_rotate on K = 4096 at M = 1 and M = 2048, three times
+        R = (torch.randn((32, 128, 128), device=dev) / 11.3).half()
+        xs = [torch.randn((M, 4096), device=dev).half() for M in (1, 2048)]
+        ys = [torch.empty_like(x) for x in xs]
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_push("tern_calls")
+        for _ in range(3):
+            for x, y in zip(xs, ys):
+                api.rotate(x, R, out=y)
+        torch.cuda.nvtx.range_pop()
+        torch.cuda.synchronize()
+        print(json.dumps({"profile": which, "calls": 6}))
+        return
     elem = 0.036 if which == "gemv_elem" else None
     pool = [draw_layer_on_device(torch, api, shapes, dev, seed=1000 + i, elem_frac=elem) for i in range(2)]
     kdim = {n: K for n, _, K in shapes}
@@ -545,6 +563,7 @@ def profile_case(torch, api, shapes, dev, which):
 def extras(torch, api, synth, pool, shapes, names, stream, dev, ws, step_fn, step_bytes, make_io, peaks,
            time_graph, capture):
     out = {}
+    kdim_of = {n: K for n, _, K in shapes}.__getitem__
     hbm = peaks["hbm_gbs"]
     # per projection at M = 1 (one launch per projection), and per group (one launch per group)
     xs1, ys1 = make_io(1)
@@ -599,6 +618,37 @@ def extras(torch, api, synth, pool, shapes, names, stream, dev, ws, step_fn, ste
                    "frac_sustained": fl / t / 1e12 / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])}
         del g, x, y, wsg
     out["gemm_m2048"] = gemm
+    # the activation-side rotation (tern_rotate, one 128 x 128 fp16 block per group): alone at M = 1
+    # and M = 2048 on K = 4096 and 12288, and the M = 1 stack with a rotation before every launch
+    # (its own blocks for each input of each of the 36 layers: 216 MB, more than L2)
+    rot = {}
+    for K in (4096, 12288):
+        R = (torch.randn((K // 128, 128, 128), device=dev) / 11.3).half()
+        for M in (1, 2048):
+            x = torch.randn((M, K), device=dev).half()
+            y = torch.empty_like(x)
+
+            def fn_rot(x=x, R=R, y=y):
+                for _ in range(20):
+                    api.rotate(x, R, out=y)
+            g = capture(torch, fn_rot, stream)
+            t = time_graph(torch, g, 20, stream) / 400
+            nbytes = R.numel() * 2 + 2 * x.numel() * 2
+            rot[f"K{K}_M{M}"] = {"us": t * 1e6, "gbs": nbytes / t / 1e9, "frac_hbm": nbytes / t / 1e9 / hbm,
+                                 "tflops": 2.0 * M * K * 128 / t / 1e12}
+            del g, x, y
+    xs, ys = make_io(1)
+    bufs = {gname: torch.empty_like(xs[gname]) for gname, _ in GROUPS}
+    rots = [{gname: ((torch.randn((kdim_of(members[0]) // 128, 128, 128), device=dev) / 11.3).half(), bufs[gname])
+             for gname, members in GROUPS} for _ in range(LAYERS)]
+    g = capture(torch, step_fn(1, xs, ys, rot=rots), stream)
+    t = time_graph(torch, g, 30, stream) / 30
+    wb, ab = step_bytes(1)
+    rb = sum(r.numel() * 2 for L in rots for r, _ in L.values())
+    rot["stack_m1_with_rotation"] = {"us_per_step": t * 1e6, "packed_gbs": wb / t / 1e9,
+                                     "bytes_gbs": (wb + rb) / t / 1e9, "rotation_bytes_per_step": rb}
+    out["rotation"] = rot
+    del g, xs, ys, rots
     # the per-group offset mu (W = mu + s1 T1 + s2 T2): the same pool with an fp16 offset per
     # (row, group) drawn U[-0.01, 0.01], the M = 1 stack and the gate GEMM at M = 2048
     gm = torch.Generator(device=dev)

@@ -206,6 +206,21 @@ tern_status tern_linear_group(const tern_weight* const* w, int32_t n, const tern
                               tern_half* const* y, void* workspace, size_t workspace_bytes,
                               const tern_weight* const* next, int32_t n_next, tern_stream stream);
 
+/* ---------------------------------------------------------------- activation rotation */
+
+/* y [M, K] = x [M, K] . blockdiag(R_0, ..., R_{G-1}) (x, y, R device, fp16, row-major): the
+ * rotation that inference applies to the activations before the linear layer when the
+ * weights were moved into a rotated basis ("Post-Training Ternarization of Qwen3-4B", section
+ * 4.2: KOTMS uses structured orthogonal matrices, and the equivalent rotation is applied to the
+ * activations; section 10.1). This library reads the structure as block-diagonal with one
+ * 128 x 128 block per 128-wide group of K: R is [K/128, 128, 128] with
+ * y[m, 128 g + j] = sum_i x[m, 128 g + i] R[g, i, j], fp32 accumulation, one rounding to fp16.
+ * K % 128 == 0; x and y must not overlap. Asynchronous on `stream`; capturable in a CUDA graph.
+ * The next kernel on the stream may start while this one runs (programmatic dependent launch):
+ * tern_linear reads its x only after this kernel has finished.                           */
+tern_status tern_rotate(const tern_half* x, int64_t M, int64_t K, const tern_half* R, tern_half* y,
+                        tern_stream stream);
+
 /* ---------------------------------------------------------------- bit accounting */
 
 typedef struct {

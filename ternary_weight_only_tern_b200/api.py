@@ -290,6 +290,23 @@ def linear_group(x: torch.Tensor, ws: list, outs: list | None = None, workspace:
     return outs
 
 
+def rotate(x: torch.Tensor, R: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """x [M, K] . blockdiag(R[0], ..., R[K/128 - 1]) with R fp16 [K/128, 128, 128] (tern_rotate)."""
+    _need(x, torch.float16, "x")
+    _need(R, torch.float16, "R", ndim=3)
+    M, K = x.shape
+    if tuple(R.shape) != (K // GROUP, GROUP, GROUP) or K % GROUP:
+        raise ValueError(f"R must have shape {(K // GROUP, GROUP, GROUP)}")
+    if out is None:
+        out = torch.empty_like(x)
+    else:
+        _need(out, torch.float16, "out")
+        if tuple(out.shape) != (M, K):
+            raise ValueError(f"out must have shape {(M, K)}")
+    _lib.check("tern_rotate", _lib.load().tern_rotate(_ptr(x), M, K, _ptr(R), _ptr(out), _stream(x.device)))
+    return out
+
+
 # ------------------------------------------------------------------------------ bits
 
 def bits_elem(N: int, K: int, masked: int, nnz2: int, group: int = GROUP, offset: bool = False) -> dict:

@@ -211,6 +211,19 @@ def test_linear_group_host_validation(lib):
     assert lib.tern_linear_group(arr(w1, w2), 2, fake, 1, Y, None, 0, arr(mk(K=100)), 1, None) == S["TERN_ERR_SHAPE"]
 
 
+def test_rotate_host_validation(lib):
+    S = _lib.STATUS
+    fake = 1 << 20
+    assert lib.tern_rotate(fake, 4, 100, fake * 2, fake * 4, None) == S["TERN_ERR_SHAPE"]
+    assert lib.tern_rotate(fake, -1, 128, fake * 2, fake * 4, None) == S["TERN_ERR_SHAPE"]
+    assert lib.tern_rotate(fake, 0, 128, None, None, None) == S["TERN_OK"]
+    assert lib.tern_rotate(None, 4, 128, fake * 2, fake * 4, None) == S["TERN_ERR_NULL"]
+    assert lib.tern_rotate(fake, 4, 128, None, fake * 4, None) == S["TERN_ERR_NULL"]
+    assert lib.tern_rotate(fake + 2, 4, 128, fake * 2, fake * 4, None) == S["TERN_ERR_ALIGN"]
+    assert lib.tern_rotate(fake, 4, 128, fake * 2 + 8, fake * 4, None) == S["TERN_ERR_ALIGN"]
+    assert lib.tern_rotate(fake, 4, 128, fake * 2, fake + 256, None) == S["TERN_ERR_SHAPE"]   # x, y overlap
+
+
 def test_pack_host_validation(lib):
     S = _lib.STATUS
     fake = 1 << 20
