@@ -42,6 +42,19 @@ integers) with numpy, with no blocking, fusion or reordering:
   128 x 128 block per 128-wide K group (the method's group size):
   x' = x . blockdiag(R_0, ..., R_{G-1}), so that x' . (W R)^T = x . W^T for
   orthogonal R.
+* The ternarization fit (an optional step before packing): E2M-ATQ fits an
+  asymmetric offset and two ternary planes with scales, then refines them for 15
+  iterations with the ternary supports held fixed (4B paper, section 4.3). Its
+  equations are not on the pages. Read here, per (row, 128-wide group), as:
+  the offset is the group mean; each plane is the sign of the residual where
+  its magnitude exceeds 0.7 times the residual's mean magnitude (the threshold
+  rule of ternary weight networks), with the mean magnitude over that support
+  as its scale; the second plane fits the first plane's residual, on the rows
+  that carry one; the refinement updates the offset, then a1, then a2, each to
+  its least-squares value with the others and both planes fixed. Every sum runs
+  in float64 over the group's 128 entries in index order, and each of the four
+  operations is rounded on its own (no fused multiply-add), so the CUDA path
+  reaches every decision with the same numbers.
 * The product: with weights in {-1, 0, +1} the matrix product reduces to adding
   and subtracting activations ("Can Ternary LLMs Hit 1.58 Bits per Weight?",
   promptzone, section "What It Is and How It Works"); the oracle computes it
@@ -399,3 +412,63 @@ def rotate(x, R) -> np.ndarray:
         cols = slice(g * GROUP, (g + 1) * GROUP)
         y[:, cols] = x[:, cols] @ R[g]
     return y
+
+
+# --------------------------------------------------------------------------------------
+# Ternarization fit (per row and 128-wide group; see the module docstring)
+# --------------------------------------------------------------------------------------
+TWN_RATIO = 0.7
+
+
+def _seq_sum(a: np.ndarray) -> np.ndarray:
+    """Sum over the last axis, in index order, in float64 (not numpy's pairwise order)."""
+    acc = np.zeros(a.shape[:-1], dtype=np.float64)
+    for k in range(a.shape[-1]):
+        acc = acc + a[..., k]
+    return acc
+
+
+def _threshold_plane(r: np.ndarray):
+    """Plane and scale of residual r [..., 128]: t = sign(r) where |r| > 0.7 mean|r|; a = mean |r| on it."""
+    delta = TWN_RATIO * (_seq_sum(np.abs(r)) / GROUP)
+    t = ((r > delta[..., None]).astype(np.int8) - (r < -delta[..., None]).astype(np.int8)).astype(np.int8)
+    n = np.count_nonzero(t, axis=-1)
+    s = _seq_sum(np.where(t != 0, np.abs(r), 0.0))
+    a = np.where(n > 0, s / np.maximum(n, 1), 0.0)
+    return t, a, n
+
+
+def fit_groups(w: np.ndarray, has2: np.ndarray, offset: bool, iters: int):
+    """The fit of groups w [..., 128] (float64); has2 [...] marks groups with a second plane.
+    Returns (T1, a1, mu, T2, a2) with the scales and the offset in float64."""
+    mu = _seq_sum(w) / GROUP if offset else np.zeros(w.shape[:-1])
+    r = w - mu[..., None]
+    T1, a1, n1 = _threshold_plane(r)
+    e = r - a1[..., None] * T1
+    T2, a2, n2 = _threshold_plane(e)
+    T2[~has2] = 0
+    a2[~has2] = 0.0
+    n2[~has2] = 0
+    for _ in range(iters):
+        if offset:
+            mu = _seq_sum((w - a1[..., None] * T1) - a2[..., None] * T2) / GROUP
+        a1 = np.where(n1 > 0, _seq_sum(((w - mu[..., None]) - a2[..., None] * T2) * T1) / np.maximum(n1, 1), 0.0)
+        a2 = np.where(n2 > 0, _seq_sum(((w - mu[..., None]) - a1[..., None] * T1) * T2) / np.maximum(n2, 1), 0.0)
+    return T1, a1, mu, T2, a2
+
+
+def ternarize(W, res_rows=None, offset: bool = True, iters: int = 15):
+    """Dense W [N, K] (fp16 -> float64, exact) -> (T1 int8 [N, K], s1 fp16 [N, G], mu fp16 [N, G] or
+    None, T2 int8 [r, K], s2 fp16 [r, G]) with the second plane on the sorted rows res_rows; each
+    scale and offset is rounded once to fp16."""
+    W = np.asarray(W, dtype=np.float16).astype(np.float64)
+    N, K = W.shape
+    if K % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    G = K // GROUP
+    res_rows = np.zeros(0, np.int64) if res_rows is None else np.asarray(res_rows, dtype=np.int64)
+    has2 = np.zeros((N, G), dtype=bool)
+    has2[res_rows] = True
+    T1, a1, mu, T2, a2 = fit_groups(W.reshape(N, G, GROUP), has2, offset, iters)
+    return (T1.reshape(N, K), a1.astype(np.float16), mu.astype(np.float16) if offset else None,
+            T2.reshape(N, K)[res_rows], a2[res_rows].astype(np.float16))

@@ -571,3 +571,81 @@ def test_rotated_activations_with_rotated_weights_give_the_layer():
     # planted mistake: the transposed blocks do not undo the basis change
     bad = oracle.rotate(x, np.transpose(blocks, (0, 2, 1))) @ (W @ Rfull).T
     assert np.abs(bad - x.astype(np.float64) @ W.T).max() > 1e-3
+
+
+
+# ---------------------------------------------------------------- ternarization fit
+def _hand_group():
+    """64 entries of 1.0 and 64 of fp16(0.4), no offset. Worked by hand: mean |w| = (64 + 64 x 0.4)
+    / 128 ~ 0.7, threshold 0.49: the first plane holds the ones (a1 = 1); its residual is 0.4 on
+    the other half, mean 0.2, threshold 0.14: the second plane holds them (a2 = fp16(0.4)); the
+    refinement keeps both, and mu + a1 T1 + a2 T2 = w exactly."""
+    w = np.array([1.0] * 64 + [0.4] * 64, dtype=np.float16)
+    return w, np.array([1] * 64 + [0] * 64, np.int8), np.array([0] * 64 + [1] * 64, np.int8)
+
+
+def test_fit_hand_worked_group():
+    w, t1, t2 = _hand_group()
+    T1, a1, mu, T2, a2 = oracle.fit_groups(w.astype(np.float64)[None], np.array([True]), False, 15)
+    assert np.array_equal(T1[0], t1) and np.array_equal(T2[0], t2)
+    assert a1[0] == 1.0 and a2[0] == float(np.float16(0.4)) and mu[0] == 0.0
+
+
+def test_planted_threshold_mistake_is_caught(monkeypatch):
+    """A fit with the threshold at 0.5 mean |r| puts the 0.4 entries into the first plane."""
+    w, t1, _ = _hand_group()
+    monkeypatch.setattr(O, "TWN_RATIO", 0.5)
+    T1, *_ = O.fit_groups(w.astype(np.float64)[None], np.array([True]), False, 15)
+    assert not np.array_equal(T1[0], t1)
+
+
+def test_fit_recovers_an_exactly_ternary_group_with_offset():
+    rng = np.random.default_rng(12)
+    t = np.array([-1] * 40 + [0] * 48 + [1] * 40, np.int8)
+    rng.shuffle(t)
+    w = (0.25 + 0.5 * t).astype(np.float16).astype(np.float64)
+    T1, a1, mu, T2, a2 = oracle.fit_groups(w[None], np.array([False]), True, 15)
+    assert np.array_equal(T1[0], t) and a1[0] == 0.5 and mu[0] == 0.25 and not T2.any() and a2[0] == 0.0
+
+
+def test_refinement_reaches_least_squares_and_never_increases_the_error():
+    rng = np.random.default_rng(13)
+    w = (rng.standard_normal((6, 128)) * 0.02 + 0.003).astype(np.float16).astype(np.float64)
+    has2 = np.array([True, False, True, True, False, True])
+    errs = []
+    for it in (0, 1, 2, 5, 15):
+        T1, a1, mu, T2, a2 = oracle.fit_groups(w, has2, True, it)
+        errs.append(((w - mu[:, None] - a1[:, None] * T1 - a2[:, None] * T2) ** 2).sum(axis=1))
+    for e0, e1 in zip(errs, errs[1:]):
+        assert np.all(e1 <= e0 * (1 + 1e-12) + 1e-300)
+    T1, a1, mu, T2, a2 = oracle.fit_groups(w, has2, True, 400)
+    for g in range(6):
+        cols = [np.ones(128), T1[g].astype(np.float64)] + ([T2[g].astype(np.float64)] if has2[g] else [])
+        sol = np.linalg.lstsq(np.stack(cols, axis=1), w[g], rcond=None)[0]
+        assert abs(sol[0] - mu[g]) < 1e-9 and abs(sol[1] - a1[g]) < 1e-9
+        if has2[g]:
+            assert abs(sol[2] - a2[g]) < 1e-9
+
+
+def test_fit_of_zero_and_constant_groups():
+    w = np.stack([np.zeros(128), np.full(128, 0.125)])
+    T1, a1, mu, T2, a2 = oracle.fit_groups(w, np.array([True, True]), True, 15)
+    assert not T1.any() and not T2.any() and np.all(a1 == 0) and np.all(a2 == 0)
+    assert mu[0] == 0 and mu[1] == 0.125
+
+
+def test_ternarize_assembles_rows_and_groups():
+    """ternarize is fit_groups over (row, group), with the second plane on the listed rows only."""
+    rng = np.random.default_rng(14)
+    W = (rng.standard_normal((9, 384)) * 0.02).astype(np.float16)
+    rows = np.array([2, 5, 8])
+    T1, s1, mu, T2, s2 = oracle.ternarize(W, rows)
+    for n in range(9):
+        for g in range(3):
+            t1, a1, m, t2, a2 = oracle.fit_groups(W[n, g * 128:(g + 1) * 128].astype(np.float64)[None],
+                                                  np.array([n in rows]), True, 15)
+            assert np.array_equal(T1[n, g * 128:(g + 1) * 128], t1[0])
+            assert s1[n, g] == np.float16(a1[0]) and mu[n, g] == np.float16(m[0])
+            if n in rows:
+                i = list(rows).index(n)
+                assert np.array_equal(T2[i, g * 128:(g + 1) * 128], t2[0]) and s2[i, g] == np.float16(a2[0])
