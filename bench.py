@@ -708,6 +708,23 @@ def extras(torch, api, synth, pool, shapes, names, stream, dev, ws, step_fn, ste
     el["gate_m2048"] = {"us": t * 1e6, "tflops": fl / t / 1e12, "frac_burst": fl / t / 1e12 / peaks["bf16_tflops"]}
     out["elem_plane"] = el
     del g, x, y, epool
+    # the ternarization fit on the gate shape (12288 x 4096 fp16, 15 % residual rows, offset, 15 rounds)
+    Wd = (torch.randn((12288, 4096), device=dev) * 0.02).half()
+    frows = torch.randperm(12288, device=dev)[:1843].sort().values.to(torch.int32)
+    api.fit(Wd, frows)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(3):
+        T1f, s1f, muf, T2f, s2f = api.fit(Wd, frows)
+    torch.cuda.synchronize()
+    dt = (time.perf_counter() - t0) / 3
+    What = (s1f.float().repeat_interleave(128, 1) * T1f.float() + muf.float().repeat_interleave(128, 1))
+    What[frows.long()] += s2f.float().repeat_interleave(128, 1) * T2f.float()
+    rel = float(((What - Wd.float()).norm() / Wd.float().norm()).item())
+    out["fit_gate"] = {"ms": dt * 1e3, "w_gbs": Wd.numel() * 2 / dt / 1e9, "groups_per_s": 12288 * 32 / dt,
+                       "relative_frobenius_error": rel,
+                       "note": "tern_fit, float64 sums; wall clock of 3 calls after a warm-up"}
+    del Wd, frows, T1f, s1f, muf, T2f, s2f, What
     # packing throughput on the gate shape
     u = torch.randint(0, 3, (12288, 4096), dtype=torch.int8, device=dev) - 1
     for fn_name, fn in (("pack_exec", api.pack_exec), ("pack_store", api.pack_store)):

@@ -169,6 +169,21 @@ tern_status tern_unpack_elem(const uint8_t* ecount, const int32_t* ebase, const 
  * own memory accesses in bounds when a slot is out of range.                            */
 tern_status tern_weight_validate(const tern_weight* w, tern_stream stream);
 
+/* Dense fp16 W [N, K] (device) -> the ternary form: T1 int8 [N, K], s1 [N, K/128], with
+ * offset != 0 mu [N, K/128], and on the rows n with res_slot[n] = j >= 0 (res_slot [N], as
+ * tern_weight.res_slot, or NULL when r == 0) T2[j] int8 [K] and s2[j] [K/128]. Per (row, 128-wide
+ * group): mu = the group mean (0 without an offset), T1 = sign(w - mu) where |w - mu| exceeds 0.7
+ * times its mean, a1 = the mean magnitude on that support, T2 and a2 the same on the residual
+ * w - mu - a1 T1, then `iters` rounds of least-squares updates of mu, a1 and a2 in turn with the
+ * planes fixed; sums in float64 in index order, each scale and offset rounded once to fp16.
+ * This is the fit the pages call E2M-ATQ (an asymmetric offset, two ternary planes with scales,
+ * 15 refinement iterations with the supports fixed: "Post-Training Ternarization of Qwen3-4B",
+ * section 4.3) in this library's reading of it (the pages give no equations). The outputs feed
+ * tern_pack_exec. W, T1 and T2 16-byte aligned; 0 <= iters <= 1000. Asynchronous on `stream`. */
+tern_status tern_fit(const tern_half* W, int64_t N, int64_t K, const int32_t* res_slot, int64_t r, int32_t offset,
+                     int32_t iters, int8_t* T1, tern_half* s1, tern_half* mu, int8_t* T2, tern_half* s2,
+                     tern_stream stream);
+
 /* ---------------------------------------------------------------- the linear layer */
 
 /* Bytes of workspace tern_linear needs for this weight and batch size (0 if none). */

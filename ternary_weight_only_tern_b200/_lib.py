@@ -31,6 +31,8 @@ EXPORTS = {
                                              _c.c_size_t, _c.c_void_p, _c.c_void_p]),
     "tern_linear_group": (_c.c_int, [_c.c_void_p, _c.c_int32, _c.c_void_p, _c.c_int64, _c.c_void_p, _c.c_void_p,
                                      _c.c_size_t, _c.c_void_p, _c.c_int32, _c.c_void_p]),
+    "tern_fit": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_int64, _c.c_void_p, _c.c_int64, _c.c_int32, _c.c_int32,
+                            _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p]),
     "tern_rotate": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_int64, _c.c_void_p, _c.c_void_p, _c.c_void_p]),
     "tern_bits": (_c.c_int, [_c.c_int64, _c.c_int64, _c.c_int64, _c.c_int32, _c.c_void_p]),
     "tern_bits_offset": (_c.c_int, [_c.c_int64, _c.c_int64, _c.c_int64, _c.c_int32, _c.c_void_p]),

@@ -290,6 +290,30 @@ def linear_group(x: torch.Tensor, ws: list, outs: list | None = None, workspace:
     return outs
 
 
+def fit(W: torch.Tensor, res_rows: torch.Tensor | None = None, offset: bool = True, iters: int = 15):
+    """Dense fp16 W [N, K] -> (T1 int8 [N, K], s1 [N, K/128], mu [N, K/128] or None, T2 int8 [r, K],
+    s2 [r, K/128]) by tern_fit, the second plane on the sorted rows res_rows."""
+    _need(W, torch.float16, "W")
+    N, K = W.shape
+    dev = W.device
+    G = K // GROUP
+    if res_rows is None or res_rows.numel() == 0:
+        res_rows = torch.zeros(0, dtype=torch.int32, device=dev)
+    res_rows = res_rows.to(device=dev, dtype=torch.int32).contiguous()
+    r = int(res_rows.numel())
+    slot = torch.full((N,), -1, dtype=torch.int32, device=dev)
+    if r:
+        slot[res_rows.long()] = torch.arange(r, dtype=torch.int32, device=dev)
+    T1 = torch.empty((N, K), dtype=torch.int8, device=dev)
+    s1 = torch.empty((N, G), dtype=torch.float16, device=dev)
+    mu = torch.empty((N, G), dtype=torch.float16, device=dev) if offset else None
+    T2 = torch.empty((r, K), dtype=torch.int8, device=dev)
+    s2 = torch.empty((r, G), dtype=torch.float16, device=dev)
+    _lib.check("tern_fit", _lib.load().tern_fit(_ptr(W), N, K, _ptr(slot) if r else None, r, int(offset), iters,
+                                                _ptr(T1), _ptr(s1), _ptr(mu), _ptr(T2), _ptr(s2), _stream(dev)))
+    return T1, s1, mu, T2, s2
+
+
 def rotate(x: torch.Tensor, R: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
     """x [M, K] . blockdiag(R[0], ..., R[K/128 - 1]) with R fp16 [K/128, 128, 128] (tern_rotate)."""
     _need(x, torch.float16, "x")

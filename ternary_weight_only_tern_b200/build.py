@@ -22,7 +22,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libtern.so")
 SOURCES = ["tern_api.cu", "tern_pack.cu", "tern_elem.cu", "tern_gemv.cu", "tern_gemm_sm100.cu",
-           "tern_rotate.cu", "tern_bits.cpp"]
+           "tern_rotate.cu", "tern_fit.cu", "tern_bits.cpp"]
 HEADERS = ["tern_internal.cuh", "tern_device.cuh", os.path.join("..", "..", "include", "tern.h")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -211,6 +211,22 @@ def test_linear_group_host_validation(lib):
     assert lib.tern_linear_group(arr(w1, w2), 2, fake, 1, Y, None, 0, arr(mk(K=100)), 1, None) == S["TERN_ERR_SHAPE"]
 
 
+def test_fit_host_validation(lib):
+    S = _lib.STATUS
+    f = 1 << 20
+    fit = lambda W=f, N=4, K=256, slot=None, r=0, off=1, it=15, T1=f * 2, s1=f * 3, mu=f * 4, T2=None, s2=None: \
+        lib.tern_fit(W, N, K, slot, r, off, it, T1, s1, mu, T2, s2, None)  # noqa: E731
+    assert fit(K=200) == S["TERN_ERR_SHAPE"]
+    assert fit(r=5) == S["TERN_ERR_SHAPE"]
+    assert fit(it=-1) == S["TERN_ERR_SHAPE"]
+    assert fit(N=0) == S["TERN_OK"]
+    assert fit(W=None) == S["TERN_ERR_NULL"]
+    assert fit(mu=None) == S["TERN_ERR_NULL"]                   # an offset needs mu
+    assert fit(r=2, slot=f * 5) == S["TERN_ERR_NULL"]           # residual rows need T2 and s2
+    assert fit(W=f + 2) == S["TERN_ERR_ALIGN"]
+    assert fit(T1=f * 2 + 8) == S["TERN_ERR_ALIGN"]
+
+
 def test_rotate_host_validation(lib):
     S = _lib.STATUS
     fake = 1 << 20
