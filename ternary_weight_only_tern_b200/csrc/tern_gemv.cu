@@ -65,9 +65,11 @@ constexpr int kMaxSplit = 16;
 constexpr int kMainChunkBytes = kRowsPerCta * 128;  // 8 KB
 constexpr int kStripBytes = kStrip * 128;           // 2 KB
 constexpr int kResChunkBytes = kResStrips * kStripBytes;
-// element plane: its staged runs and per-row starts live in the residual tile's space, which
-// that form does not use
-constexpr int kEStageBytes = kMaxChunks * kResChunkBytes - kMaxGpc * kRowsPerCta * 4;
+// element plane: its staged runs, per-row starts, counts and scales and the run ends live in the
+// residual tile's space, which that form does not use
+constexpr int kEMetaBytes = kMaxGpc * kRowsPerCta * (4 + 1 + 2) + kMaxGpc * 8;
+constexpr int kEStageBytes = (kMaxChunks * kResChunkBytes - kEMetaBytes) / 16 * 16;
+static_assert(kEStageBytes > 0, "element-plane staging space");
 static_assert(kRowsPerCta == kElemBlock, "one element-plane block per CTA");
 
 constexpr int kMaxGroup = kMaxGemvGroup;            // weights sharing x in one launch
@@ -600,6 +602,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
         constexpr int kTok = kOne ? 1 : 8 * NT;
         uint8_t* ebuf = wt2;
         int* estart = reinterpret_cast<int*>(wt2 + kEStageBytes);      // [kMaxGpc][64]
+        uint8_t* ecnt = wt2 + kEStageBytes + kMaxGpc * kRowsPerCta * 4;  // [kMaxGpc][64]
+        __half* esc = reinterpret_cast<__half*>(ecnt + kMaxGpc * kRowsPerCta);   // [kMaxGpc][64]
+        int64_t* erend = reinterpret_cast<int64_t*>(esc + kMaxGpc * kRowsPerCta);  // [kMaxGpc]
         int64_t b0 = 0, b1 = 0;
         if (lane < ng) {
             const int64_t cell = int64_t(g_begin + lane) * W.nb + blk;
@@ -687,11 +692,24 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
             const int base = int(__shfl_sync(0xffffffffu, rbase, gi));
             estart[gi * kRowsPerCta + lane] = base + i0 - c0;
             estart[gi * kRowsPerCta + 32 + lane] = base + tot0 + i1 - c1;
+            const int64_t run_end = __shfl_sync(0xffffffffu, rend, gi);
+            if (NT == 1) {
+                // for the block-wide pass below: counts, scales and the run end of each cell
+                ecnt[gi * kRowsPerCta + lane] = uint8_t(c0);
+                ecnt[gi * kRowsPerCta + 32 + lane] = uint8_t(c1);
+                esc[gi * kRowsPerCta + lane] =
+                    __ushort_as_half(static_cast<unsigned short>((spk[0][gi >> 1] >> (16 * (gi & 1))) & 0xffffu));
+                esc[gi * kRowsPerCta + 32 + lane] =
+                    __ushort_as_half(static_cast<unsigned short>((spk[1][gi >> 1] >> (16 * (gi & 1))) & 0xffffu));
+                if (lane == 0) erend[gi] = run_end;
+            }
         }
         __syncwarp();
         const uint8_t* src = staged ? ebuf : W.eidx;
+        if (NT == 1 && lane == 0) misc[2] = staged ? 1 : 0;
+        // M > 8: this warp sums the listed trits itself; M <= 8: every warp does, below
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < 2 && NT == 2; ++h) {
             const int lr = lane + 32 * h;
             float acc[kTok];
 #pragma unroll
@@ -727,6 +745,54 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
 #pragma unroll
             for (int t = 0; t < kTok; ++t)
                 if (t < M) push(recv_res, lr, t, acc[t]);
+        }
+    }
+
+    if (kElem && NT == 1) {
+        // Element plane, M <= 8: all 160 threads take (group, row) cells once the main strips are
+        // done and warp 4 has staged the runs; each cell's scaled sum goes to shared memory (in
+        // the main tile's space, now free), then each (row, token) adds its cells in group order
+        // and sends the sum to the owning rank.
+        asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
+        const uint8_t* ebuf = wt2;
+        const int* estart = reinterpret_cast<const int*>(wt2 + kEStageBytes);
+        const uint8_t* ecnt = wt2 + kEStageBytes + kMaxGpc * kRowsPerCta * 4;
+        const __half* esc = reinterpret_cast<const __half*>(ecnt + kMaxGpc * kRowsPerCta);
+        const int64_t* erend = reinterpret_cast<const int64_t*>(esc + kMaxGpc * kRowsPerCta);
+        const uint8_t* src = misc[2] ? ebuf : W.eidx;
+        float* csum = reinterpret_cast<float*>(wt1);            // [cell][M], M <= 8
+        constexpr int kTok = kOne ? 1 : 8;
+        for (int c = threadIdx.x; c < ng * kRowsPerCta; c += kThreads) {
+            const int gi = c / kRowsPerCta;
+            const int cnt = ecnt[c], st = estart[c];
+            const int64_t end = erend[gi];
+            float gs[kTok];
+#pragma unroll
+            for (int t = 0; t < kTok; ++t) gs[t] = 0.f;
+            for (int e = 0; e < cnt; ++e) {
+                if (st + e >= end) break;       // only with inconsistent counts
+                const uint32_t v = src[st + e];
+                const uint32_t kk = v >> 1, w = kk >> 4, j = kk & 15;
+                const int off = gi * kGroup + int((((w & 1) << 2) | (w >> 1)) * 16 + (((j & 7) << 1) | (j >> 3)));
+#pragma unroll
+                for (int t = 0; t < kTok; ++t) {
+                    if (t < M) {
+                        const float xv = __half2float(xs[size_t(t) * xs_stride + off]);
+                        gs[t] += (v & 1) ? -xv : xv;
+                    }
+                }
+            }
+            const float sc = __half2float(esc[c]);
+#pragma unroll
+            for (int t = 0; t < kTok; ++t)
+                if (t < M) csum[c * M + t] = sc * gs[t];
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
+        for (int i = threadIdx.x; i < kRowsPerCta * M; i += kThreads) {
+            const int lr = i % kRowsPerCta, t = i / kRowsPerCta;
+            float sum = 0.f;
+            for (int gi = 0; gi < ng; ++gi) sum += csum[(gi * kRowsPerCta + lr) * M + t];
+            push(recv_res, lr, t, sum);
         }
     }
 
