@@ -46,8 +46,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 KERNEL_TRAFFIC = {
     "gemv": {"sources": ["ternary_weight_only_tern_b200/csrc/tern_gemv.cu",
                          "ternary_weight_only_tern_b200/csrc/tern_device.cuh"],
-             "sha256": "999783d04b7d19b94ad4c7def044890540992f9fdf51ae8fd7ef32301bb3d1f8",
-             "bytes": 30935808},
+             "sha256": "f47ea014a055ec5a5e16a0607e089581d4f638a7192d8a77076031b29d9b63e8",
+             "bytes": 30926336},
 }
 
 
