@@ -286,6 +286,90 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
     // x (this call's output, possibly) only after griddepcontrol.wait.
     grid_launch_dependents();
 
+    // Element plane of this block's 64 rows over the slice, staged by warp 4 with the other weight
+    // reads: lane gi reads group gi's run bounds, the warp copies the runs (16-byte aligned spans)
+    // into the residual tile's space with cp.async (or leaves them in global memory when they do
+    // not fit), and each (group, row) cell's start, count and scale go to shared memory.
+    auto elem_stage = [&]() {
+        uint8_t* ebuf = wt2;
+        int* estart = reinterpret_cast<int*>(wt2 + kEStageBytes);                // [kMaxGpc][64]
+        uint8_t* ecnt = wt2 + kEStageBytes + kMaxGpc * kRowsPerCta * 4;          // [kMaxGpc][64]
+        __half* esc = reinterpret_cast<__half*>(ecnt + kMaxGpc * kRowsPerCta);   // [kMaxGpc][64]
+        int64_t* erend = reinterpret_cast<int64_t*>(esc + kMaxGpc * kRowsPerCta);  // [kMaxGpc]
+        int64_t b0 = 0, b1 = 0;
+        if (lane < ng) {
+            const int64_t cell = int64_t(g_begin + lane) * W.nb + blk;
+            b0 = min(max(int64_t(__ldg(W.ebase + cell)), int64_t(0)), W.nnz2);
+            b1 = min(max(int64_t(__ldg(W.ebase + cell + 1)), b0), W.nnz2);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int64_t n = n0 + lane + 32 * h;
+            for (int gi = 0; gi < kMaxGpc; ++gi) {
+                uint32_t c = 0;
+                __half sc = __float2half(0.f);
+                if (gi < ng && n < W.N) {
+                    c = min(uint32_t(__ldg(W.ecount + int64_t(g_begin + gi) * W.N + n)), uint32_t(kGroup));
+                    sc = W.escale[n * a.G + g_begin + gi];
+                }
+                ecnt[gi * kRowsPerCta + lane + 32 * h] = uint8_t(c);
+                esc[gi * kRowsPerCta + lane + 32 * h] = sc;
+            }
+        }
+        const int64_t a0 = b0 & ~int64_t(15), a1 = (b1 + 15) & ~int64_t(15);
+        const int nchunk = lane < ng ? int((a1 - a0) >> 4) : 0;
+        int coff = nchunk;                             // inclusive scan of the chunk counts
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, coff, o);
+            if (lane >= o) coff += u;
+        }
+        const int total = __shfl_sync(0xffffffffu, coff, 31);
+        coff -= nchunk;
+        const bool staged = total * 16 <= kEStageBytes;
+        if (staged) {
+            // chunk j of the copy belongs to the last group whose first chunk is <= j
+            int cof[kMaxGpc], src0[kMaxGpc];
+#pragma unroll
+            for (int gi = 0; gi < kMaxGpc; ++gi) {
+                cof[gi] = __shfl_sync(0xffffffffu, coff, gi);
+                src0[gi] = int(__shfl_sync(0xffffffffu, a0, gi) >> 4);
+            }
+            for (int j = lane; j < total; j += 32) {
+                int from = src0[0] + j - cof[0];
+#pragma unroll
+                for (int q2 = 1; q2 < kMaxGpc; ++q2)
+                    if (q2 < ng && cof[q2] <= j) from = src0[q2] + j - cof[q2];
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(ebuf + 16 * j)),
+                             "l"(W.eidx + int64_t(from) * 16)
+                             : "memory");
+            }
+        }
+        // run base of each group in the source: the staged copy or the global list
+        const int64_t rbase = staged ? int64_t(coff) * 16 + (b0 - a0) : b0;
+        const int64_t rend = rbase + (b1 - b0);
+        __syncwarp();
+        for (int gi = 0; gi < ng; ++gi) {
+            const int c0 = ecnt[gi * kRowsPerCta + lane], c1 = ecnt[gi * kRowsPerCta + 32 + lane];
+            int i0 = c0, i1 = c1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u0 = __shfl_up_sync(0xffffffffu, i0, o), u1 = __shfl_up_sync(0xffffffffu, i1, o);
+                if (lane >= o) {
+                    i0 += u0;
+                    i1 += u1;
+                }
+            }
+            const int tot0 = __shfl_sync(0xffffffffu, i0, 31);
+            const int base = int(__shfl_sync(0xffffffffu, rbase, gi));
+            const int64_t run_end = __shfl_sync(0xffffffffu, rend, gi);
+            estart[gi * kRowsPerCta + lane] = base + i0 - c0;
+            estart[gi * kRowsPerCta + 32 + lane] = base + tot0 + i1 - c1;
+            if (lane == 0) erend[gi] = run_end;
+        }
+        if (lane == 0) misc[2] = staged ? 1 : 0;
+    };
+
     int s_lo = 0, nres = 0;
     // Everything the weight determines, issued at once: TMA of the main tile (thread 0); the
     // block's residual slots, their TMA and scales (warp 4); the main scales (warps 0-3).
@@ -326,6 +410,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
                                     (g_begin + c * kChunkGroups) * kWordsPerGroup, s_lo + j * kStrip, &mbar2[c]);
                 }
             }
+            if (kElem) elem_stage();
             // residual scales: lane g of each 8-lane quarter loads group g of rows quarter, +4, ...
             const int g = lane & 7;
             if (g < ng)
@@ -595,164 +680,60 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const _
             }
         }
     } else if (kElem) {
-        // Element plane of this block's 64 rows over the slice. Lane gi reads group gi's run
-        // bounds, the warp copies the runs (16-byte aligned spans) into shared memory, each lane
-        // finds the start of rows lane and lane + 32 in them (scan of the counts), then sums
-        // +-x over its rows' listed trits per group and scales by s2e.
-        constexpr int kTok = kOne ? 1 : 8 * NT;
-        uint8_t* ebuf = wt2;
-        int* estart = reinterpret_cast<int*>(wt2 + kEStageBytes);      // [kMaxGpc][64]
-        uint8_t* ecnt = wt2 + kEStageBytes + kMaxGpc * kRowsPerCta * 4;  // [kMaxGpc][64]
-        __half* esc = reinterpret_cast<__half*>(ecnt + kMaxGpc * kRowsPerCta);   // [kMaxGpc][64]
-        int64_t* erend = reinterpret_cast<int64_t*>(esc + kMaxGpc * kRowsPerCta);  // [kMaxGpc]
-        int64_t b0 = 0, b1 = 0;
-        if (lane < ng) {
-            const int64_t cell = int64_t(g_begin + lane) * W.nb + blk;
-            b0 = min(max(int64_t(__ldg(W.ebase + cell)), int64_t(0)), W.nnz2);
-            b1 = min(max(int64_t(__ldg(W.ebase + cell + 1)), b0), W.nnz2);
-        }
-        uint32_t cpk[2][2] = {{0u, 0u}, {0u, 0u}};   // counts of rows lane, lane + 32: 8 bits per group
-        uint32_t spk[2][kMaxGpc / 2];                 // their scales s2e, fp16 pairs
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int64_t n = n0 + lane + 32 * h;
-#pragma unroll
-            for (int gi = 0; gi < kMaxGpc; gi += 2) {
-                uint32_t s01 = 0u;
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    if (gi + u < ng && n < W.N) {
-                        const uint32_t c = __ldg(W.ecount + int64_t(g_begin + gi + u) * W.N + n);
-                        cpk[h][(gi + u) >> 2] |= min(c, uint32_t(kGroup)) << (8 * ((gi + u) & 3));
-                        s01 |= uint32_t(__half_as_ushort(W.escale[n * a.G + g_begin + gi + u])) << (16 * u);
-                    }
-                }
-                spk[h][gi >> 1] = s01;
-            }
-        }
-        const int64_t a0 = b0 & ~int64_t(15), a1 = (b1 + 15) & ~int64_t(15);
-        const int nchunk = lane < ng ? int((a1 - a0) >> 4) : 0;
-        int coff = nchunk;                             // inclusive scan of the chunk counts
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int u = __shfl_up_sync(0xffffffffu, coff, o);
-            if (lane >= o) coff += u;
-        }
-        const int total = __shfl_sync(0xffffffffu, coff, 31);
-        coff -= nchunk;
-        const bool staged = total * 16 <= kEStageBytes;
-        if (staged) {
-            // chunk j of the copy belongs to the last group whose first chunk is <= j
-            int cof[kMaxGpc], src0[kMaxGpc];
-#pragma unroll
-            for (int gi = 0; gi < kMaxGpc; ++gi) {
-                cof[gi] = __shfl_sync(0xffffffffu, coff, gi);
-                src0[gi] = int(__shfl_sync(0xffffffffu, a0, gi) >> 4);
-            }
-            const uint4* gsrc = reinterpret_cast<const uint4*>(W.eidx);
-            uint4* sdst = reinterpret_cast<uint4*>(ebuf);
-            for (int j0 = 0; j0 < total; j0 += 64) {
-                uint4 v[2];
-                int dj[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int j = j0 + 32 * u + lane;
-                    dj[u] = -1;
-                    if (j < total) {
-                        int from = src0[0] + j - cof[0];
-#pragma unroll
-                        for (int q2 = 1; q2 < kMaxGpc; ++q2)
-                            if (q2 < ng && cof[q2] <= j) from = src0[q2] + j - cof[q2];
-                        v[u] = __ldg(gsrc + from);
-                        dj[u] = j;
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 2; ++u)
-                    if (dj[u] >= 0) sdst[dj[u]] = v[u];
-            }
-        }
-        // run base of each group in the source: the staged copy or the global list
-        const int64_t rbase = staged ? int64_t(coff) * 16 + (b0 - a0) : b0;
-        const int64_t rend = rbase + (b1 - b0);
-#pragma unroll
-        for (int gi = 0; gi < kMaxGpc; ++gi) {
-            if (gi >= ng) break;
-            const int c0 = (cpk[0][gi >> 2] >> (8 * (gi & 3))) & 0xff, c1 = (cpk[1][gi >> 2] >> (8 * (gi & 3))) & 0xff;
-            int i0 = c0, i1 = c1;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int u0 = __shfl_up_sync(0xffffffffu, i0, o), u1 = __shfl_up_sync(0xffffffffu, i1, o);
-                if (lane >= o) {
-                    i0 += u0;
-                    i1 += u1;
-                }
-            }
-            const int tot0 = __shfl_sync(0xffffffffu, i0, 31);
-            const int base = int(__shfl_sync(0xffffffffu, rbase, gi));
-            estart[gi * kRowsPerCta + lane] = base + i0 - c0;
-            estart[gi * kRowsPerCta + 32 + lane] = base + tot0 + i1 - c1;
-            const int64_t run_end = __shfl_sync(0xffffffffu, rend, gi);
-            if (NT == 1) {
-                // for the block-wide pass below: counts, scales and the run end of each cell
-                ecnt[gi * kRowsPerCta + lane] = uint8_t(c0);
-                ecnt[gi * kRowsPerCta + 32 + lane] = uint8_t(c1);
-                esc[gi * kRowsPerCta + lane] =
-                    __ushort_as_half(static_cast<unsigned short>((spk[0][gi >> 1] >> (16 * (gi & 1))) & 0xffffu));
-                esc[gi * kRowsPerCta + 32 + lane] =
-                    __ushort_as_half(static_cast<unsigned short>((spk[1][gi >> 1] >> (16 * (gi & 1))) & 0xffffu));
-                if (lane == 0) erend[gi] = run_end;
-            }
-        }
+        // Element plane: the runs were staged with cp.async at the start (elem_stage); M > 8: this
+        // warp sums +-x over its rows' listed trits per group and scales by s2e; M <= 8: every
+        // warp does, below.
+        asm volatile("cp.async.wait_all;" ::: "memory");
         __syncwarp();
-        const uint8_t* src = staged ? ebuf : W.eidx;
-        if (NT == 1 && lane == 0) misc[2] = staged ? 1 : 0;
-        // M > 8: this warp sums the listed trits itself; M <= 8: every warp does, below
+        if (NT == 2) {
+            constexpr int kTok = 8 * NT;
+            const uint8_t* src = misc[2] ? wt2 : W.eidx;
+            const int* estart = reinterpret_cast<const int*>(wt2 + kEStageBytes);
+            const uint8_t* ecnt = wt2 + kEStageBytes + kMaxGpc * kRowsPerCta * 4;
+            const __half* esc = reinterpret_cast<const __half*>(ecnt + kMaxGpc * kRowsPerCta);
+            const int64_t* erend = reinterpret_cast<const int64_t*>(esc + kMaxGpc * kRowsPerCta);
 #pragma unroll
-        for (int h = 0; h < 2 && NT == 2; ++h) {
-            const int lr = lane + 32 * h;
-            float acc[kTok];
+            for (int h = 0; h < 2; ++h) {
+                const int lr = lane + 32 * h;
+                float acc[kTok];
 #pragma unroll
-            for (int t = 0; t < kTok; ++t) acc[t] = 0.f;
+                for (int t = 0; t < kTok; ++t) acc[t] = 0.f;
+                for (int gi = 0; gi < ng; ++gi) {
+                    const int c = ecnt[gi * kRowsPerCta + lr], st = estart[gi * kRowsPerCta + lr];
+                    const int64_t end = erend[gi];
+                    float gs[kTok];
 #pragma unroll
-            for (int gi = 0; gi < kMaxGpc; ++gi) {
-                if (gi >= ng) break;
-                const int c = (cpk[h][gi >> 2] >> (8 * (gi & 3))) & 0xff;
-                const int64_t end = __shfl_sync(0xffffffffu, rend, gi);
-                if (c == 0) continue;
-                const int st = estart[gi * kRowsPerCta + lr];
-                float gs[kTok];
+                    for (int t = 0; t < kTok; ++t) gs[t] = 0.f;
+                    for (int e = 0; e < c; ++e) {
+                        if (st + e >= end) break;       // only with inconsistent counts
+                        const uint32_t v = src[st + e];
+                        const uint32_t kk = v >> 1, w = kk >> 4, j = kk & 15;
+                        const int off =
+                            gi * kGroup + int((((w & 1) << 2) | (w >> 1)) * 16 + (((j & 7) << 1) | (j >> 3)));
 #pragma unroll
-                for (int t = 0; t < kTok; ++t) gs[t] = 0.f;
-                for (int e = 0; e < c; ++e) {
-                    if (st + e >= end) break;       // only with inconsistent counts
-                    const uint32_t v = src[st + e];
-                    const uint32_t kk = v >> 1, w = kk >> 4, j = kk & 15;
-                    const int off = gi * kGroup + int((((w & 1) << 2) | (w >> 1)) * 16 + (((j & 7) << 1) | (j >> 3)));
-#pragma unroll
-                    for (int t = 0; t < kTok; ++t) {
-                        if (t < M) {
-                            const float xv = __half2float(xs[size_t(t) * xs_stride + off]);
-                            gs[t] += (v & 1) ? -xv : xv;
+                        for (int t = 0; t < kTok; ++t) {
+                            if (t < M) {
+                                const float xv = __half2float(xs[size_t(t) * xs_stride + off]);
+                                gs[t] += (v & 1) ? -xv : xv;
+                            }
                         }
                     }
+                    const float sc = __half2float(esc[gi * kRowsPerCta + lr]);
+#pragma unroll
+                    for (int t = 0; t < kTok; ++t) acc[t] = fmaf(sc, gs[t], acc[t]);
                 }
-                const uint32_t sp = spk[h][gi >> 1] >> (16 * (gi & 1));
-                const float sc = __half2float(__ushort_as_half(static_cast<unsigned short>(sp & 0xffffu)));
 #pragma unroll
-                for (int t = 0; t < kTok; ++t) acc[t] = fmaf(sc, gs[t], acc[t]);
+                for (int t = 0; t < kTok; ++t)
+                    if (t < M) push(recv_res, lr, t, acc[t]);
             }
-#pragma unroll
-            for (int t = 0; t < kTok; ++t)
-                if (t < M) push(recv_res, lr, t, acc[t]);
         }
     }
 
     if (kElem && NT == 1) {
         // Element plane, M <= 8: all 160 threads take (group, row) cells once the main strips are
-        // done and warp 4 has staged the runs; each cell's scaled sum goes to shared memory (in
-        // the main tile's space, now free), then each (row, token) adds its cells in group order
-        // and sends the sum to the owning rank.
+        // done and warp 4's staged runs have landed; each cell's scaled sum goes to shared memory
+        // (in the main tile's space, now free), then each (row, token) adds its cells in group
+        // order and sends the sum to the owning rank.
         asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
         const uint8_t* ebuf = wt2;
         const int* estart = reinterpret_cast<const int*>(wt2 + kEStageBytes);
