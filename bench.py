@@ -46,8 +46,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 KERNEL_TRAFFIC = {
     "gemv": {"sources": ["ternary_weight_only_tern_b200/csrc/tern_gemv.cu",
                          "ternary_weight_only_tern_b200/csrc/tern_device.cuh"],
-             "sha256": "f47ea014a055ec5a5e16a0607e089581d4f638a7192d8a77076031b29d9b63e8",
-             "bytes": 30926336},
+             "sha256": "39508d230af327d476e81e8fe4d8e9cba38ee5613844d51775ab999668960ce5",
+             "bytes": 30928640},
 }
 
 
