@@ -85,3 +85,51 @@ def test_rotation_then_linear_on_the_rotated_weight(M):
     x_rot_ref = oracle.round_fp16(oracle.rotate(t.x, R))
     y_ref = oracle.linear(x_rot_ref, t.T1, t.s1, t.res_rows, t.T2, t.s2)
     assert oracle.rel_err(y.cpu().numpy().astype(np.float64), y_ref) <= TOL
+
+
+@pytest.mark.parametrize("M", [1, 4, 130])
+def test_rotation_and_groups_chained_in_a_cuda_graph(M):
+    """rotate -> linear_group -> rotate -> linear, captured once in a CUDA graph and replayed with new
+    inputs: every launch (several with programmatic dependent launch) reads what the one before
+    it wrote, and each replay matches the oracle's chain."""
+    rng = np.random.default_rng(90 + M)
+    K = 1024
+    R1 = _orthogonal(rng, K // 128).astype(np.float16)
+    ts = [synth.draw_tensor(rng, f"g{i}", 1024, K, M, p_zero=0.4, res_pct=10) for i in range(2)]
+    ws = [api.TernWeight.from_numpy(t.T1, t.s1, t.res_rows, t.T2, t.s2) for t in ts]
+    for w in ws:
+        w.static = True
+    R1d = torch.from_numpy(R1).cuda()
+    x = torch.zeros((M, K), dtype=torch.float16, device="cuda")
+    xr = torch.empty_like(x)
+    ys = [torch.empty((M, 1024), dtype=torch.float16, device="cuda") for _ in range(2)]
+    hr = torch.empty_like(x)
+    out = torch.empty((M, 1024), dtype=torch.float16, device="cuda")
+
+    def step():
+        api.rotate(x, R1d, out=xr)
+        api.linear_group(xr, ws, outs=ys)
+        api.rotate(ys[0], R1d, out=hr)
+        api.linear(hr, ws[1], out=out)
+
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    for rep in range(2):
+        xh = synth.draw_x(rng, M, K)
+        x.copy_(torch.from_numpy(xh))
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        a = oracle.round_fp16(oracle.rotate(xh, R1))
+        y0 = oracle.round_fp16(oracle.linear(a, ts[0].T1, ts[0].s1, ts[0].res_rows, ts[0].T2, ts[0].s2))
+        y1 = oracle.linear(a, ts[1].T1, ts[1].s1, ts[1].res_rows, ts[1].T2, ts[1].s2)
+        b = oracle.round_fp16(oracle.rotate(y0, R1))
+        y2 = oracle.linear(b, ts[1].T1, ts[1].s1, ts[1].res_rows, ts[1].T2, ts[1].s2)
+        assert oracle.rel_err(ys[1].cpu().numpy().astype(np.float64), y1) <= TOL
+        assert oracle.rel_err(out.cpu().numpy().astype(np.float64), y2) <= 5e-3
+    del g
