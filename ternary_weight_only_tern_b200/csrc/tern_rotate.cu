@@ -12,7 +12,8 @@
 // (32 KB) and the tokens' 128 activations in shared memory with cp.async (rows padded to 272
 // bytes, so the ldmatrix reads of 8 rows hit 32 distinct banks), and each of its 4 warps runs
 // 8 k-steps x 16 n-tiles of mma.sync m16n8k16 (fp16 in, fp32 accumulate) for 16 tokens; the
-// result is rounded to fp16 once. Everything is read after griddepcontrol.wait; the dependent
+// result is rounded to fp16 once and, for a warp with 16 real tokens, leaves through its own rows of
+// the staged tile as 16-byte stores. Everything is read after griddepcontrol.wait; the dependent
 // launch is triggered at entry, so the next kernel's weight loads overlap this one.
 #include <mutex>
 
@@ -93,14 +94,38 @@ __global__ void __launch_bounds__(kRotThreads) rotate_kernel(const __half* __res
             mma_16816(acc[2 * n + 1], a, b[2], b[3]);
         }
     }
-    // D: lane holds rows lane/4 and lane/4 + 8 of the warp's tokens, columns 2 (lane % 4) + {0, 1}
-    const int64_t r0 = m0 + warp * 16 + (lane >> 2), r1 = r0 + 8;
-    const int c0 = 2 * (lane & 3);
+    // D: lane holds rows lane/4 and lane/4 + 8 of the warp's tokens, columns 2 (lane % 4) + {0, 1}.
+    if (m0 + warp * 16 + 16 > M) {
+        // a partial tile (few tokens): each lane stores its pairs
+        const int64_t r0 = m0 + warp * 16 + (lane >> 2), r1 = r0 + 8;
+        const int c0 = 2 * (lane & 3);
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+            const int64_t col = g * kGroup + n * 8 + c0;
+            if (r0 < M) *reinterpret_cast<__half2*>(y + r0 * K + col) = __floats2half2_rn(acc[n][0], acc[n][1]);
+            if (r1 < M) *reinterpret_cast<__half2*>(y + r1 * K + col) = __floats2half2_rn(acc[n][2], acc[n][3]);
+        }
+        return;
+    }
+    // A full tile: the warp's 16 rows go, rounded, into its own rows of the x tile (which only this
+    // warp read) and leave as 16-byte stores.
+    __syncwarp();
+    const uint32_t rowa = sX + ((warp * 16 + (lane >> 2)) * kPitch + 2 * (lane & 3)) * 2;
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
-        const int64_t col = g * kGroup + n * 8 + c0;
-        if (r0 < M) *reinterpret_cast<__half2*>(y + r0 * K + col) = __floats2half2_rn(acc[n][0], acc[n][1]);
-        if (r1 < M) *reinterpret_cast<__half2*>(y + r1 * K + col) = __floats2half2_rn(acc[n][2], acc[n][3]);
+        const __half2 v0 = __floats2half2_rn(acc[n][0], acc[n][1]), v1 = __floats2half2_rn(acc[n][2], acc[n][3]);
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(rowa + n * 16), "r"(*reinterpret_cast<const uint32_t*>(&v0))
+                     : "memory");
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(rowa + n * 16 + 8 * kPitch * 2),
+                     "r"(*reinterpret_cast<const uint32_t*>(&v1))
+                     : "memory");
+    }
+    __syncwarp();
+    for (int c = lane; c < 16 * 16; c += 32) {
+        const int row = c >> 4, col = c & 15;
+        const int64_t m = m0 + warp * 16 + row;
+        *reinterpret_cast<uint4*>(y + m * K + g * kGroup + col * 8) =
+            lds_u4(sX + ((warp * 16 + row) * kPitch + col * 8) * 2);
     }
 }
 
