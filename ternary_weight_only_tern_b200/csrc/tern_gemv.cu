@@ -219,7 +219,7 @@ __device__ __forceinline__ void strip_sums(int ng, int q, int rr, uint32_t sc, u
 // ------------------------------------------------------------------ the kernel
 // kElem: the weight carries an element plane (a separate instantiation; warp 4 then sums it)
 template <int NT, bool kOne, bool kElem>
-__global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 4) gemv_kernel(const __grid_constant__ GemvMaps maps,
+__global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 3) gemv_kernel(const __grid_constant__ GemvMaps maps,
                                                                       const __grid_constant__ GemvArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
