@@ -46,8 +46,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 KERNEL_TRAFFIC = {
     "gemv": {"sources": ["ternary_weight_only_tern_b200/csrc/tern_gemv.cu",
                          "ternary_weight_only_tern_b200/csrc/tern_device.cuh"],
-             "sha256": "39508d230af327d476e81e8fe4d8e9cba38ee5613844d51775ab999668960ce5",
-             "bytes": 30928640},
+             "sha256": "846da767d2e21362d59dd522627c3b9f62eccc699dab95c78629f02a844d3491",
+             "bytes": 30941440},
 }
 
 
