@@ -46,7 +46,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 KERNEL_TRAFFIC = {
     "gemv": {"sources": ["ternary_weight_only_tern_b200/csrc/tern_gemv.cu",
                          "ternary_weight_only_tern_b200/csrc/tern_device.cuh"],
-             "sha256": "846da767d2e21362d59dd522627c3b9f62eccc699dab95c78629f02a844d3491",
+             "sha256": "dfc417d5311d539d471482404c15871dcd4a96b6bd9cd1af63cf2cbbd05f2fac",
              "bytes": 30941440},
 }
 

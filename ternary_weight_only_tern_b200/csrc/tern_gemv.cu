@@ -13,9 +13,13 @@
 //    swizzle), of the residual-plane rows that belong to those 64 rows and of their scales,
 //    so the HBM stream starts at once and no later step waits on another global round trip
 //    except the read of x.
-//  * The K-slices of a 64-row block form a thread-block cluster. Partial sums meet in
-//    distributed shared memory in a fixed order (no global partials, no atomics, no
-//    spin-waits on other CTAs); the CTA of cluster rank c writes rows [c*64/S, (c+1)*64/S).
+//  * The K-slices of a 64-row block form a thread-block cluster. Each CTA sends its partial
+//    sums to the rank that owns the row as asynchronous stores into that rank's shared memory
+//    (st.async, completing on the owner's receive barrier); the owner adds them in rank order
+//    (no global partials, no atomics, a deterministic result) and the CTA of cluster rank c
+//    writes rows [c*64/S, (c+1)*64/S). No CTA waits for its peers to finish.
+//  * Up to 4 weights that share x run as one launch: each weight's 64-row blocks are blocks of
+//    the same grid, and a CTA finds its weight from blockIdx.y.
 //  * Warps 0-3 each own a 16-row strip of the main plane. Warp 4 owns the residual rows of the
 //    block: since R is sorted, they are the contiguous slots [s_lo, s_lo + nres) of the
 //    residual plane, taken 16 rows at a time. Their sums join the main rows' sums before the
@@ -30,9 +34,14 @@
 //    so a word of 16 trits costs 2 shifts and 8 LOP3. Since c = t + 1, the MMA sums
 //    (B_p + 1 + t) * x from zero, and C = sum (B_p + 1) * x is subtracted once per group. C is
 //    computed once per CTA by the same MMA on the constant pattern B_p + 1 in the same K order
-//    and accumulator split (hidden behind the weight loads), so a zero plane cancels bit for bit. The bases are 4, 16 and 64, so the offsets
-//    are small and every partial sum is exact on integer inputs. A non-finite activation
-//    makes every output of its token non-finite (NaN where the dense product has +-inf).
+//    and accumulator split (hidden behind the weight loads), so a zero plane cancels bit for
+//    bit. The bases are 4, 16 and 64, so the offsets are small and every partial sum is exact
+//    on integer inputs. A non-finite activation makes every output of its token non-finite
+//    (NaN where the dense product has +-inf).
+//  * Options: a per-group offset mu (section 4.3's asymmetric offset) adds mu * X_g, the
+//    group sums X_g coming from one more MMA chain on an all-ones pattern; an element-level
+//    second plane (section 4.4's salience masks) is staged by warp 4 and summed on the CUDA
+//    cores.
 //  * The contraction order over K is free, so the MMA's K order follows the packed words
 //    (pair j = trits j and j+8 of a word); x is staged in shared memory in that order, with
 //    the words of a group arranged so that one MMA step's activation fragments are 128
