@@ -1,22 +1,25 @@
 """Benchmark of the W1.58A16 ternary linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--quick]
+                    [--profile gemv|gemv_elem|gemm|rotate]
 
 A step is one decode pass (M = 1) over the 252 ternarized linear tensors of a 36-layer
 Qwen3-8B-shaped stack (q, k, v, o, gate, up, down per layer; 15% of rows carry a residual
-plane), i.e. 252 tern_linear calls, replayed from a CUDA graph. Weights come from a pool of
-8 distinct layers (about 470 MB of packed planes, several times the 126 MB L2), assigned to
-the 36 layer slots round-robin, so every call streams its weights from HBM.
+plane): per layer four tern_linear_group launches, one per input the projections share (q+k+v,
+o, gate+up, down), 144 per step, replayed from a CUDA graph. Weights come from a pool of 8
+distinct layers (about 470 MB of packed planes, several times the 126 MB L2), assigned to the 36
+layer slots round-robin, so every call streams its weights from HBM.
 
 value     : packed-weight GB/s = (2-bit planes + fp16 scales + slot map) bytes per step / time.
-roofline  : the dominant op (the gate projection's tern_linear at M = 1), algorithmic bytes
-            (packed weight + activations) per call / its average call time, against the
-            measured HBM copy bandwidth.
-e2e       : the same metric through the Python API with the step's activations copied from
-            pinned host memory and its outputs copied back, every step.
+roofline  : the dominant launch (gate + up at M = 1), algorithmic bytes (packed weights +
+            activations) per launch / its average launch time, against the measured HBM copy
+            bandwidth; traffic = the DRAM bytes of one such launch from an ncu capture.
+e2e       : the same metric through the Python API with the step's inputs copied from pinned
+            host memory and its outputs copied back, every step.
 cpu_baseline / --impl reference: the CPU oracle (numpy float64) on a bounded sample.
-extra     : per-projection and per-M decode figures, the M = 2048 prefill GEMM in TFLOP/s,
-            packing throughput, bit accounting, and dense fp16 cuBLAS on the same shapes.
+extra     : per-projection, per-group and per-M decode figures, the M = 2048 prefill GEMM in
+            TFLOP/s, the offset, element-plane, rotation and fit measurements, packing throughput,
+            bit accounting, and dense fp16 cuBLAS on the same shapes.
 
 For --gpus N > 1 (torchrun) every rank runs the same workload on its own GPU (replicas; the
 path has no data exchange), the timed region is bracketed by barriers, and the time is the
