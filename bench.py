@@ -311,7 +311,7 @@ def main():
                     help="how many following launches' weights each launch brings into L2 (with grouped "
                          "launches 0 measured best: 1824 us per step against 1840 for 1 and 1971 for 2)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline")
-    ap.add_argument("--profile", choices=["gemv", "gemv_elem", "gemm", "rotate"], default=None,
+    ap.add_argument("--profile", choices=["gemv", "gemv_elem", "gemm", "gemm_elem", "rotate"], default=None,
                     help="run a few calls of one op on one pool layer and exit (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -536,7 +536,7 @@ def main():
 def profile_case(torch, api, shapes, dev, which):
     """A minimal run for ncu, three repetitions over two layers: at M = 1 (gemv) the bench's four
     launches per layer (q+k+v, o, gate+up, down), or (gemv_elem) the same with element planes
-    (3.6 % masked) in place of residual rows; at M = 2048 (gemm) gate, up and down."""
+    (3.6 % masked) in place of residual rows; at M = 2048 (gemm, gemm_elem) gate, up and down."""
     if which == "rotate":
         # tern_rotate on K = 4096 at M = 1 and M = 2048, three times
         R = (torch.randn((32, 128, 128), device=dev) / 11.3).half()
@@ -551,11 +551,12 @@ def profile_case(torch, api, shapes, dev, which):
         torch.cuda.synchronize()
         print(json.dumps({"profile": which, "calls": 6}))
         return
-    elem = 0.036 if which == "gemv_elem" else None
+    elem = 0.036 if which in ("gemv_elem", "gemm_elem") else None
     pool = [draw_layer_on_device(torch, api, shapes, dev, seed=1000 + i, elem_frac=elem) for i in range(2)]
     kdim = {n: K for n, _, K in shapes}
-    groups = GROUPS if which != "gemm" else [("gate", ("gate",)), ("up", ("up",)), ("down", ("down",))]
-    M = 2048 if which == "gemm" else 1
+    prefill = which in ("gemm", "gemm_elem")
+    groups = GROUPS if not prefill else [("gate", ("gate",)), ("up", ("up",)), ("down", ("down",))]
+    M = 2048 if prefill else 1
     xs = {g: torch.randn((M, kdim[m[0]]), device=dev).half() for g, m in groups}
     ys = {n: torch.empty((M, N), dtype=torch.float16, device=dev) for n, N, _ in shapes}
     torch.cuda.synchronize()
