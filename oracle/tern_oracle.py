@@ -195,6 +195,13 @@ def row_bitmap(N: int, res_rows: np.ndarray) -> np.ndarray:
     return np.packbits(bits, bitorder="little")
 
 
+def rows_from_bitmap(N: int, bitmap: np.ndarray) -> np.ndarray:
+    """The inverse of row_bitmap: int32 [r], the rows whose bit is set, in increasing order.
+    Bits of the last byte past row N - 1 are not rows (they must be 0 in a canonical bitmap)."""
+    bits = np.unpackbits(np.asarray(bitmap, dtype=np.uint8), bitorder="little")[:N]
+    return np.nonzero(bits)[0].astype(np.int32)
+
+
 # --------------------------------------------------------------------------------------
 # Element-level second plane: the nonzero trits of T2e, one byte each,
 #   byte = (k % 128) << 1 | (t < 0),

@@ -789,7 +789,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 6 : 3) gemv_kernel(const _
     // Epilogue: once the partial sums of this rank's rows have arrived from every rank (the
     // receive barrier counts their bytes) they are summed in rank order, the residual rows' sums
     // added, and rounded once. No CTA reads another's memory, so none waits for its peers to end.
-    if (ok) ok = mbar_wait(rbar, 0);
+    // The wait runs whatever `ok` is: every rank pushes its partial sums on every path, and a CTA
+    // that left early would take stores into the shared memory of an exited CTA.
+    ok = mbar_wait(rbar, 0) && ok;
     {
         for (int i = threadIdx.x; i < nrows * M; i += kThreads) {
             const int tok = i / nrows, lo = i - tok * nrows, lr = lr0 + lo;

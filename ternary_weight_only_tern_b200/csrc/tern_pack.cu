@@ -272,8 +272,8 @@ extern "C" tern_status tern_weight_validate(const tern_weight* w, tern_stream s)
     if (w->N < 0 || w->K <= 0 || w->K % kGroup || w->group != kGroup || w->r < 0 || w->r > w->N)
         return TERN_ERR_SHAPE;
     if (w->N == 0) return TERN_OK;
-    if (!w->plane1 || !w->scale1 || !w->res_slot) return TERN_ERR_NULL;
-    if (w->r > 0 && (!w->plane2 || !w->scale2 || !w->res_rows)) return TERN_ERR_NULL;
+    if (!w->plane1 || !w->scale1) return TERN_ERR_NULL;
+    if (w->r > 0 && (!w->plane2 || !w->scale2 || !w->res_rows || !w->res_slot)) return TERN_ERR_NULL;
     cudaStream_t st = as_cuda(s);
     const int64_t n1 = w->N * (w->K / kCodesPerWord);
     const int64_t n2 = w->r * (w->K / kCodesPerWord);
@@ -282,8 +282,11 @@ extern "C" tern_status tern_weight_validate(const tern_weight* w, tern_stream s)
     const tern_status cs = run_checked(st, [&](unsigned int* f) {
         validate_codes_kernel<<<grid_for(n1, 256), 256, 0, st>>>(w->plane1, n1, f);
         if (n2) validate_codes_kernel<<<grid_for(n2, 256), 256, 0, st>>>(w->plane2, n2, f);
-        validate_residual_kernel<<<grid_for(w->N + w->r, 256), 256, 0, st>>>(w->res_rows, w->res_slot, w->N,
-                                                                            w->r, f);
+        // without residual rows the slot map may be absent (as tern_linear accepts); when given
+        // it must hold -1 everywhere
+        if (w->res_slot)
+            validate_residual_kernel<<<grid_for(w->N + w->r, 256), 256, 0, st>>>(w->res_rows, w->res_slot, w->N,
+                                                                                w->r, f);
     }, TERN_ERR_BAD_CODE);
     if (cs != TERN_OK || !w->ecount) return cs;
     return elem_check(*w, st);

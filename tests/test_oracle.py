@@ -649,3 +649,38 @@ def test_ternarize_assembles_rows_and_groups():
             if n in rows:
                 i = list(rows).index(n)
                 assert np.array_equal(T2[i, g * 128:(g + 1) * 128], t2[0]) and s2[i, g] == np.float16(a2[0])
+
+
+# ------------------------------------------------------------------ residual-row metadata
+# The second plane lives on a sorted subset R of rows ("Post-Training Ternarization of
+# Qwen3-4B", section 4.4; the 8B paper's representation paragraph). Its execution form is the
+# slot map (row -> index in R, or -1), its storage form a bitmap of the rows.
+
+def test_slot_map_and_bitmap_hand_worked():
+    rows = np.array([1, 2, 9], np.int32)
+    assert oracle.slot_map(11, rows).tolist() == [-1, 0, 1, -1, -1, -1, -1, -1, -1, 2, -1]
+    # rows 1, 2 -> byte 0 = 0b00000110; row 9 -> byte 1 = 0b00000010
+    assert oracle.row_bitmap(11, rows).tolist() == [6, 2]
+    assert O.rows_from_bitmap(11, np.array([6, 2], np.uint8)).tolist() == [1, 2, 9]
+
+
+@pytest.mark.parametrize("N", [1, 7, 8, 9, 63, 64, 65, 1000, 12288])
+def test_residual_metadata_against_python_integers(N):
+    rng = np.random.default_rng(N)
+    for frac in (0.0, 0.15, 1.0):
+        r = int(round(frac * N))
+        rows = np.sort(rng.choice(N, size=r, replace=False)).astype(np.int32)
+        # the bitmap is the little-endian bytes of the integer sum of 2^n over R
+        as_int = sum(1 << int(n) for n in rows)
+        want = np.frombuffer(as_int.to_bytes(-(-N // 8), "little"), dtype=np.uint8)
+        assert np.array_equal(oracle.row_bitmap(N, rows), want)
+        # the slot map, element by element from its definition
+        slot = oracle.slot_map(N, rows)
+        pos = {int(n): i for i, n in enumerate(rows)}
+        assert all(int(slot[n]) == pos.get(n, -1) for n in range(N))
+        assert np.array_equal(O.rows_from_bitmap(N, want), rows)
+
+
+def test_rows_from_bitmap_ignores_bits_past_n():
+    # byte 1 holds rows 8..15; with N = 10 only rows 8 and 9 exist
+    assert O.rows_from_bitmap(10, np.array([0, 0xFF], np.uint8)).tolist() == [8, 9]
