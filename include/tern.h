@@ -88,7 +88,8 @@ typedef struct {
     int64_t r;                   /* rows with a second plane, 0 <= r <= N               */
     const int32_t* res_rows;     /* [r] strictly increasing row indices (R); read only by
                                     tern_weight_validate                                 */
-    const int32_t* res_slot;     /* [N] -1, or rho(n) for n in R                        */
+    const int32_t* res_slot;     /* [N] -1, or rho(n) for n in R (tern_pack_residual);
+                                    may be NULL when r == 0                              */
     const uint32_t* plane2;      /* [r, K/16]   exec codes of T2                        */
     const tern_half* scale2;     /* [r, K/128]  s2                                      */
     uint32_t flags;              /* 0 or TERN_WEIGHT_STATIC                             */
@@ -161,9 +162,32 @@ tern_status tern_pack_elem(const int8_t* t, int64_t N, int64_t K, uint8_t* ecoun
 tern_status tern_unpack_elem(const uint8_t* ecount, const int32_t* ebase, const uint8_t* eidx, int64_t nnz2,
                              int64_t N, int64_t K, int8_t* out, tern_stream stream);
 
+/* Residual-row metadata. The second plane is carried by a salience-selected subset R of the
+ * output rows ("Post-Training Ternarization of Qwen3-4B", section 4.4; the Qwen3-8B scale-up
+ * paper, representation paragraph), which this library keeps as whole rows. Its execution form
+ * is the slot map res_slot [N] int32 (-1, or rho(n) = n's index in R), which the linear kernels
+ * read; its storage form is a row bitmap [ceil(N/8)] uint8 (bit n % 8 of byte n / 8 set for n in
+ * R, the bits past row N - 1 zero), the one counted by tern_bits' store_bits.
+ *
+ * tern_pack_residual: res_rows [r] (device; strictly increasing, in [0, N)) -> res_slot [N]
+ * (device, required when N > 0) and, when row_bitmap is not NULL, the bitmap (device). Rows out
+ * of range or not strictly increasing return TERN_ERR_RESIDUAL; the outputs are then written
+ * but describe no valid weight. int32 pointers 4-byte aligned. Synchronous on `stream`.     */
+tern_status tern_pack_residual(const int32_t* res_rows, int64_t r, int64_t N, int32_t* res_slot,
+                               uint8_t* row_bitmap, tern_stream stream);
+
+/* tern_unpack_residual: row bitmap [ceil(N/8)] (device) -> *r = |R| (host), and, when not
+ * NULL, res_rows [r] (device, capacity r_cap entries) in increasing order and res_slot [N]
+ * (device). Call with res_rows == NULL to learn *r. A bit set past row N - 1 is not a row and
+ * returns TERN_ERR_BAD_CODE (the outputs still hold the rows below N); more than r_cap rows
+ * return TERN_ERR_WORKSPACE (the first r_cap are written). Synchronous on `stream`.        */
+tern_status tern_unpack_residual(const uint8_t* row_bitmap, int64_t N, int32_t* res_rows, int64_t r_cap,
+                                 int64_t* r, int32_t* res_slot, tern_stream stream);
+
 /* Checks a weight descriptor's device data: every code of plane1/plane2 is in {0,1,2},
  * res_rows is strictly increasing in [0, N), and res_slot[n] == i exactly when
- * res_rows[i] == n (else -1); an element plane is checked as by tern_unpack_elem.
+ * res_rows[i] == n (else -1; a NULL res_slot is accepted when r == 0); an element plane is
+ * checked as by tern_unpack_elem.
  * Returns TERN_OK, TERN_ERR_BAD_CODE, TERN_ERR_RESIDUAL or TERN_ERR_ELEM.
  * Synchronous on `stream`. tern_linear does not repeat these checks; it only keeps its
  * own memory accesses in bounds when a slot is out of range.                            */

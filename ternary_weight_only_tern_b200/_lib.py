@@ -42,6 +42,9 @@ EXPORTS = {
                                   _c.c_int64, _c.c_void_p, _c.c_void_p]),
     "tern_unpack_elem": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_int64, _c.c_int64,
                                     _c.c_void_p, _c.c_void_p]),
+    "tern_pack_residual": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_int64, _c.c_void_p, _c.c_void_p, _c.c_void_p]),
+    "tern_unpack_residual": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_void_p, _c.c_int64, _c.c_void_p, _c.c_void_p,
+                                        _c.c_void_p]),
     "tern_device_status": (_c.c_int, [_c.c_void_p]),
     "tern_status_string": (_c.c_char_p, [_c.c_int]),
     "tern_version": (_c.c_int, []),

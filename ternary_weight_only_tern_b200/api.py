@@ -73,6 +73,36 @@ def unpack_store(data: torch.Tensor, K: int) -> torch.Tensor:
     return out
 
 
+def pack_residual(res_rows: torch.Tensor, N: int, bitmap: bool = True):
+    """Sorted residual rows int32 [r] -> (slot map int32 [N], row bitmap uint8 [ceil(N/8)] or None)
+    by tern_pack_residual."""
+    _need(res_rows, torch.int32, "res_rows", ndim=1)
+    dev = res_rows.device
+    slot = torch.empty(N, dtype=torch.int32, device=dev)
+    bm = torch.empty(-(-N // 8), dtype=torch.uint8, device=dev) if bitmap else None
+    _lib.check("tern_pack_residual", _lib.load().tern_pack_residual(
+        _ptr(res_rows), int(res_rows.numel()), N, _ptr(slot), _ptr(bm), _stream(dev)))
+    return slot, bm
+
+
+def unpack_residual(bitmap: torch.Tensor, N: int):
+    """Row bitmap uint8 [ceil(N/8)] -> (residual rows int32 [r], slot map int32 [N]) by
+    tern_unpack_residual (two calls: the count, then the rows)."""
+    _need(bitmap, torch.uint8, "bitmap", ndim=1)
+    if bitmap.numel() != -(-N // 8):
+        raise ValueError("bitmap must hold ceil(N/8) bytes")
+    dev = bitmap.device
+    lib = _lib.load()
+    r = ctypes.c_int64(0)
+    _lib.check("tern_unpack_residual", lib.tern_unpack_residual(_ptr(bitmap), N, None, 0, ctypes.byref(r), None,
+                                                                _stream(dev)))
+    rows = torch.empty(max(1, r.value), dtype=torch.int32, device=dev)
+    slot = torch.empty(N, dtype=torch.int32, device=dev)
+    _lib.check("tern_unpack_residual", lib.tern_unpack_residual(_ptr(bitmap), N, _ptr(rows), rows.numel(),
+                                                                ctypes.byref(r), _ptr(slot), _stream(dev)))
+    return rows[: r.value], slot
+
+
 @dataclass
 class ElemPlane:
     """An element-level second plane in its listed form (tern_pack_elem): the nonzero trits of
@@ -185,9 +215,7 @@ class TernWeight:
             s2 = torch.zeros((0, K // GROUP), dtype=torch.float16, device=dev)
         res_rows = res_rows.to(device=dev, dtype=torch.int32).contiguous()
         r = int(res_rows.numel())
-        slot = torch.full((N,), -1, dtype=torch.int32, device=dev)
-        if r:
-            slot[res_rows.long()] = torch.arange(r, dtype=torch.int32, device=dev)
+        slot, _ = pack_residual(res_rows, N, bitmap=False)
         plane2 = pack_exec(T2) if r else torch.zeros((0, K // 16), dtype=torch.int32, device=dev)
         if mu is not None:
             _need(mu, torch.float16, "mu")
@@ -301,9 +329,7 @@ def fit(W: torch.Tensor, res_rows: torch.Tensor | None = None, offset: bool = Tr
         res_rows = torch.zeros(0, dtype=torch.int32, device=dev)
     res_rows = res_rows.to(device=dev, dtype=torch.int32).contiguous()
     r = int(res_rows.numel())
-    slot = torch.full((N,), -1, dtype=torch.int32, device=dev)
-    if r:
-        slot[res_rows.long()] = torch.arange(r, dtype=torch.int32, device=dev)
+    slot, _ = pack_residual(res_rows, N, bitmap=False)
     T1 = torch.empty((N, K), dtype=torch.int8, device=dev)
     s1 = torch.empty((N, G), dtype=torch.float16, device=dev)
     mu = torch.empty((N, G), dtype=torch.float16, device=dev) if offset else None

@@ -197,6 +197,102 @@ __global__ void validate_residual_kernel(const int32_t* __restrict__ rows, const
     if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, kBadResidual);
 }
 
+// Residual-row metadata: the sorted rows R -> the slot map (execution form) and the row bitmap
+// (storage form), and back.
+__global__ void slot_fill_kernel(int32_t* __restrict__ slot, int64_t N) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < N; i += (int64_t)gridDim.x * blockDim.x)
+        slot[i] = -1;
+}
+
+__global__ void slot_scatter_kernel(const int32_t* __restrict__ rows, int64_t r, int64_t N, int32_t* __restrict__ slot,
+                                    unsigned int* status) {
+    bool bad = false;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < r; i += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t n = rows[i];
+        if (n < 0 || n >= N) {
+            bad = true;
+            continue;
+        }
+        if (i + 1 < r && rows[i + 1] <= n) bad = true;   // not strictly increasing
+        slot[n] = int32_t(i);
+    }
+    if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, kBadResidual);
+}
+
+// Byte j of the bitmap: bit b is set when row 8 j + b has a slot.
+__global__ void bitmap_from_slots_kernel(const int32_t* __restrict__ slot, int64_t N, uint8_t* __restrict__ bitmap) {
+    const int64_t nbytes = (N + 7) / 8;
+    for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < nbytes;
+         j += (int64_t)gridDim.x * blockDim.x) {
+        uint32_t v = 0;
+        for (int b = 0; b < 8; ++b) {
+            const int64_t n = 8 * j + b;
+            if (n < N && slot[n] >= 0) v |= 1u << b;
+        }
+        bitmap[j] = uint8_t(v);
+    }
+}
+
+// One CTA walks the bitmap in order, kRowsThreads bytes per round: each thread counts its
+// byte's rows, a block scan gives each its first index, and the rows (and slots) are written.
+// count receives r; a bit set past row N - 1 is reported as non-canonical.
+constexpr int kRowsThreads = 1024;
+__global__ void __launch_bounds__(kRowsThreads) rows_from_bitmap_kernel(const uint8_t* __restrict__ bitmap, int64_t N,
+                                                                        int32_t* __restrict__ rows, int64_t r_cap,
+                                                                        int32_t* __restrict__ slot,
+                                                                        unsigned int* count, unsigned int* status) {
+    __shared__ unsigned int warp_tot[kRowsThreads / 32];
+    __shared__ unsigned int base_s;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t nbytes = (N + 7) / 8;
+    if (threadIdx.x == 0) base_s = 0;
+    __syncthreads();
+    bool bad = false;
+    for (int64_t j0 = 0; j0 < nbytes; j0 += kRowsThreads) {
+        const int64_t j = j0 + threadIdx.x;
+        uint32_t v = j < nbytes ? bitmap[j] : 0u;
+        const int valid = int(min(int64_t(8), N - 8 * j));   // rows held by this byte
+        if (j < nbytes && valid < 8) {
+            bad |= (v >> valid) != 0u;
+            v &= (1u << valid) - 1u;
+        }
+        const unsigned int c = __popc(v);
+        unsigned int inc = c;   // inclusive scan within the warp
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned int u = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += u;
+        }
+        if (lane == 31) warp_tot[warp] = inc;
+        __syncthreads();
+        if (warp == 0) {
+            unsigned int t = warp_tot[lane], ti = t;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned int u = __shfl_up_sync(0xffffffffu, ti, o);
+                if (lane >= o) ti += u;
+            }
+            warp_tot[lane] = ti - t;   // exclusive prefix of the warps
+        }
+        __syncthreads();
+        unsigned int idx = base_s + warp_tot[warp] + inc - c;
+        if (j < nbytes) {
+            for (int b = 0; b < valid; ++b) {
+                const int64_t n = 8 * j + b;
+                const bool set = (v >> b) & 1u;
+                if (set && rows && int64_t(idx) < r_cap) rows[idx] = int32_t(n);
+                if (slot) slot[n] = set ? int32_t(idx) : -1;
+                idx += set ? 1u : 0u;
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x == kRowsThreads - 1) base_s += warp_tot[warp] + inc;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) *count = base_s;
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, kBadInput);
+}
+
 int grid_for(int64_t items, int threads) {
     const int64_t want = (items + threads - 1) / threads;
     const int64_t cap = static_cast<int64_t>(sm_count()) * 32;
@@ -305,4 +401,44 @@ extern "C" tern_status tern_device_status(tern_stream s) {
         return TERN_ERR_TIMEOUT;
     }
     return TERN_OK;
+}
+
+extern "C" tern_status tern_pack_residual(const int32_t* res_rows, int64_t r, int64_t N, int32_t* res_slot,
+                                          uint8_t* row_bitmap, tern_stream s) {
+    if (N < 0 || r < 0 || r > N || N > (int64_t(1) << 31) - 1) return TERN_ERR_SHAPE;
+    if (N == 0) return TERN_OK;
+    if (!res_slot || (r > 0 && !res_rows)) return TERN_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(res_slot) & 3u) || (reinterpret_cast<uintptr_t>(res_rows) & 3u))
+        return TERN_ERR_ALIGN;
+    cudaStream_t st = as_cuda(s);
+    return run_checked(st, [&](unsigned int* f) {
+        slot_fill_kernel<<<grid_for(N, 256), 256, 0, st>>>(res_slot, N);
+        if (r > 0) slot_scatter_kernel<<<grid_for(r, 256), 256, 0, st>>>(res_rows, r, N, res_slot, f);
+        if (row_bitmap) bitmap_from_slots_kernel<<<grid_for((N + 7) / 8, 256), 256, 0, st>>>(res_slot, N, row_bitmap);
+    }, TERN_ERR_RESIDUAL);
+}
+
+extern "C" tern_status tern_unpack_residual(const uint8_t* row_bitmap, int64_t N, int32_t* res_rows, int64_t r_cap,
+                                            int64_t* r, int32_t* res_slot, tern_stream s) {
+    if (N < 0 || r_cap < 0 || N > (int64_t(1) << 31) - 1) return TERN_ERR_SHAPE;
+    if (!r) return TERN_ERR_NULL;
+    *r = 0;
+    if (N == 0) return TERN_OK;
+    if (!row_bitmap) return TERN_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(res_slot) & 3u) || (reinterpret_cast<uintptr_t>(res_rows) & 3u))
+        return TERN_ERR_ALIGN;
+    cudaStream_t st = as_cuda(s);
+    unsigned int* count = acquire_flag_slot(st);
+    if (!count) return TERN_ERR_CUDA;
+    const tern_status rs = run_checked(st, [&](unsigned int* f) {
+        rows_from_bitmap_kernel<<<1, kRowsThreads, 0, st>>>(row_bitmap, N, res_rows, res_rows ? r_cap : 0, res_slot,
+                                                            count, f);
+    }, TERN_ERR_BAD_CODE);
+    if (rs != TERN_OK && rs != TERN_ERR_BAD_CODE) return rs;
+    unsigned int c = 0;
+    const tern_status cs = read_flag_slot(count, st, &c);
+    if (cs != TERN_OK) return cs;
+    *r = int64_t(c);
+    if (rs != TERN_OK) return rs;
+    return (res_rows && int64_t(c) > r_cap) ? TERN_ERR_WORKSPACE : TERN_OK;
 }

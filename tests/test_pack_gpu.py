@@ -129,3 +129,59 @@ def test_weight_validate_catches_corruption():
     w = api.TernWeight.from_numpy(t.T1, t.s1, t.res_rows, t.T2, t.s2)
     w.res_rows[0], w.res_rows[1] = int(t.res_rows[1]), int(t.res_rows[0])
     expect_status(api.weight_validate, w, status="TERN_ERR_RESIDUAL")
+
+
+# ------------------------------------------------------------------ residual-row metadata
+@pytest.mark.parametrize("N", [1, 7, 9, 64, 65, 1000, 4096, 12288])
+def test_residual_metadata_bit_exact(N):
+    rng = np.random.default_rng(N + 5)
+    for frac in (0.0, 0.1, 0.15, 1.0):
+        r = int(round(frac * N))
+        rows = np.sort(rng.choice(N, size=r, replace=False)).astype(np.int32)
+        slot, bm = api.pack_residual(dev(rows), N)
+        assert np.array_equal(slot.cpu().numpy(), oracle.slot_map(N, rows))
+        assert np.array_equal(bm.cpu().numpy(), oracle.row_bitmap(N, rows))
+        rows2, slot2 = api.unpack_residual(bm, N)
+        assert np.array_equal(rows2.cpu().numpy(), rows)
+        assert np.array_equal(slot2.cpu().numpy(), oracle.slot_map(N, rows))
+
+
+def test_residual_metadata_large_n_spans_several_scan_rounds():
+    # 8 bytes per thread round trip: 1024 threads x 8 rows per round, so N = 3e5 takes ~37 rounds
+    N = 300_001
+    rng = np.random.default_rng(3)
+    rows = np.sort(rng.choice(N, size=45_000, replace=False)).astype(np.int32)
+    slot, bm = api.pack_residual(dev(rows), N)
+    assert np.array_equal(bm.cpu().numpy(), oracle.row_bitmap(N, rows))
+    rows2, slot2 = api.unpack_residual(bm, N)
+    assert np.array_equal(rows2.cpu().numpy(), rows)
+    assert np.array_equal(slot2.cpu().numpy(), oracle.slot_map(N, rows))
+
+
+@pytest.mark.parametrize("bad", [[3, 3], [5, 2], [-1, 4], [2, 10]])
+def test_pack_residual_rejects_unsorted_or_out_of_range(bad):
+    expect_status(api.pack_residual, dev(np.array(bad, np.int32)), 10, status="TERN_ERR_RESIDUAL")
+
+
+def test_unpack_residual_flags_bits_past_n_and_small_capacity():
+    lib = _lib.load()
+    bm = dev(np.array([0b00000101, 0b11000001], np.uint8))     # rows 0, 2, 8 valid; bits 14, 15 past N = 10
+    import ctypes
+    r = ctypes.c_int64(0)
+    rows = torch.full((8,), -7, dtype=torch.int32, device="cuda")
+    st = lib.tern_unpack_residual(api._ptr(bm), 10, api._ptr(rows), 8, ctypes.byref(r), None, api._stream())
+    assert st == S["TERN_ERR_BAD_CODE"] and r.value == 3
+    assert rows.cpu().numpy()[:3].tolist() == [0, 2, 8]
+    ok = dev(np.array([0b00000101, 0b00000001], np.uint8))
+    st = lib.tern_unpack_residual(api._ptr(ok), 10, api._ptr(rows), 2, ctypes.byref(r), None, api._stream())
+    assert st == S["TERN_ERR_WORKSPACE"] and r.value == 3
+
+
+def test_validate_accepts_a_null_slot_map_without_residual_rows():
+    rng = np.random.default_rng(1)
+    t = synth.draw_tensor(rng, "t", 64, 256, 1, p_zero=0.4, res_pct=0)
+    w = api.TernWeight.from_numpy(t.T1, t.s1, t.res_rows, t.T2, t.s2)
+    c = w.c_struct()
+    c.res_slot = None
+    import ctypes
+    assert _lib.load().tern_weight_validate(ctypes.byref(c), api._stream()) == 0
