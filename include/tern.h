@@ -298,6 +298,14 @@ tern_status tern_bits_elem(int64_t N, int64_t K, int64_t masked, int64_t nnz2, i
  * wait (its output is then undefined), else TERN_OK. Synchronous on `stream`.            */
 tern_status tern_device_status(tern_stream stream);
 
+/* The failure path of the bounded device-side waits, exercised on purpose: one thread waits on
+ * a shared-memory barrier that nothing completes, bounded by `cycles` SM clock cycles
+ * (1 <= cycles <= 2^32), and then records the timeout in the device's sticky status word as a
+ * linear kernel whose wait ran out does; no copy or MMA is in flight meanwhile, and the context
+ * stays usable. A following tern_device_status returns TERN_ERR_TIMEOUT and clears the word.
+ * For tests of error handling. Asynchronous on `stream`.                                   */
+tern_status tern_selftest_timeout(int64_t cycles, tern_stream stream);
+
 /* A static, human-readable name for a status code. */
 const char* tern_status_string(tern_status s);
 

@@ -46,6 +46,7 @@ EXPORTS = {
     "tern_unpack_residual": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_void_p, _c.c_int64, _c.c_void_p, _c.c_void_p,
                                         _c.c_void_p]),
     "tern_device_status": (_c.c_int, [_c.c_void_p]),
+    "tern_selftest_timeout": (_c.c_int, [_c.c_int64, _c.c_void_p]),
     "tern_status_string": (_c.c_char_p, [_c.c_int]),
     "tern_version": (_c.c_int, []),
 }

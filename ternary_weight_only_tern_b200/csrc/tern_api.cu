@@ -109,6 +109,7 @@ tern_status linear_group(const tern_weight* const* w, int n, const tern_half* x,
     const __half* xh = reinterpret_cast<const __half*>(x);
     __half* yh[kMaxGemvGroup];
     for (int i = 0; i < n; ++i) yh[i] = reinterpret_cast<__half*>(y[i]);
+    if (M == 1 && decode1_supported(w, n)) return decode1_launch_group(w, n, xh, yh, next, nnext, st);
     if (M <= kGemvMaxM) return gemv_launch_group(w, n, xh, int(M), yh, next, nnext, st);
     for (int i = 0; i < n; ++i) {
         const tern_status s = gemm_launch(*w[i], xh, M, yh[i], workspace, st);

@@ -89,9 +89,9 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 }
 
 
-// Bounded wait for the completion of the phase with the given parity: false after
-// kWaitLimitCycles.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Bounded wait for the completion of the phase with the given parity: false after `limit` SM
+// clock cycles.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint64_t limit) {
     const uint32_t addr = smem_u32(bar);
     uint64_t t0 = 0;
     for (uint32_t i = 0;; ++i) {
@@ -106,8 +106,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
         if (done) return true;
         const uint64_t t = clock64();
         if (i == 0) t0 = t;
-        else if (t - t0 > kWaitLimitCycles) return false;
+        else if (t - t0 > limit) return false;
     }
+}
+
+// Bounded wait with the library's limit (kWaitLimitCycles).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    return mbar_wait_for(bar, parity, kWaitLimitCycles);
 }
 
 // 2D tiled TMA load into this CTA's shared memory, completing on `bar` (no multicast).

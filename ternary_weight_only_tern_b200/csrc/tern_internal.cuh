@@ -34,6 +34,12 @@ tern_status gemv_launch_group(const tern_weight* const* ws, int nw, const __half
                               const tern_weight* const* next, int nnext, cudaStream_t stream);
 size_t gemv_workspace_bytes(const tern_weight& w, int64_t M);
 
+// Decode GEMV for one token on a persistent, warp-specialised grid (tern_decode1.cu): row-level
+// residual planes and offsets, K % 512 == 0; decode1_supported tells whether it takes the call.
+bool decode1_supported(const tern_weight* const* ws, int nw);
+tern_status decode1_launch_group(const tern_weight* const* ws, int nw, const __half* x, __half* const* ys,
+                                 const tern_weight* const* next, int nnext, cudaStream_t stream);
+
 // Prefill GEMM on tcgen05 (tern_gemm_sm100.cu), M > 16.
 tern_status gemm_launch(const tern_weight& w, const __half* x, int64_t M, __half* y, void* workspace,
                         cudaStream_t stream);

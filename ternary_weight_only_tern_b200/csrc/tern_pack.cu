@@ -14,7 +14,7 @@
 #include <atomic>
 #include <mutex>
 
-#include "tern_internal.cuh"
+#include "tern_device.cuh"
 
 namespace tern {
 
@@ -293,6 +293,15 @@ __global__ void __launch_bounds__(kRowsThreads) rows_from_bitmap_kernel(const ui
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, kBadInput);
 }
 
+// The failure path of the bounded waits, on its own: one thread waits on a barrier that nothing
+// completes and, when the bound runs out, records the timeout as a linear kernel would.
+__global__ void selftest_timeout_kernel(uint64_t cycles, unsigned int* status) {
+    __shared__ uint64_t bar;
+    dev::mbar_init(&bar, 1);
+    dev::fence_barrier_init();
+    if (!dev::mbar_wait_for(&bar, 0, cycles) && status) atomicOr(status, 1u);
+}
+
 int grid_for(int64_t items, int threads) {
     const int64_t want = (items + threads - 1) / threads;
     const int64_t cap = static_cast<int64_t>(sm_count()) * 32;
@@ -441,4 +450,12 @@ extern "C" tern_status tern_unpack_residual(const uint8_t* row_bitmap, int64_t N
     *r = int64_t(c);
     if (rs != TERN_OK) return rs;
     return (res_rows && int64_t(c) > r_cap) ? TERN_ERR_WORKSPACE : TERN_OK;
+}
+
+extern "C" tern_status tern_selftest_timeout(int64_t cycles, tern_stream s) {
+    if (cycles < 1 || cycles > (int64_t(1) << 32)) return TERN_ERR_SHAPE;
+    unsigned int* w = async_status_word();
+    if (!w) return TERN_ERR_CUDA;
+    selftest_timeout_kernel<<<1, 1, 0, as_cuda(s)>>>(uint64_t(cycles), w);
+    return cudaGetLastError() == cudaSuccess ? TERN_OK : TERN_ERR_CUDA;
 }
