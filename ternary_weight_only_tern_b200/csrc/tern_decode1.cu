@@ -12,12 +12,14 @@
 //  * Persistent grid, one CTA per SM. The 16-row strips of all weights of the launch are split
 //    into contiguous ranges that differ by at most one strip, one per CTA, so every output row is
 //    finished inside one CTA: no partial sum leaves the SM and no workspace is needed.
-//  * Warp-specialised CTA: a producer warp streams each strip's plane as 3D TMA boxes (16 rows x
-//    up to SB 512-wide K slabs, 128-byte swizzle, no multicast) into a ring of NS stages, and
-//    its 32 lanes copy the strip's scales (and offsets) beside them with cp.async; W consumer
-//    warps each own a fixed share of the K groups of every stage; an epilogue warp adds the
-//    consumers' partial sums in warp order, keeps the sums of the current segment (up to 256
-//    rows) in shared memory, adds the residual rows' sums and writes y.
+//  * Warp-specialised CTA. A bulk or TMA copy holds its issuing thread until the copy before it
+//    has landed, so four producer warps issue the strips' planes (one 3D TMA box each: 16 rows x
+//    up to SB 512-wide K slabs, 128-byte swizzle, no multicast) and four more the strips' scales
+//    and offsets (one bulk copy each), every one taking every fourth stage of a ring of NS. W
+//    consumer warps each own a fixed share of the K groups of every stage; once a warp has its
+//    words and scales in registers the stage is free again. An epilogue warp adds the consumers'
+//    partial sums in warp order, keeps the sums of the current segment (up to 256 rows) in shared
+//    memory, adds the residual rows' sums and writes y.
 //  * Residual rows: since R is sorted, the residual rows of a segment are the contiguous slots
 //    [s_a, s_a + span) of the residual plane; they stream as extra 16-slot strips after the
 //    segment's main strips, and each row's residual sum joins its main sum before the single
@@ -29,7 +31,7 @@
 //    groups, and each group accumulates in its own registers, whose column 2 g alone is read
 //    (the other columns multiply other groups' activations and are ignored). Lane q then holds
 //    group q's sums for its two rows, and the per-group scaling costs a few instructions per
-//    32 MMAs.
+//    32 MMAs. The groups' MMA chains are interleaved step by step with their decode.
 //  * Decode is branch-free: one LOP3 writes two 2-bit codes (trits p and p+8 of a word) into
 //    the mantissas of an fp16 pair (B_p + c) (tern_device.cuh); the MMA sums (B_p + 1 + t) x,
 //    and C = sum (B_p + 1) x, computed once per kernel by the same MMA chain on the constant
@@ -41,8 +43,8 @@
 //    weights its weight and slot-map reads start before griddepcontrol.wait, x is read and y is
 //    written only after it.
 //  * Every wait is bounded; a wait that runs out records TERN_ERR_TIMEOUT in the sticky status
-//    word and the warps leave their loops; the producer first waits, again bounded, for the TMA
-//    copies it issued.
+//    word and the warps leave their loops; the producers first wait, again bounded, for the TMA
+//    copies they issued.
 #include <algorithm>
 #include <mutex>
 
@@ -59,6 +61,12 @@ constexpr int kSegRows = kSegStrips * kStrip;
 constexpr int kMaxSegs = 8;                // segments per CTA
 constexpr int kSlabTile = kStrip * 128;    // bytes of one strip's slab: 16 rows x 128 B
 constexpr int kMaxNW = kMaxGemvGroup;      // weights per launch
+// A bulk or TMA copy holds its issuing thread until the copy before it has landed, so the bytes
+// in flight are (issuing threads) x (bytes per copy). Four warps issue the planes' boxes and four
+// the scales' (and offsets') runs, each taking every fourth stage.
+constexpr int kIssuePerKind = 4;
+constexpr int kStages = 8;                 // ring stages (fewer when shared memory runs short)
+constexpr int kProducers = 2 * kIssuePerKind;
 constexpr int kPfPerWeight = 6;
 constexpr int kPfRanges = kPfPerWeight * kMaxNW;
 
@@ -144,12 +152,45 @@ __device__ __forceinline__ void walk_jobs(const D1Args& a, int j0, int j1, const
     }
 }
 
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+// 1D bulk copy global -> this CTA's shared memory (16-byte aligned, bytes a multiple of 16),
+// completing as transaction bytes on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
 }
 
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+// The scales of rows [row0, row0 + rows) of a [*, G] fp16 array are one contiguous run. They
+// reach shared memory at dst as one bulk copy from the 16-byte boundary at or below the run's start
+// (the run then begins `skew` bytes into dst) and, for the last bytes that do not fill 16, plain
+// loads and stores. stage_plan writes those last bytes and returns the bulk copy's source offset
+// and size; stage_issue issues it (after the barrier expects its bytes).
+struct RowRun {
+    uint64_t a0;      // byte offset of the bulk copy's source
+    uint32_t bytes;   // bulk copy size (a multiple of 16, may be 0)
+};
+
+__device__ __forceinline__ RowRun stage_plan(uint32_t dst, const __half* base, int64_t row0, int rows, int G) {
+    RowRun r{0, 0};
+    if (rows <= 0) return r;
+    const uint64_t start = uint64_t(row0) * G * 2, end = start + uint64_t(rows) * G * 2;
+    const uint64_t a0 = start & ~uint64_t(15), a1 = end & ~uint64_t(15);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(base);
+    for (uint64_t b = a1; b < end; b += 2) {
+        const unsigned short h = __ldg(reinterpret_cast<const unsigned short*>(src + b));
+        asm volatile("st.shared.u16 [%0], %1;" ::"r"(dst + uint32_t(b - a0)), "h"(h) : "memory");
+    }
+    r.a0 = a0;
+    r.bytes = uint32_t(a1 - a0);
+    return r;
+}
+
+__device__ __forceinline__ void stage_issue(uint32_t dst, const __half* base, RowRun r, uint64_t* bar) {
+    if (r.bytes) bulk_load(dst, reinterpret_cast<const uint8_t*>(base) + r.a0, r.bytes, bar);
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
 // 3D tiled TMA load (no multicast) into this CTA's shared memory, completing on `bar`.
@@ -160,6 +201,28 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         "[%5];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Bounded wait that polls the barrier with the non-blocking test_wait: a warp suspended in
+// try_wait was measured to resume about a microsecond after the phase completed, which at this
+// kernel's stage rate costs more than the issue slots the polling takes.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
+    const uint32_t addr = smem_u32(bar);
+    uint64_t t0 = 0;
+    for (uint32_t i = 0;; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(addr), "r"(parity)
+            : "memory");
+        if (done) return true;
+        const uint64_t t = clock64();
+        if (i == 0) t0 = t;
+        else if (t - t0 > kWaitLimitCycles) return false;
+    }
 }
 
 __device__ __forceinline__ float sel4(int q, float a0, float a1, float a2, float a3) {
@@ -178,8 +241,10 @@ __device__ __forceinline__ void warp_groups(int gc, int w, int W, int& g0, int& 
 // tile fall in 32 distinct banks.
 __device__ __forceinline__ int lane_row(int rr) { return rr < 4 ? 2 * rr : 2 * (rr - 4) + 1; }
 
-template <int W>
-__global__ void __launch_bounds__((W + 2) * 32, 1) decode1_kernel(const __grid_constant__ D1Maps maps,
+// W consumer warps; GW groups per warp per stage (a warp with fewer groups in a stage repeats
+// its last one and discards the extra sums).
+template <int W, int GW>
+__global__ void __launch_bounds__((W + kProducers + 1) * 32, 1) decode1_kernel(const __grid_constant__ D1Maps maps,
                                                                   const __grid_constant__ D1Args a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -188,13 +253,15 @@ __global__ void __launch_bounds__((W + 2) * 32, 1) decode1_kernel(const __grid_c
     const int gcmax = 4 * SB;                                   // groups per full chunk
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + a.o_bar);
     uint64_t* redfull = full + NS;
-    uint64_t* empty = redfull + NS;
-    uint64_t* meta_bar = empty + NS;
+    uint64_t* empty = redfull + NS;                             // the stage's tile and scales are free
+    uint64_t* redempty = empty + NS;                            // the stage's partial sums were read
+    uint64_t* meta_bar = redempty + NS;
     int* abort_flag = reinterpret_cast<int*>(meta_bar + 1);
     const uint32_t stage0 = smem_u32(smem);
     const int stage_bytes = SB * kSlabTile;
-    __half* sc_base = reinterpret_cast<__half*>(smem + a.o_sc);  // [NS][16][gcmax]
-    __half* mu_base = reinterpret_cast<__half*>(smem + a.o_mu);  // [NS][16][gcmax]
+    const int sc_stride = (32 * a.G + 16 + 15) & ~15;          // bytes per stage: 16 rows x G, + skew
+    uint8_t* sc_base = smem + a.o_sc;                            // [NS][16 rows][G] fp16 (skewed)
+    uint8_t* mu_base = smem + a.o_mu;                            // [NS][16 rows][G] fp16
     float* red = reinterpret_cast<float*>(smem + a.o_red);       // [NS][W][16]
     __half* xs = reinterpret_cast<__half*>(smem + a.o_xs);       // [K], pairs adjacent
     float* cofs = reinterpret_cast<float*>(smem + a.o_cofs);     // [nchunk][W][4]
@@ -206,9 +273,10 @@ __global__ void __launch_bounds__((W + 2) * 32, 1) decode1_kernel(const __grid_c
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
-            mbar_init(&full[s], 1 + 32);
+            mbar_init(&full[s], 2);             // the plane's issuer and the scales' issuer
             mbar_init(&redfull[s], W);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], W);
+            mbar_init(&redempty[s], 1);
         }
         mbar_init(meta_bar, 1);
         *abort_flag = 0;
@@ -225,20 +293,33 @@ __global__ void __launch_bounds__((W + 2) * 32, 1) decode1_kernel(const __grid_c
         if (a.status) atomicOr(a.status, 1u);
     };
     auto meta_wait = [&]() -> bool {
-        if (mbar_wait(meta_bar, 0)) return true;
+        if (mbar_wait_sleep(meta_bar, 0)) return true;
         fail();
         return false;
     };
 
-    if (warp == W) {
-        // ------------------------------------------------------------ producer
+    if (warp >= W && warp < W + kProducers) {
+        // ------------------------------------------------------------ producers
+        // producer warp p < kIssuePerKind issues the planes of the jobs u with
+        // u % kIssuePerKind == p, warp kIssuePerKind + p their scales and offsets
+        const int pw = (warp - W) % kIssuePerKind;
+        const bool planes = (warp - W) < kIssuePerKind;
+        if (warp == W && lane < a.nw) {
+            prefetch_tensormap(&maps.m1[lane]);
+            prefetch_tensormap(&maps.m2[lane]);
+        }
         if (!a.static_weights) grid_dependency_wait();
-        int job = 0;
+        int job = 0, last_mine = -1;
         walk_jobs(a, j0, j1, meta, meta_wait, [&](int kind, int k, const Seg& sg, int jj, int c) -> bool {
             if (*vabort) return false;
+            if (job % kIssuePerKind != pw) {
+                ++job;
+                return true;
+            }
+            last_mine = job;
             const D1Weight& Wt = a.w[sg.wi];
             const int s = job % NS, round = job / NS;
-            if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1)) {
+            if (round > 0 && !mbar_wait_sleep(&empty[s], (round - 1) & 1)) {
                 fail();
                 return false;
             }
@@ -247,39 +328,36 @@ __global__ void __launch_bounds__((W + 2) * 32, 1) decode1_kernel(const __grid_c
             const int64_t nrows = kind ? Wt.r : Wt.N;
             const __half* scale = kind ? Wt.scale2 : Wt.scale1;
             const __half* mu = kind == 0 ? Wt.mu : nullptr;
-            const int gc = min(gcmax, a.G - c * gcmax);
-            if (lane == 0) {
+            if (lane == 0 && planes) {
+                // the strip's plane: one TMA box, counted as transaction bytes on the barrier
                 mbar_arrive_expect_tx(&full[s], uint32_t(stage_bytes));
                 tma_load_3d(stage0 + s * stage_bytes, map, 0, int(row0), c * SB, &full[s]);
+            } else if (lane == 0) {
+                // its 16 rows of scales (and offsets); the barrier expects the bytes first
+                const int rows = int(max(int64_t(0), min(int64_t(kStrip), nrows - row0)));
+                const uint32_t scd = smem_u32(sc_base + s * sc_stride), mud = smem_u32(mu_base + s * sc_stride);
+                const RowRun rs = stage_plan(scd, scale, row0, rows, a.G);
+                const RowRun rm = mu ? stage_plan(mud, mu, row0, rows, a.G) : RowRun{0, 0};
+                mbar_arrive_expect_tx(&full[s], rs.bytes + rm.bytes);
+                stage_issue(scd, scale, rs, &full[s]);
+                if (mu) stage_issue(mud, mu, rm, &full[s]);
             }
-            // scales (and offsets) of the 16 rows for the chunk's groups, 8 bytes at a time
-            const int per_row = gc / 4;
-            const uint32_t scd = smem_u32(sc_base + s * kStrip * gcmax), mud = smem_u32(mu_base + s * kStrip * gcmax);
-            for (int p = lane; p < kStrip * per_row; p += 32) {
-                const int row = p / per_row, col = p - row * per_row;
-                const bool v = row0 + row < nrows;
-                const int64_t off = (v ? (row0 + row) * a.G : 0) + int64_t(c) * gcmax + 4 * col;
-                const uint32_t d = uint32_t(row * gcmax + 4 * col) * 2;
-                cp_async8(scd + d, scale + off, v ? 8u : 0u);
-                if (mu) cp_async8(mud + d, mu + off, v ? 8u : 0u);
-            }
-            cp_async_arrive_noinc(&full[s]);
             ++job;
             return true;
         });
         // the next call's weights into L2 (a hint), then wait for the copies still in flight
-        if (lane == 0) {
+        if (lane == 0 && warp == W) {
             for (int i = 0; i < a.npf; ++i) {
                 const int64_t lo = int64_t(b) * a.pf_per[i], hi = min(a.pf_bytes[i], lo + a.pf_per[i]);
                 if (lo < hi) prefetch_l2_bulk(a.pf_ptr[i] + lo, uint32_t(hi - lo));
             }
         }
-        for (int u = max(0, job - NS); u < job; ++u)
-            if (!mbar_wait(&full[u % NS], (u / NS) & 1)) break;
+        for (int u = max(0, job - NS); u <= last_mine; ++u)
+            if (u % kIssuePerKind == pw && !mbar_wait(&full[u % NS], (u / NS) & 1)) break;
         return;
     }
 
-    if (warp == W + 1) {
+    if (warp == W + kProducers) {
         // ------------------------------------------------------------ epilogue
         // segment metadata: the slots of the segment's residual rows
         if (!a.static_weights) grid_dependency_wait();
@@ -347,7 +425,7 @@ __global__ void __launch_bounds__((W + 2) * 32, 1) decode1_kernel(const __grid_c
                 cur = sg;
             }
             const int s = job % NS, round = job / NS;
-            if (!mbar_wait(&redfull[s], round & 1)) {
+            if (!mbar_wait_sleep(&redfull[s], round & 1)) {
                 fail();
                 return false;
             }
@@ -359,7 +437,7 @@ __global__ void __launch_bounds__((W + 2) * 32, 1) decode1_kernel(const __grid_c
                 dst[idx] = c ? dst[idx] + v : v;
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
+            if (lane == 0) mbar_arrive(&redempty[s]);
             ++job;
             return true;
         });
@@ -403,7 +481,8 @@ __global__ void __launch_bounds__((W + 2) * 32, 1) decode1_kernel(const __grid_c
     // C and X of every chunk's groups of this warp: one MMA chain each on the constant patterns
     for (int c = 0; c < nchunk; ++c) {
         load_x(c);
-        float cz[4] = {0.f, 0.f, 0.f, 0.f}, co[4] = {0.f, 0.f, 0.f, 0.f};
+        // the same chain as the main sums (both words of the lane into one accumulator)
+        float cz[4] = {}, co[4] = {};
         const uint32_t one[4] = {kHalf2One, kHalf2One, kHalf2One, kHalf2One};
 #pragma unroll
         for (int h = 0; h < 2; ++h)
@@ -423,6 +502,48 @@ __global__ void __launch_bounds__((W + 2) * 32, 1) decode1_kernel(const __grid_c
     }
     __syncwarp();
     if (nchunk == 1) load_x(0);
+    if (!meta_wait()) return;
+
+    struct Sc {
+        unsigned short sa, sb, ma, mb;
+    };
+    // A job's accumulators and what its epilogue (per-group scaling, quad reduction, hand-off of
+    // the 16 row sums to the epilogue warp) needs.
+    struct Pending {
+        float acc[4][4];
+        Sc sc;
+        int s, round, c, ng, mu;
+    };
+    auto finish = [&](const Pending& pd) -> bool {
+        float p0 = 0.f, p1 = 0.f;
+        if (q < pd.ng) {
+            const float v0 = sel4(q, pd.acc[0][0], pd.acc[1][0], pd.acc[2][0], pd.acc[3][0]);
+            const float v1 = sel4(q, pd.acc[0][2], pd.acc[1][2], pd.acc[2][2], pd.acc[3][2]);
+            const float C = cofs[(pd.c * W + warp) * 4 + q];
+            p0 = __half2float(__ushort_as_half(pd.sc.sa)) * (v0 - C);
+            p1 = __half2float(__ushort_as_half(pd.sc.sb)) * (v1 - C);
+            if (pd.mu) {
+                const float X = xsum[(pd.c * W + warp) * 4 + q];
+                p0 = fmaf(__half2float(__ushort_as_half(pd.sc.ma)), X, p0);
+                p1 = fmaf(__half2float(__ushort_as_half(pd.sc.mb)), X, p1);
+            }
+        }
+        p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
+        p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
+        p0 += __shfl_xor_sync(0xffffffffu, p0, 2);
+        p1 += __shfl_xor_sync(0xffffffffu, p1, 2);
+        if (pd.round > 0 && !mbar_wait_sleep(&redempty[pd.s], (pd.round - 1) & 1)) {
+            fail();
+            return false;
+        }
+        if (q == 0) {
+            red[(pd.s * W + warp) * kStrip + pr] = p0;
+            red[(pd.s * W + warp) * kStrip + pr + 8] = p1;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&redfull[pd.s]);
+        return true;
+    };
 
     int job = 0;
     walk_jobs(a, j0, j1, meta, meta_wait, [&](int kind, int k, const Seg& sg, int jj, int c) -> bool {
@@ -432,57 +553,73 @@ __global__ void __launch_bounds__((W + 2) * 32, 1) decode1_kernel(const __grid_c
         const int gc = min(gcmax, a.G - c * gcmax);
         warp_groups(gc, warp, W, g0, ng);
         if (nchunk > 1) load_x(c);
-        if (!mbar_wait(&full[s], round & 1)) {
+        if (!mbar_wait_sleep(&full[s], round & 1)) {
             fail();
             return false;
         }
         const uint32_t tile = stage0 + s * stage_bytes;
-        float acc[4][4];
+        // the words of the warp's GW groups (rows pr and pr + 8, words 2q and 2q + 1 of each)
+        uint2 wa[GW], wb[GW];
 #pragma unroll
-        for (int gi = 0; gi < 4; ++gi) acc[gi][0] = acc[gi][1] = acc[gi][2] = acc[gi][3] = 0.f;
-#pragma unroll
-        for (int gi = 0; gi < 4; ++gi) {
-            if (gi < ng) {
-                const int g = g0 + gi;                      // group within the chunk
-                const int slab = g >> 2, wofs = (g & 3) * 8 + 2 * q;
-                const uint32_t sw = (uint32_t((wofs >> 2) ^ (pr & 7)) << 4) | uint32_t((wofs & 3) * 4);
-                const uint32_t base = tile + slab * kSlabTile + sw;
-                const uint2 wa = lds_u2(base + pr * 128), wb = lds_u2(base + (pr + 8) * 128);
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t A[4][4];
-                    decode_word_pair(h ? wa.y : wa.x, h ? wb.y : wb.x, A);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) mma_16816(acc[gi], A[i], xr[8 * h + 2 * i], xr[8 * h + 2 * i + 1]);
-                }
-            }
+        for (int gi = 0; gi < GW; ++gi) {
+            const int g = g0 + min(gi, max(ng - 1, 0));     // group within the chunk
+            const int slab = g >> 2, wofs = (g & 3) * 8 + 2 * q;
+            const uint32_t sw = (uint32_t((wofs >> 2) ^ (pr & 7)) << 4) | uint32_t((wofs & 3) * 4);
+            const uint32_t base = tile + slab * kSlabTile + sw;
+            wa[gi] = lds_u2(base + pr * 128);
+            wb[gi] = lds_u2(base + (pr + 8) * 128);
         }
-        // lane q: group q's sums for rows pr and pr + 8 (column 2q of its accumulator)
-        float p0 = 0.f, p1 = 0.f;
+        // this lane's scales (and offsets): rows pr and pr + 8, group q of the warp's groups
+        Sc cur{0, 0, 0, 0};
+        const bool has_mu = kind == 0 && a.w[sg.wi].mu;
         if (q < ng) {
-            const float v0 = sel4(q, acc[0][0], acc[1][0], acc[2][0], acc[3][0]);
-            const float v1 = sel4(q, acc[0][2], acc[1][2], acc[2][2], acc[3][2]);
-            const float C = cofs[(c * W + warp) * 4 + q];
-            const __half* sc = sc_base + s * kStrip * gcmax + g0 + q;
-            p0 = __half2float(sc[pr * gcmax]) * (v0 - C);
-            p1 = __half2float(sc[(pr + 8) * gcmax]) * (v1 - C);
-            if (kind == 0 && a.w[sg.wi].mu) {
-                const float X = xsum[(c * W + warp) * 4 + q];
-                const __half* m = mu_base + s * kStrip * gcmax + g0 + q;
-                p0 = fmaf(__half2float(m[pr * gcmax]), X, p0);
-                p1 = fmaf(__half2float(m[(pr + 8) * gcmax]), X, p1);
+            const int64_t row0 = kind ? int64_t(meta[2 * k]) + int64_t(jj) * kStrip : int64_t(jj) * kStrip;
+            const int skew = int((uint64_t(row0) * a.G * 2) & 15);
+            const int gq = c * gcmax + g0 + q;
+            const unsigned short* sc = reinterpret_cast<const unsigned short*>(sc_base + s * sc_stride + skew) + gq;
+            cur.sa = sc[pr * a.G];
+            cur.sb = sc[(pr + 8) * a.G];
+            if (has_mu) {
+                const unsigned short* m = reinterpret_cast<const unsigned short*>(mu_base + s * sc_stride + skew) + gq;
+                cur.ma = m[pr * a.G];
+                cur.mb = m[(pr + 8) * a.G];
             }
         }
-        p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
-        p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
-        p0 += __shfl_xor_sync(0xffffffffu, p0, 2);
-        p1 += __shfl_xor_sync(0xffffffffu, p1, 2);
-        if (q == 0) {
-            red[(s * W + warp) * kStrip + pr] = p0;
-            red[(s * W + warp) * kStrip + pr + 8] = p1;
-        }
+        // the words and scales are in registers: the stage may be refilled
         __syncwarp();
-        if (lane == 0) mbar_arrive(&redfull[s]);
+        if (lane == 0) mbar_arrive(&empty[s]);
+        // GW independent accumulator chains, their MMAs interleaved step by step
+        Pending nw;
+#pragma unroll
+        for (int gi = 0; gi < 4; ++gi) nw.acc[gi][0] = nw.acc[gi][1] = nw.acc[gi][2] = nw.acc[gi][3] = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t sh[GW][6];
+#pragma unroll
+            for (int gi = 0; gi < GW; ++gi) {
+                const uint32_t a0 = h ? wa[gi].y : wa[gi].x, b0 = h ? wb[gi].y : wb[gi].x;
+                sh[gi][0] = a0; sh[gi][1] = a0 << 6; sh[gi][2] = a0 >> 6;
+                sh[gi][3] = b0; sh[gi][4] = b0 << 6; sh[gi][5] = b0 >> 6;
+            }
+#define TERN_D1_STEP(I)                                                                                \
+    _Pragma("unroll") for (int gi = 0; gi < GW; ++gi) {                                                \
+        uint32_t A[4];                                                                                 \
+        decode_mma<I>(sh[gi][0], sh[gi][1], sh[gi][2], sh[gi][3], sh[gi][4], sh[gi][5], A);            \
+        mma_16816(nw.acc[gi], A, xr[8 * h + 2 * (I)], xr[8 * h + 2 * (I) + 1]);                        \
+    }
+            TERN_D1_STEP(0)
+            TERN_D1_STEP(1)
+            TERN_D1_STEP(2)
+            TERN_D1_STEP(3)
+#undef TERN_D1_STEP
+        }
+        nw.sc = cur;
+        nw.s = s;
+        nw.round = round;
+        nw.c = c;
+        nw.ng = ng;
+        nw.mu = has_mu ? 1 : 0;
+        if (!finish(nw)) return false;
         ++job;
         return true;
     });
@@ -503,45 +640,41 @@ bool slab_map(CUtensorMap* map, const uint32_t* plane, int64_t rows, int64_t K, 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+
 struct Layout {
-    int W, SB, nchunk, NS;
+    int W, SB, GW, nchunk, NS;
     int o_sc, o_mu, o_red, o_xs, o_cofs, o_xsum, o_meta, o_bslot, o_mainy, o_resy, o_bar, total;
 };
 
-// Consumer warps and slabs per stage: the chunk's groups split over W warps (at most 4 each); W
-// is 8 or 10, whichever loses less to the uneven split.
-void plan_warps(int G, int& W, int& SB) {
+// Consumer warps, slabs per stage and groups per warp: every warp computes GW groups per stage
+// (ceil of the chunk's groups over W), so the split that wastes the fewest computed groups wins;
+// W is 8 or 10 (ties: 8).
+void plan_warps(int G, int& W, int& SB, int& GW) {
     double best = -1.0;
     for (int w : {8, 10}) {
         const int sb = std::min(G / 4, w);
-        const int gcmax = 4 * sb;
-        int tot = 0, mx = 0;
-        for (int g = 0; g < G; g += gcmax) {
-            const int gc = std::min(gcmax, G - g);
-            tot += gc;
-            int m = 0;
-            for (int i = 0; i < w; ++i) m = std::max(m, ((i + 1) * gc) / w - (i * gc) / w);
-            mx += m;
-        }
-        const double eff = double(tot) / (double(mx) * w) + (w == 8 ? 1e-9 : 0.0);   // ties: fewer warps
-        if (eff > best) {
+        const int gcmax = 4 * sb, nchunk = (G + gcmax - 1) / gcmax;
+        const int gw = (gcmax + w - 1) / w;
+        const double eff = double(G) / (double(nchunk) * gw * w);
+        if (eff > best + 1e-9) {
             best = eff;
             W = w;
             SB = sb;
+            GW = gw;
         }
     }
 }
 
 bool make_layout(int K, int NSwant, Layout& L) {
     const int G = K / kGroup;
-    plan_warps(G, L.W, L.SB);
+    plan_warps(G, L.W, L.SB, L.GW);
     L.nchunk = (G + 4 * L.SB - 1) / (4 * L.SB);
-    const int gcmax = 4 * L.SB;
     auto up = [](int v, int a) { return (v + a - 1) / a * a; };
     for (int NS = NSwant; NS >= 2; --NS) {
         int o = NS * L.SB * kSlabTile;
-        L.o_sc = o; o += up(NS * kStrip * gcmax * 2, 16);
-        L.o_mu = o; o += up(NS * kStrip * gcmax * 2, 16);
+        const int sc_stride = (32 * G + 16 + 15) & ~15;
+        L.o_sc = o; o += NS * sc_stride;
+        L.o_mu = o; o += NS * sc_stride;
         L.o_red = o; o += up(NS * L.W * kStrip * 4, 16);
         L.o_xs = o; o += up(K * 2, 16);
         L.o_cofs = o; o += up(L.nchunk * L.W * 4 * 4, 16);
@@ -550,7 +683,7 @@ bool make_layout(int K, int NSwant, Layout& L) {
         L.o_bslot = o; o += up(kMaxSegs * kSegRows * 2, 16);
         L.o_mainy = o; o += kSegRows * 4;
         L.o_resy = o; o += kSegRows * 4;
-        L.o_bar = o; o += up((3 * NS + 1) * 8 + 8, 16);
+        L.o_bar = o; o += up((4 * NS + 1) * 8 + 8, 16);
         L.total = o + 1024;     // alignment slack
         L.NS = NS;
         if (L.total <= 200 * 1024) return true;
@@ -558,14 +691,10 @@ bool make_layout(int K, int NSwant, Layout& L) {
     return false;
 }
 
-int env_int(const char* name, int dflt) {
-    const char* s = getenv(name);
-    return s ? atoi(s) : dflt;
-}
 
-template <int W>
+template <int W, int GW>
 tern_status launch1(const D1Maps& maps, const D1Args& args, int grid, size_t smem, cudaStream_t stream) {
-    auto kernel = decode1_kernel<W>;
+    auto kernel = decode1_kernel<W, GW>;
     static std::mutex mu;
     static bool configured[64] = {false};
     int dev = 0;
@@ -580,7 +709,7 @@ tern_status launch1(const D1Maps& maps, const D1Args& args, int grid, size_t sme
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(grid), 1, 1);
-    cfg.blockDim = dim3((W + 2) * 32, 1, 1);
+    cfg.blockDim = dim3((W + kProducers + 1) * 32, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -590,6 +719,16 @@ tern_status launch1(const D1Maps& maps, const D1Args& args, int grid, size_t sme
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kernel, maps, args) != cudaSuccess) return TERN_ERR_CUDA;
     return TERN_OK;
+}
+
+template <int W>
+tern_status launch_w(const Layout& L, const D1Maps& maps, const D1Args& args, int grid, cudaStream_t stream) {
+    switch (L.GW) {
+        case 1: return launch1<W, 1>(maps, args, grid, size_t(L.total), stream);
+        case 2: return launch1<W, 2>(maps, args, grid, size_t(L.total), stream);
+        case 3: return launch1<W, 3>(maps, args, grid, size_t(L.total), stream);
+        default: return launch1<W, 4>(maps, args, grid, size_t(L.total), stream);
+    }
 }
 
 }  // namespace
@@ -616,7 +755,7 @@ tern_status decode1_launch_group(const tern_weight* const* ws, int nw, const __h
     D1Args a = {};
     const int64_t K = ws[0]->K;
     Layout L;
-    if (!make_layout(int(K), env_int("TERN_DECODE_STAGES", 4), L)) return TERN_ERR_SHAPE;
+    if (!make_layout(int(K), kStages, L)) return TERN_ERR_SHAPE;
     int64_t S = 0;
     bool all_static = true, has_mu = false;
     for (int i = 0; i < nw; ++i) {
@@ -668,8 +807,7 @@ tern_status decode1_launch_group(const tern_weight* const* ws, int nw, const __h
         }
     }
     for (int i = 0; i < a.npf; ++i) a.pf_per[i] = ((a.pf_bytes[i] + grid - 1) / grid + 15) / 16 * 16;
-    if (L.W == 10) return launch1<10>(maps, a, grid, size_t(L.total), stream);
-    return launch1<8>(maps, a, grid, size_t(L.total), stream);
+    return L.W == 10 ? launch_w<10>(L, maps, a, grid, stream) : launch_w<8>(L, maps, a, grid, stream);
 }
 
 }  // namespace tern

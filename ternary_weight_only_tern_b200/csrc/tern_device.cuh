@@ -211,6 +211,18 @@ __device__ __forceinline__ void decode_word_pair(uint32_t wa, uint32_t wb, uint3
     A[3][2] = decode_pair<7>(wa, wal, war); A[3][3] = decode_pair<7>(wb, wbl, wbr);
 }
 
+// The A fragment of MMA I (pairs 2I, 2I+1) of a word pair, decoded on its own so that the MMAs
+// of several independent chains can be interleaved with their decode; wal/war (wbl/wbr) are the
+// word shifted left/right by 6.
+template <int I>
+__device__ __forceinline__ void decode_mma(uint32_t wa, uint32_t wal, uint32_t war, uint32_t wb, uint32_t wbl,
+                                           uint32_t wbr, uint32_t (&A)[4]) {
+    A[0] = decode_pair<2 * I>(wa, wal, war);
+    A[1] = decode_pair<2 * I>(wb, wbl, wbr);
+    A[2] = decode_pair<2 * I + 1>(wa, wal, war);
+    A[3] = decode_pair<2 * I + 1>(wb, wbl, wbr);
+}
+
 constexpr uint32_t kHalf2One = 0x3C003C00u;   // the fp16 pair (1, 1)
 
 // B_p + 1 (the decoded value of trit 0) for the pairs of MMA i (pairs 2*(i%4) and 2*(i%4)+1),

@@ -37,8 +37,9 @@ constexpr int BM = 256;                             // tokens per CTA tile
 constexpr int kUmmaM = 128;                         // tokens per MMA (two MMAs per K step)
 constexpr int BN = 256;
 constexpr int BK = 64;
-constexpr int kStages = 2;                          // x tile + dequantised W tile
-constexpr int kStagesP = 8;                         // packed codes
+constexpr int kStagesA = 3;                         // x tiles (from L2: the deeper ring covers its latency)
+constexpr int kStages = 2;                          // dequantised W tiles
+constexpr int kStagesP = 6;                         // packed codes
 constexpr int kDequantThreads = 256;
 constexpr int kThreads = 64 + kDequantThreads;
 constexpr int kABytes = BM * BK * 2;
@@ -69,11 +70,11 @@ struct GemmArgs {
 
 struct SmemLayout {
     static constexpr int a_off = 0;
-    static constexpr int b_off = a_off + kStages * kABytes;
+    static constexpr int b_off = a_off + kStagesA * kABytes;
     static constexpr int p1_off = b_off + kStages * kBBytes;                    // [kStagesP][256][16 B]
     static constexpr int p2_off = p1_off + kStagesP * kPBytes;                  // [kStagesP][256][16 B]
     static constexpr int bar_off = p2_off + kStagesP * kPBytes;
-    static constexpr int nbar = 3 * kStages + 2 * kStagesP + 1;
+    static constexpr int nbar = 2 * kStagesA + 2 * kStages + 2 * kStagesP + 1;
     static constexpr int tmem_off = bar_off + nbar * 8;
     static constexpr int cnt_off = tmem_off + 16;                               // 8 warp counts + total
     static constexpr int list_off = cnt_off + 48;                               // int2 [BN]
@@ -159,8 +160,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     uint8_t* smem_p1 = smem + SmemLayout::p1_off;
     uint8_t* smem_p2 = smem + SmemLayout::p2_off;
     uint64_t* full_a = reinterpret_cast<uint64_t*>(smem + SmemLayout::bar_off);
-    uint64_t* full_b = full_a + kStages;
-    uint64_t* empty = full_b + kStages;
+    uint64_t* empty_a = full_a + kStagesA;
+    uint64_t* full_b = empty_a + kStagesA;
+    uint64_t* empty = full_b + kStages;                // the dequantised W stage is free again
     uint64_t* full_p = empty + kStages;
     uint64_t* empty_p = full_p + kStagesP;
     uint64_t* tmem_full = empty_p + kStagesP;
@@ -174,8 +176,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     const int num_kb = int(a.K / BK);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kStagesA; ++s) {
             mbar_init(&full_a[s], 1);
+            mbar_init(&empty_a[s], 1);
+        }
+        for (int s = 0; s < kStages; ++s) {
             mbar_init(&full_b[s], kDequantThreads);
             mbar_init(&empty[s], 1);
         }
@@ -240,8 +245,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                                     p_issued * (BK / kCodesPerWord), s_lo + j * kResBox, &full_p[sp]);
                 }
                 if (!ok) break;
-                const int s = kb % kStages;
-                if (kb >= kStages) ok = mbar_wait(&empty[s], ((kb / kStages) - 1) & 1);
+                const int s = kb % kStagesA;
+                if (kb >= kStagesA) ok = mbar_wait(&empty_a[s], ((kb / kStagesA) - 1) & 1);
                 if (!ok) break;
                 mbar_arrive_expect_tx(&full_a[s], kABytes);
                 tma_load_2d(smem_a + s * kABytes, &tmap_x, kb * BK, int(m0), &full_a[s]);
@@ -249,20 +254,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                 issued = kb + 1;
             }
             // drain: every issued copy lands before the CTA may exit
-            for (int kb = issued - 1; kb >= 0 && kb >= issued - kStages; --kb)
-                if (!mbar_wait(&full_a[kb % kStages], (kb / kStages) & 1)) ok = false;
+            for (int kb = issued - 1; kb >= 0 && kb >= issued - kStagesA; --kb)
+                if (!mbar_wait(&full_a[kb % kStagesA], (kb / kStagesA) & 1)) ok = false;
             for (int kb = p_issued - 1; kb >= 0 && kb >= p_issued - kStagesP; --kb)
                 if (!mbar_wait(&full_p[kb % kStagesP], (kb / kStagesP) & 1)) ok = false;
         }
     } else if (warp == 1) {
         if (lane == 0) {
             for (int kb = 0; kb < num_kb && ok; ++kb) {
-                const int s = kb % kStages;
-                const uint32_t par = (kb / kStages) & 1;
-                ok = mbar_wait(&full_a[s], par) && mbar_wait(&full_b[s], par);
+                const int s = kb % kStages, sa = kb % kStagesA;
+                ok = mbar_wait(&full_a[sa], (kb / kStagesA) & 1) && mbar_wait(&full_b[s], (kb / kStages) & 1);
                 if (!ok) break;
                 tc_fence_after();
-                const uint8_t* as = smem_a + s * kABytes;
+                const uint8_t* as = smem_a + sa * kABytes;
                 const uint8_t* bs = smem_b + s * kBBytes;
 #pragma unroll
                 for (int k = 0; k < BK / 16; ++k) {
@@ -271,6 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
                     umma_f16(tmem_base, umma_desc_sw128(as + 32 * k), bd, acc);
                     umma_f16(tmem_base + uint32_t(BN), umma_desc_sw128(as + kABytes / 2 + 32 * k), bd, acc);
                 }
+                umma_commit(&empty_a[sa]);
                 umma_commit(&empty[s]);
             }
             umma_commit(tmem_full);          // also on a timeout: every issued MMA retires first
