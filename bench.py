@@ -47,10 +47,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 # kernel is built from: when they change, the number no longer describes the kernel and the
 # bench reports null until it is captured again.
 KERNEL_TRAFFIC = {
-    "gemv": {"sources": ["ternary_weight_only_tern_b200/csrc/tern_gemv.cu",
+    "gemv": {"sources": ["ternary_weight_only_tern_b200/csrc/tern_decode1.cu",
                          "ternary_weight_only_tern_b200/csrc/tern_device.cuh"],
-             "sha256": "dfc417d5311d539d471482404c15871dcd4a96b6bd9cd1af63cf2cbbd05f2fac",
-             "bytes": 30941440},
+             "sha256": None,
+             "bytes": None},
 }
 
 
@@ -168,13 +168,14 @@ def replica_value(world: int, units_per_rank: float, max_secs: float) -> float:
 
 
 # ------------------------------------------------------------------------------ workload
-def draw_layer_on_device(torch, api, shapes, dev, seed, elem_frac=None):
+def draw_layer_on_device(torch, api, shapes, dev, seed, elem_frac=None, res_pct=None, uniform=False):
     """One layer's projections, drawn on the device with a seeded torch generator (same
-    distributions as the host recipe: P(0) = 0.4, P(+-1) = 0.3; s1 ~ U[0.005, 0.02];
-    s2 ~ U[0.001, 0.005]; 15% residual rows uniformly without replacement) and packed with
-    tern_pack_exec. With elem_frac, the second plane is element-level instead: each weight is
-    masked with probability elem_frac and a masked weight draws a trit like the main plane, with
-    s2e ~ U[0.001, 0.005] per (row, group)."""
+    distributions as the host recipe: P(0) = 0.4, P(+-1) = 0.3, or 1/3 each with uniform;
+    s1 ~ U[0.005, 0.02]; s2 ~ U[0.001, 0.005]; res_pct (default 15) % residual rows uniformly
+    without replacement) and packed with tern_pack_exec. With elem_frac, the second plane is
+    element-level instead: each weight is masked with probability elem_frac and a masked weight
+    draws a trit like the main plane, with s2e ~ U[0.001, 0.005] per (row, group)."""
+    res_pct = RES_PCT if res_pct is None else res_pct
     from ternary_weight_only_tern_b200.synth import residual_count
     g = torch.Generator(device=dev)
     g.manual_seed(seed)
@@ -183,6 +184,8 @@ def draw_layer_on_device(torch, api, shapes, dev, seed, elem_frac=None):
         G = K // 128
 
         def trits(rows):
+            if uniform:
+                return torch.randint(0, 3, (rows, K), dtype=torch.int8, generator=g, device=dev) - 1
             u = torch.randint(0, 10, (rows, K), dtype=torch.uint8, generator=g, device=dev)
             return (u >= 7).to(torch.int8) - (u < 3).to(torch.int8)
 
@@ -197,7 +200,7 @@ def draw_layer_on_device(torch, api, shapes, dev, seed, elem_frac=None):
             out[name] = w
             del T1, T2e, mask
             continue
-        r = residual_count(N, RES_PCT)
+        r = residual_count(N, res_pct)
         rows = torch.randperm(N, generator=g, device=dev)[:r].sort().values.to(torch.int32)
         T2 = trits(r)
         s2 = (torch.rand((r, G), generator=g, device=dev) * 0.004 + 0.001).half()
@@ -210,6 +213,136 @@ def draw_layer_on_device(torch, api, shapes, dev, seed, elem_frac=None):
 
 def packed_bytes(w) -> int:
     return w.nbytes()
+
+
+COLD_BYTES = 384e6        # > 3x the 126 MB L2: a pool this large cycles every call's weight out of L2
+
+
+def cold_pool(torch, api, dev, shapes, seed, res_pct, uniform=False, max_copies=512):
+    """Distinct copies of one group of projections (shapes [(name, N, K)]), enough of them that
+    their packed bytes exceed COLD_BYTES, so that calls taken in turn each stream from HBM."""
+    first = draw_layer_on_device(torch, api, shapes, dev, seed, res_pct=res_pct, uniform=uniform)
+    per = sum(w.nbytes() for w in first.values())
+    n = int(min(max_copies, max(8, -(-COLD_BYTES // per))))
+    return [first] + [draw_layer_on_device(torch, api, shapes, dev, seed + i, res_pct=res_pct, uniform=uniform)
+                      for i in range(1, n)]
+
+
+def time_cold_calls(torch, api, dev, stream, pool, members, M, capture, time_graph, reps=5):
+    """Seconds per call of api.linear_group over the weights `members` of every pool entry in
+    turn (one launch each), replayed from a CUDA graph; and the algorithmic bytes per call."""
+    K = pool[0][members[0]].K
+    x = torch.randn((M, K), device=dev).half()
+    ys = [torch.empty((M, pool[0][n].N), dtype=torch.float16, device=dev) for n in members]
+
+    def fn():
+        for layer in pool:
+            api.linear_group(x, [layer[n] for n in members], outs=ys)
+    g = capture(torch, fn, stream)
+    t = time_graph(torch, g, reps, stream) / (reps * len(pool))
+    del g
+    wb = sum(pool[0][n].nbytes() for n in members)
+    ab = 2 * M * (K + sum(pool[0][n].N for n in members))
+    return t, wb, ab
+
+
+def workload_extras(torch, api, synth, dev, stream, peaks, capture, time_graph):
+    """The other workloads of the layer, each call on a cold weight: the single 4096 x 2560 GEMV
+    (trits 1/3 each, no residual rows), one Qwen3-4B layer's 7 projections, the 36-layer
+    Qwen3-4B stack at M = 1, 4 and 16 (four grouped launches per layer, like the 8B step), and
+    the Qwen3-8B projections one by one at M = 1, 4, 8 and 16."""
+    hbm = peaks["hbm_gbs"]
+    out = {}
+
+    def entry(t, wb, ab):
+        return {"us": t * 1e6, "packed_gbs": wb / t / 1e9, "frac": (wb + ab) / t / 1e9 / hbm,
+                "frac_of_8000": (wb + ab) / t / 1e9 / 8000.0}
+
+    # config 1
+    pool = cold_pool(torch, api, dev, [("single", 4096, 2560)], 5000, res_pct=0, uniform=True)
+    t, wb, ab = time_cold_calls(torch, api, dev, stream, pool, ["single"], 1, capture, time_graph)
+    out["single_gemv_4096x2560_m1"] = dict(entry(t, wb, ab), distinct_weights=len(pool))
+    del pool
+    # config 2: one launch per projection
+    shapes4 = [(n, N, K) for n, (N, K) in synth.QWEN3_4B.items()]
+    per = {}
+    for n, N, K in shapes4:
+        pool = cold_pool(torch, api, dev, [(n, N, K)], 6000, res_pct=10)
+        t, wb, ab = time_cold_calls(torch, api, dev, stream, pool, [n], 1, capture, time_graph)
+        per[n] = dict(entry(t, wb, ab), distinct_weights=len(pool))
+        del pool
+    out["qwen3_4b_layer_m1"] = {"per_projection": per,
+                                "layer_us": sum(v["us"] for v in per.values()),
+                                "note": "7 launches, one per projection, 10% residual rows"}
+    # config 3: the 36-layer stack, grouped launches, weights from an 8-layer pool (237 MB)
+    pool = [draw_layer_on_device(torch, api, shapes4, dev, seed=7000 + i, res_pct=10) for i in range(POOL_LAYERS)]
+    kd = {n: K for n, _, K in shapes4}
+    nd = {n: N for n, N, _ in shapes4}
+    stack = {}
+    for M in (1, 4, 16):
+        xs = {g: torch.randn((M, kd[m[0]]), device=dev).half() for g, m in GROUPS}
+        flat = torch.empty(LAYERS * M * sum(nd.values()), dtype=torch.float16, device=dev)
+        ys, off = [], 0
+        for _ in range(LAYERS):
+            d = {}
+            for n in nd:
+                d[n] = flat[off:off + M * nd[n]].view(M, nd[n])
+                off += M * nd[n]
+            ys.append(d)
+
+        def fn(xs=xs, ys=ys):
+            for layer in range(LAYERS):
+                for g, members in GROUPS:
+                    api.linear_group(xs[g], [pool[layer % POOL_LAYERS][n] for n in members],
+                                     outs=[ys[layer][n] for n in members])
+        g = capture(torch, fn, stream)
+        t = time_graph(torch, g, 20, stream) / 20
+        del g
+        wb = LAYERS * sum(pool[0][n].nbytes() for n in nd)
+        ab = LAYERS * sum(2 * M * (kd[m[0]] + sum(nd[n] for n in m)) for _, m in GROUPS)
+        stack[str(M)] = {"us_per_step": t * 1e6, "packed_gbs": wb / t / 1e9, "frac": (wb + ab) / t / 1e9 / hbm,
+                         "launches": LAYERS * len(GROUPS)}
+        del xs, ys, flat
+    out["qwen3_4b_stack"] = dict(stack, pool_mb=sum(w.nbytes() for L in pool for w in L.values()) / 1e6)
+    del pool
+    # config 4: the 8B projections, one launch each, at every M
+    per = {}
+    for n, (N, K) in synth.QWEN3_8B.items():
+        pool = cold_pool(torch, api, dev, [(n, N, K)], 8000, res_pct=15)
+        per[n] = {}
+        for M in (1, 4, 8, 16):
+            t, wb, ab = time_cold_calls(torch, api, dev, stream, pool, [n], M, capture, time_graph)
+            per[n][str(M)] = entry(t, wb, ab)
+        del pool
+    out["qwen3_8b_projections"] = per
+    return out
+
+
+def oracle_configs():
+    """The oracle on the host cores for each workload: one call per projection (config 3: one
+    layer, times 36, stated)."""
+    import oracle
+    from ternary_weight_only_tern_b200 import synth
+    out = {}
+
+    def timed(ts, M):
+        t0 = time.perf_counter()
+        nb = 0
+        for t in ts:
+            oracle.linear(t.x[:M], t.T1, t.s1, t.res_rows, t.T2, t.s2)
+            nb += (t.N + t.r) * t.K // 4 + 2 * (t.N + t.r) * (t.K // 128) + 4 * t.N
+        return time.perf_counter() - t0, nb
+
+    s, nb = timed(list(synth.draw_workload(synth.WORKLOADS[1])), 1)
+    out["single_gemv_4096x2560_m1"] = {"s": s, "packed_gbs": nb / s / 1e9}
+    layer = list(synth.draw_workload(synth.WORKLOADS[2]))
+    s, nb = timed(layer, 1)
+    out["qwen3_4b_layer_m1"] = {"s": s, "packed_gbs": nb / s / 1e9}
+    out["qwen3_4b_stack_m1"] = {"s": 36 * s, "packed_gbs": nb / s / 1e9, "note": "one layer timed, times 36"}
+    t8 = list(synth.draw_workload(synth.WORKLOADS[4]))
+    s, nb = timed(t8, 16)
+    out["qwen3_8b_projections_m16"] = {"s": s, "packed_gbs": nb / s / 1e9}
+    return out
 
 
 def time_graph(torch, graph, reps, stream):
@@ -457,9 +590,10 @@ def main():
     if not args.quick and world == 1:
         extra = extras(torch, api, synth, pool, shapes, names, stream, dev, ws, step_fn, step_bytes, make_io, peaks,
                        time_graph, capture)
+        extra["workloads"] = workload_extras(torch, api, synth, dev, stream, peaks, capture, time_graph)
 
     # ---------------- e2e through the Python API with host buffers
-    e2e_steps = max(3, min(20, args.steps // 100))
+    e2e_steps = 20
     xh = {gname: torch.randn((1, kdim[members[0]])).half().pin_memory() for gname, members in GROUPS}
     yh = torch.empty(flat1.numel(), dtype=torch.float16).pin_memory()
     h2d = sum(2 * kdim[members[0]] for _, members in GROUPS)
@@ -497,18 +631,22 @@ def main():
         e2e_step_eager()
     eager_secs = max_over_ranks(time.perf_counter() - t0)
     del g_e2e
-    e2e = {"value": world * wb * e2e_steps / e2e_secs / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+    e2e = {"value": world * wb * e2e_steps / eager_secs / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-           "eager_value": world * wb * e2e_steps / eager_secs / 1e9,
-           "note": "144 api.linear_group calls per step (q+k+v, o, gate+up, down per layer) with the step's 4 "
-                   "inputs copied in from pinned host memory and all 252 outputs (one buffer) copied back, captured once into a CUDA graph and replayed (wall clock "
-                   "around replay + synchronize); eager_value: the same calls issued from Python each step"}
+           "graph_value": world * wb * e2e_steps / e2e_secs / 1e9,
+           "note": "value: every step issues the 144 api.linear_group calls (q+k+v, o, gate+up, down per layer) "
+                   "from Python through the C ABI, with the step's 4 inputs copied in from pinned host memory "
+                   "and all 252 outputs (one buffer) copied back; wall clock around the step and its stream "
+                   "synchronize. graph_value: the same calls and copies captured once into a CUDA graph and "
+                   "replayed each step"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         nb, cs, threads, desc = oracle_sample()
         cpu = {"value": nb / cs / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
                "seconds": cs}
+        if not args.quick:
+            cpu["per_workload"] = oracle_configs()
 
     if world > 1:
         dist.destroy_process_group()
@@ -575,23 +713,16 @@ def extras(torch, api, synth, pool, shapes, names, stream, dev, ws, step_fn, ste
     out = {}
     kdim_of = {n: K for n, _, K in shapes}.__getitem__
     hbm = peaks["hbm_gbs"]
-    # per projection at M = 1 (one launch per projection), and per group (one launch per group)
+    # per group at M = 1 (one launch per group), each call on a cold weight (a pool of distinct
+    # copies larger than three L2s)
     xs1, ys1 = make_io(1)
     per = {}
-    for n in names:
-        g = capture(torch, step_fn(1, xs1, ys1, only=n, grouped=False), stream)
-        t = time_graph(torch, g, 50, stream) / (50 * LAYERS)
-        wb, ab = step_bytes(1, only=n, grouped=False)
-        per[n] = {"us": t * 1e6, "packed_gbs": wb / LAYERS / t / 1e9, "frac": (wb + ab) / LAYERS / t / 1e9 / hbm}
-        del g
-    out["per_projection_m1"] = per
-    per = {}
-    for gname, _ in GROUPS:
-        g = capture(torch, step_fn(1, xs1, ys1, only=gname), stream)
-        t = time_graph(torch, g, 50, stream) / (50 * LAYERS)
-        wb, ab = step_bytes(1, only=gname)
-        per[gname] = {"us": t * 1e6, "packed_gbs": wb / LAYERS / t / 1e9, "frac": (wb + ab) / LAYERS / t / 1e9 / hbm}
-        del g
+    for gi, (gname, members) in enumerate(GROUPS):
+        cp = cold_pool(torch, api, dev, [s_ for s_ in shapes if s_[0] in members], 9000 + 1000 * gi, res_pct=RES_PCT)
+        t, wb, ab = time_cold_calls(torch, api, dev, stream, cp, list(members), 1, capture, time_graph)
+        per[gname] = {"us": t * 1e6, "packed_gbs": wb / t / 1e9, "frac": (wb + ab) / t / 1e9 / hbm,
+                      "distinct_weights": len(cp)}
+        del cp
     out["per_group_m1"] = per
     # the whole stack with one launch per projection (252 per step), for comparison
     g = capture(torch, step_fn(1, xs1, ys1, grouped=False), stream)

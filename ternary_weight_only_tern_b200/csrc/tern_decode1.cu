@@ -33,7 +33,8 @@
 //    group q's sums for its two rows, and the per-group scaling costs a few instructions per
 //    32 MMAs. The groups' MMA chains are interleaved step by step with their decode.
 //  * Decode is branch-free: one LOP3 writes two 2-bit codes (trits p and p+8 of a word) into
-//    the mantissas of an fp16 pair (B_p + c) (tern_device.cuh); the MMA sums (B_p + 1 + t) x,
+//    the mantissas of an fp16 pair (B_p + c); pairs 0-4 read the codes in place and pairs 5-7
+//    after one shift of the word (tern_device.cuh); the MMA sums (B_p + 1 + t) x,
 //    and C = sum (B_p + 1) x, computed once per kernel by the same MMA chain on the constant
 //    pattern, is subtracted once per group, so a zero plane cancels bit for bit. With an offset,
 //    the group sums X_g come from the same chain on an all-ones pattern.
@@ -262,7 +263,7 @@ __global__ void __launch_bounds__((W + kProducers + 1) * 32, 1) decode1_kernel(c
     const int sc_stride = (32 * a.G + 16 + 15) & ~15;          // bytes per stage: 16 rows x G, + skew
     uint8_t* sc_base = smem + a.o_sc;                            // [NS][16 rows][G] fp16 (skewed)
     uint8_t* mu_base = smem + a.o_mu;                            // [NS][16 rows][G] fp16
-    float* red = reinterpret_cast<float*>(smem + a.o_red);       // [NS][W][16]
+    float* red = reinterpret_cast<float*>(smem + a.o_red);       // [NS][W][4 groups][16 rows]
     __half* xs = reinterpret_cast<__half*>(smem + a.o_xs);       // [K], pairs adjacent
     float* cofs = reinterpret_cast<float*>(smem + a.o_cofs);     // [nchunk][W][4]
     float* xsum = reinterpret_cast<float*>(smem + a.o_xsum);     // [nchunk][W][4]
@@ -431,7 +432,10 @@ __global__ void __launch_bounds__((W + kProducers + 1) * 32, 1) decode1_kernel(c
             }
             if (lane < kStrip) {
                 float v = 0.f;
-                for (int w = 0; w < W; ++w) v += red[(s * W + w) * kStrip + lane];
+                // every consumer warp's group sums, in warp order, then group order
+                for (int w = 0; w < W; ++w)
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) v += red[((s * W + w) * 4 + g) * kStrip + lane];
                 const int idx = kind ? jj * kStrip + lane : (jj - sg.ja) * kStrip + lane;
                 float* dst = kind ? res_y : main_y;
                 dst[idx] = c ? dst[idx] + v : v;
@@ -489,7 +493,7 @@ __global__ void __launch_bounds__((W + kProducers + 1) * 32, 1) decode1_kernel(c
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 uint32_t Z[4];
-                zero_trit_pattern(i, Z[0], Z[2]);
+                zero_trit_pattern_in_place(i, Z[0], Z[2]);
                 Z[1] = Z[0];
                 Z[3] = Z[2];
                 mma_16816(cz, Z, xr[8 * h + 2 * i], xr[8 * h + 2 * i + 1]);
@@ -507,8 +511,8 @@ __global__ void __launch_bounds__((W + kProducers + 1) * 32, 1) decode1_kernel(c
     struct Sc {
         unsigned short sa, sb, ma, mb;
     };
-    // A job's accumulators and what its epilogue (per-group scaling, quad reduction, hand-off of
-    // the 16 row sums to the epilogue warp) needs.
+    // A job's accumulators and what its epilogue (per-group scaling and the hand-off of each
+    // lane's two row sums of its group to the epilogue warp, which adds them) needs.
     struct Pending {
         float acc[4][4];
         Sc sc;
@@ -528,18 +532,13 @@ __global__ void __launch_bounds__((W + kProducers + 1) * 32, 1) decode1_kernel(c
                 p1 = fmaf(__half2float(__ushort_as_half(pd.sc.mb)), X, p1);
             }
         }
-        p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
-        p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
-        p0 += __shfl_xor_sync(0xffffffffu, p0, 2);
-        p1 += __shfl_xor_sync(0xffffffffu, p1, 2);
         if (pd.round > 0 && !mbar_wait_sleep(&redempty[pd.s], (pd.round - 1) & 1)) {
             fail();
             return false;
         }
-        if (q == 0) {
-            red[(pd.s * W + warp) * kStrip + pr] = p0;
-            red[(pd.s * W + warp) * kStrip + pr + 8] = p1;
-        }
+        float* rq = red + ((pd.s * W + warp) * 4 + q) * kStrip;
+        rq[pr] = p0;
+        rq[pr + 8] = p1;
         __syncwarp();
         if (lane == 0) mbar_arrive(&redfull[pd.s]);
         return true;
@@ -594,17 +593,17 @@ __global__ void __launch_bounds__((W + kProducers + 1) * 32, 1) decode1_kernel(c
         for (int gi = 0; gi < 4; ++gi) nw.acc[gi][0] = nw.acc[gi][1] = nw.acc[gi][2] = nw.acc[gi][3] = 0.f;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            uint32_t sh[GW][6];
+            uint32_t sh[GW][4];
 #pragma unroll
             for (int gi = 0; gi < GW; ++gi) {
                 const uint32_t a0 = h ? wa[gi].y : wa[gi].x, b0 = h ? wb[gi].y : wb[gi].x;
-                sh[gi][0] = a0; sh[gi][1] = a0 << 6; sh[gi][2] = a0 >> 6;
-                sh[gi][3] = b0; sh[gi][4] = b0 << 6; sh[gi][5] = b0 >> 6;
+                sh[gi][0] = a0; sh[gi][1] = a0 >> 6;
+                sh[gi][2] = b0; sh[gi][3] = b0 >> 6;
             }
 #define TERN_D1_STEP(I)                                                                                \
     _Pragma("unroll") for (int gi = 0; gi < GW; ++gi) {                                                \
         uint32_t A[4];                                                                                 \
-        decode_mma<I>(sh[gi][0], sh[gi][1], sh[gi][2], sh[gi][3], sh[gi][4], sh[gi][5], A);            \
+        decode_mma_in_place<I>(sh[gi][0], sh[gi][1], sh[gi][2], sh[gi][3], A);                         \
         mma_16816(nw.acc[gi], A, xr[8 * h + 2 * (I)], xr[8 * h + 2 * (I) + 1]);                        \
     }
             TERN_D1_STEP(0)
@@ -675,7 +674,7 @@ bool make_layout(int K, int NSwant, Layout& L) {
         const int sc_stride = (32 * G + 16 + 15) & ~15;
         L.o_sc = o; o += NS * sc_stride;
         L.o_mu = o; o += NS * sc_stride;
-        L.o_red = o; o += up(NS * L.W * kStrip * 4, 16);
+        L.o_red = o; o += up(NS * L.W * 4 * kStrip * 4, 16);
         L.o_xs = o; o += up(K * 2, 16);
         L.o_cofs = o; o += up(L.nchunk * L.W * 4 * 4, 16);
         L.o_xsum = o; o += up(L.nchunk * L.W * 4 * 4, 16);

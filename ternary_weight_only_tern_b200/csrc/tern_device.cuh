@@ -223,6 +223,45 @@ __device__ __forceinline__ void decode_mma(uint32_t wa, uint32_t wal, uint32_t w
     A[3] = decode_pair<2 * I + 1>(wb, wbl, wbr);
 }
 
+// A second decode with one shift per word instead of two: pairs 0-4 read their codes in place
+// (bits 2p, 2p+1 of each half) under the bases B_p = 1024, 256, 64, 16, 4, whose fp16 ulps are
+// 1, 1/4, 1/16, 1/64, 1/256, so the code lands as an integer; pairs 5-7 come from wr = w >> 6
+// under 64, 16, 4. Every B_p + c stays exact in fp16, and the MMA's products with fp16
+// activations stay exact in fp32.
+template <int P>
+__device__ __forceinline__ uint32_t decode_pair_in_place(uint32_t w, uint32_t wr) {
+    if (P == 0) return lop3_and_or(w, 0x00030003u, 0x64006400u);
+    if (P == 1) return lop3_and_or(w, 0x000C000Cu, 0x5C005C00u);
+    if (P == 2) return lop3_and_or(w, 0x00300030u, 0x54005400u);
+    if (P == 3) return lop3_and_or(w, 0x00C000C0u, 0x4C004C00u);
+    if (P == 4) return lop3_and_or(w, 0x03000300u, 0x44004400u);
+    if (P == 5) return lop3_and_or(wr, 0x00300030u, 0x54005400u);
+    if (P == 6) return lop3_and_or(wr, 0x00C000C0u, 0x4C004C00u);
+    return lop3_and_or(wr, 0x03000300u, 0x44004400u);
+}
+
+// The A fragment of MMA I (pairs 2I, 2I+1) of rows rr (word wa) and rr+8 (word wb) under the
+// in-place decode; war, wbr are the words shifted right by 6.
+template <int I>
+__device__ __forceinline__ void decode_mma_in_place(uint32_t wa, uint32_t war, uint32_t wb, uint32_t wbr,
+                                                    uint32_t (&A)[4]) {
+    A[0] = decode_pair_in_place<2 * I>(wa, war);
+    A[1] = decode_pair_in_place<2 * I>(wb, wbr);
+    A[2] = decode_pair_in_place<2 * I + 1>(wa, war);
+    A[3] = decode_pair_in_place<2 * I + 1>(wb, wbr);
+}
+
+// B_p + 1 of the in-place decode for the pairs of MMA i, as fp16x2 bits:
+// 1025 = 0x6401, 257 = 0x5C04, 65 = 0x5410, 17 = 0x4C40, 5 = 0x4500.
+__device__ __forceinline__ void zero_trit_pattern_in_place(int i4, uint32_t& lo, uint32_t& hi) {
+    switch (i4) {
+        case 0: lo = 0x64016401u; hi = 0x5C045C04u; break;   // pairs 0, 1: bases 1024, 256
+        case 1: lo = 0x54105410u; hi = 0x4C404C40u; break;   // pairs 2, 3: bases 64, 16
+        case 2: lo = 0x45004500u; hi = 0x54105410u; break;   // pairs 4, 5: bases 4, 64
+        default: lo = 0x4C404C40u; hi = 0x45004500u; break;  // pairs 6, 7: bases 16, 4
+    }
+}
+
 constexpr uint32_t kHalf2One = 0x3C003C00u;   // the fp16 pair (1, 1)
 
 // B_p + 1 (the decoded value of trit 0) for the pairs of MMA i (pairs 2*(i%4) and 2*(i%4)+1),
