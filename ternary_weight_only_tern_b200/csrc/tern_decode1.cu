@@ -12,32 +12,36 @@
 //  * Persistent grid, one CTA per SM. The 16-row strips of all weights of the launch are split
 //    into contiguous ranges that differ by at most one strip, one per CTA, so every output row is
 //    finished inside one CTA: no partial sum leaves the SM and no workspace is needed.
-//  * Warp-specialised CTA. A bulk or TMA copy holds its issuing thread until the copy before it
-//    has landed, so four producer warps issue the strips' planes (one 3D TMA box each: 16 rows x
-//    up to SB 512-wide K slabs, 128-byte swizzle, no multicast) and four more the strips' scales
-//    and offsets (one bulk copy each), every one taking every fourth stage of a ring of NS. W
-//    consumer warps each own a fixed share of the K groups of every stage; once a warp has its
-//    words and scales in registers the stage is free again. An epilogue warp adds the consumers'
-//    partial sums in warp order, keeps the sums of the current segment (up to 256 rows) in shared
-//    memory, adds the residual rows' sums and writes y.
+//  * A CTA walks its range as blocks of Sb strips (Sb = 1, 2, 4 or 8, chosen per launch from the
+//    strips per CTA and K). A block streams through a ring of NS stages, each stage SB 512-wide
+//    K slabs of the block's 16 Sb rows (one 3D TMA box, 128-byte swizzle, no multicast). Each of
+//    the W = 8 consumer warps owns one strip of the block and a fixed share of the K groups of
+//    every stage, and keeps its rows' sums in registers across the block's stages: partial sums
+//    leave a warp once per block, not once per stage.
+//  * Four producer warps issue the planes' boxes (a bulk or TMA copy holds its issuing thread for
+//    a while, so they take every fourth stage each) and two more the blocks' scales (and
+//    offsets), one bulk copy per block into one of two block buffers. An epilogue warp adds the
+//    warps' sums of each strip in warp order, keeps the sums of the current segment (up to 256
+//    rows) in shared memory, adds the residual rows' sums and writes y.
 //  * Residual rows: since R is sorted, the residual rows of a segment are the contiguous slots
-//    [s_a, s_a + span) of the residual plane; they stream as extra 16-slot strips after the
-//    segment's main strips, and each row's residual sum joins its main sum before the single
-//    rounding to fp16.
+//    [s_a, s_a + span) of the residual plane; they stream as extra blocks after the segment's
+//    main blocks, and each row's residual sum joins its main sum before the single rounding to
+//    fp16.
 //  * The signed sums run on the tensor pipe as mma.sync m16n8k16 (fp16 in, fp32 accumulate),
 //    A = 16 weight rows x 16 K of decoded trits. With one token, each of a warp's (up to 4)
 //    groups keeps the token in its own MMA column: lanes of row index rr = 2 g hold group g's
 //    activations, so one set of 16 activation registers per lane serves all of the warp's
 //    groups, and each group accumulates in its own registers, whose column 2 g alone is read
 //    (the other columns multiply other groups' activations and are ignored). Lane q then holds
-//    group q's sums for its two rows, and the per-group scaling costs a few instructions per
-//    32 MMAs. The groups' MMA chains are interleaved step by step with their decode.
+//    group q's sums for its two rows and scales them into its running row sums; the four lanes
+//    of a quad add theirs at the end of the block. The groups' MMA chains are interleaved step
+//    by step with their decode.
 //  * Decode is branch-free: one LOP3 writes two 2-bit codes (trits p and p+8 of a word) into
 //    the mantissas of an fp16 pair (B_p + c); pairs 0-4 read the codes in place and pairs 5-7
-//    after one shift of the word (tern_device.cuh); the MMA sums (B_p + 1 + t) x,
-//    and C = sum (B_p + 1) x, computed once per kernel by the same MMA chain on the constant
-//    pattern, is subtracted once per group, so a zero plane cancels bit for bit. With an offset,
-//    the group sums X_g come from the same chain on an all-ones pattern.
+//    after one shift of the word (tern_device.cuh); the MMA sums (B_p + 1 + t) x, and
+//    C = sum (B_p + 1) x, computed once per kernel and group by the same MMA chain on the
+//    constant pattern, is subtracted once per group, so a zero plane cancels bit for bit. With an
+//    offset, the group sums X_g come from the same chain on an all-ones pattern.
 //  * x is staged once per CTA in shared memory with the two activations of each decoded pair
 //    adjacent (pair p of word w = activations 16 w + p and 16 w + p + 8).
 //  * Programmatic dependent launch: the CTA lets the next kernel launch at once; with static
@@ -60,14 +64,29 @@ constexpr int kStrip = 16;                 // rows per strip (the MMA's M)
 constexpr int kSegStrips = 16;             // strips per segment
 constexpr int kSegRows = kSegStrips * kStrip;
 constexpr int kMaxSegs = 8;                // segments per CTA
-constexpr int kSlabTile = kStrip * 128;    // bytes of one strip's slab: 16 rows x 128 B
+constexpr int kSlabBytes = 128;            // one row of one 512-wide K slab
 constexpr int kMaxNW = kMaxGemvGroup;      // weights per launch
-// A bulk or TMA copy holds its issuing thread until the copy before it has landed, so the bytes
-// in flight are (issuing threads) x (bytes per copy). Four warps issue the planes' boxes and four
-// the scales' (and offsets') runs, each taking every fourth stage.
-constexpr int kIssuePerKind = 4;
+#ifndef TERN_D1_W
+#define TERN_D1_W 8
+#endif
+#ifndef TERN_D1_PLANE_ISSUERS
+#define TERN_D1_PLANE_ISSUERS 2
+#endif
+#ifndef TERN_D1_SCALE_ISSUERS
+#define TERN_D1_SCALE_ISSUERS 1
+#endif
+constexpr int kW = TERN_D1_W;                          // consumer warps
+constexpr int kPlaneIssuers = TERN_D1_PLANE_ISSUERS;   // warps issuing the planes' boxes
+constexpr int kScaleIssuers = TERN_D1_SCALE_ISSUERS;   // warps issuing the blocks' scales and offsets
+constexpr int kProducers = kPlaneIssuers + kScaleIssuers;
+constexpr int kThreads = (kW + kProducers + 1) * 32;
+#ifndef TERN_D1_RAMP
+#define TERN_D1_RAMP 0
+#endif
+constexpr int kRamp = TERN_D1_RAMP;        // stages in flight at the start before the first lands
 constexpr int kStages = 8;                 // ring stages (fewer when shared memory runs short)
-constexpr int kProducers = 2 * kIssuePerKind;
+constexpr int kScaleBufs = 2;              // block scale buffers
+constexpr int kRedBufs = 2;                // block partial-sum buffers
 constexpr int kPfPerWeight = 6;
 constexpr int kPfRanges = kPfPerWeight * kMaxNW;
 
@@ -82,7 +101,7 @@ struct D1Weight {
 };
 
 struct D1Maps {
-    CUtensorMap m1[kMaxNW];   // plane1 viewed as [slab][row][32 words]: box {32, 16, SB}
+    CUtensorMap m1[kMaxNW];   // plane1 viewed as [slab][row][32 words]: box {32, 16 Sb, SB}
     CUtensorMap m2[kMaxNW];   // plane2, the same
 };
 
@@ -91,15 +110,17 @@ struct D1Args {
     int32_t nw;
     const __half* x;          // [K]
     unsigned int* status;
-    int32_t K, G;
-    int32_t SB;               // slabs per stage (per TMA box)
-    int32_t nchunk;           // stages per strip = ceil(K / (512 SB))
+    int32_t K, G, nslab;
+    int32_t Sb;               // strips per block
+    int32_t SB;               // slabs per stage
+    int32_t nstage;           // stages per block = ceil(nslab / SB)
     int32_t NS;               // ring stages
     int32_t S;                // strips of the launch
     int32_t static_weights;
     int32_t has_mu;
     // shared-memory offsets in bytes from the 1024-aligned base (the stages start at 0)
     int32_t o_sc, o_mu, o_red, o_xs, o_cofs, o_xsum, o_meta, o_bslot, o_mainy, o_resy, o_bar;
+    int32_t sc_stride;        // bytes of one block scale buffer (16 Sb rows x G fp16, + skew)
     // L2 prefetch of the next call's weights: each CTA takes pf_per bytes of each range
     const uint8_t* pf_ptr[kPfRanges];
     int64_t pf_bytes[kPfRanges];
@@ -128,27 +149,46 @@ __device__ __forceinline__ bool next_seg(const D1Args& a, int& j, int j1, Seg& s
     return true;
 }
 
-// Every role walks the same job sequence: per segment, its main strips (nchunk stages each),
-// then its residual strips (known once the epilogue warp has published the segment metadata).
-// fn(kind, segment index, segment, strip within the kind, chunk) returns false to stop.
-template <typename Fn, typename MetaWait>
-__device__ __forceinline__ void walk_jobs(const D1Args& a, int j0, int j1, const int* meta, MetaWait meta_wait,
-                                          Fn fn) {
-    int j = j0, k = 0;
+// One block: Sb (or, at the end of a segment, fewer) strips of one plane of one weight.
+struct Blk {
+    int kind;      // 0 main plane, 1 residual plane
+    int k;         // segment index within the CTA
     Seg sg;
+    int first;     // first strip: of the weight (main) or of the segment's residual slots
+    int n;         // strips in the block (1..Sb)
+    int64_t row0;  // first row of the plane
+};
+
+// Every role walks the same block sequence: per segment, its main blocks, then its residual
+// blocks (known once the epilogue warp has published the segment metadata).
+// fn(block) returns false to stop.
+template <typename Fn, typename MetaWait>
+__device__ __forceinline__ void walk_blocks(const D1Args& a, int j0, int j1, const int* meta, MetaWait meta_wait,
+                                            Fn fn) {
+    int j = j0, k = 0;
+    Blk bk;
     bool have_meta = false;
-    while (k < kMaxSegs && next_seg(a, j, j1, sg)) {
-        for (int jj = sg.ja; jj < sg.jb; ++jj)
-            for (int c = 0; c < a.nchunk; ++c)
-                if (!fn(0, k, sg, jj, c)) return;
+    while (k < kMaxSegs && next_seg(a, j, j1, bk.sg)) {
+        bk.k = k;
+        bk.kind = 0;
+        for (int f = bk.sg.ja; f < bk.sg.jb; f += a.Sb) {
+            bk.first = f;
+            bk.n = min(a.Sb, bk.sg.jb - f);
+            bk.row0 = int64_t(f) * kStrip;
+            if (!fn(bk)) return;
+        }
         if (!have_meta) {
             if (!meta_wait()) return;
             have_meta = true;
         }
         const int nrs = meta[2 * k + 1];
-        for (int t = 0; t < nrs; ++t)
-            for (int c = 0; c < a.nchunk; ++c)
-                if (!fn(1, k, sg, t, c)) return;
+        bk.kind = 1;
+        for (int f = 0; f < nrs; f += a.Sb) {
+            bk.first = f;
+            bk.n = min(a.Sb, nrs - f);
+            bk.row0 = int64_t(meta[2 * k]) + int64_t(f) * kStrip;
+            if (!fn(bk)) return;
+        }
         ++k;
     }
 }
@@ -204,11 +244,13 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
-// Bounded wait that polls the barrier with the non-blocking test_wait: a warp suspended in
-// try_wait was measured to resume about a microsecond after the phase completed, which at this
-// kernel's stage rate costs more than the issue slots the polling takes.
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
-    const uint32_t addr = smem_u32(bar);
+// Pause between two polls of a barrier by the warps off the critical path (producers, epilogue).
+constexpr unsigned kIdlePauseNs = 64;
+
+// Bounded wait that polls the barrier with the non-blocking test_wait, pausing pause_ns between
+// polls: a warp suspended in try_wait was measured to resume about a microsecond after the phase
+// completed, which at this kernel's stage rate is too late.
+__device__ __forceinline__ bool mbar_poll_addr(uint32_t addr, uint32_t parity, unsigned pause_ns) {
     uint64_t t0 = 0;
     for (uint32_t i = 0;; ++i) {
         uint32_t done;
@@ -223,7 +265,16 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) 
         const uint64_t t = clock64();
         if (i == 0) t0 = t;
         else if (t - t0 > kWaitLimitCycles) return false;
+        if (pause_ns) __nanosleep(pause_ns);
     }
+}
+
+__device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity, unsigned pause_ns) {
+    return mbar_poll_addr(smem_u32(bar), parity, pause_ns);
+}
+
+__device__ __forceinline__ void mbar_arrive_addr(uint32_t addr) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(addr) : "memory");
 }
 
 __device__ __forceinline__ float sel4(int q, float a0, float a1, float a2, float a3) {
@@ -231,42 +282,51 @@ __device__ __forceinline__ float sel4(int q, float a0, float a1, float a2, float
     return (q & 2) ? hi : lo;
 }
 
-// Groups [g0, g0 + ng) of a chunk of gc groups belong to consumer warp w of W.
-__device__ __forceinline__ void warp_groups(int gc, int w, int W, int& g0, int& ng) {
-    g0 = (w * gc) / W;
-    ng = ((w + 1) * gc) / W - g0;
-}
-
 // Lane rows: lane row index rr of the MMA handles strip rows pi(rr) and pi(rr) + 8, with
 // pi = 0, 2, 4, 6, 1, 3, 5, 7, so that each half-warp's 8-byte reads of the 128-byte-swizzled
 // tile fall in 32 distinct banks.
 __device__ __forceinline__ int lane_row(int rr) { return rr < 4 ? 2 * rr : 2 * (rr - 4) + 1; }
 
-// W consumer warps; GW groups per warp per stage (a warp with fewer groups in a stage repeats
-// its last one and discards the extra sums).
-template <int W, int GW>
-__global__ void __launch_bounds__((W + kProducers + 1) * 32, 1) decode1_kernel(const __grid_constant__ D1Maps maps,
-                                                                  const __grid_constant__ D1Args a) {
+
+__device__ __forceinline__ unsigned short lds_u16(uint32_t addr) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return v;
+}
+
+// A consumer warp's share of a stage of gs groups: groups [g0, g0 + ng) (wi of the wps warps of
+// its strip).
+__device__ __forceinline__ void warp_share(int gs, int wi, int wps, int& g0, int& ng) {
+    g0 = (wi * gs) / wps;
+    ng = ((wi + 1) * gs) / wps - g0;
+}
+
+// GW: groups per consumer warp per stage at most (a warp with fewer repeats its last one and
+// discards the extra sums).
+template <int GW>
+__global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_constant__ D1Maps maps,
+                                                             const __grid_constant__ D1Args a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int NS = a.NS, SB = a.SB, nchunk = a.nchunk;
-    const int gcmax = 4 * SB;                                   // groups per full chunk
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + a.o_bar);
-    uint64_t* redfull = full + NS;
-    uint64_t* empty = redfull + NS;                             // the stage's tile and scales are free
-    uint64_t* redempty = empty + NS;                            // the stage's partial sums were read
-    uint64_t* meta_bar = redempty + NS;
+    const int NS = a.NS, SB = a.SB, Sb = a.Sb, nstage = a.nstage;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + a.o_bar);   // [NS] the stage's box landed
+    uint64_t* empty = full + NS;                  // [NS] every consumer has its words of the stage
+    uint64_t* sfull = empty + NS;                 // [kScaleBufs] the block's scales landed
+    uint64_t* sempty = sfull + kScaleBufs;        // [kScaleBufs] the block's scales are no longer read
+    uint64_t* redfull = sempty + kScaleBufs;      // [kRedBufs] the block's partial sums are written
+    uint64_t* redempty = redfull + kRedBufs;      // [kRedBufs] ... and were read
+    uint64_t* meta_bar = redempty + kRedBufs;
     int* abort_flag = reinterpret_cast<int*>(meta_bar + 1);
     const uint32_t stage0 = smem_u32(smem);
-    const int stage_bytes = SB * kSlabTile;
-    const int sc_stride = (32 * a.G + 16 + 15) & ~15;          // bytes per stage: 16 rows x G, + skew
-    uint8_t* sc_base = smem + a.o_sc;                            // [NS][16 rows][G] fp16 (skewed)
-    uint8_t* mu_base = smem + a.o_mu;                            // [NS][16 rows][G] fp16
-    float* red = reinterpret_cast<float*>(smem + a.o_red);       // [NS][W][4 groups][16 rows]
+    const int slab_bytes = Sb * kStrip * kSlabBytes;             // one slab of a stage: 16 Sb rows
+    const int stage_bytes = SB * slab_bytes;
+    uint8_t* sc_base = smem + a.o_sc;                            // [kScaleBufs][16 Sb rows][G] (skewed)
+    uint8_t* mu_base = smem + a.o_mu;                            // the same for the offsets
+    float* red = reinterpret_cast<float*>(smem + a.o_red);       // [kRedBufs][W][16 rows]
     __half* xs = reinterpret_cast<__half*>(smem + a.o_xs);       // [K], pairs adjacent
-    float* cofs = reinterpret_cast<float*>(smem + a.o_cofs);     // [nchunk][W][4]
-    float* xsum = reinterpret_cast<float*>(smem + a.o_xsum);     // [nchunk][W][4]
+    float* cofs = reinterpret_cast<float*>(smem + a.o_cofs);     // [G] C of every group
+    float* xsum = reinterpret_cast<float*>(smem + a.o_xsum);     // [G] X of every group
     int* meta = reinterpret_cast<int*>(smem + a.o_meta);         // [kMaxSegs][2]: s_a, residual strips
     int16_t* bslot = reinterpret_cast<int16_t*>(smem + a.o_bslot);  // [kMaxSegs][256]
     float* main_y = reinterpret_cast<float*>(smem + a.o_mainy);  // [256]
@@ -274,10 +334,16 @@ __global__ void __launch_bounds__((W + kProducers + 1) * 32, 1) decode1_kernel(c
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
-            mbar_init(&full[s], 2);             // the plane's issuer and the scales' issuer
-            mbar_init(&redfull[s], W);
-            mbar_init(&empty[s], W);
-            mbar_init(&redempty[s], 1);
+            mbar_init(&full[s], 1);              // the plane's issuer (plus the box's bytes)
+            mbar_init(&empty[s], kW);
+        }
+        for (int i = 0; i < kScaleBufs; ++i) {
+            mbar_init(&sfull[i], 1);             // the scales' issuer (plus the copies' bytes)
+            mbar_init(&sempty[i], kW);
+        }
+        for (int i = 0; i < kRedBufs; ++i) {
+            mbar_init(&redfull[i], kW);
+            mbar_init(&redempty[i], 1);
         }
         mbar_init(meta_bar, 1);
         *abort_flag = 0;
@@ -294,71 +360,96 @@ __global__ void __launch_bounds__((W + kProducers + 1) * 32, 1) decode1_kernel(c
         if (a.status) atomicOr(a.status, 1u);
     };
     auto meta_wait = [&]() -> bool {
-        if (mbar_wait_sleep(meta_bar, 0)) return true;
+        if (mbar_poll(meta_bar, 0, 0)) return true;
         fail();
         return false;
     };
 
-    if (warp >= W && warp < W + kProducers) {
-        // ------------------------------------------------------------ producers
-        // producer warp p < kIssuePerKind issues the planes of the jobs u with
-        // u % kIssuePerKind == p, warp kIssuePerKind + p their scales and offsets
-        const int pw = (warp - W) % kIssuePerKind;
-        const bool planes = (warp - W) < kIssuePerKind;
-        if (warp == W && lane < a.nw) {
+    if (warp >= kW && warp < kW + kPlaneIssuers) {
+        // ------------------------------------------------------------ plane issuers
+        // warp p issues the boxes of the jobs u (block stages, in walk order) with u % 4 == p
+        const int pw = warp - kW;
+        if (pw == 0 && lane < a.nw) {
             prefetch_tensormap(&maps.m1[lane]);
             prefetch_tensormap(&maps.m2[lane]);
         }
         if (!a.static_weights) grid_dependency_wait();
         int job = 0, last_mine = -1;
-        walk_jobs(a, j0, j1, meta, meta_wait, [&](int kind, int k, const Seg& sg, int jj, int c) -> bool {
+        walk_blocks(a, j0, j1, meta, meta_wait, [&](const Blk& bk) -> bool {
             if (*vabort) return false;
-            if (job % kIssuePerKind != pw) {
-                ++job;
-                return true;
+            const CUtensorMap* map = bk.kind ? &maps.m2[bk.sg.wi] : &maps.m1[bk.sg.wi];
+            for (int t = 0; t < nstage; ++t, ++job) {
+                if (job % kPlaneIssuers != pw) continue;
+                last_mine = job;
+                const int s = job % NS, round = job / NS;
+                if (round > 0 && !mbar_poll(&empty[s], (round - 1) & 1, kIdlePauseNs)) {
+                    fail();
+                    return false;
+                }
+                if (kRamp > 0 && round == 0 && job >= kRamp && !mbar_poll(&full[job - kRamp], 0, 0)) {
+                    fail();
+                    return false;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[s], uint32_t(stage_bytes));
+                    tma_load_3d(stage0 + s * stage_bytes, map, 0, int(bk.row0), t * SB, &full[s]);
+                }
             }
-            last_mine = job;
-            const D1Weight& Wt = a.w[sg.wi];
-            const int s = job % NS, round = job / NS;
-            if (round > 0 && !mbar_wait_sleep(&empty[s], (round - 1) & 1)) {
-                fail();
-                return false;
-            }
-            const CUtensorMap* map = kind ? &maps.m2[sg.wi] : &maps.m1[sg.wi];
-            const int64_t row0 = kind ? int64_t(meta[2 * k]) + int64_t(jj) * kStrip : int64_t(jj) * kStrip;
-            const int64_t nrows = kind ? Wt.r : Wt.N;
-            const __half* scale = kind ? Wt.scale2 : Wt.scale1;
-            const __half* mu = kind == 0 ? Wt.mu : nullptr;
-            if (lane == 0 && planes) {
-                // the strip's plane: one TMA box, counted as transaction bytes on the barrier
-                mbar_arrive_expect_tx(&full[s], uint32_t(stage_bytes));
-                tma_load_3d(stage0 + s * stage_bytes, map, 0, int(row0), c * SB, &full[s]);
-            } else if (lane == 0) {
-                // its 16 rows of scales (and offsets); the barrier expects the bytes first
-                const int rows = int(max(int64_t(0), min(int64_t(kStrip), nrows - row0)));
-                const uint32_t scd = smem_u32(sc_base + s * sc_stride), mud = smem_u32(mu_base + s * sc_stride);
-                const RowRun rs = stage_plan(scd, scale, row0, rows, a.G);
-                const RowRun rm = mu ? stage_plan(mud, mu, row0, rows, a.G) : RowRun{0, 0};
-                mbar_arrive_expect_tx(&full[s], rs.bytes + rm.bytes);
-                stage_issue(scd, scale, rs, &full[s]);
-                if (mu) stage_issue(mud, mu, rm, &full[s]);
-            }
-            ++job;
             return true;
         });
         // the next call's weights into L2 (a hint), then wait for the copies still in flight
-        if (lane == 0 && warp == W) {
+        if (lane == 0 && pw == 0) {
             for (int i = 0; i < a.npf; ++i) {
                 const int64_t lo = int64_t(b) * a.pf_per[i], hi = min(a.pf_bytes[i], lo + a.pf_per[i]);
                 if (lo < hi) prefetch_l2_bulk(a.pf_ptr[i] + lo, uint32_t(hi - lo));
             }
         }
         for (int u = max(0, job - NS); u <= last_mine; ++u)
-            if (u % kIssuePerKind == pw && !mbar_wait(&full[u % NS], (u / NS) & 1)) break;
+            if (u % kPlaneIssuers == pw && !mbar_wait(&full[u % NS], (u / NS) & 1)) break;
         return;
     }
 
-    if (warp == W + kProducers) {
+    if (warp >= kW + kPlaneIssuers && warp < kW + kProducers) {
+        // ------------------------------------------------------------ scale issuers
+        // warp p issues the scales (and offsets) of the blocks v with v % 2 == p: the block's rows
+        // of the [*, G] arrays are one contiguous run
+        const int pw = warp - kW - kPlaneIssuers;
+        if (!a.static_weights) grid_dependency_wait();
+        int blk = 0, last_mine = -1;
+        walk_blocks(a, j0, j1, meta, meta_wait, [&](const Blk& bk) -> bool {
+            if (*vabort) return false;
+            if (blk % kScaleIssuers != pw) {
+                ++blk;
+                return true;
+            }
+            last_mine = blk;
+            const int nb = blk % kScaleBufs, round = blk / kScaleBufs;
+            if (round > 0 && !mbar_poll(&sempty[nb], (round - 1) & 1, kIdlePauseNs)) {
+                fail();
+                return false;
+            }
+            if (lane == 0) {
+                const D1Weight& Wt = a.w[bk.sg.wi];
+                const int64_t nrows = bk.kind ? Wt.r : Wt.N;
+                const int rows = int(max(int64_t(0), min(int64_t(bk.n * kStrip), nrows - bk.row0)));
+                const __half* scale = bk.kind ? Wt.scale2 : Wt.scale1;
+                const __half* mu = bk.kind == 0 ? Wt.mu : nullptr;
+                const uint32_t scd = smem_u32(sc_base + nb * a.sc_stride), mud = smem_u32(mu_base + nb * a.sc_stride);
+                const RowRun rs = stage_plan(scd, scale, bk.row0, rows, a.G);
+                const RowRun rm = mu ? stage_plan(mud, mu, bk.row0, rows, a.G) : RowRun{0, 0};
+                mbar_arrive_expect_tx(&sfull[nb], rs.bytes + rm.bytes);
+                stage_issue(scd, scale, rs, &sfull[nb]);
+                if (mu) stage_issue(mud, mu, rm, &sfull[nb]);
+            }
+            ++blk;
+            return true;
+        });
+        for (int u = max(0, blk - kScaleBufs); u <= last_mine; ++u)
+            if (u % kScaleIssuers == pw && !mbar_wait(&sfull[u % kScaleBufs], (u / kScaleBufs) & 1)) break;
+        return;
+    }
+
+    if (warp == kW + kProducers) {
         // ------------------------------------------------------------ epilogue
         // segment metadata: the slots of the segment's residual rows
         if (!a.static_weights) grid_dependency_wait();
@@ -401,7 +492,8 @@ __global__ void __launch_bounds__((W + kProducers + 1) * 32, 1) decode1_kernel(c
             if (lane == 0) mbar_arrive(meta_bar);
         }
         grid_dependency_wait();       // y may still be read by the previous kernel
-        int job = 0;
+        const int wps = kW / Sb;
+        int blk = 0;
         int cur_k = -1;
         Seg cur{};
         auto flush = [&]() {          // write the finished segment's rows
@@ -418,31 +510,29 @@ __global__ void __launch_bounds__((W + kProducers + 1) * 32, 1) decode1_kernel(c
             }
             __syncwarp();
         };
-        walk_jobs(a, j0, j1, meta, [] { return true; }, [&](int kind, int k, const Seg& sg, int jj, int c) -> bool {
+        walk_blocks(a, j0, j1, meta, [] { return true; }, [&](const Blk& bk) -> bool {
             if (*vabort) return false;
-            if (k != cur_k) {
+            if (bk.k != cur_k) {
                 flush();
-                cur_k = k;
-                cur = sg;
+                cur_k = bk.k;
+                cur = bk.sg;
             }
-            const int s = job % NS, round = job / NS;
-            if (!mbar_wait_sleep(&redfull[s], round & 1)) {
+            const int nr = blk % kRedBufs, round = blk / kRedBufs;
+            if (!mbar_poll(&redfull[nr], round & 1, kIdlePauseNs)) {
                 fail();
                 return false;
             }
-            if (lane < kStrip) {
+            // row r of strip st: the sums of the strip's warps st, st + Sb, ... in warp order
+            float* dst = bk.kind ? res_y + bk.first * kStrip : main_y + (bk.first - bk.sg.ja) * kStrip;
+            for (int e = lane; e < bk.n * kStrip; e += 32) {
+                const int st = e >> 4, r = e & (kStrip - 1);
                 float v = 0.f;
-                // every consumer warp's group sums, in warp order, then group order
-                for (int w = 0; w < W; ++w)
-#pragma unroll
-                    for (int g = 0; g < 4; ++g) v += red[((s * W + w) * 4 + g) * kStrip + lane];
-                const int idx = kind ? jj * kStrip + lane : (jj - sg.ja) * kStrip + lane;
-                float* dst = kind ? res_y : main_y;
-                dst[idx] = c ? dst[idx] + v : v;
+                for (int i = 0; i < wps; ++i) v += red[(nr * kW + st + Sb * i) * kStrip + r];
+                dst[e] = v;
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&redempty[s]);
-            ++job;
+            if (lane == 0) mbar_arrive(&redempty[nr]);
+            ++blk;
             return true;
         });
         if (!*vabort) flush();
@@ -454,7 +544,7 @@ __global__ void __launch_bounds__((W + kProducers + 1) * 32, 1) decode1_kernel(c
     const int pr = lane_row(rr);
     grid_dependency_wait();
     // stage x with the two activations of each pair adjacent
-    for (int i = threadIdx.x; i < a.K / 16; i += W * 32) {
+    for (int i = threadIdx.x; i < a.K / 16; i += kW * 32) {
         const uint4* src = reinterpret_cast<const uint4*>(a.x + int64_t(i) * 16);
         const uint4 lo = __ldg(src), hi = __ldg(src + 1);
         uint4 o0, o1;
@@ -466,26 +556,30 @@ __global__ void __launch_bounds__((W + kProducers + 1) * 32, 1) decode1_kernel(c
         dst[0] = o0;
         dst[1] = o1;
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(W * 32) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kW * 32) : "memory");
 
-    // The lane's activation registers for chunk c: words 2q, 2q+1 of the warp's group rr / 2
-    // (group 0 of the warp for the lanes whose column is not read).
+    // The lane's activation registers for groups [g, g + ng) of the K axis: words 2q, 2q+1 of
+    // group g + rr / 2 (group g for the lanes whose column is not read).
     uint32_t xr[16];
-    auto load_x = [&](int c) {
-        int g0, ng;
-        warp_groups(min(gcmax, a.G - c * gcmax), warp, W, g0, ng);
+    auto load_x = [&](int g, int ng) {
         const int gl = (rr & 1) == 0 && (rr >> 1) < ng ? (rr >> 1) : 0;
-        const uint32_t src = smem_u32(xs) + uint32_t(((c * gcmax + g0 + gl) * kGroup + 32 * q) * 2);
+        const uint32_t src = smem_u32(xs) + uint32_t(((g + gl) * kGroup + 32 * q) * 2);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const uint4 v = lds_u4(src + 16 * i);
             xr[4 * i] = v.x; xr[4 * i + 1] = v.y; xr[4 * i + 2] = v.z; xr[4 * i + 3] = v.w;
         }
     };
-    // C and X of every chunk's groups of this warp: one MMA chain each on the constant patterns
-    for (int c = 0; c < nchunk; ++c) {
-        load_x(c);
-        // the same chain as the main sums (both words of the lane into one accumulator)
+    auto load_x_at = [&](uint32_t src) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4 v = lds_u4(src + 16 * i);
+            xr[4 * i] = v.x; xr[4 * i + 1] = v.y; xr[4 * i + 2] = v.z; xr[4 * i + 3] = v.w;
+        }
+    };
+    // C and X of every group, four groups (one slab) per chain: the same chain as the main sums
+    for (int sl = warp; sl < a.nslab; sl += kW) {
+        load_x(4 * sl, 4);
         float cz[4] = {}, co[4] = {};
         const uint32_t one[4] = {kHalf2One, kHalf2One, kHalf2One, kHalf2One};
 #pragma unroll
@@ -499,201 +593,244 @@ __global__ void __launch_bounds__((W + kProducers + 1) * 32, 1) decode1_kernel(c
                 mma_16816(cz, Z, xr[8 * h + 2 * i], xr[8 * h + 2 * i + 1]);
                 if (a.has_mu) mma_16816(co, one, xr[8 * h + 2 * i], xr[8 * h + 2 * i + 1]);
             }
-        if (rr == 0) {     // column 2q: group q of the warp
-            cofs[(c * W + warp) * 4 + q] = cz[0];
-            xsum[(c * W + warp) * 4 + q] = co[0];
+        if (rr == 0) {     // column 2q: group 4 sl + q
+            cofs[4 * sl + q] = cz[0];
+            xsum[4 * sl + q] = co[0];
         }
     }
-    __syncwarp();
-    if (nchunk == 1) load_x(0);
-    if (!meta_wait()) return;
+    asm volatile("bar.sync 1, %0;" ::"n"(kW * 32) : "memory");
 
-    struct Sc {
-        unsigned short sa, sb, ma, mb;
-    };
-    // A job's accumulators and what its epilogue (per-group scaling and the hand-off of each
-    // lane's two row sums of its group to the epilogue warp, which adds them) needs.
-    struct Pending {
-        float acc[4][4];
-        Sc sc;
-        int s, round, c, ng, mu;
-    };
-    auto finish = [&](const Pending& pd) -> bool {
-        float p0 = 0.f, p1 = 0.f;
-        if (q < pd.ng) {
-            const float v0 = sel4(q, pd.acc[0][0], pd.acc[1][0], pd.acc[2][0], pd.acc[3][0]);
-            const float v1 = sel4(q, pd.acc[0][2], pd.acc[1][2], pd.acc[2][2], pd.acc[3][2]);
-            const float C = cofs[(pd.c * W + warp) * 4 + q];
-            p0 = __half2float(__ushort_as_half(pd.sc.sa)) * (v0 - C);
-            p1 = __half2float(__ushort_as_half(pd.sc.sb)) * (v1 - C);
-            if (pd.mu) {
-                const float X = xsum[(pd.c * W + warp) * 4 + q];
-                p0 = fmaf(__half2float(__ushort_as_half(pd.sc.ma)), X, p0);
-                p1 = fmaf(__half2float(__ushort_as_half(pd.sc.mb)), X, p1);
-            }
-        }
-        if (pd.round > 0 && !mbar_wait_sleep(&redempty[pd.s], (pd.round - 1) & 1)) {
-            fail();
-            return false;
-        }
-        float* rq = red + ((pd.s * W + warp) * 4 + q) * kStrip;
-        rq[pr] = p0;
-        rq[pr + 8] = p1;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&redfull[pd.s]);
-        return true;
-    };
+    // the warp's strip of every block and its share of the groups of a full and of the last stage
+    const int st = warp % Sb, wps = kW / Sb, wi = warp / Sb;
+    int g0f, ngf, g0l, ngl;
+    warp_share(4 * SB, wi, wps, g0f, ngf);
+    warp_share(4 * (a.nslab - (nstage - 1) * SB), wi, wps, g0l, ngl);
+    // Per-warp constants, so that a stage costs few instructions besides the decode: the byte
+    // offsets within a stage of the lane's word pair (row pr) of each of its groups, and the
+    // shared-memory addresses of its activations and of its groups' C and X for stage 0.
+    uint32_t offf[GW], offl[GW];
+#pragma unroll
+    for (int gi = 0; gi < GW; ++gi) {
+        const int gf = g0f + min(gi, max(ngf - 1, 0)), gl = g0l + min(gi, max(ngl - 1, 0));
+        const int wf = (gf & 3) * 8 + 2 * q, wl = (gl & 3) * 8 + 2 * q;
+        offf[gi] = uint32_t((gf >> 2) * slab_bytes + (st * kStrip + pr) * kSlabBytes) +
+                   ((uint32_t((wf >> 2) ^ (pr & 7)) << 4) | uint32_t((wf & 3) * 4));
+        offl[gi] = uint32_t((gl >> 2) * slab_bytes + (st * kStrip + pr) * kSlabBytes) +
+                   ((uint32_t((wl >> 2) ^ (pr & 7)) << 4) | uint32_t((wl & 3) * 4));
+    }
+    const int xgf = (rr & 1) == 0 && (rr >> 1) < ngf ? (rr >> 1) : 0;
+    const int xgl = (rr & 1) == 0 && (rr >> 1) < ngl ? (rr >> 1) : 0;
+    const uint32_t xsf = smem_u32(xs) + uint32_t(((g0f + xgf) * kGroup + 32 * q) * 2);
+    const uint32_t xsl = smem_u32(xs) + uint32_t((((nstage - 1) * 4 * SB + g0l + xgl) * kGroup + 32 * q) * 2);
+    const uint32_t xstep = uint32_t(4 * SB * kGroup * 2);      // bytes of x per stage
+    const int gqf = g0f + q, gql = (nstage - 1) * 4 * SB + g0l + q;
+    const bool lanef = q < ngf, lanel = q < ngl;
+    const uint32_t ring_end = stage0 + uint32_t(NS * stage_bytes);
+    if (nstage == 1) load_x_at(xsl);      // the same activations for every stage
 
-    int job = 0;
-    walk_jobs(a, j0, j1, meta, meta_wait, [&](int kind, int k, const Seg& sg, int jj, int c) -> bool {
+    uint32_t tile = stage0;                 // the next job's stage
+    uint32_t fullb = smem_u32(full), emptyb = smem_u32(empty);
+    uint32_t ph = 0;
+    int blk = 0;
+    walk_blocks(a, j0, j1, meta, meta_wait, [&](const Blk& bk) -> bool {
         if (*vabort) return false;
-        const int s = job % NS, round = job / NS;
-        int g0, ng;
-        const int gc = min(gcmax, a.G - c * gcmax);
-        warp_groups(gc, warp, W, g0, ng);
-        if (nchunk > 1) load_x(c);
-        if (!mbar_wait_sleep(&full[s], round & 1)) {
-            fail();
-            return false;
-        }
-        const uint32_t tile = stage0 + s * stage_bytes;
-        // the words of the warp's GW groups (rows pr and pr + 8, words 2q and 2q + 1 of each)
-        uint2 wa[GW], wb[GW];
-#pragma unroll
-        for (int gi = 0; gi < GW; ++gi) {
-            const int g = g0 + min(gi, max(ng - 1, 0));     // group within the chunk
-            const int slab = g >> 2, wofs = (g & 3) * 8 + 2 * q;
-            const uint32_t sw = (uint32_t((wofs >> 2) ^ (pr & 7)) << 4) | uint32_t((wofs & 3) * 4);
-            const uint32_t base = tile + slab * kSlabTile + sw;
-            wa[gi] = lds_u2(base + pr * 128);
-            wb[gi] = lds_u2(base + (pr + 8) * 128);
-        }
-        // this lane's scales (and offsets): rows pr and pr + 8, group q of the warp's groups
-        Sc cur{0, 0, 0, 0};
-        const bool has_mu = kind == 0 && a.w[sg.wi].mu;
-        if (q < ng) {
-            const int64_t row0 = kind ? int64_t(meta[2 * k]) + int64_t(jj) * kStrip : int64_t(jj) * kStrip;
-            const int skew = int((uint64_t(row0) * a.G * 2) & 15);
-            const int gq = c * gcmax + g0 + q;
-            const unsigned short* sc = reinterpret_cast<const unsigned short*>(sc_base + s * sc_stride + skew) + gq;
-            cur.sa = sc[pr * a.G];
-            cur.sb = sc[(pr + 8) * a.G];
-            if (has_mu) {
-                const unsigned short* m = reinterpret_cast<const unsigned short*>(mu_base + s * sc_stride + skew) + gq;
-                cur.ma = m[pr * a.G];
-                cur.mb = m[(pr + 8) * a.G];
+        const bool active = st < bk.n;
+        const int nb = blk % kScaleBufs;
+        bool sc_ready = false;        // the block's scales are waited for when first needed
+        const bool has_mu = bk.kind == 0 && a.w[bk.sg.wi].mu != nullptr;
+        const int skew = int((uint64_t(bk.row0) * a.G * 2) & 15);
+        const uint32_t sca = smem_u32(sc_base + nb * a.sc_stride + skew) + uint32_t((st * kStrip + pr) * a.G * 2);
+        const uint32_t scb = sca + uint32_t(8 * a.G * 2);
+        const uint32_t mud = uint32_t(a.o_mu - a.o_sc);
+        float p0 = 0.f, p1 = 0.f;
+        // one stage: its words (then the stage is released), x, the MMA chains, the scaling
+        auto stage = [&](const uint32_t (&off)[GW], uint32_t xsrc, bool reload_x, int gq, bool lane_on,
+                         bool work) -> bool {
+            if (!mbar_poll_addr(fullb, ph, 0)) {
+                fail();
+                return false;
             }
-        }
-        // the words and scales are in registers: the stage may be refilled
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-        // GW independent accumulator chains, their MMAs interleaved step by step
-        Pending nw;
+            uint2 wa[GW], wb[GW];
+            if (work) {
 #pragma unroll
-        for (int gi = 0; gi < 4; ++gi) nw.acc[gi][0] = nw.acc[gi][1] = nw.acc[gi][2] = nw.acc[gi][3] = 0.f;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            uint32_t sh[GW][4];
-#pragma unroll
-            for (int gi = 0; gi < GW; ++gi) {
-                const uint32_t a0 = h ? wa[gi].y : wa[gi].x, b0 = h ? wb[gi].y : wb[gi].x;
-                sh[gi][0] = a0; sh[gi][1] = a0 >> 6;
-                sh[gi][2] = b0; sh[gi][3] = b0 >> 6;
+                for (int gi = 0; gi < GW; ++gi) {
+                    wa[gi] = lds_u2(tile + off[gi]);
+                    wb[gi] = lds_u2(tile + off[gi] + 8 * kSlabBytes);
+                }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive_addr(emptyb);
+            tile += uint32_t(stage_bytes);
+            fullb += 8;
+            emptyb += 8;
+            if (tile == ring_end) {
+                tile = stage0;
+                fullb = smem_u32(full);
+                emptyb = smem_u32(empty);
+                ph ^= 1;
+            }
+            if (!work) return true;
+            if (reload_x) load_x_at(xsrc);
+            float acc[4][4];
+#pragma unroll
+            for (int gi = 0; gi < 4; ++gi) acc[gi][0] = acc[gi][1] = acc[gi][2] = acc[gi][3] = 0.f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t sh[GW][4];
+#pragma unroll
+                for (int gi = 0; gi < GW; ++gi) {
+                    const uint32_t a0 = h ? wa[gi].y : wa[gi].x, b0 = h ? wb[gi].y : wb[gi].x;
+                    sh[gi][0] = a0; sh[gi][1] = a0 >> 6;
+                    sh[gi][2] = b0; sh[gi][3] = b0 >> 6;
+                }
 #define TERN_D1_STEP(I)                                                                                \
     _Pragma("unroll") for (int gi = 0; gi < GW; ++gi) {                                                \
         uint32_t A[4];                                                                                 \
         decode_mma_in_place<I>(sh[gi][0], sh[gi][1], sh[gi][2], sh[gi][3], A);                         \
-        mma_16816(nw.acc[gi], A, xr[8 * h + 2 * (I)], xr[8 * h + 2 * (I) + 1]);                        \
+        mma_16816(acc[gi], A, xr[8 * h + 2 * (I)], xr[8 * h + 2 * (I) + 1]);                           \
     }
-            TERN_D1_STEP(0)
-            TERN_D1_STEP(1)
-            TERN_D1_STEP(2)
-            TERN_D1_STEP(3)
+                TERN_D1_STEP(0)
+                TERN_D1_STEP(1)
+                TERN_D1_STEP(2)
+                TERN_D1_STEP(3)
 #undef TERN_D1_STEP
+            }
+            if (!sc_ready) {
+                if (!mbar_poll(&sfull[nb], (blk / kScaleBufs) & 1, 0)) {
+                    fail();
+                    return false;
+                }
+                sc_ready = true;
+            }
+            // lane q: group q's sums for rows pr and pr + 8 (column 2q of its accumulators)
+            if (lane_on) {
+                const float v0 = sel4(q, acc[0][0], acc[1][0], acc[2][0], acc[3][0]);
+                const float v1 = sel4(q, acc[0][2], acc[1][2], acc[2][2], acc[3][2]);
+                const float C = cofs[gq];
+                p0 = fmaf(__half2float(__ushort_as_half(lds_u16(sca + 2 * gq))), v0 - C, p0);
+                p1 = fmaf(__half2float(__ushort_as_half(lds_u16(scb + 2 * gq))), v1 - C, p1);
+                if (has_mu) {
+                    const float X = xsum[gq];
+                    p0 = fmaf(__half2float(__ushort_as_half(lds_u16(sca + mud + 2 * gq))), X, p0);
+                    p1 = fmaf(__half2float(__ushort_as_half(lds_u16(scb + mud + 2 * gq))), X, p1);
+                }
+            }
+            return true;
+        };
+        const bool reload = nstage > 1;
+        for (int t = 0; t + 1 < nstage; ++t)
+            if (!stage(offf, xsf + uint32_t(t) * xstep, reload, gqf + t * 4 * SB, lanef, active && ngf > 0))
+                return false;
+        if (!stage(offl, xsl, reload, gql, lanel, active && ngl > 0)) return false;
+        // the block's scales are no longer read (a warp with no work in the block still waits for
+        // them, so that the buffer's phases stay in step)
+        if (!sc_ready && !mbar_poll(&sfull[nb], (blk / kScaleBufs) & 1, 0)) {
+            fail();
+            return false;
         }
-        nw.sc = cur;
-        nw.s = s;
-        nw.round = round;
-        nw.c = c;
-        nw.ng = ng;
-        nw.mu = has_mu ? 1 : 0;
-        if (!finish(nw)) return false;
-        ++job;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sempty[nb]);
+        // the quad's four lanes hold the row sums of different groups
+        p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
+        p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
+        p0 += __shfl_xor_sync(0xffffffffu, p0, 2);
+        p1 += __shfl_xor_sync(0xffffffffu, p1, 2);
+        const int nr = blk % kRedBufs, round = blk / kRedBufs;
+        if (round > 0 && !mbar_poll(&redempty[nr], (round - 1) & 1, 0)) {
+            fail();
+            return false;
+        }
+        if (q == 0) {
+            red[(nr * kW + warp) * kStrip + pr] = p0;
+            red[(nr * kW + warp) * kStrip + pr + 8] = p1;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&redfull[nr]);
+        ++blk;
         return true;
     });
 }
 
 // ------------------------------------------------------------------ host side
 // plane [rows, K/16] uint32 viewed as [slab][row][32 words]: dims {32, rows, K/512}, box
-// {32, 16, SB}, 128-byte swizzle.
-bool slab_map(CUtensorMap* map, const uint32_t* plane, int64_t rows, int64_t K, int SB) {
+// {32, 16 Sb, SB}, 128-byte swizzle.
+bool slab_map(CUtensorMap* map, const uint32_t* plane, int64_t rows, int64_t K, int Sb, int SB) {
     auto enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[3] = {32, cuuint64_t(rows > 0 ? rows : 1), cuuint64_t(K / 512)};
     const cuuint64_t strides[2] = {cuuint64_t(K / 4), 128};
-    const cuuint32_t box[3] = {32, kStrip, cuuint32_t(SB)};
+    const cuuint32_t box[3] = {32, cuuint32_t(kStrip * Sb), cuuint32_t(SB)};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(plane), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-
 struct Layout {
-    int W, SB, GW, nchunk, NS;
+    int Sb, SB, GW, nstage, NS, sc_stride;
     int o_sc, o_mu, o_red, o_xs, o_cofs, o_xsum, o_meta, o_bslot, o_mainy, o_resy, o_bar, total;
 };
 
-// Consumer warps, slabs per stage and groups per warp: every warp computes GW groups per stage
-// (ceil of the chunk's groups over W), so the split that wastes the fewest computed groups wins;
-// W is 8 or 10 (ties: 8).
-void plan_warps(int G, int& W, int& SB, int& GW) {
-    double best = -1.0;
-    for (int w : {8, 10}) {
-        const int sb = std::min(G / 4, w);
-        const int gcmax = 4 * sb, nchunk = (G + gcmax - 1) / gcmax;
-        const int gw = (gcmax + w - 1) / w;
-        const double eff = double(G) / (double(nchunk) * gw * w);
-        if (eff > best + 1e-9) {
-            best = eff;
-            W = w;
-            SB = sb;
-            GW = gw;
+constexpr int kSmemMax = 227 * 1024;
+
+// Strips per block and slabs per stage. A consumer warp's time per stage grows with the groups
+// it computes (GW, rounded up over the warps of its strip) plus a fixed cost per stage, and per
+// block a fixed cost for the hand-off; blocks are rounded up to Sb strips, and a CTA's residual
+// strips (res of them) form blocks of their own. Costs in units of one group (8 MMAs of one
+// warp): about 0.7 per stage and 1.8 per block (measured).
+void plan_blocks(int nslab, int64_t per, int64_t res, int& Sb, int& SB, int& GW) {
+    double best = 1e30;
+    Sb = 1;
+    SB = 1;
+    GW = 4;
+    for (int sb = 1; sb <= 8; sb *= 2) {
+        const int wps = kW / sb;
+        for (int slabs = 1; slabs <= std::min(nslab, 8 / sb); ++slabs) {
+            const int gw = (4 * slabs + wps - 1) / wps;
+            if (gw > 4) continue;
+            const int nst = (nslab + slabs - 1) / slabs;
+            const double blocks = double((per + sb - 1) / sb) + double((res + sb - 1) / sb);
+            const double cost = blocks * (nst * (gw + 0.7) + 1.8);
+            if (cost < best - 1e-9) {
+                best = cost;
+                Sb = sb;
+                SB = slabs;
+                GW = gw;
+            }
         }
     }
 }
 
-bool make_layout(int K, int NSwant, Layout& L) {
-    const int G = K / kGroup;
-    plan_warps(G, L.W, L.SB, L.GW);
-    L.nchunk = (G + 4 * L.SB - 1) / (4 * L.SB);
+bool make_layout(int K, int64_t per, int64_t res, bool has_mu, Layout& L) {
+    const int G = K / kGroup, nslab = K / 512;
+    plan_blocks(nslab, per, res, L.Sb, L.SB, L.GW);
+    L.nstage = (nslab + L.SB - 1) / L.SB;
     auto up = [](int v, int a) { return (v + a - 1) / a * a; };
-    for (int NS = NSwant; NS >= 2; --NS) {
-        int o = NS * L.SB * kSlabTile;
-        const int sc_stride = (32 * G + 16 + 15) & ~15;
-        L.o_sc = o; o += NS * sc_stride;
-        L.o_mu = o; o += NS * sc_stride;
-        L.o_red = o; o += up(NS * L.W * 4 * kStrip * 4, 16);
+    const int stage_bytes = L.Sb * L.SB * kStrip * kSlabBytes;
+    L.sc_stride = up(kStrip * L.Sb * G * 2 + 16, 16);
+    for (int NS = kStages; NS >= 2; --NS) {
+        int o = NS * stage_bytes;
+        L.o_sc = o; o += kScaleBufs * L.sc_stride;
+        L.o_mu = o; o += has_mu ? kScaleBufs * L.sc_stride : 0;
+        L.o_red = o; o += kRedBufs * kW * kStrip * 4;
         L.o_xs = o; o += up(K * 2, 16);
-        L.o_cofs = o; o += up(L.nchunk * L.W * 4 * 4, 16);
-        L.o_xsum = o; o += up(L.nchunk * L.W * 4 * 4, 16);
+        L.o_cofs = o; o += up(G * 4, 16);
+        L.o_xsum = o; o += up(G * 4, 16);
         L.o_meta = o; o += up(kMaxSegs * 2 * 4, 16);
         L.o_bslot = o; o += up(kMaxSegs * kSegRows * 2, 16);
         L.o_mainy = o; o += kSegRows * 4;
         L.o_resy = o; o += kSegRows * 4;
-        L.o_bar = o; o += up((4 * NS + 1) * 8 + 8, 16);
+        L.o_bar = o; o += up((2 * NS + 2 * kScaleBufs + 2 * kRedBufs + 1) * 8 + 8, 16);
         L.total = o + 1024;     // alignment slack
         L.NS = NS;
-        if (L.total <= 200 * 1024) return true;
+        if (L.total <= kSmemMax) return true;
     }
     return false;
 }
 
-
-template <int W, int GW>
+template <int GW>
 tern_status launch1(const D1Maps& maps, const D1Args& args, int grid, size_t smem, cudaStream_t stream) {
-    auto kernel = decode1_kernel<W, GW>;
+    auto kernel = decode1_kernel<GW>;
     static std::mutex mu;
     static bool configured[64] = {false};
     int dev = 0;
@@ -701,14 +838,14 @@ tern_status launch1(const D1Maps& maps, const D1Args& args, int grid, size_t sme
     {
         std::lock_guard<std::mutex> lock(mu);
         if (!configured[dev]) {
-            if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) != cudaSuccess)
+            if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) != cudaSuccess)
                 return TERN_ERR_CUDA;
             configured[dev] = true;
         }
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(grid), 1, 1);
-    cfg.blockDim = dim3((W + kProducers + 1) * 32, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -720,14 +857,19 @@ tern_status launch1(const D1Maps& maps, const D1Args& args, int grid, size_t sme
     return TERN_OK;
 }
 
-template <int W>
-tern_status launch_w(const Layout& L, const D1Maps& maps, const D1Args& args, int grid, cudaStream_t stream) {
-    switch (L.GW) {
-        case 1: return launch1<W, 1>(maps, args, grid, size_t(L.total), stream);
-        case 2: return launch1<W, 2>(maps, args, grid, size_t(L.total), stream);
-        case 3: return launch1<W, 3>(maps, args, grid, size_t(L.total), stream);
-        default: return launch1<W, 4>(maps, args, grid, size_t(L.total), stream);
+// Strips of the launch, strips per CTA (the largest range) and the residual strips of such a
+// range (its rows' share of the residual rows, rounded up).
+void launch_strips(const tern_weight* const* ws, int nw, int64_t& S, int64_t& P, int64_t& per, int64_t& res) {
+    S = 0;
+    int64_t rows = 0, rrows = 0;
+    for (int i = 0; i < nw; ++i) {
+        S += (ws[i]->N + kStrip - 1) / kStrip;
+        rows += ws[i]->N;
+        rrows += ws[i]->r;
     }
+    P = std::max<int64_t>(1, std::min<int64_t>(sm_count(), S));
+    per = (S + P - 1) / P;
+    res = rrows > 0 ? (per * kStrip * rrows / std::max<int64_t>(rows, 1) + kStrip - 1) / kStrip : 0;
 }
 
 }  // namespace
@@ -735,17 +877,17 @@ tern_status launch_w(const Layout& L, const D1Maps& maps, const D1Args& args, in
 bool decode1_supported(const tern_weight* const* ws, int nw) {
     const int64_t K = ws[0]->K;
     if (K % 512 != 0 || K / 512 > 4096) return false;
-    int64_t S = 0;
+    bool has_mu = false;
     for (int i = 0; i < nw; ++i) {
         if (ws[i]->ecount) return false;
-        S += (ws[i]->N + kStrip - 1) / kStrip;
+        has_mu = has_mu || ws[i]->mu != nullptr;
     }
-    const int64_t P = std::min<int64_t>(sm_count(), S);
-    const int64_t per = (S + P - 1) / P;
+    int64_t S, P, per, res;
+    launch_strips(ws, nw, S, P, per, res);
     // segments of one CTA: its strips in pieces of kSegStrips, plus one more per weight boundary
     if ((per + kSegStrips - 1) / kSegStrips + (nw - 1) > kMaxSegs) return false;
     Layout L;
-    return make_layout(int(K), 4, L);
+    return make_layout(int(K), per, res, has_mu, L);
 }
 
 tern_status decode1_launch_group(const tern_weight* const* ws, int nw, const __half* x, __half* const* ys,
@@ -753,14 +895,21 @@ tern_status decode1_launch_group(const tern_weight* const* ws, int nw, const __h
     D1Maps maps;
     D1Args a = {};
     const int64_t K = ws[0]->K;
-    Layout L;
-    if (!make_layout(int(K), kStages, L)) return TERN_ERR_SHAPE;
-    int64_t S = 0;
+    int64_t S, P, per, res;
+    launch_strips(ws, nw, S, P, per, res);
     bool all_static = true, has_mu = false;
     for (int i = 0; i < nw; ++i) {
+        all_static = all_static && (ws[i]->flags & TERN_WEIGHT_STATIC);
+        has_mu = has_mu || ws[i]->mu != nullptr;
+    }
+    Layout L;
+    if (!make_layout(int(K), per, res, has_mu, L)) return TERN_ERR_SHAPE;
+    int64_t S0 = 0;
+    for (int i = 0; i < nw; ++i) {
         const tern_weight& w = *ws[i];
-        if (!slab_map(&maps.m1[i], w.plane1, w.N, K, L.SB)) return TERN_ERR_CUDA;
-        if (!slab_map(&maps.m2[i], w.r > 0 ? w.plane2 : w.plane1, w.r > 0 ? w.r : w.N, K, L.SB)) return TERN_ERR_CUDA;
+        if (!slab_map(&maps.m1[i], w.plane1, w.N, K, L.Sb, L.SB)) return TERN_ERR_CUDA;
+        if (!slab_map(&maps.m2[i], w.r > 0 ? w.plane2 : w.plane1, w.r > 0 ? w.r : w.N, K, L.Sb, L.SB))
+            return TERN_ERR_CUDA;
         D1Weight& g = a.w[i];
         g.scale1 = reinterpret_cast<const __half*>(w.scale1);
         g.scale2 = reinterpret_cast<const __half*>(w.r > 0 ? w.scale2 : w.scale1);
@@ -769,19 +918,19 @@ tern_status decode1_launch_group(const tern_weight* const* ws, int nw, const __h
         g.y = ys[i];
         g.N = w.N;
         g.r = w.r;
-        g.strip0 = int32_t(S);
+        g.strip0 = int32_t(S0);
         g.nstrips = int32_t((w.N + kStrip - 1) / kStrip);
-        S += g.nstrips;
-        all_static = all_static && (w.flags & TERN_WEIGHT_STATIC);
-        has_mu = has_mu || w.mu != nullptr;
+        S0 += g.nstrips;
     }
     a.nw = nw;
     a.x = x;
     a.status = async_status_word();
     a.K = int32_t(K);
     a.G = int32_t(K / kGroup);
+    a.nslab = int32_t(K / 512);
+    a.Sb = L.Sb;
     a.SB = L.SB;
-    a.nchunk = L.nchunk;
+    a.nstage = L.nstage;
     a.NS = L.NS;
     a.S = int32_t(S);
     a.static_weights = all_static ? 1 : 0;
@@ -789,7 +938,8 @@ tern_status decode1_launch_group(const tern_weight* const* ws, int nw, const __h
     a.o_sc = L.o_sc; a.o_mu = L.o_mu; a.o_red = L.o_red; a.o_xs = L.o_xs; a.o_cofs = L.o_cofs;
     a.o_xsum = L.o_xsum; a.o_meta = L.o_meta; a.o_bslot = L.o_bslot; a.o_mainy = L.o_mainy;
     a.o_resy = L.o_resy; a.o_bar = L.o_bar;
-    const int grid = int(std::min<int64_t>(sm_count(), S));
+    a.sc_stride = L.sc_stride;
+    const int grid = int(P);
     for (int j = 0; j < nnext; ++j) {
         const tern_weight* nx = next[j];
         const int64_t G = nx->K / kGroup, rn = nx->r;
@@ -806,7 +956,12 @@ tern_status decode1_launch_group(const tern_weight* const* ws, int nw, const __h
         }
     }
     for (int i = 0; i < a.npf; ++i) a.pf_per[i] = ((a.pf_bytes[i] + grid - 1) / grid + 15) / 16 * 16;
-    return L.W == 10 ? launch_w<10>(L, maps, a, grid, stream) : launch_w<8>(L, maps, a, grid, stream);
+    switch (L.GW) {
+        case 1: return launch1<1>(maps, a, grid, size_t(L.total), stream);
+        case 2: return launch1<2>(maps, a, grid, size_t(L.total), stream);
+        case 3: return launch1<3>(maps, a, grid, size_t(L.total), stream);
+        default: return launch1<4>(maps, a, grid, size_t(L.total), stream);
+    }
 }
 
 }  // namespace tern
