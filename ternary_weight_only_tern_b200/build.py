@@ -21,9 +21,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libtern.so")
-SOURCES = ["tern_api.cu", "tern_pack.cu", "tern_elem.cu", "tern_gemv.cu", "tern_decode1.cu", "tern_gemm_sm100.cu",
+SOURCES = ["tern_api.cu", "tern_pack.cu", "tern_elem.cu", "tern_gemv.cu", "tern_decode1.cu", "tern_decodem.cu", "tern_gemm_sm100.cu",
            "tern_rotate.cu", "tern_fit.cu", "tern_bits.cpp"]
-HEADERS = ["tern_internal.cuh", "tern_device.cuh", os.path.join("..", "..", "include", "tern.h")]
+HEADERS = ["tern_internal.cuh", "tern_device.cuh", "tern_stream.cuh", os.path.join("..", "..", "include", "tern.h")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

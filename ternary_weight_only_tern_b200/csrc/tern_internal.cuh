@@ -40,6 +40,13 @@ bool decode1_supported(const tern_weight* const* ws, int nw);
 tern_status decode1_launch_group(const tern_weight* const* ws, int nw, const __half* x, __half* const* ys,
                                  const tern_weight* const* next, int nnext, cudaStream_t stream);
 
+// Decode GEMV for 2..16 tokens on the same persistent grid (tern_decodem.cu): the tokens are
+// the MMA's columns, x streams beside the weights; decodem_supported tells whether it takes the call.
+constexpr int64_t kDecodemMinM = 9;    // the smallest M the dispatch gives it
+bool decodem_supported(const tern_weight* const* ws, int nw, int64_t M, const void* x);
+tern_status decodem_launch_group(const tern_weight* const* ws, int nw, const __half* x, int64_t M, __half* const* ys,
+                                 const tern_weight* const* next, int nnext, cudaStream_t stream);
+
 // Prefill GEMM on tcgen05 (tern_gemm_sm100.cu), M > 16.
 tern_status gemm_launch(const tern_weight& w, const __half* x, int64_t M, __half* y, void* workspace,
                         cudaStream_t stream);
