@@ -1,7 +1,7 @@
 """Benchmark of the W1.58A16 ternary linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--quick]
-                    [--profile gemv|gemv_elem|gemm|rotate]
+                    [--profile gemv|gemv16|gemv_elem|gemm|gemm_elem|rotate]
 
 A step is one decode pass (M = 1) over the 252 ternarized linear tensors of a 36-layer
 Qwen3-8B-shaped stack (q, k, v, o, gate, up, down per layer; 15% of rows carry a residual
@@ -48,9 +48,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 # bench reports null until it is captured again.
 KERNEL_TRAFFIC = {
     "gemv": {"sources": ["ternary_weight_only_tern_b200/csrc/tern_decode1.cu",
-                         "ternary_weight_only_tern_b200/csrc/tern_device.cuh"],
-             "sha256": None,
-             "bytes": None},
+                         "ternary_weight_only_tern_b200/csrc/tern_device.cuh",
+                         "ternary_weight_only_tern_b200/csrc/tern_stream.cuh"],
+             "sha256": "1e8e2a20c1b570c84872987e4e7a06cc318b9ec3640134ed2346f2727ad2ee11",
+             "bytes": 30953728},
 }
 
 
@@ -444,7 +445,7 @@ def main():
                     help="how many following launches' weights each launch brings into L2 (with grouped "
                          "launches 0 measured best: 1824 us per step against 1840 for 1 and 1971 for 2)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline")
-    ap.add_argument("--profile", choices=["gemv", "gemv_elem", "gemm", "gemm_elem", "rotate"], default=None,
+    ap.add_argument("--profile", choices=["gemv", "gemv16", "gemv_elem", "gemm", "gemm_elem", "rotate"], default=None,
                     help="run a few calls of one op on one pool layer and exit (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -672,8 +673,8 @@ def main():
 
 
 def profile_case(torch, api, shapes, dev, which):
-    """A minimal run for ncu, three repetitions over two layers: at M = 1 (gemv) the bench's four
-    launches per layer (q+k+v, o, gate+up, down), or (gemv_elem) the same with element planes
+    """A minimal run for ncu, three repetitions over two layers: at M = 1 (gemv) or M = 16 (gemv16) the
+    bench's four launches per layer (q+k+v, o, gate+up, down), or (gemv_elem) the same with element planes
     (3.6 % masked) in place of residual rows; at M = 2048 (gemm, gemm_elem) gate, up and down."""
     if which == "rotate":
         # tern_rotate on K = 4096 at M = 1 and M = 2048, three times
@@ -694,7 +695,7 @@ def profile_case(torch, api, shapes, dev, which):
     kdim = {n: K for n, _, K in shapes}
     prefill = which in ("gemm", "gemm_elem")
     groups = GROUPS if not prefill else [("gate", ("gate",)), ("up", ("up",)), ("down", ("down",))]
-    M = 2048 if prefill else 1
+    M = 2048 if prefill else (16 if which == "gemv16" else 1)
     xs = {g: torch.randn((M, kdim[m[0]]), device=dev).half() for g, m in groups}
     ys = {n: torch.empty((M, N), dtype=torch.float16, device=dev) for n, N, _ in shapes}
     torch.cuda.synchronize()
