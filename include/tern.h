@@ -74,8 +74,10 @@ typedef enum {
     TERN_ERR_WORKSPACE = 7,  /* workspace smaller than tern_linear_workspace_bytes() or NULL */
     TERN_ERR_CUDA = 8,       /* a CUDA runtime call failed (launch error, no device, ...) */
     TERN_ERR_TIMEOUT = 9,    /* a bounded device-side wait ran out (see tern_device_status) */
-    TERN_ERR_ELEM = 10       /* unpack_elem / validate: element-plane counts, bases or order
+    TERN_ERR_ELEM = 10,      /* unpack_elem / validate: element-plane counts, bases or order
                                 inconsistent */
+    TERN_ERR_BOUNDS = 11     /* a TERN_DEBUG build's device-side bounds check failed (the access was
+                                skipped; outputs since the last tern_device_status are undefined) */
 } tern_status;
 
 /* A ternarized weight W [N, K] in execution form. Every pointer is device memory,
@@ -295,8 +297,15 @@ tern_status tern_bits_elem(int64_t N, int64_t K, int64_t masked, int64_t nnz2, i
 
 /* Reports, and clears, the current device's sticky status word for asynchronous work: returns
  * TERN_ERR_TIMEOUT if a tern_linear kernel since the last call gave up a bounded device-side
- * wait (its output is then undefined), else TERN_OK. Synchronous on `stream`.            */
+ * wait (its output is then undefined), TERN_ERR_BOUNDS if, in a TERN_DEBUG build, one of its
+ * device-side bounds checks failed (that access was skipped; the output is undefined), else
+ * TERN_OK. Synchronous on `stream`.                                                       */
 tern_status tern_device_status(tern_stream stream);
+
+/* 1 for a TERN_DEBUG build (libtern_debug.so: the decode kernels check their shared- and global-
+ * memory indices before each access and report a failure through tern_device_status instead of
+ * faulting), 0 for the release build. No counterpart on the pages: a test aid.            */
+int tern_debug_build(void);
 
 /* The failure path of the bounded device-side waits, exercised on purpose: one thread waits on
  * a shared-memory barrier that nothing completes, bounded by `cycles` SM clock cycles

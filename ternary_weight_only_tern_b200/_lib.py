@@ -6,13 +6,14 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libtern.so")
+# TERN_LIBRARY=debug selects the TERN_DEBUG build (device-side bounds checks; build with --debug)
+LIB_PATH = os.path.join(_HERE, "libtern_debug.so" if os.environ.get("TERN_LIBRARY") == "debug" else "libtern.so")
 
 TERN_OK = 0
 STATUS_NAMES = {
     0: "TERN_OK", 1: "TERN_ERR_NULL", 2: "TERN_ERR_SHAPE", 3: "TERN_ERR_ALIGN", 4: "TERN_ERR_BAD_TRIT",
     5: "TERN_ERR_BAD_CODE", 6: "TERN_ERR_RESIDUAL", 7: "TERN_ERR_WORKSPACE", 8: "TERN_ERR_CUDA",
-    9: "TERN_ERR_TIMEOUT", 10: "TERN_ERR_ELEM",
+    9: "TERN_ERR_TIMEOUT", 10: "TERN_ERR_ELEM", 11: "TERN_ERR_BOUNDS",
 }
 STATUS = {v: k for k, v in STATUS_NAMES.items()}
 
@@ -47,6 +48,7 @@ EXPORTS = {
                                         _c.c_void_p]),
     "tern_device_status": (_c.c_int, [_c.c_void_p]),
     "tern_selftest_timeout": (_c.c_int, [_c.c_int64, _c.c_void_p]),
+    "tern_debug_build": (_c.c_int, []),
     "tern_status_string": (_c.c_char_p, [_c.c_int]),
     "tern_version": (_c.c_int, []),
 }

@@ -85,6 +85,7 @@ extern "C" const char* tern_status_string(tern_status s) {
         case TERN_ERR_CUDA: return "CUDA error";
         case TERN_ERR_TIMEOUT: return "device wait timed out";
         case TERN_ERR_ELEM: return "inconsistent element-plane metadata";
+        case TERN_ERR_BOUNDS: return "a device-side bounds check of the debug build failed";
     }
     return "unknown status";
 }

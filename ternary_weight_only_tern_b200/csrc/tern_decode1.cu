@@ -205,8 +205,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
                     return false;
                 }
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[s], uint32_t(stage_bytes));
-                    tma_load_3d(stage0 + s * stage_bytes, map, 0, int(bk.row0), t * SB, &full[s]);
+                    // (a box that would start outside the plane is a planning error: no copy)
+                    [[maybe_unused]] const int64_t prow = bk.kind ? a.w[bk.sg.wi].r : a.w[bk.sg.wi].N;
+                    const bool ok = TERN_BOUNDS(a.status, bk.row0 < prow && t * SB < a.nslab);
+                    mbar_arrive_expect_tx(&full[s], ok ? uint32_t(stage_bytes) : 0u);
+                    if (ok) tma_load_3d(stage0 + s * stage_bytes, map, 0, int(bk.row0), t * SB, &full[s]);
                 }
             }
             return true;
@@ -319,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
             for (int lr = lane; lr < rows; lr += 32) {
                 float v = main_y[lr];
                 const int bs = bslot[cur_k * kSegRows + lr];
-                if (bs >= 0) v += res_y[bs];
+                if (bs >= 0 && TERN_BOUNDS(a.status, bs < kSegRows)) v += res_y[bs];
                 Wt.y[n_a + lr] = __float2half_rn(v);
             }
             __syncwarp();
@@ -337,12 +340,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
                 return false;
             }
             // row r of strip st: the sums of the strip's warps st, st + Sb, ... in warp order
-            float* dst = bk.kind ? res_y + bk.first * kStrip : main_y + (bk.first - bk.sg.ja) * kStrip;
+            const int d0 = bk.kind ? bk.first * kStrip : (bk.first - bk.sg.ja) * kStrip;
+            float* dst = (bk.kind ? res_y : main_y) + d0;
             for (int e = lane; e < bk.n * kStrip; e += 32) {
                 const int st = e >> 4, r = e & (kStrip - 1);
                 float v = 0.f;
                 for (int i = 0; i < wps; ++i) v += red[(nr * kW + st + Sb * i) * kStrip + r];
-                dst[e] = v;
+                if (TERN_BOUNDS(a.status, d0 + e < kSegRows)) dst[e] = v;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&redempty[nr]);
@@ -385,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
         }
     };
     auto load_x_at = [&](uint32_t src) {
+        if (!TERN_BOUNDS(a.status, src >= smem_u32(xs) && src - smem_u32(xs) + 64 <= uint32_t(a.K * 2))) return;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const uint4 v = lds_u4(src + 16 * i);
@@ -456,6 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
         const uint32_t sca = smem_u32(sc_base + nb * a.sc_stride + skew) + uint32_t((st * kStrip + pr) * a.G * 2);
         const uint32_t scb = sca + uint32_t(8 * a.G * 2);
         const uint32_t mud = uint32_t(a.o_mu - a.o_sc);
+        [[maybe_unused]] const uint32_t sc_end = smem_u32(sc_base + (nb + 1) * a.sc_stride);   // (debug checks)
         float p0 = 0.f, p1 = 0.f;
         // one stage: its words (then the stage is released), x, the MMA chains, the scaling
         auto stage = [&](const uint32_t (&off)[GW], uint32_t xsrc, bool reload_x, int gq, bool lane_on,
@@ -468,8 +474,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
             if (work) {
 #pragma unroll
                 for (int gi = 0; gi < GW; ++gi) {
-                    wa[gi] = lds_u2(tile + off[gi]);
-                    wb[gi] = lds_u2(tile + off[gi] + 8 * kSlabBytes);
+                    if (TERN_BOUNDS(a.status, tile - stage0 + off[gi] + 8 * kSlabBytes + 8 <= uint32_t(NS * stage_bytes))) {
+                        wa[gi] = lds_u2(tile + off[gi]);
+                        wb[gi] = lds_u2(tile + off[gi] + 8 * kSlabBytes);
+                    } else {
+                        wa[gi] = wb[gi] = make_uint2(0u, 0u);
+                    }
                 }
             }
             __syncwarp();
@@ -518,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
                 sc_ready = true;
             }
             // lane q: group q's sums for rows pr and pr + 8 (column 2q of its accumulators)
-            if (lane_on) {
+            if (lane_on && TERN_BOUNDS(a.status, gq < a.G && scb + 2 * gq + 2 <= sc_end)) {
                 const float v0 = sel4(q, acc[0][0], acc[1][0], acc[2][0], acc[3][0]);
                 const float v1 = sel4(q, acc[0][2], acc[1][2], acc[2][2], acc[3][2]);
                 const float C = cofs[gq];
@@ -555,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
             fail();
             return false;
         }
-        if (q == 0) {
+        if (q == 0 && TERN_BOUNDS(a.status, (nr * kW + warp) * kStrip + pr + 8 < kRedBufs * kW * kStrip)) {
             red[(nr * kW + warp) * kStrip + pr] = p0;
             red[(nr * kW + warp) * kStrip + pr + 8] = p1;
         }

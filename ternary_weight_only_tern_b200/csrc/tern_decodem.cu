@@ -184,10 +184,15 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
                     return false;
                 }
                 if (lane == 0) {
+                    // (a box that would start outside the plane is a planning error: no copy)
                     const uint32_t dst = stage0 + s * stage_bytes;
-                    mbar_arrive_expect_tx(&full[s], uint32_t(stage_bytes));
-                    tma_load_3d(dst, map, 0, int(bk.row0), t * SB, &full[s]);
-                    tma_load_3d(dst + plane_stage, &maps.xm, 0, 0, t * 8 * SB, &full[s]);
+                    [[maybe_unused]] const int64_t prow = bk.kind ? a.w[bk.sg.wi].r : a.w[bk.sg.wi].N;
+                    const bool ok = TERN_BOUNDS(a.status, bk.row0 < prow && t * SB < a.nslab);
+                    mbar_arrive_expect_tx(&full[s], ok ? uint32_t(stage_bytes) : 0u);
+                    if (ok) {
+                        tma_load_3d(dst, map, 0, int(bk.row0), t * SB, &full[s]);
+                        tma_load_3d(dst + plane_stage, &maps.xm, 0, 0, t * 8 * SB, &full[s]);
+                    }
                 }
             }
             return true;
@@ -330,6 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
         const bool has_mu = bk.kind == 0 && Wt.mu != nullptr;
         const int skew = int((uint64_t(bk.row0) * a.G * 2) & 15);
         const uint32_t sc0 = smem_u32(sc_base + nb * a.sc_stride + skew);
+        [[maybe_unused]] const uint32_t sc_end = smem_u32(sc_base + (nb + 1) * a.sc_stride);   // (debug checks)
         const uint32_t mud = uint32_t(a.o_mu - a.o_sc);
         float run[kStripsPerWarp][MT][4];
 #pragma unroll
@@ -347,11 +353,13 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
             if (work) {
 #pragma unroll
                 for (int o = 0; o < MT; ++o) {
-                    uint32_t nat[16];
+                    uint32_t nat[16] = {};
+                    if (TERN_BOUNDS(a.status, xrow[o] + 128 <= uint32_t(stage_bytes))) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint4 v = lds_u4(tile + xrow[o] + ((uint32_t(4 * (q & 1) + i) ^ xsw[o]) << 4));
-                        nat[4 * i] = v.x; nat[4 * i + 1] = v.y; nat[4 * i + 2] = v.z; nat[4 * i + 3] = v.w;
+                        for (int i = 0; i < 4; ++i) {
+                            const uint4 v = lds_u4(tile + xrow[o] + ((uint32_t(4 * (q & 1) + i) ^ xsw[o]) << 4));
+                            nat[4 * i] = v.x; nat[4 * i + 1] = v.y; nat[4 * i + 2] = v.z; nat[4 * i + 3] = v.w;
+                        }
                     }
                     pair_order(nat, xr[o]);
                 }
@@ -363,8 +371,12 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
                 if (work) {
 #pragma unroll
                     for (int kk = 0; kk < kSpp; ++kk) {
-                        wa[kk] = lds_u2(tile + off[pass * kSpp + kk]);
-                        wb[kk] = lds_u2(tile + off[pass * kSpp + kk] + 8 * kSlabBytes);
+                        if (TERN_BOUNDS(a.status, off[pass * kSpp + kk] + 8 * kSlabBytes + 8 <= plane_stage)) {
+                            wa[kk] = lds_u2(tile + off[pass * kSpp + kk]);
+                            wb[kk] = lds_u2(tile + off[pass * kSpp + kk] + 8 * kSlabBytes);
+                        } else {
+                            wa[kk] = wb[kk] = make_uint2(0u, 0u);
+                        }
                     }
                 }
                 {
@@ -445,6 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
                     const int k = pass * kSpp + kk;
                     const uint32_t ra = sc0 + uint32_t(((sw0 + ss * k) * kStrip + pr) * a.G * 2 + gq * 2);
                     const uint32_t rb = ra + uint32_t(8 * a.G * 2);
+                    if (!TERN_BOUNDS(a.status, rb + 2 <= sc_end && gq < a.G)) continue;
                     const float fa = __half2float(__ushort_as_half(lds_u16(ra)));
                     const float fb = __half2float(__ushort_as_half(lds_u16(rb)));
                     float ma = 0.f, mb = 0.f;
@@ -496,6 +509,8 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
                 const int n0 = 8 * o + 2 * q;
                 float* ra = red + ((warp * kStripsPerWarp + k) * kStrip + pr) * M;
                 float* rb = ra + 8 * M;
+                if (!TERN_BOUNDS(a.status, (warp * kStripsPerWarp + k) * kStrip + pr + 8 < kW * kStripsPerWarp * kStrip))
+                    continue;
                 if (n0 < M) {
                     ra[n0] = run[k][o][0];
                     rb[n0] = run[k][o][2];
@@ -526,14 +541,15 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
                     for (int g = 0; g < gs4; ++g) v += red[(((w0 + g) * kStripsPerWarp + k) * kStrip + r) * M + m];
                     if (bk.kind == 0) {
                         const int lr = (bk.first - bk.sg.ja) * kStrip + R;
-                        if (n_a + lr < Nw) {
+                        if (n_a + lr < Nw && TERN_BOUNDS(a.status, lr < kSegRows)) {
                             if (bslot[bk.k * kSegRows + lr] < 0) yw[int64_t(m) * Nw + n_a + lr] = __float2half_rn(v);
                             else main_y[m * kSegRows + lr] = v;
                         }
                     } else {
                         const int d = bk.first * kStrip + R;
                         const int lr = d < kSegRows ? rslot[bk.k * kSegRows + d] : -1;
-                        if (lr >= 0) yw[int64_t(m) * Nw + n_a + lr] = __float2half_rn(main_y[m * kSegRows + lr] + v);
+                        if (lr >= 0 && TERN_BOUNDS(a.status, lr < kSegRows && n_a + lr < Nw))
+                            yw[int64_t(m) * Nw + n_a + lr] = __float2half_rn(main_y[m * kSegRows + lr] + v);
                     }
                 }
             }

@@ -18,6 +18,23 @@ namespace dev {
 // first poll fails does not pay a slow timer read.
 constexpr uint64_t kWaitLimitCycles = 1ull << 32;
 
+// Bits of the sticky status word of the asynchronous kernels.
+constexpr unsigned int kStatusTimeout = 1u;    // a bounded wait ran out
+constexpr unsigned int kStatusBounds = 2u;     // a TERN_DEBUG bounds check failed
+
+// TERN_BOUNDS(status, cond): in a TERN_DEBUG build, cond is checked before an access it guards; when
+// it fails the status word gets kStatusBounds and the caller skips the access (no trap, no fault).
+// In the release build it is `true` and costs nothing.
+#ifdef TERN_DEBUG
+__device__ __forceinline__ bool bounds_ok(unsigned int* status, bool cond) {
+    if (!cond && status) atomicOr(status, kStatusBounds);
+    return cond;
+}
+#define TERN_BOUNDS(status, cond) (::tern::dev::bounds_ok((status), (cond)))
+#else
+#define TERN_BOUNDS(status, cond) true
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -407,9 +407,17 @@ extern "C" tern_status tern_device_status(tern_stream s) {
     if (v) {
         if (cudaMemsetAsync(w, 0, sizeof(unsigned int), st) != cudaSuccess) return TERN_ERR_CUDA;
         if (cudaStreamSynchronize(st) != cudaSuccess) return TERN_ERR_CUDA;
-        return TERN_ERR_TIMEOUT;
+        return (v & dev::kStatusBounds) ? TERN_ERR_BOUNDS : TERN_ERR_TIMEOUT;
     }
     return TERN_OK;
+}
+
+extern "C" int tern_debug_build(void) {
+#ifdef TERN_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
 }
 
 extern "C" tern_status tern_pack_residual(const int32_t* res_rows, int64_t r, int64_t N, int32_t* res_slot,

@@ -24,3 +24,16 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _no_failed_device_checks(request):
+    """Under TERN_CHECK_DEVICE_STATUS=1 (set by test_debug_gpu for its runs against the TERN_DEBUG
+    build), every GPU test must leave the sticky device status clean: no bounded wait ran out and no
+    bounds check of the debug build failed."""
+    yield
+    if os.environ.get("TERN_CHECK_DEVICE_STATUS") != "1" or "gpu" not in request.keywords:
+        return
+    from ternary_weight_only_tern_b200 import _lib, api
+    st = _lib.load().tern_device_status(api._stream())
+    assert st == 0, f"device status after the test: {_lib.STATUS_NAMES.get(st, st)}"

@@ -43,9 +43,24 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(10):
+    for code in range(12):
         assert lib.tern_status_string(code)
     assert lib.tern_status_string(99) == b"unknown status"
+
+
+def test_release_and_debug_builds_identify_themselves(lib):
+    """The TERN_DEBUG build (libtern_debug.so) exports the same boundary and says it is the debug
+    build; the release build says it is not; TERN_LIBRARY=debug loads the debug build."""
+    assert lib.tern_debug_build() == (1 if os.environ.get("TERN_LIBRARY") == "debug" else 0)
+    path = os.path.join(os.path.dirname(_lib.LIB_PATH), "libtern_debug.so")
+    if not os.path.exists(path):
+        from ternary_weight_only_tern_b200 import build
+        build.build(debug=True)
+    dbg = ctypes.CDLL(path)
+    for name in header_functions():
+        assert hasattr(dbg, name), name
+    dbg.tern_debug_build.restype = ctypes.c_int
+    assert dbg.tern_debug_build() == 1
 
 
 @pytest.mark.parametrize("N,K,r", [(4096, 2560, 0), (9728, 2560, 973), (12288, 4096, 1843), (13, 384, 13),
