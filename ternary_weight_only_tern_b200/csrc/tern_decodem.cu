@@ -87,6 +87,8 @@ struct DMArgs {
     int32_t stage_bytes;      // plane box + x box
     int32_t sc_stride;
     int32_t o_sc, o_mu, o_red, o_cofs, o_xsum, o_meta, o_bslot, o_rslot, o_mainy, o_bar;
+    int32_t o_xs;             // resident x: [M][K + 8] fp16, pair order (XRES)
+    int32_t static_weights;
     const uint8_t* pf_ptr[kPfRanges];
     int64_t pf_bytes[kPfRanges];
     int64_t pf_per[kPfRanges];
@@ -103,8 +105,10 @@ __device__ __forceinline__ void pair_order(const uint32_t (&nat)[16], uint32_t (
             xr[8 * h + p] = prmt(nat[8 * h + p / 2], nat[8 * h + p / 2 + 4], (p & 1) ? 0x7632u : 0x5410u);
 }
 
-// MT: 8-token column blocks (1 for M <= 8, 2 for M <= 16).
-template <int MT>
+// MT: 8-token column blocks (1 for M <= 8, 2 for M <= 16). XRES: x is staged once per CTA in
+// shared memory (all tokens, in pair order) when it fits, and the stages carry the plane alone;
+// otherwise each stage carries its K range of x beside the plane.
+template <int MT, bool XRES>
 __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_constant__ DMMaps maps,
                                                               const __grid_constant__ DMArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -169,8 +173,10 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
             prefetch_tensormap(&maps.m1[lane]);
             prefetch_tensormap(&maps.m2[lane]);
         }
-        if (pw == 0 && lane == 0) prefetch_tensormap(&maps.xm);
-        grid_dependency_wait();                  // x may be written by the previous kernel
+        if (!XRES && pw == 0 && lane == 0) prefetch_tensormap(&maps.xm);
+        // x may be written by the previous kernel; with x resident the stages hold static weights
+        // only, which may stream before the wait
+        if (!XRES || !a.static_weights) grid_dependency_wait();
         int job = 0, last_mine = -1;
         walk_blocks(a, j0, j1, meta, meta_wait, [&](const Blk& bk) -> bool {
             if (*vabort) return false;
@@ -191,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
                     mbar_arrive_expect_tx(&full[s], ok ? uint32_t(stage_bytes) : 0u);
                     if (ok) {
                         tma_load_3d(dst, map, 0, int(bk.row0), t * SB, &full[s]);
-                        tma_load_3d(dst + plane_stage, &maps.xm, 0, 0, t * 8 * SB, &full[s]);
+                        if (!XRES) tma_load_3d(dst + plane_stage, &maps.xm, 0, 0, t * 8 * SB, &full[s]);
                     }
                 }
             }
@@ -292,6 +298,26 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
     const int gw = warp % gs4;                    // the warp's group within a stage
     const int sw0 = warp / gs4, ss = kW / gs4;    // its strips: sw0 + ss k, k < kStripsPerWarp
     grid_dependency_wait();
+    const int xstride = a.K + 8;                  // halves per resident token row (spreads the banks)
+    __half* xs = reinterpret_cast<__half*>(smem + a.o_xs);
+    if (XRES) {
+        // every token's x with the two activations of each decoded pair adjacent
+        const int per_tok = a.K / 16;
+        for (int u = threadIdx.x; u < M * per_tok; u += kW * 32) {
+            const int m = u / per_tok, i = u - m * per_tok;
+            const uint4* src = reinterpret_cast<const uint4*>(a.x + int64_t(m) * a.K + int64_t(i) * 16);
+            const uint4 lo = __ldg(src), hi = __ldg(src + 1);
+            uint4 o0, o1;
+            o0.x = prmt(lo.x, hi.x, 0x5410u); o0.y = prmt(lo.x, hi.x, 0x7632u);
+            o0.z = prmt(lo.y, hi.y, 0x5410u); o0.w = prmt(lo.y, hi.y, 0x7632u);
+            o1.x = prmt(lo.z, hi.z, 0x5410u); o1.y = prmt(lo.z, hi.z, 0x7632u);
+            o1.z = prmt(lo.w, hi.w, 0x5410u); o1.w = prmt(lo.w, hi.w, 0x7632u);
+            uint4* dst = reinterpret_cast<uint4*>(xs + int64_t(m) * xstride + int64_t(i) * 16);
+            dst[0] = o0;
+            dst[1] = o1;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kW * 32) : "memory");
+    }
 
     // per-warp constants: the word offsets (row pr) of its four strips' words of its group within
     // a stage, and the x tile offsets of its group's activations for each token block
@@ -304,12 +330,13 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
     }
     // x tile row of token block o: (2 gw + q / 2) M + token; its 16-byte pieces 4 (q & 1) + i,
     // swizzled with the row
+    // (resident x: token row n, words 2q and 2q + 1 of the group, the pair order staged above)
     uint32_t xrow[MT], xsw[MT];
 #pragma unroll
     for (int o = 0; o < MT; ++o) {
         const int n = min(8 * o + rr, M - 1);
         const int row = (2 * gw + (q >> 1)) * M + n;
-        xrow[o] = plane_stage + uint32_t(row * 128);
+        xrow[o] = XRES ? smem_u32(xs) + uint32_t((n * xstride + gw * kGroup + 32 * q) * 2) : plane_stage + uint32_t(row * 128);
         xsw[o] = uint32_t(row & 7);
     }
     const uint32_t ring_end = stage0 + uint32_t(NS * stage_bytes);
@@ -350,7 +377,23 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
                 return false;
             }
             uint32_t xr[MT][16];
-            if (work) {
+            if (work && XRES) {
+                // the group's activations of stage t from the resident rows
+                const uint32_t xt = uint32_t(t * gs4 * kGroup * 2);
+#pragma unroll
+                for (int o = 0; o < MT; ++o) {
+                    if (TERN_BOUNDS(a.status, xrow[o] + xt + 64 <= smem_u32(xs) + uint32_t(M * xstride * 2))) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint4 v = lds_u4(xrow[o] + xt + 16 * i);
+                            xr[o][4 * i] = v.x; xr[o][4 * i + 1] = v.y; xr[o][4 * i + 2] = v.z; xr[o][4 * i + 3] = v.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) xr[o][i] = 0u;
+                    }
+                }
+            } else if (work) {
 #pragma unroll
                 for (int o = 0; o < MT; ++o) {
                     uint32_t nat[16] = {};
@@ -588,7 +631,8 @@ bool x_map(CUtensorMap* map, const __half* x, int M, int64_t K, int SB) {
 
 struct LayoutM {
     int Sb, SB, nstage, NS, stage_bytes, sc_stride;
-    int o_sc, o_mu, o_red, o_cofs, o_xsum, o_meta, o_bslot, o_rslot, o_mainy, o_bar, total;
+    bool xres;
+    int o_sc, o_mu, o_red, o_cofs, o_xsum, o_meta, o_bslot, o_rslot, o_mainy, o_xs, o_bar, total;
 };
 
 // A stage holds 2 spw strip slabs (spw strips per warp): Sb = 2 spw strips x 1 slab, or spw strips
@@ -612,30 +656,37 @@ bool make_layout_m(int K, int M, int64_t per, int64_t res, bool has_mu, LayoutM&
         }
     }
     auto up = [](int v, int a) { return (v + a - 1) / a * a; };
-    L.stage_bytes = L.Sb * L.SB * kStrip * kSlabBytes + M * L.SB * 1024;
     L.sc_stride = up(kStrip * L.Sb * G * 2 + 16, 16);
-    for (int NS = kMaxStages; NS >= 3; --NS) {
-        int o = NS * L.stage_bytes;
-        L.o_sc = o; o += kScaleBufs * L.sc_stride;
-        L.o_mu = o; o += has_mu ? kScaleBufs * L.sc_stride : 0;
-        L.o_red = o; o += kW * spw * kStrip * M * 4;
-        L.o_cofs = o; o += up(G * kTokPad * 4, 16);
-        L.o_xsum = o; o += up(G * kTokPad * 4, 16);
-        L.o_meta = o; o += up(kMaxSegs * 2 * 4, 16);
-        L.o_bslot = o; o += kMaxSegs * kSegRows * 2;
-        L.o_rslot = o; o += kMaxSegs * kSegRows * 2;
-        L.o_mainy = o; o += M * kSegRows * 4;
-        L.o_bar = o; o += up((2 * NS + 2 * kScaleBufs + 2) * 8 + 8, 16);
-        L.total = o + 1024;
-        L.NS = NS;
-        if (L.total <= kSmemMaxM) return true;
+    // x resident (stages of plane alone, at least 4 of them), else x streamed with each stage
+    // (at least 3 stages)
+    for (int xres = 1; xres >= 0; --xres) {
+        L.xres = xres == 1;
+        const int plane = L.Sb * L.SB * kStrip * kSlabBytes;
+        L.stage_bytes = plane + (L.xres ? 0 : M * L.SB * 1024);
+        for (int NS = kMaxStages; NS >= (L.xres ? 4 : 3); --NS) {
+            int o = NS * L.stage_bytes;
+            L.o_sc = o; o += kScaleBufs * L.sc_stride;
+            L.o_mu = o; o += has_mu ? kScaleBufs * L.sc_stride : 0;
+            L.o_red = o; o += kW * spw * kStrip * M * 4;
+            L.o_cofs = o; o += up(G * kTokPad * 4, 16);
+            L.o_xsum = o; o += up(G * kTokPad * 4, 16);
+            L.o_meta = o; o += up(kMaxSegs * 2 * 4, 16);
+            L.o_bslot = o; o += kMaxSegs * kSegRows * 2;
+            L.o_rslot = o; o += kMaxSegs * kSegRows * 2;
+            L.o_mainy = o; o += M * kSegRows * 4;
+            L.o_xs = o; o += L.xres ? up(M * (K + 8) * 2, 16) : 0;
+            L.o_bar = o; o += up((2 * NS + 2 * kScaleBufs + 2) * 8 + 8, 16);
+            L.total = o + 1024;
+            L.NS = NS;
+            if (L.total <= kSmemMaxM) return true;
+        }
     }
     return false;
 }
 
-template <int MT>
+template <int MT, bool XRES>
 tern_status launch_m(const DMMaps& maps, const DMArgs& args, int grid, size_t smem, cudaStream_t stream) {
-    auto kernel = decodem_kernel<MT>;
+    auto kernel = decodem_kernel<MT, XRES>;
     static std::mutex mu;
     static bool configured[64] = {false};
     int dev = 0;
@@ -739,6 +790,10 @@ tern_status decodem_launch_group(const tern_weight* const* ws, int nw, const __h
     a.sc_stride = L.sc_stride;
     a.o_sc = L.o_sc; a.o_mu = L.o_mu; a.o_red = L.o_red; a.o_cofs = L.o_cofs; a.o_xsum = L.o_xsum;
     a.o_meta = L.o_meta; a.o_bslot = L.o_bslot; a.o_rslot = L.o_rslot; a.o_mainy = L.o_mainy; a.o_bar = L.o_bar;
+    a.o_xs = L.o_xs;
+    bool all_static = true;
+    for (int i = 0; i < nw; ++i) all_static = all_static && (ws[i]->flags & TERN_WEIGHT_STATIC);
+    a.static_weights = all_static ? 1 : 0;
     const int grid = int(P);
     for (int j = 0; j < nnext; ++j) {
         const tern_weight* nx = next[j];
@@ -756,7 +811,8 @@ tern_status decodem_launch_group(const tern_weight* const* ws, int nw, const __h
         }
     }
     for (int i = 0; i < a.npf; ++i) a.pf_per[i] = ((a.pf_bytes[i] + grid - 1) / grid + 15) / 16 * 16;
-    return launch_m<2>(maps, a, grid, size_t(L.total), stream);
+    return L.xres ? launch_m<2, true>(maps, a, grid, size_t(L.total), stream)
+                  : launch_m<2, false>(maps, a, grid, size_t(L.total), stream);
 }
 
 }  // namespace tern
