@@ -110,9 +110,9 @@ tern_status linear_group(const tern_weight* const* w, int n, const tern_half* x,
     __half* yh[kMaxGemvGroup];
     for (int i = 0; i < n; ++i) yh[i] = reinterpret_cast<__half*>(y[i]);
     if (M == 1 && decode1_supported(w, n)) return decode1_launch_group(w, n, xh, yh, next, nnext, st);
-    // two 8-token column blocks per decoded fragment pay off from 9 tokens on; up to 8 the cluster
-    // kernel's occupancy wins (measured on the 8B layer)
-    if (M >= kDecodemMinM && decodem_supported(w, n, M, xh))
+    // the multi-token kernel: from 9 tokens on, and up to 8 on launches with many strips per CTA
+    // (decodem_supported); the cluster kernel otherwise (measured on the 4B and 8B layers)
+    if (M >= 2 && decodem_supported(w, n, M, xh))
         return decodem_launch_group(w, n, xh, M, yh, next, nnext, st);
     if (M <= kGemvMaxM) return gemv_launch_group(w, n, xh, int(M), yh, next, nnext, st);
     for (int i = 0; i < n; ++i) {

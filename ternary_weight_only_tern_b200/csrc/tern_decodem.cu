@@ -1,4 +1,4 @@
-// Decode GEMV for 9 to 16 tokens: y[M, N] = x[M, K] . W^T with W on packed 2-bit ternary planes.
+// Decode GEMV for 2 to 16 tokens: y[M, N] = x[M, K] . W^T with W on packed 2-bit ternary planes.
 //
 // What it computes is the representation of "Post-Training Ternarization of Qwen3-4B"
 // (arXiv 2609.01962v1), sections 4.3-4.5: one ternary plane T1 with an fp16 scale per
@@ -18,9 +18,9 @@
 //    so the activations of a group (one B fragment set per 8 tokens, permuted in registers into
 //    the order of the decoded pairs) serve four strips. A decoded A fragment (16 rows x 16 K of
 //    trits, one LOP3 per pair of trits; tern_device.cuh) feeds one mma.sync m16n8k16 per 8
-//    tokens, so the decode costs the same for 9 and for 16 tokens. (The kernel is written for one
-//    or two column blocks; the call gives it 9 to 16 tokens, where two blocks per decoded fragment
-//    pay off; up to 8 tokens the cluster kernel of tern_gemv.cu was measured faster.)
+//    tokens, so the decode costs the same for 2 and for 16 tokens. The call gives it 9 to 16
+//    tokens, and 8 tokens on launches of at least 10 strips per CTA; the cluster kernel of
+//    tern_gemv.cu was measured faster on the other calls up to 8 tokens.
 //  * Lane (rr, q) of the D fragment holds rows rr and rr+8, tokens 2q and 2q+1; it scales each
 //    stage's sums by the row's group scale (after subtracting C = sum (B_p + 1) x of the group
 //    and token, computed once per kernel by the same MMA chain on the constant pattern, so a zero
@@ -730,7 +730,7 @@ void strips_m(const tern_weight* const* ws, int nw, int64_t& S, int64_t& P, int6
 
 bool decodem_supported(const tern_weight* const* ws, int nw, int64_t M, const void* x) {
     const int64_t K = ws[0]->K;
-    if (M < kDecodemMinM || M > 16 || K % 512 != 0 || K / 512 > 4096 || !aligned16(x)) return false;
+    if (M < 2 || M > 16 || K % 512 != 0 || K / 512 > 4096 || !aligned16(x)) return false;
     bool has_mu = false;
     for (int i = 0; i < nw; ++i) {
         if (ws[i]->ecount) return false;
@@ -738,6 +738,11 @@ bool decodem_supported(const tern_weight* const* ws, int nw, int64_t M, const vo
     }
     int64_t S, P, per, res;
     strips_m(ws, nw, S, P, per, res);
+    // below 9 tokens the cluster kernel is faster on launches of few strips per CTA, and at 4
+    // tokens on every launch of the 8B stack (measured: this kernel wins its gate+up launch, 12
+    // strips per CTA, at 8 tokens and in isolation at 4, but the stack at 4 tokens is faster with
+    // the cluster kernel throughout)
+    if (M < kDecodemMinM && (M < kDecodemStripsMinM || per < kDecodemMinStrips)) return false;
     if ((per + kSegStrips - 1) / kSegStrips + (nw - 1) > kMaxSegs) return false;
     LayoutM L;
     return make_layout_m(int(K), int(M), per, res, has_mu, L);
@@ -811,6 +816,9 @@ tern_status decodem_launch_group(const tern_weight* const* ws, int nw, const __h
         }
     }
     for (int i = 0; i < a.npf; ++i) a.pf_per[i] = ((a.pf_bytes[i] + grid - 1) / grid + 15) / 16 * 16;
+    if (M <= 8)
+        return L.xres ? launch_m<1, true>(maps, a, grid, size_t(L.total), stream)
+                      : launch_m<1, false>(maps, a, grid, size_t(L.total), stream);
     return L.xres ? launch_m<2, true>(maps, a, grid, size_t(L.total), stream)
                   : launch_m<2, false>(maps, a, grid, size_t(L.total), stream);
 }

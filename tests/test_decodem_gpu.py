@@ -1,6 +1,6 @@
-"""GPU parity of the multi-token decode kernel (the call takes it for 9 <= M <= 16, K a multiple of
-512; smaller M run the cluster kernel and are covered here too): the persistent GEMV whose MMA
-columns are the tokens. Cases aimed at its structure: one and two 8-token column
+"""GPU parity of the multi-token decode kernel (the call takes it for 9 <= M <= 16, and for M = 8
+on launches of at least 10 strips per CTA; K a multiple of 512; the other calls run the cluster
+kernel and are covered here too): the persistent GEMV whose MMA columns are the tokens. Cases aimed at its structure: one and two 8-token column
 blocks and ragged token counts, blocks of 8 and 4 strips (1 and 2 slabs per stage), ranges that
 span several segments and weight boundaries, residual rows that fill whole segments, K with an
 odd number of 512-wide slabs, offsets, and chains of calls under programmatic dependent launch.
@@ -44,6 +44,18 @@ def run(x, w):
 def test_shapes_tokens_and_residual_fractions(M, K, N, pct):
     rng = np.random.default_rng(M * 7 + K + N + pct)
     t = synth.draw_tensor(rng, "dm", N, K, M, p_zero=0.4, res_pct=pct)
+    check(run(t.x, weight(t)), oracle.linear(t.x, t.T1, t.s1, t.res_rows, t.T2, t.s2))
+
+
+@pytest.mark.parametrize("M", [2, 5, 8])
+@pytest.mark.parametrize("K,pct", [(4096, 15), (12288, 10), (2560, 100)])
+def test_one_token_block_on_large_launches(M, K, pct):
+    """11 strips per CTA: at M = 8 one 8-token column block in this kernel, x resident in shared
+    memory (K = 4096, 2560) or streamed with the stages (K = 12288); at M = 2 and 5 the cluster
+    kernel on the same shapes."""
+    rng = np.random.default_rng(M * 100 + K + pct)
+    N = 148 * 16 * 11 + 5
+    t = synth.draw_tensor(rng, "l", N, K, M, p_zero=0.4, res_pct=pct)
     check(run(t.x, weight(t)), oracle.linear(t.x, t.T1, t.s1, t.res_rows, t.T2, t.s2))
 
 
