@@ -50,8 +50,8 @@ KERNEL_TRAFFIC = {
     "gemv": {"sources": ["ternary_weight_only_tern_b200/csrc/tern_decode1.cu",
                          "ternary_weight_only_tern_b200/csrc/tern_device.cuh",
                          "ternary_weight_only_tern_b200/csrc/tern_stream.cuh"],
-             "sha256": "1e8e2a20c1b570c84872987e4e7a06cc318b9ec3640134ed2346f2727ad2ee11",
-             "bytes": 30953728},
+             "sha256": "3a10bcd2147430c31422fcf4364b348dc0767912240785f64f0a4cfdf6b3332d",
+             "bytes": 30946048},
 }
 
 
