@@ -33,9 +33,10 @@
 //    activations, so one set of 16 activation registers per lane serves all of the warp's
 //    groups, and each group accumulates in its own registers, whose column 2 g alone is read
 //    (the other columns multiply other groups' activations and are ignored). Lane q then holds
-//    group q's sums for its two rows and scales them into its running row sums; the four lanes
-//    of a quad add theirs at the end of the block. The groups' MMA chains are interleaved step
-//    by step with their decode.
+//    group q's sums for its two rows and scales them into its running row sums; at the end of a
+//    block every lane leaves its two row sums in shared memory (no shuffles on the consumers'
+//    path) and the epilogue warp adds the quad's four. The groups' MMA chains are interleaved
+//    step by step with their decode.
 //  * Decode is branch-free: one LOP3 writes two 2-bit codes (trits p and p+8 of a word) into
 //    the mantissas of an fp16 pair (B_p + c); pairs 0-4 read the codes in place and pairs 5-7
 //    after one shift of the word (tern_device.cuh); the MMA sums (B_p + 1 + t) x, and
@@ -70,7 +71,7 @@ constexpr int kThreads = (kW + kProducers + 1) * 32;
 
 constexpr int kStages = 8;                 // ring stages (fewer when shared memory runs short)
 constexpr int kScaleBufs = 2;              // block scale buffers
-constexpr int kRedBufs = 2;                // block partial-sum buffers
+constexpr int kRedBufs = 4;                // block partial-sum buffers
 constexpr int kPfPerWeight = 6;
 constexpr int kPfRanges = kPfPerWeight * kMaxNW;
 
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
     const int stage_bytes = SB * slab_bytes;
     uint8_t* sc_base = smem + a.o_sc;                            // [kScaleBufs][16 Sb rows][G] (skewed)
     uint8_t* mu_base = smem + a.o_mu;                            // the same for the offsets
-    float* red = reinterpret_cast<float*>(smem + a.o_red);       // [kRedBufs][W][16 rows]
+    float* red = reinterpret_cast<float*>(smem + a.o_red);       // [kRedBufs][W][16 rows][4 quad lanes]
     __half* xs = reinterpret_cast<__half*>(smem + a.o_xs);       // [K], pairs adjacent
     float* cofs = reinterpret_cast<float*>(smem + a.o_cofs);     // [G] C of every group
     float* xsum = reinterpret_cast<float*>(smem + a.o_xsum);     // [G] X of every group
@@ -171,7 +172,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
     grid_launch_dependents();
 
     const int P = gridDim.x, b = blockIdx.x;
-    const int j0 = int((int64_t(b) * a.S) / P), j1 = int((int64_t(b + 1) * a.S) / P);
+    // the CTA's strips [j0, j1) = [b S / P, (b + 1) S / P), in 32-bit arithmetic: the host keeps S
+    // below 2^24 and P is at most the SM count, so (b + 1) S fits (a 64-bit division here cost
+    // hundreds of cycles before the first copy of every launch)
+    const uint32_t uS = uint32_t(a.S), uP = uint32_t(P);
+    const int j0 = int(uint32_t(b) * uS / uP), j1 = int(uint32_t(b + 1) * uS / uP);
     volatile int* vabort = abort_flag;
     auto fail = [&]() {
         *vabort = 1;
@@ -192,14 +197,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
             prefetch_tensormap(&maps.m2[lane]);
         }
         if (!a.static_weights) grid_dependency_wait();
-        int job = 0, last_mine = -1;
+        int job = 0, last_mine = -1, js = 0, jr = 0;     // job = jr NS + js (no division per job)
         walk_blocks(a, j0, j1, meta, meta_wait, [&](const Blk& bk) -> bool {
             if (*vabort) return false;
             const CUtensorMap* map = bk.kind ? &maps.m2[bk.sg.wi] : &maps.m1[bk.sg.wi];
             for (int t = 0; t < nstage; ++t, ++job) {
+                const int s = js, round = jr;
+                if (++js == NS) {
+                    js = 0;
+                    ++jr;
+                }
                 if (job % kPlaneIssuers != pw) continue;
                 last_mine = job;
-                const int s = job % NS, round = job / NS;
                 if (round > 0 && !mbar_poll(&empty[s], (round - 1) & 1, kIdlePauseNs)) {
                     fail();
                     return false;
@@ -339,13 +348,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
                 fail();
                 return false;
             }
-            // row r of strip st: the sums of the strip's warps st, st + Sb, ... in warp order
+            // row r of strip st: the sums of the strip's warps st, st + Sb, ... in warp order, each
+            // the sum of its quad's lanes (lanes 0 + 1, 2 + 3, then the two)
             const int d0 = bk.kind ? bk.first * kStrip : (bk.first - bk.sg.ja) * kStrip;
             float* dst = (bk.kind ? res_y : main_y) + d0;
             for (int e = lane; e < bk.n * kStrip; e += 32) {
                 const int st = e >> 4, r = e & (kStrip - 1);
                 float v = 0.f;
-                for (int i = 0; i < wps; ++i) v += red[(nr * kW + st + Sb * i) * kStrip + r];
+                for (int i = 0; i < wps; ++i) {
+                    const float4 c = *reinterpret_cast<const float4*>(red + ((nr * kW + st + Sb * i) * kStrip + r) * 4);
+                    v += (c.x + c.y) + (c.z + c.w);
+                }
                 if (TERN_BOUNDS(a.status, d0 + e < kSegRows)) dst[e] = v;
             }
             __syncwarp();
@@ -543,10 +556,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
             return true;
         };
         const bool reload = nstage > 1;
-        for (int t = 0; t + 1 < nstage; ++t)
-            if (!stage(offf, xsf + uint32_t(t) * xstep, reload, gqf + t * 4 * SB, lanef, active && ngf > 0))
+        // one call site, so that the stage body is inlined once (the last stage takes its own
+        // offsets): a shorter loop for the instruction cache, measured faster than a separate copy
+#pragma unroll 1
+        for (int t = 0; t < nstage; ++t) {
+            const bool last = t + 1 == nstage;
+            uint32_t off[GW];
+#pragma unroll
+            for (int gi = 0; gi < GW; ++gi) off[gi] = last ? offl[gi] : offf[gi];
+            if (!stage(off, last ? xsl : xsf + uint32_t(t) * xstep, reload, last ? gql : gqf + t * 4 * SB,
+                       last ? lanel : lanef, active && (last ? ngl : ngf) > 0))
                 return false;
-        if (!stage(offl, xsl, reload, gql, lanel, active && ngl > 0)) return false;
+        }
         // the block's scales are no longer read (a warp with no work in the block still waits for
         // them, so that the buffer's phases stay in step)
         if (!sc_ready && !mbar_poll(&sfull[nb], (blk / kScaleBufs) & 1, 0)) {
@@ -555,19 +576,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sempty[nb]);
-        // the quad's four lanes hold the row sums of different groups
-        p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
-        p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
-        p0 += __shfl_xor_sync(0xffffffffu, p0, 2);
-        p1 += __shfl_xor_sync(0xffffffffu, p1, 2);
         const int nr = blk % kRedBufs, round = blk / kRedBufs;
         if (round > 0 && !mbar_poll(&redempty[nr], (round - 1) & 1, 0)) {
             fail();
             return false;
         }
-        if (q == 0 && TERN_BOUNDS(a.status, (nr * kW + warp) * kStrip + pr + 8 < kRedBufs * kW * kStrip)) {
-            red[(nr * kW + warp) * kStrip + pr] = p0;
-            red[(nr * kW + warp) * kStrip + pr + 8] = p1;
+        if (TERN_BOUNDS(a.status, ((nr * kW + warp) * kStrip + pr + 8) * 4 + q < kRedBufs * kW * kStrip * 4)) {
+            red[((nr * kW + warp) * kStrip + pr) * 4 + q] = p0;
+            red[((nr * kW + warp) * kStrip + pr + 8) * 4 + q] = p1;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&redfull[nr]);
@@ -637,7 +653,7 @@ bool make_layout(int K, int64_t per, int64_t res, bool has_mu, Layout& L) {
         int o = NS * stage_bytes;
         L.o_sc = o; o += kScaleBufs * L.sc_stride;
         L.o_mu = o; o += has_mu ? kScaleBufs * L.sc_stride : 0;
-        L.o_red = o; o += kRedBufs * kW * kStrip * 4;
+        L.o_red = o; o += kRedBufs * kW * kStrip * 4 * 4;
         L.o_xs = o; o += up(K * 2, 16);
         L.o_cofs = o; o += up(G * 4, 16);
         L.o_xsum = o; o += up(G * 4, 16);
@@ -709,6 +725,7 @@ bool decode1_supported(const tern_weight* const* ws, int nw) {
     }
     int64_t S, P, per, res;
     launch_strips(ws, nw, S, P, per, res);
+    if (S >= kMaxLaunchStrips || P > 256) return false;      // the CTA ranges' 32-bit arithmetic
     // segments of one CTA: its strips in pieces of kSegStrips, plus one more per weight boundary
     if ((per + kSegStrips - 1) / kSegStrips + (nw - 1) > kMaxSegs) return false;
     Layout L;

@@ -154,7 +154,11 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
     grid_launch_dependents();
 
     const int P = gridDim.x, b = blockIdx.x;
-    const int j0 = int((int64_t(b) * a.S) / P), j1 = int((int64_t(b + 1) * a.S) / P);
+    // the CTA's strips [j0, j1) = [b S / P, (b + 1) S / P), in 32-bit arithmetic: the host keeps S
+    // below 2^24 and P is at most the SM count, so (b + 1) S fits (a 64-bit division here cost
+    // hundreds of cycles before the first copy of every launch)
+    const uint32_t uS = uint32_t(a.S), uP = uint32_t(P);
+    const int j0 = int(uint32_t(b) * uS / uP), j1 = int(uint32_t(b + 1) * uS / uP);
     volatile int* vabort = abort_flag;
     auto fail = [&]() {
         *vabort = 1;
@@ -177,14 +181,18 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
         // x may be written by the previous kernel; with x resident the stages hold static weights
         // only, which may stream before the wait
         if (!XRES || !a.static_weights) grid_dependency_wait();
-        int job = 0, last_mine = -1;
+        int job = 0, last_mine = -1, js = 0, jr = 0;     // job = jr NS + js (no division per job)
         walk_blocks(a, j0, j1, meta, meta_wait, [&](const Blk& bk) -> bool {
             if (*vabort) return false;
             const CUtensorMap* map = bk.kind ? &maps.m2[bk.sg.wi] : &maps.m1[bk.sg.wi];
             for (int t = 0; t < nstage; ++t, ++job) {
+                const int s = js, round = jr;
+                if (++js == NS) {
+                    js = 0;
+                    ++jr;
+                }
                 if (job % kPlaneIssuers != pw) continue;
                 last_mine = job;
-                const int s = job % NS, round = job / NS;
                 if (round > 0 && !mbar_poll(&empty[s], (round - 1) & 1, kIdlePauseNs)) {
                     fail();
                     return false;
@@ -738,6 +746,7 @@ bool decodem_supported(const tern_weight* const* ws, int nw, int64_t M, const vo
     }
     int64_t S, P, per, res;
     strips_m(ws, nw, S, P, per, res);
+    if (S >= kMaxLaunchStrips || P > 256) return false;      // the CTA ranges' 32-bit arithmetic
     // below 9 tokens the cluster kernel is faster on launches of few strips per CTA, and at 4
     // tokens on every launch of the 8B stack (measured: this kernel wins its gate+up launch, 12
     // strips per CTA, at 8 tokens and in isolation at 4, but the stack at 4 tokens is faster with

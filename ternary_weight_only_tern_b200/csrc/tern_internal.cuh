@@ -36,6 +36,7 @@ size_t gemv_workspace_bytes(const tern_weight& w, int64_t M);
 
 // Decode GEMV for one token on a persistent, warp-specialised grid (tern_decode1.cu): row-level
 // residual planes and offsets, K % 512 == 0; decode1_supported tells whether it takes the call.
+constexpr int64_t kMaxLaunchStrips = int64_t(1) << 24;   // 16-row strips of one persistent decode launch
 bool decode1_supported(const tern_weight* const* ws, int nw);
 tern_status decode1_launch_group(const tern_weight* const* ws, int nw, const __half* x, __half* const* ys,
                                  const tern_weight* const* next, int nnext, cudaStream_t stream);
