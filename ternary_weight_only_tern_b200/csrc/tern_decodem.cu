@@ -48,11 +48,13 @@ constexpr int kW = 8;                      // consumer warps
 constexpr int kPlaneIssuers = 2;
 constexpr int kScaleIssuers = 1;
 constexpr int kProducers = kPlaneIssuers + kScaleIssuers;
-constexpr int kThreads = (kW + kProducers) * 32;    // the scale issuer also writes the segment metadata
+constexpr int kThreads = (kW + kProducers + 1) * 32;    // + the epilogue warp; the scale issuer also writes
+                                                        // the segment metadata
 // strips per consumer warp: 4 with one token block, 2 with two (the registers for both blocks'
 // activations and sums); a stage then holds 2 x that many strip slabs (16 or 8 KB of plane)
 __host__ __device__ constexpr int strips_per_warp(int mt) { return mt == 1 ? 4 : 2; }
 constexpr int kScaleBufs = 2;
+constexpr int kRedBufs = 2;                // block partial-sum buffers (consumers -> epilogue)
 constexpr int kMaxStages = 6;
 constexpr int kTokPad = 16;                // tokens per row of the C and X tables
 constexpr int kSmemMaxM = 227 * 1024;
@@ -122,13 +124,17 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
     uint64_t* sfull = empty + NS;                 // [kScaleBufs] the block's scales landed
     uint64_t* sempty = sfull + kScaleBufs;        // [kScaleBufs] the block's scales are no longer read
     uint64_t* meta_bar = sempty + kScaleBufs;
-    uint64_t* cbar = meta_bar + 1;                // the consumer warps' block-end barrier
-    int* abort_flag = reinterpret_cast<int*>(cbar + 1);
+    uint64_t* cbar = meta_bar + 1;                // the consumer warps' barrier after the first block
+    uint64_t* redfull = cbar + 1;                 // [kRedBufs] the block's partial sums are written
+    uint64_t* redempty = redfull + kRedBufs;      // [kRedBufs] ... and were read
+    int* abort_flag = reinterpret_cast<int*>(redempty + kRedBufs);
     const uint32_t stage0 = smem_u32(smem);
     const int stage_bytes = a.stage_bytes;
     const int slab_bytes = Sb * kStrip * kSlabBytes;
     uint8_t* sc_base = smem + a.o_sc;                            // [kScaleBufs][16 Sb rows][G] (skewed)
-    float* red = reinterpret_cast<float*>(smem + a.o_red);       // [W][strips per warp][16 rows][M]
+    float* red = reinterpret_cast<float*>(smem + a.o_red);       // [kRedBufs][W][strips per warp][16 rows][M + 1]
+    const int Mp = M + 1;                                        // (odd: the epilogue's reads spread the banks)
+    const int red_stride = kW * kStripsPerWarp * kStrip * Mp;
     float* cofs = reinterpret_cast<float*>(smem + a.o_cofs);     // [G][16 tokens]
     float* xsum = reinterpret_cast<float*>(smem + a.o_xsum);     // [G][16 tokens]
     int* meta = reinterpret_cast<int*>(smem + a.o_meta);         // [kMaxSegs][2]: s_a, residual strips
@@ -147,6 +153,10 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
         }
         mbar_init(meta_bar, 1);
         mbar_init(cbar, kW);
+        for (int i = 0; i < kRedBufs; ++i) {
+            mbar_init(&redfull[i], kW);
+            mbar_init(&redempty[i], 1);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -299,6 +309,72 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
         return;
     }
 
+    if (warp == kW + kProducers) {
+        // ------------------------------------------------------------ epilogue
+        // per block: the (row, token) sums over the strip's warps, in warp order (strip st's warps
+        // are (st % ss) gs4 + g, g < gs4, each with it as its strip st / ss); a main row without a
+        // residual row is written at once, the others wait in main_y for their residual block.
+        // Lanes take tokens fastest (the partial sums' token rows are padded to an odd length).
+        grid_dependency_wait();       // y may still be read by the previous kernel
+        if (!meta_wait()) return;     // the segments' slot tables
+        const int gs4 = 4 * SB, ss = kW / gs4;
+        int blk = 0;
+        walk_blocks(a, j0, j1, meta, meta_wait, [&](const Blk& bk) -> bool {
+            if (*vabort) return false;
+            const int nr = blk % kRedBufs, rround = blk / kRedBufs;
+            if (!mbar_poll(&redfull[nr], rround & 1, kIdlePauseNs)) {
+                fail();
+                return false;
+            }
+            const float* redb = red + nr * red_stride;
+            const DMWeight& Wt = a.w[bk.sg.wi];
+            __half* yw = Wt.y;
+            const int64_t Nw = Wt.N;
+            const int64_t n_a = int64_t(bk.sg.ja) * kStrip;
+            const int cells = bk.n * kStrip * M;
+            const int gstride = kStripsPerWarp * kStrip * Mp;      // from one warp's sums to the next's
+            for (int e = lane; e < cells; e += 32) {
+                const int R = e / M, m = e - R * M;
+                const int st = R >> 4, r = R & (kStrip - 1);
+                const int w0 = (st % ss) * gs4, k = st / ss;
+                const float* src = redb + ((w0 * kStripsPerWarp + k) * kStrip + r) * Mp + m;
+                // gs4 is 4 or 8: all loads first, then the sum in warp order
+                float t[8];
+                float v;
+                if (gs4 == 8) {
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) t[g] = src[g * gstride];
+                    v = 0.f;
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) v += t[g];
+                } else {
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) t[g] = src[g * gstride];
+                    v = 0.f;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) v += t[g];
+                }
+                if (bk.kind == 0) {
+                    const int lr = (bk.first - bk.sg.ja) * kStrip + R;
+                    if (n_a + lr < Nw && TERN_BOUNDS(a.status, lr < kSegRows)) {
+                        if (bslot[bk.k * kSegRows + lr] < 0) yw[int64_t(m) * Nw + n_a + lr] = __float2half_rn(v);
+                        else main_y[m * kSegRows + lr] = v;
+                    }
+                } else {
+                    const int d = bk.first * kStrip + R;
+                    const int lr = d < kSegRows ? rslot[bk.k * kSegRows + d] : -1;
+                    if (lr >= 0 && TERN_BOUNDS(a.status, lr < kSegRows && n_a + lr < Nw))
+                        yw[int64_t(m) * Nw + n_a + lr] = __float2half_rn(main_y[m * kSegRows + lr] + v);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&redempty[nr]);
+            ++blk;
+            return true;
+        });
+        return;
+    }
+
     // ---------------------------------------------------------------- consumers
     const int q = lane & 3, rr = lane >> 2;
     const int pr = lane_row(rr);
@@ -349,8 +425,6 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
     }
     const uint32_t ring_end = stage0 + uint32_t(NS * stage_bytes);
     uint32_t tile = stage0, fullb = smem_u32(full), emptyb = smem_u32(empty), ph = 0;
-    const int tid = threadIdx.x;           // consumer threads: 0 .. 255
-    bool have_meta = false;
     // a bounded barrier of the consumer warps (a warp that gave up makes the others give up too)
     uint32_t cph = 0;
     auto csync = [&]() -> bool {
@@ -552,14 +626,21 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sempty[nb]);
-        // the warp's running sums: red[warp][k][row][token]
+        // the warp's running sums into partial-sum buffer nr (red[nr][warp][k][row][token]), for the
+        // epilogue warp; the consumers go on with the next block
+        const int nr = blk % kRedBufs, rround = blk / kRedBufs;
+        if (rround > 0 && !mbar_poll(&redempty[nr], (rround - 1) & 1, 0)) {
+            fail();
+            return false;
+        }
+        float* redb = red + nr * red_stride;
 #pragma unroll
         for (int k = 0; k < kStripsPerWarp; ++k)
 #pragma unroll
             for (int o = 0; o < MT; ++o) {
                 const int n0 = 8 * o + 2 * q;
-                float* ra = red + ((warp * kStripsPerWarp + k) * kStrip + pr) * M;
-                float* rb = ra + 8 * M;
+                float* ra = redb + ((warp * kStripsPerWarp + k) * kStrip + pr) * Mp;
+                float* rb = ra + 8 * Mp;
                 if (!TERN_BOUNDS(a.status, (warp * kStripsPerWarp + k) * kStrip + pr + 8 < kW * kStripsPerWarp * kStrip))
                     continue;
                 if (n0 < M) {
@@ -571,41 +652,10 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
                     rb[n0 + 1] = run[k][o][3];
                 }
             }
-        if (!csync()) return false;
-        if (!have_meta) {
-            if (!meta_wait()) return false;
-            have_meta = true;
-        }
-        // (row, token) sums over the strip's warps in warp order; rows are written once complete.
-        // Thread tid takes token tid / 16 and rows tid % 16 + 16 i of the block; strip st's warps
-        // are (st % ss) gs4 + g, g < gs4, each with it as strip st / ss.
-        {
-            const int m = tid >> 4;
-            __half* yw = Wt.y;
-            const int64_t Nw = Wt.N;
-            const int64_t n_a = int64_t(bk.sg.ja) * kStrip;
-            if (m < M) {
-                for (int R = tid & 15; R < bk.n * kStrip; R += 16) {
-                    const int st = R >> 4, r = R & (kStrip - 1);
-                    const int w0 = (st % ss) * gs4, k = st / ss;
-                    float v = 0.f;
-                    for (int g = 0; g < gs4; ++g) v += red[(((w0 + g) * kStripsPerWarp + k) * kStrip + r) * M + m];
-                    if (bk.kind == 0) {
-                        const int lr = (bk.first - bk.sg.ja) * kStrip + R;
-                        if (n_a + lr < Nw && TERN_BOUNDS(a.status, lr < kSegRows)) {
-                            if (bslot[bk.k * kSegRows + lr] < 0) yw[int64_t(m) * Nw + n_a + lr] = __float2half_rn(v);
-                            else main_y[m * kSegRows + lr] = v;
-                        }
-                    } else {
-                        const int d = bk.first * kStrip + R;
-                        const int lr = d < kSegRows ? rslot[bk.k * kSegRows + d] : -1;
-                        if (lr >= 0 && TERN_BOUNDS(a.status, lr < kSegRows && n_a + lr < Nw))
-                            yw[int64_t(m) * Nw + n_a + lr] = __float2half_rn(main_y[m * kSegRows + lr] + v);
-                    }
-                }
-            }
-        }
-        if (!csync()) return false;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&redfull[nr]);
+        // the C and X tables of the first block are read by other warps from the second block on
+        if (blk == 0 && !csync()) return false;
         ++blk;
         return true;
     });
@@ -665,17 +715,16 @@ bool make_layout_m(int K, int M, int64_t per, int64_t res, bool has_mu, LayoutM&
     }
     auto up = [](int v, int a) { return (v + a - 1) / a * a; };
     L.sc_stride = up(kStrip * L.Sb * G * 2 + 16, 16);
-    // x resident (stages of plane alone, at least 4 of them), else x streamed with each stage
-    // (at least 3 stages)
+    // x resident (stages of plane alone), else x streamed with each stage; at least 3 stages
     for (int xres = 1; xres >= 0; --xres) {
         L.xres = xres == 1;
         const int plane = L.Sb * L.SB * kStrip * kSlabBytes;
         L.stage_bytes = plane + (L.xres ? 0 : M * L.SB * 1024);
-        for (int NS = kMaxStages; NS >= (L.xres ? 4 : 3); --NS) {
+        for (int NS = kMaxStages; NS >= 3; --NS) {
             int o = NS * L.stage_bytes;
             L.o_sc = o; o += kScaleBufs * L.sc_stride;
             L.o_mu = o; o += has_mu ? kScaleBufs * L.sc_stride : 0;
-            L.o_red = o; o += kW * spw * kStrip * M * 4;
+            L.o_red = o; o += kRedBufs * kW * spw * kStrip * (M + 1) * 4;
             L.o_cofs = o; o += up(G * kTokPad * 4, 16);
             L.o_xsum = o; o += up(G * kTokPad * 4, 16);
             L.o_meta = o; o += up(kMaxSegs * 2 * 4, 16);
@@ -683,7 +732,7 @@ bool make_layout_m(int K, int M, int64_t per, int64_t res, bool has_mu, LayoutM&
             L.o_rslot = o; o += kMaxSegs * kSegRows * 2;
             L.o_mainy = o; o += M * kSegRows * 4;
             L.o_xs = o; o += L.xres ? up(M * (K + 8) * 2, 16) : 0;
-            L.o_bar = o; o += up((2 * NS + 2 * kScaleBufs + 2) * 8 + 8, 16);
+            L.o_bar = o; o += up((2 * NS + 2 * kScaleBufs + 2 + 2 * kRedBufs) * 8 + 8, 16);
             L.total = o + 1024;
             L.NS = NS;
             if (L.total <= kSmemMaxM) return true;
