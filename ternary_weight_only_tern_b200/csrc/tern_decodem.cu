@@ -89,7 +89,7 @@ struct DMArgs {
     int32_t stage_bytes;      // plane box + x box
     int32_t sc_stride;
     int32_t o_sc, o_mu, o_red, o_cofs, o_xsum, o_meta, o_bslot, o_rslot, o_mainy, o_bar;
-    int32_t o_xs;             // resident x: [M][K + 8] fp16, pair order (XRES)
+    int32_t o_xs;             // resident x: [M][K + 32] fp16, pair order, pieces transposed (XRES)
     int32_t static_weights;
     const uint8_t* pf_ptr[kPfRanges];
     int64_t pf_bytes[kPfRanges];
@@ -382,13 +382,18 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
     const int gw = warp % gs4;                    // the warp's group within a stage
     const int sw0 = warp / gs4, ss = kW / gs4;    // its strips: sw0 + ss k, k < kStripsPerWarp
     grid_dependency_wait();
-    const int xstride = a.K + 8;                  // halves per resident token row (spreads the banks)
+    // Resident x: token rows of K + 32 halves (2K + 64 bytes: consecutive tokens 64 bytes apart
+    // modulo 128), and within each group's 256 bytes the 16-byte piece i of lane q's 64 bytes
+    // (q < 4, i < 4) stored at piece 4 i + q: the eight lanes of a quarter warp (two tokens, four
+    // q) then read eight different 16-byte bank groups with each load
+    const int xstride = a.K + 32;
     __half* xs = reinterpret_cast<__half*>(smem + a.o_xs);
     if (XRES) {
         // every token's x with the two activations of each decoded pair adjacent
         const int per_tok = a.K / 16;
         for (int u = threadIdx.x; u < M * per_tok; u += kW * 32) {
             const int m = u / per_tok, i = u - m * per_tok;
+            const int g = i >> 3, uu = i & 7;         // group, and unit (pieces 2 uu, 2 uu + 1) in it
             const uint4* src = reinterpret_cast<const uint4*>(a.x + int64_t(m) * a.K + int64_t(i) * 16);
             const uint4 lo = __ldg(src), hi = __ldg(src + 1);
             uint4 o0, o1;
@@ -396,9 +401,10 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
             o0.z = prmt(lo.y, hi.y, 0x5410u); o0.w = prmt(lo.y, hi.y, 0x7632u);
             o1.x = prmt(lo.z, hi.z, 0x5410u); o1.y = prmt(lo.z, hi.z, 0x7632u);
             o1.z = prmt(lo.w, hi.w, 0x5410u); o1.w = prmt(lo.w, hi.w, 0x7632u);
-            uint4* dst = reinterpret_cast<uint4*>(xs + int64_t(m) * xstride + int64_t(i) * 16);
-            dst[0] = o0;
-            dst[1] = o1;
+            uint4* grp = reinterpret_cast<uint4*>(xs + int64_t(m) * xstride + int64_t(g) * kGroup);
+            const int p0 = 8 * (uu & 1) + (uu >> 1);  // piece c -> 4 (c % 4) + c / 4, c = 2 uu, 2 uu + 1
+            grp[p0] = o0;
+            grp[p0 + 4] = o1;
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kW * 32) : "memory");
     }
@@ -414,13 +420,13 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
     }
     // x tile row of token block o: (2 gw + q / 2) M + token; its 16-byte pieces 4 (q & 1) + i,
     // swizzled with the row
-    // (resident x: token row n, words 2q and 2q + 1 of the group, the pair order staged above)
+    // (resident x: token row n, lane q's pieces 4 i + q of the group, as staged above)
     uint32_t xrow[MT], xsw[MT];
 #pragma unroll
     for (int o = 0; o < MT; ++o) {
         const int n = min(8 * o + rr, M - 1);
         const int row = (2 * gw + (q >> 1)) * M + n;
-        xrow[o] = XRES ? smem_u32(xs) + uint32_t((n * xstride + gw * kGroup + 32 * q) * 2) : plane_stage + uint32_t(row * 128);
+        xrow[o] = XRES ? smem_u32(xs) + uint32_t((n * xstride + gw * kGroup) * 2 + 16 * q) : plane_stage + uint32_t(row * 128);
         xsw[o] = uint32_t(row & 7);
     }
     const uint32_t ring_end = stage0 + uint32_t(NS * stage_bytes);
@@ -464,10 +470,10 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
                 const uint32_t xt = uint32_t(t * gs4 * kGroup * 2);
 #pragma unroll
                 for (int o = 0; o < MT; ++o) {
-                    if (TERN_BOUNDS(a.status, xrow[o] + xt + 64 <= smem_u32(xs) + uint32_t(M * xstride * 2))) {
+                    if (TERN_BOUNDS(a.status, xrow[o] + xt + 64 * 3 + 16 <= smem_u32(xs) + uint32_t(M * xstride * 2))) {
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const uint4 v = lds_u4(xrow[o] + xt + 16 * i);
+                            const uint4 v = lds_u4(xrow[o] + xt + 64 * i);
                             xr[o][4 * i] = v.x; xr[o][4 * i + 1] = v.y; xr[o][4 * i + 2] = v.z; xr[o][4 * i + 3] = v.w;
                         }
                     } else {
@@ -731,7 +737,7 @@ bool make_layout_m(int K, int M, int64_t per, int64_t res, bool has_mu, LayoutM&
             L.o_bslot = o; o += kMaxSegs * kSegRows * 2;
             L.o_rslot = o; o += kMaxSegs * kSegRows * 2;
             L.o_mainy = o; o += M * kSegRows * 4;
-            L.o_xs = o; o += L.xres ? up(M * (K + 8) * 2, 16) : 0;
+            L.o_xs = o; o += L.xres ? up(M * (K + 32) * 2, 16) : 0;
             L.o_bar = o; o += up((2 * NS + 2 * kScaleBufs + 2 + 2 * kRedBufs) * 8 + 8, 16);
             L.total = o + 1024;
             L.NS = NS;
