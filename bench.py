@@ -50,8 +50,8 @@ KERNEL_TRAFFIC = {
     "gemv": {"sources": ["ternary_weight_only_tern_b200/csrc/tern_decode1.cu",
                          "ternary_weight_only_tern_b200/csrc/tern_device.cuh",
                          "ternary_weight_only_tern_b200/csrc/tern_stream.cuh"],
-             "sha256": "3a10bcd2147430c31422fcf4364b348dc0767912240785f64f0a4cfdf6b3332d",
-             "bytes": 30946048},
+             "sha256": "65a0df0ff98dfa93501b9408177c3e2a8b16b335ec8b17036144a569b0266539",
+             "bytes": 30931712},
 }
 
 
