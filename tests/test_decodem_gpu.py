@@ -1,5 +1,5 @@
-"""GPU parity of the multi-token decode kernel (the call takes it for 9 <= M <= 16, and for M = 8
-on launches of at least 10 strips per CTA; K a multiple of 512; the other calls run the cluster
+"""GPU parity of the multi-token decode kernel (the call takes it for 9 <= M <= 16, and for
+4 <= M <= 8 on launches of at least 10 strips per CTA; K a multiple of 512; the other calls run the cluster
 kernel and are covered here too): the persistent GEMV whose MMA columns are the tokens. Cases aimed at its structure: one and two 8-token column
 blocks and ragged token counts, blocks of 8 and 4 strips (1 and 2 slabs per stage), ranges that
 span several segments and weight boundaries, residual rows that fill whole segments, K with an
@@ -47,12 +47,12 @@ def test_shapes_tokens_and_residual_fractions(M, K, N, pct):
     check(run(t.x, weight(t)), oracle.linear(t.x, t.T1, t.s1, t.res_rows, t.T2, t.s2))
 
 
-@pytest.mark.parametrize("M", [2, 5, 8])
+@pytest.mark.parametrize("M", [2, 3, 4, 5, 7, 8])
 @pytest.mark.parametrize("K,pct", [(4096, 15), (12288, 10), (2560, 100)])
 def test_one_token_block_on_large_launches(M, K, pct):
-    """11 strips per CTA: at M = 8 one 8-token column block in this kernel, x resident in shared
-    memory (K = 4096, 2560) or streamed with the stages (K = 12288); at M = 2 and 5 the cluster
-    kernel on the same shapes."""
+    """11 strips per CTA: at M = 4 to 8 one (ragged) 8-token column block in this kernel, x resident
+    in shared memory (K = 4096, 2560) or streamed with the stages (K = 12288); at M = 2 and 3 the
+    cluster kernel on the same shapes."""
     rng = np.random.default_rng(M * 100 + K + pct)
     N = 148 * 16 * 11 + 5
     t = synth.draw_tensor(rng, "l", N, K, M, p_zero=0.4, res_pct=pct)
@@ -84,7 +84,7 @@ def test_group_boundaries_inside_cta_ranges(M):
 
 
 @pytest.mark.parametrize("M,N,K,r", [(2, 256, 512, 40), (8, 1024 + 5, 4096, 1024 + 5), (16, 130, 12288, 13),
-                                     (11, 4000, 2560, 600)])
+                                     (11, 4000, 2560, 600), (5, 148 * 16 * 11, 4096, 3000)])
 def test_exact_case_bit_exact(M, N, K, r):
     rng = np.random.default_rng(M + N * 3 + K + r)
     t = synth.draw_exact_tensor(rng, N, K, M, r)
