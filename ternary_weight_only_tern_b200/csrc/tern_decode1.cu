@@ -21,8 +21,9 @@
 //  * Two producer warps issue the planes' boxes (a bulk or TMA copy holds its issuing thread for
 //    a while, so they take every other stage each) and one more the blocks' scales (and
 //    offsets), one bulk copy per block into one of two block buffers. An epilogue warp adds the
-//    warps' sums of each strip in warp order, keeps the sums of the current segment (up to 256
-//    rows) in shared memory, adds the residual rows' sums and writes y.
+//    warps' sums of each strip in warp order and writes a row at once unless it has a residual
+//    row; those rows' main sums wait in shared memory for their residual block, which adds its
+//    sums and writes them (so the tail after the last block is one block's rows, not a segment's).
 //  * Residual rows: since R is sorted, the residual rows of a segment are the contiguous slots
 //    [s_a, s_a + span) of the residual plane; they stream as extra blocks after the segment's
 //    main blocks, and each row's residual sum joins its main sum before the single rounding to
@@ -104,7 +105,7 @@ struct D1Args {
     int32_t static_weights;
     int32_t has_mu;
     // shared-memory offsets in bytes from the 1024-aligned base (the stages start at 0)
-    int32_t o_sc, o_mu, o_red, o_xs, o_cofs, o_xsum, o_meta, o_bslot, o_mainy, o_resy, o_bar;
+    int32_t o_sc, o_mu, o_red, o_xs, o_cofs, o_xsum, o_meta, o_bslot, o_rslot, o_mainy, o_bar;
     int32_t sc_stride;        // bytes of one block scale buffer (16 Sb rows x G fp16, + skew)
     // L2 prefetch of the next call's weights: each CTA takes pf_per bytes of each range
     const uint8_t* pf_ptr[kPfRanges];
@@ -147,9 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
     float* cofs = reinterpret_cast<float*>(smem + a.o_cofs);     // [G] C of every group
     float* xsum = reinterpret_cast<float*>(smem + a.o_xsum);     // [G] X of every group
     int* meta = reinterpret_cast<int*>(smem + a.o_meta);         // [kMaxSegs][2]: s_a, residual strips
-    int16_t* bslot = reinterpret_cast<int16_t*>(smem + a.o_bslot);  // [kMaxSegs][256]
-    float* main_y = reinterpret_cast<float*>(smem + a.o_mainy);  // [256]
-    float* res_y = reinterpret_cast<float*>(smem + a.o_resy);    // [256]
+    int16_t* bslot = reinterpret_cast<int16_t*>(smem + a.o_bslot);  // [kMaxSegs][256] row -> slot - s_a
+    int16_t* rslot = reinterpret_cast<int16_t*>(smem + a.o_rslot);  // [kMaxSegs][256] slot - s_a -> row
+    float* main_y = reinterpret_cast<float*>(smem + a.o_mainy);  // [256] main sums of rows with a residual
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -277,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
 
     if (warp == kW + kProducers) {
         // ------------------------------------------------------------ epilogue
-        // segment metadata: the slots of the segment's residual rows
+        // segment metadata: the slots of the segment's residual rows, both ways
         if (!a.static_weights) grid_dependency_wait();
         {
             int j = j0, k = 0;
@@ -299,14 +300,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
                         smin = min(smin, v);
                         smax = max(smax, v);
                     }
+                    rslot[k * kSegRows + lr] = -1;
                 }
                 smin = __reduce_min_sync(0xffffffffu, smin);
                 smax = __reduce_max_sync(0xffffffffu, smax);
                 const int span = smax >= 0 ? min(smax - smin + 1, kSegRows) : 0;
+                __syncwarp();
 #pragma unroll
                 for (int i = 0; i < kSegRows / 32; ++i) {
                     const int d = sl[i] - smin;
-                    bslot[k * kSegRows + lane + 32 * i] = int16_t((sl[i] >= 0 && d < span) ? d : -1);
+                    const bool has = sl[i] >= 0 && d < span;
+                    bslot[k * kSegRows + lane + 32 * i] = int16_t(has ? d : -1);
+                    if (has) rslot[k * kSegRows + d] = int16_t(lane + 32 * i);
                 }
                 if (lane == 0) {
                     meta[2 * k] = smax >= 0 ? smin : 0;
@@ -320,38 +325,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
         grid_dependency_wait();       // y may still be read by the previous kernel
         const int wps = kW / Sb;
         int blk = 0;
-        int cur_k = -1;
-        Seg cur{};
-        auto flush = [&]() {          // write the finished segment's rows
-            if (cur_k < 0) return;
-            const D1Weight& Wt = a.w[cur.wi];
-            const int64_t n_a = int64_t(cur.ja) * kStrip;
-            const int rows = int(min(int64_t(cur.jb) * kStrip, Wt.N) - n_a);
-            __syncwarp();
-            for (int lr = lane; lr < rows; lr += 32) {
-                float v = main_y[lr];
-                const int bs = bslot[cur_k * kSegRows + lr];
-                if (bs >= 0 && TERN_BOUNDS(a.status, bs < kSegRows)) v += res_y[bs];
-                Wt.y[n_a + lr] = __float2half_rn(v);
-            }
-            __syncwarp();
-        };
+        // per block: row r of strip st is the sum of the strip's warps st, st + Sb, ... in warp order,
+        // each the sum of its quad's lanes (lanes 0 + 1, 2 + 3, then the two). A main row without a
+        // residual row is written at once; the others wait in main_y for their residual block, whose
+        // slots map back to their rows, so nothing is left to write when the last block is done.
         walk_blocks(a, j0, j1, meta, [] { return true; }, [&](const Blk& bk) -> bool {
             if (*vabort) return false;
-            if (bk.k != cur_k) {
-                flush();
-                cur_k = bk.k;
-                cur = bk.sg;
-            }
             const int nr = blk % kRedBufs, round = blk / kRedBufs;
             if (!mbar_poll(&redfull[nr], round & 1, kIdlePauseNs)) {
                 fail();
                 return false;
             }
-            // row r of strip st: the sums of the strip's warps st, st + Sb, ... in warp order, each
-            // the sum of its quad's lanes (lanes 0 + 1, 2 + 3, then the two)
+            const D1Weight& Wt = a.w[bk.sg.wi];
+            const int64_t n_a = int64_t(bk.sg.ja) * kStrip;
             const int d0 = bk.kind ? bk.first * kStrip : (bk.first - bk.sg.ja) * kStrip;
-            float* dst = (bk.kind ? res_y : main_y) + d0;
             for (int e = lane; e < bk.n * kStrip; e += 32) {
                 const int st = e >> 4, r = e & (kStrip - 1);
                 float v = 0.f;
@@ -359,14 +346,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode1_kernel(const __grid_const
                     const float4 c = *reinterpret_cast<const float4*>(red + ((nr * kW + st + Sb * i) * kStrip + r) * 4);
                     v += (c.x + c.y) + (c.z + c.w);
                 }
-                if (TERN_BOUNDS(a.status, d0 + e < kSegRows)) dst[e] = v;
+                const int d = d0 + e;
+                if (!TERN_BOUNDS(a.status, d < kSegRows)) continue;
+                if (bk.kind == 0) {
+                    if (n_a + d >= Wt.N) continue;
+                    if (bslot[bk.k * kSegRows + d] < 0) Wt.y[n_a + d] = __float2half_rn(v);
+                    else main_y[d] = v;
+                } else {
+                    const int lr = rslot[bk.k * kSegRows + d];
+                    if (lr >= 0 && TERN_BOUNDS(a.status, lr < kSegRows && n_a + lr < Wt.N))
+                        Wt.y[n_a + lr] = __float2half_rn(main_y[lr] + v);
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&redempty[nr]);
             ++blk;
             return true;
         });
-        if (!*vabort) flush();
         return;
     }
 
@@ -609,7 +605,7 @@ bool slab_map(CUtensorMap* map, const uint32_t* plane, int64_t rows, int64_t K, 
 
 struct Layout {
     int Sb, SB, GW, nstage, NS, sc_stride;
-    int o_sc, o_mu, o_red, o_xs, o_cofs, o_xsum, o_meta, o_bslot, o_mainy, o_resy, o_bar, total;
+    int o_sc, o_mu, o_red, o_xs, o_cofs, o_xsum, o_meta, o_bslot, o_rslot, o_mainy, o_bar, total;
 };
 
 constexpr int kSmemMax = 227 * 1024;
@@ -659,8 +655,8 @@ bool make_layout(int K, int64_t per, int64_t res, bool has_mu, Layout& L) {
         L.o_xsum = o; o += up(G * 4, 16);
         L.o_meta = o; o += up(kMaxSegs * 2 * 4, 16);
         L.o_bslot = o; o += up(kMaxSegs * kSegRows * 2, 16);
+        L.o_rslot = o; o += up(kMaxSegs * kSegRows * 2, 16);
         L.o_mainy = o; o += kSegRows * 4;
-        L.o_resy = o; o += kSegRows * 4;
         L.o_bar = o; o += up((2 * NS + 2 * kScaleBufs + 2 * kRedBufs + 1) * 8 + 8, 16);
         L.total = o + 1024;     // alignment slack
         L.NS = NS;
@@ -778,8 +774,8 @@ tern_status decode1_launch_group(const tern_weight* const* ws, int nw, const __h
     a.static_weights = all_static ? 1 : 0;
     a.has_mu = has_mu ? 1 : 0;
     a.o_sc = L.o_sc; a.o_mu = L.o_mu; a.o_red = L.o_red; a.o_xs = L.o_xs; a.o_cofs = L.o_cofs;
-    a.o_xsum = L.o_xsum; a.o_meta = L.o_meta; a.o_bslot = L.o_bslot; a.o_mainy = L.o_mainy;
-    a.o_resy = L.o_resy; a.o_bar = L.o_bar;
+    a.o_xsum = L.o_xsum; a.o_meta = L.o_meta; a.o_bslot = L.o_bslot; a.o_rslot = L.o_rslot;
+    a.o_mainy = L.o_mainy; a.o_bar = L.o_bar;
     a.sc_stride = L.sc_stride;
     const int grid = int(P);
     for (int j = 0; j < nnext; ++j) {
