@@ -50,8 +50,8 @@ KERNEL_TRAFFIC = {
     "gemv": {"sources": ["ternary_weight_only_tern_b200/csrc/tern_decode1.cu",
                          "ternary_weight_only_tern_b200/csrc/tern_device.cuh",
                          "ternary_weight_only_tern_b200/csrc/tern_stream.cuh"],
-             "sha256": "65a0df0ff98dfa93501b9408177c3e2a8b16b335ec8b17036144a569b0266539",
-             "bytes": 30931712},
+             "sha256": "8ba4c6d092030926afbdc55525a892640598107fda41a041f6aa1d780813045f",
+             "bytes": 30930176},
 }
 
 
