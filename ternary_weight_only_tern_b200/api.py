@@ -14,7 +14,14 @@ from . import _lib
 GROUP = 128
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(device: torch.device | None = None) -> ctypes.c_void_p:
+    """The current CUDA stream of `device` (torch's raw accessor where it exists: it is read on
+    every call, and the stream object costs microseconds to build)."""
+    if _raw_stream is not None and device is not None and device.index is not None:
+        return ctypes.c_void_p(_raw_stream(device.index))
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
@@ -167,6 +174,13 @@ class TernWeight:
     def device(self) -> torch.device:
         return self.plane1.device
 
+    def __setattr__(self, name, value):
+        # a changed field drops the cached C descriptor and workspace sizes
+        object.__setattr__(self, name, value)
+        if name not in ("_c", "_ws"):
+            object.__setattr__(self, "_c", None)
+            object.__setattr__(self, "_ws", None)
+
     def c_struct(self) -> _lib.TernWeightC:
         c = getattr(self, "_c", None)
         if c is None:
@@ -255,7 +269,15 @@ def weight_validate(w: TernWeight) -> None:
 # ------------------------------------------------------------------------------ linear
 
 def workspace_bytes(w: TernWeight, M: int) -> int:
-    return int(_lib.load().tern_linear_workspace_bytes(ctypes.byref(w.c_struct()), M))
+    """tern_linear_workspace_bytes, remembered per weight and M."""
+    cache = getattr(w, "_ws", None)
+    if cache is None:
+        cache = {}
+        object.__setattr__(w, "_ws", cache)
+    n = cache.get(M)
+    if n is None:
+        n = cache[M] = int(_lib.load().tern_linear_workspace_bytes(ctypes.byref(w.c_struct()), M))
+    return n
 
 
 def linear(x: torch.Tensor, w: TernWeight, out: torch.Tensor | None = None,
@@ -288,6 +310,21 @@ def linear(x: torch.Tensor, w: TernWeight, out: torch.Tensor | None = None,
     return out
 
 
+def _weight_array(ws: list):
+    """The C array of the weights' descriptor addresses, kept on the first weight per group (the
+    key holds the descriptors' addresses, which stay valid while the entry holds them)."""
+    structs = [w.c_struct() for w in ws]
+    key = tuple(ctypes.addressof(c) for c in structs)
+    cache = getattr(ws[0], "_groups", None)
+    if cache is None:
+        cache = {}
+        object.__setattr__(ws[0], "_groups", cache)
+    hit = cache.get(key)
+    if hit is None:
+        hit = cache[key] = ((ctypes.c_void_p * len(ws))(*key), structs)
+    return hit[0]
+
+
 def linear_group(x: torch.Tensor, ws: list, outs: list | None = None, workspace: torch.Tensor | None = None,
                  prefetch: list | None = None) -> list:
     """[x . W_i^T for W_i in ws]: weights that share the input x (same K), one decode launch for
@@ -306,8 +343,7 @@ def linear_group(x: torch.Tensor, ws: list, outs: list | None = None, workspace:
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    structs = [w.c_struct() for w in ws]
-    warr = (ctypes.c_void_p * len(ws))(*[ctypes.addressof(c) for c in structs])
+    warr = _weight_array(ws)
     yarr = (ctypes.c_void_p * len(ws))(*[o.data_ptr() for o in outs])
     pf = list(prefetch or [])
     pstructs = [w.c_struct() for w in pf]
