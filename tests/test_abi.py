@@ -266,3 +266,36 @@ def test_pack_host_validation(lib):
     assert lib.tern_pack_store(None, 4, 7, fake, None) == S["TERN_ERR_NULL"]
     assert lib.tern_unpack_store(fake, 4, -7, fake, None) == S["TERN_ERR_SHAPE"]
     assert lib.tern_weight_validate(None, None) == S["TERN_ERR_NULL"]
+
+
+def test_binding_caches_follow_the_weight(lib):
+    """The binding remembers a weight's C descriptor, its workspace sizes and a group's pointer
+    array; changing a field of the weight must give a fresh descriptor (host logic only: the
+    tensors stay on the host and no kernel runs)."""
+    import torch
+    from ternary_weight_only_tern_b200 import api
+
+    N, K = 64, 256
+
+    def weight():
+        return api.TernWeight(N, K, torch.zeros((N, K // 16), dtype=torch.int32),
+                              torch.zeros((N, K // 128), dtype=torch.float16),
+                              torch.zeros(0, dtype=torch.int32), torch.full((N,), -1, dtype=torch.int32),
+                              torch.zeros((0, K // 16), dtype=torch.int32),
+                              torch.zeros((0, K // 128), dtype=torch.float16))
+
+    w, v = weight(), weight()
+    c1 = w.c_struct()
+    assert c1 is w.c_struct() and c1.flags == 0
+    w.static = True
+    c2 = w.c_struct()
+    assert c2 is not c1 and c2.flags == _lib.WEIGHT_STATIC and c2.N == N and c2.K == K
+    assert api.workspace_bytes(w, 1) == lib.tern_linear_workspace_bytes(ctypes.byref(c2), 1)
+    assert 1 in w._ws
+    a1 = api._weight_array([w, v])
+    assert a1 is api._weight_array([w, v])
+    assert [a1[0], a1[1]] == [ctypes.addressof(w.c_struct()), ctypes.addressof(v.c_struct())]
+    v.static = True                       # a new descriptor for v: a new array
+    a2 = api._weight_array([w, v])
+    assert a2 is not a1 and a2[1] == ctypes.addressof(v.c_struct())
+    assert w._ws is not None and v._ws is None
