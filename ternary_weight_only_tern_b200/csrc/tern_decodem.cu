@@ -10,26 +10,30 @@
 //
 // Design: the pipeline of the one-token kernel (tern_decode1.cu) with the tokens as MMA columns.
 //  * Persistent grid, one CTA per SM, each CTA a contiguous range of 16-row strips walked as
-//    blocks of Sb = 8 (or 4) strips; a block streams through a ring of NS stages, each stage one
-//    (or two) 512-wide K slabs of the block's rows (3D TMA box, 128-byte swizzle, no multicast)
-//    and beside it the same K range of x for all tokens (a second box: 64 activations x M tokens
-//    x 8 slab chunks). Two producer warps issue the boxes, one more the blocks' scales.
-//  * Each of the 8 consumer warps takes one K group of every stage and four strips of the block,
-//    so the activations of a group (one B fragment set per 8 tokens, permuted in registers into
-//    the order of the decoded pairs) serve four strips. A decoded A fragment (16 rows x 16 K of
-//    trits, one LOP3 per pair of trits; tern_device.cuh) feeds one mma.sync m16n8k16 per 8
-//    tokens, so the decode costs the same for 2 and for 16 tokens. The call gives it 9 to 16
-//    tokens, and 8 tokens on launches of at least 10 strips per CTA; the cluster kernel of
-//    tern_gemv.cu was measured faster on the other calls up to 8 tokens.
+//    blocks of Sb strips; a block streams through a ring of NS stages, each stage one or two
+//    512-wide K slabs of the block's rows (3D TMA box, 128-byte swizzle, no multicast). x is
+//    either resident (all tokens copied once into shared memory, in pair order, each group's
+//    16-byte pieces stored transposed so that a quarter warp's loads hit eight bank groups) or,
+//    when it does not fit, streamed beside each stage as a second box (64 activations x M tokens
+//    x 8 slab chunks, permuted in registers). Two producer warps issue the boxes, one more the
+//    blocks' scales and the segment metadata, and an epilogue warp reduces the blocks.
+//  * Each of the 8 consumer warps takes one K group of every stage and two strips (four with one
+//    token block) of the block, so the activations of a group (one B fragment set per 8 tokens)
+//    serve every strip. A decoded A fragment (16 rows x 16 K of trits, one LOP3 per pair of
+//    trits; tern_device.cuh) feeds one mma.sync m16n8k16 per 8 tokens, so the decode costs the
+//    same for 2 and for 16 tokens. The call gives it 9 to 16 tokens, and 4 to 8 tokens on launches
+//    of at least 10 strips per CTA; the cluster kernel of tern_gemv.cu was measured faster on the
+//    other calls up to 8 tokens.
 //  * Lane (rr, q) of the D fragment holds rows rr and rr+8, tokens 2q and 2q+1; it scales each
 //    stage's sums by the row's group scale (after subtracting C = sum (B_p + 1) x of the group
-//    and token, computed once per kernel by the same MMA chain on the constant pattern, so a zero
-//    plane cancels bit for bit) into running sums held across the block's stages.
-//  * At the end of a block the warps leave their running sums in shared memory and, after a
-//    barrier of the consumer warps, add them per (row, token) in warp order: a main row without
-//    a residual row is rounded and written at once, the others wait in shared memory for their
-//    residual block (the segment's residual rows are the contiguous slots [s_a, s_a + span) of
-//    the residual plane, since R is sorted), which adds its sum and writes the row.
+//    and token, computed in the first block by the same MMA chain on the constant pattern, so a
+//    zero plane cancels bit for bit) into running sums held across the block's stages.
+//  * At the end of a block each consumer warp leaves its running sums in one of two partial-sum
+//    buffers (token rows padded to an odd length) and goes on; the epilogue warp adds them per
+//    (row, token) in warp order: a main row without a residual row is rounded and written at
+//    once, the others wait in shared memory for their residual block (the segment's residual
+//    rows are the contiguous slots [s_a, s_a + span) of the residual plane, since R is sorted),
+//    which adds its sum and writes the row. The consumers meet once, after the first block.
 //  * Programmatic dependent launch: the next kernel may launch at once; x is read and y written
 //    only after griddepcontrol.wait. Every wait is bounded and records TERN_ERR_TIMEOUT.
 #include <algorithm>
