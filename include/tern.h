@@ -81,7 +81,7 @@ typedef enum {
 } tern_status;
 
 /* A ternarized weight W [N, K] in execution form. Every pointer is device memory,
- * caller-owned, 16-byte aligned.                                                       */
+ * caller-owned, 16-byte aligned, except res_per_strip (host memory).                   */
 typedef struct {
     int64_t N, K;                /* output and input features; K % 128 == 0            */
     int32_t group;               /* scale group width along K; must be 128             */
@@ -103,6 +103,12 @@ typedef struct {
     const uint8_t* eidx;         /* [nnz2] listed trits, allocated to a multiple of 16 bytes */
     const tern_half* escale;     /* [N, K/128]  s2e                                     */
     int64_t nnz2;                /* number of listed trits                              */
+    /* HOST memory, optional (NULL: none): [ceil(N/16)] the number of residual rows among rows
+     * 16 j .. 16 j + 15, for each strip j. With it on every weight of a call that has residual
+     * rows, the decode launch splits its strips among the CTAs so that their main and residual
+     * blocks even out, instead of splitting the strips evenly (a planning hint read on the host
+     * during the call: the results do not depend on it).                                 */
+    const uint16_t* res_per_strip;
 } tern_weight;
 
 /* With an offset the weight is W[n, k] = mu[n, k/128] + s1[n, k/128] T1[n, k]

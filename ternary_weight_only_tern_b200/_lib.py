@@ -64,6 +64,7 @@ class TernWeightC(ctypes.Structure):
         ("mu", ctypes.c_void_p),
         ("ecount", ctypes.c_void_p), ("ebase", ctypes.c_void_p), ("eidx", ctypes.c_void_p),
         ("escale", ctypes.c_void_p), ("nnz2", ctypes.c_int64),
+        ("res_per_strip", ctypes.c_void_p),
     ]
 
 

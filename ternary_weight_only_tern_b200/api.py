@@ -165,6 +165,7 @@ class TernWeight:
     mu: torch.Tensor | None = None   # float16 [N, K/128] per-group offset: W = mu + s1 T1 (+ s2 T2)
     elem: ElemPlane | None = None    # element-level second plane (then r == 0)
     escale: torch.Tensor | None = None   # float16 [N, K/128] its scales s2e
+    res_hint: torch.Tensor | None = None  # host int16 [ceil(N/16)] residual rows per strip (a launch hint)
 
     @property
     def r(self) -> int:
@@ -189,7 +190,7 @@ class TernWeight:
                 self.res_rows.data_ptr() if self.r else None, self.res_slot.data_ptr(),
                 self.plane2.data_ptr() if self.r else None, self.scale2.data_ptr() if self.r else None,
                 _lib.WEIGHT_STATIC if self.static else 0, self.mu.data_ptr() if self.mu is not None else None,
-                *self._elem_fields())
+                *self._elem_fields(), self.res_hint.data_ptr() if self.res_hint is not None else None)
             object.__setattr__(self, "_c", c)
         return c
 
@@ -247,9 +248,12 @@ class TernWeight:
                 raise ValueError(f"s2e must have shape {(N, K // GROUP)}")
             elem = pack_elem(T2e.to(dev).contiguous())
             s2e = s2e.to(dev).contiguous()
+        # residual rows per 16-row strip, kept on the host for the decode launches' CTA split
+        hint = (torch.bincount(res_rows.long() // 16, minlength=(N + 15) // 16).to(torch.int16).cpu()
+                if r else None)
         return cls(N, K, pack_exec(T1), s1.contiguous(), res_rows, slot, plane2,
                    s2.contiguous() if r else torch.zeros((0, K // GROUP), dtype=torch.float16, device=dev), mu=mu,
-                   elem=elem, escale=s2e if elem is not None else None)
+                   elem=elem, escale=s2e if elem is not None else None, res_hint=hint)
 
     @classmethod
     def from_numpy(cls, T1, s1, res_rows, T2, s2, device="cuda", mu=None, T2e=None, s2e=None) -> "TernWeight":

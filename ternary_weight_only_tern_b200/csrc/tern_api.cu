@@ -6,11 +6,104 @@
 // M (prefill) runs the dequantise-into-tcgen05 GEMM. Both read the packed planes directly,
 // never a floating reconstruction of W (section 14: native kernels consume the ternary
 // planes; section 15: a lossless native kernel).
+#include <algorithm>
+#include <map>
 #include <mutex>
+#include <vector>
 
 #include "tern_internal.cuh"
 
 namespace tern {
+
+namespace {
+std::mutex g_plan_mu;
+std::map<std::vector<int64_t>, std::vector<int32_t>> g_plans;   // balanced splits by weights and plan
+constexpr size_t kMaxPlans = 4096;
+}  // namespace
+
+bool balanced_ranges(const tern_weight* const* ws, int nw, int64_t S, int64_t P, int Sb, int nstage,
+                     int seg_strips, int max_segs, int32_t* jb) {
+    bool any_res = false;
+    int64_t nstrips = 0;
+    for (int i = 0; i < nw; ++i) {
+        if (ws[i]->r > 0) {
+            if (!ws[i]->res_per_strip) return false;
+            any_res = true;
+        }
+        nstrips += (ws[i]->N + 15) / 16;
+    }
+    if (!any_res || P < 1 || P > kMaxBalancedGrid || nstrips != S || Sb < 1 || nstage < 1) return false;
+    std::vector<int64_t> key = {S, P, Sb, nstage, seg_strips, max_segs};
+    for (int i = 0; i < nw; ++i) {
+        key.push_back(int64_t(reinterpret_cast<uintptr_t>(ws[i]->plane1)));
+        key.push_back(int64_t(reinterpret_cast<uintptr_t>(ws[i]->res_per_strip)));
+        key.push_back(ws[i]->N);
+        key.push_back(ws[i]->r);
+    }
+    {
+        std::lock_guard<std::mutex> lock(g_plan_mu);
+        auto it = g_plans.find(key);
+        if (it != g_plans.end()) {
+            std::copy(it->second.begin(), it->second.end(), jb);
+            return true;
+        }
+    }
+    // every strip's weight and residual rows
+    std::vector<int32_t> wi(size_t(S), 0), rr(size_t(S), 0);
+    for (int i = 0, j = 0; i < nw; ++i)
+        for (int64_t t = 0; t < (ws[i]->N + 15) / 16; ++t, ++j) {
+            wi[size_t(j)] = i;
+            rr[size_t(j)] = ws[i]->r > 0 ? int32_t(ws[i]->res_per_strip[t]) : 0;
+        }
+    auto cdiv = [](int64_t a, int64_t b) { return (a + b - 1) / b; };
+    auto seg_cost = [&](int64_t nmain, int64_t rows) { return (cdiv(nmain, Sb) + cdiv(cdiv(rows, 16), Sb)) * nstage; };
+    // can P ranges of cost <= T each cover the strips? (greedy, the kernel's segmentation)
+    std::vector<int32_t> out(size_t(P) + 1);
+    auto fill = [&](int64_t T) -> bool {
+        int64_t start = 0;
+        for (int64_t b = 0; b < P; ++b) {
+            out[size_t(b)] = int32_t(start);
+            int64_t done = 0, segs = 0, seg0 = start, smain = 0, srows = 0, end = start;
+            while (end < S) {
+                const bool fresh = end == start || wi[size_t(end)] != wi[size_t(seg0)] || end - seg0 >= seg_strips;
+                int64_t d = done, ns = segs, s0 = seg0, m = smain, rws = srows;
+                if (fresh) {
+                    if (end > start) d += seg_cost(smain, srows);
+                    ++ns;
+                    s0 = end;
+                    m = 0;
+                    rws = 0;
+                }
+                ++m;
+                rws += rr[size_t(end)];
+                if (ns > max_segs || d + seg_cost(m, rws) > T) break;
+                done = d;
+                segs = ns;
+                seg0 = s0;
+                smain = m;
+                srows = rws;
+                ++end;
+            }
+            if (end == start && start < S) return false;
+            start = end;
+        }
+        out[size_t(P)] = int32_t(S);
+        return start >= S;
+    };
+    int64_t lo = 1, hi = int64_t(1) << 40;
+    if (!fill(hi)) return false;
+    while (lo < hi) {
+        const int64_t mid = lo + (hi - lo) / 2;
+        if (fill(mid)) hi = mid;
+        else lo = mid + 1;
+    }
+    if (!fill(lo)) return false;
+    std::copy(out.begin(), out.end(), jb);
+    std::lock_guard<std::mutex> lock(g_plan_mu);
+    if (g_plans.size() >= kMaxPlans) g_plans.clear();
+    g_plans.emplace(std::move(key), out);
+    return true;
+}
 
 int sm_count() {
     static std::mutex mu;

@@ -99,6 +99,10 @@ struct DMArgs {
     int64_t pf_bytes[kPfRanges];
     int64_t pf_per[kPfRanges];
     int32_t npf;
+    // the CTAs' strip ranges [jb[b], jb[b + 1]) when balanced by their residual strips (else
+    // an even split)
+    int32_t balanced;
+    int32_t jb[kMaxBalancedGrid + 1];
 };
 
 // Natural-order activations (nat[8h + i] = halves 16h + 2i, 16h + 2i + 1) into the order of the
@@ -168,11 +172,13 @@ __global__ void __launch_bounds__(kThreads, 1) decodem_kernel(const __grid_const
     grid_launch_dependents();
 
     const int P = gridDim.x, b = blockIdx.x;
-    // the CTA's strips [j0, j1) = [b S / P, (b + 1) S / P), in 32-bit arithmetic: the host keeps S
-    // below 2^24 and P is at most the SM count, so (b + 1) S fits (a 64-bit division here cost
-    // hundreds of cycles before the first copy of every launch)
+    // the CTA's strips [j0, j1): the host's split balanced by residual strips when it has one, else
+    // [b S / P, (b + 1) S / P) in 32-bit arithmetic (the host keeps S below 2^24 and P is at most
+    // the SM count, so (b + 1) S fits; a 64-bit division here cost hundreds of cycles before the
+    // first copy of every launch)
     const uint32_t uS = uint32_t(a.S), uP = uint32_t(P);
-    const int j0 = int(uint32_t(b) * uS / uP), j1 = int(uint32_t(b + 1) * uS / uP);
+    const int j0 = a.balanced ? a.jb[b] : int(uint32_t(b) * uS / uP);
+    const int j1 = a.balanced ? a.jb[b + 1] : int(uint32_t(b + 1) * uS / uP);
     volatile int* vabort = abort_flag;
     auto fail = [&]() {
         *vabort = 1;
@@ -861,6 +867,7 @@ tern_status decodem_launch_group(const tern_weight* const* ws, int nw, const __h
     a.has_mu = has_mu ? 1 : 0;
     a.stage_bytes = L.stage_bytes;
     a.sc_stride = L.sc_stride;
+    a.balanced = balanced_ranges(ws, nw, S, P, L.Sb, L.nstage, kSegStrips, kMaxSegs, a.jb) ? 1 : 0;
     a.o_sc = L.o_sc; a.o_mu = L.o_mu; a.o_red = L.o_red; a.o_cofs = L.o_cofs; a.o_xsum = L.o_xsum;
     a.o_meta = L.o_meta; a.o_bslot = L.o_bslot; a.o_rslot = L.o_rslot; a.o_mainy = L.o_mainy; a.o_bar = L.o_bar;
     a.o_xs = L.o_xs;

@@ -36,6 +36,16 @@ size_t gemv_workspace_bytes(const tern_weight& w, int64_t M);
 
 // Decode GEMV for one token on a persistent, warp-specialised grid (tern_decode1.cu): row-level
 // residual planes and offsets, K % 512 == 0; decode1_supported tells whether it takes the call.
+// The persistent decode kernels' split of a launch's S strips (the weights' strips in order)
+// among P CTAs, balanced by what each CTA walks: per segment (at most seg_strips strips of one
+// weight, starting at the CTA's first strip), ceil(main strips / Sb) + ceil(residual strips / Sb)
+// blocks of nstage stages, a segment's residual strips being ceil(its residual rows / 16); at
+// most max_segs segments per CTA. CTA b takes strips [jb[b], jb[b + 1]). False (the caller
+// splits evenly) when a weight with residual rows has no res_per_strip, no weight has residual
+// rows, or P > kMaxBalancedGrid. Cached per weights and plan.
+constexpr int kMaxBalancedGrid = 192;
+bool balanced_ranges(const tern_weight* const* ws, int nw, int64_t S, int64_t P, int Sb, int nstage,
+                     int seg_strips, int max_segs, int32_t* jb);
 constexpr int64_t kMaxLaunchStrips = int64_t(1) << 24;   // 16-row strips of one persistent decode launch
 bool decode1_supported(const tern_weight* const* ws, int nw);
 tern_status decode1_launch_group(const tern_weight* const* ws, int nw, const __half* x, __half* const* ys,

@@ -163,3 +163,40 @@ def test_graph_replay_with_new_inputs():
         g.replay()
         torch.cuda.synchronize()
         check(y.cpu().numpy(), oracle.linear(xn, t.T1, t.s1, t.res_rows, t.T2, t.s2))
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+@pytest.mark.parametrize("pct", [15, 100])
+def test_balanced_split_gives_the_same_bits(M, pct):
+    """A launch whose CTAs' strip ranges are balanced by the weights' residual rows per strip
+    (the host hint) computes every row in the same order as the even split: the outputs are
+    bit-identical, and within the bar against the oracle. Gate-and-up-like group of two weights
+    (11 strips per CTA), rows with residual rows bunched at one end."""
+    import dataclasses
+
+    rng = np.random.default_rng(300 + M + pct)
+    K = 2048
+    x = synth.draw_x(rng, M, K)
+    ts, hinted, plain = [], [], []
+    for i, N in enumerate((148 * 16 * 6, 148 * 16 * 5 + 7)):
+        t = synth.draw_tensor(rng, "bal", N, K, M, p_zero=0.4, res_pct=pct)
+        if pct < 100:   # residual rows bunched into the first third of the rows
+            r = t.res_rows.size
+            rows = np.sort(rng.choice(N // 3, size=min(r, N // 3), replace=False)).astype(np.int32)
+            T2 = synth.draw_trits(rng, (rows.size, K), p_zero=0.4)
+            s2 = synth.draw_scales(rng, rows.size, K, 0.001, 0.005)
+            t = synth.TernTensor("bal", N, K, x, t.T1, t.s1, rows, T2, s2)
+        else:
+            t = synth.TernTensor("bal", N, K, x, t.T1, t.s1, t.res_rows, t.T2, t.s2)
+        ts.append(t)
+        w = weight(t)
+        assert w.res_hint is not None and int(w.res_hint.sum()) == t.res_rows.size
+        hinted.append(w)
+        plain.append(dataclasses.replace(w, res_hint=None))
+    xt = torch.from_numpy(x).cuda()
+    ya = api.linear_group(xt, hinted)
+    yb = api.linear_group(xt, plain)
+    torch.cuda.synchronize()
+    for a, b, t in zip(ya, yb, ts):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+        check(a.cpu().numpy(), oracle.linear(x, t.T1, t.s1, t.res_rows, t.T2, t.s2))
