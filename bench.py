@@ -50,8 +50,8 @@ KERNEL_TRAFFIC = {
     "gemv": {"sources": ["ternary_weight_only_tern_b200/csrc/tern_decode1.cu",
                          "ternary_weight_only_tern_b200/csrc/tern_device.cuh",
                          "ternary_weight_only_tern_b200/csrc/tern_stream.cuh"],
-             "sha256": "8ba4c6d092030926afbdc55525a892640598107fda41a041f6aa1d780813045f",
-             "bytes": 30930176},
+             "sha256": "2559bec6f68d385a1ddbf6c0d83fe5b9282cc903381a1cc38ef912ea6aaba515",
+             "bytes": 30926848},
 }
 
 
