@@ -253,6 +253,20 @@ tern_status tern_linear_group(const tern_weight* const* w, int32_t n, const tern
                               tern_half* const* y, void* workspace, size_t workspace_bytes,
                               const tern_weight* const* next, int32_t n_next, tern_stream stream);
 
+/* The CTA split of the persistent decode launch that tern_linear_group(w, n, x, M, ...) makes
+ * (tern_linear: n = 1), for inspection and tests: CTA b walks the 16-row strips
+ * [ranges[b], ranges[b + 1]) of the weights' strips in order (weight i's after those of weights
+ * 0 .. i-1), in blocks of *strips_per_block strips of *stages_per_block stages (either pointer
+ * may be NULL). With res_per_strip on every weight that has residual rows the split is balanced
+ * by the blocks each CTA walks, else even. *n_ctas = 0 when that call runs no persistent decode
+ * kernel (M > 16, element planes, a 2-8-token launch the cluster kernel takes). ranges holds
+ * max_ctas + 1 entries; TERN_ERR_SHAPE when the launch needs more CTAs (its CTA count is the
+ * current device's SM count, 148 without a device). Host function: reads the descriptors and
+ * res_per_strip, no device memory; the weights' validity rules of tern_linear apply.       */
+tern_status tern_decode_ranges(const tern_weight* const* w, int32_t n, int64_t M, int32_t* ranges,
+                               int32_t max_ctas, int32_t* n_ctas, int32_t* strips_per_block,
+                               int32_t* stages_per_block);
+
 /* ---------------------------------------------------------------- activation rotation */
 
 /* y [M, K] = x [M, K] . blockdiag(R_0, ..., R_{G-1}) (x, y, R device, fp16, row-major): the

@@ -329,6 +329,18 @@ def _weight_array(ws: list):
     return hit[0]
 
 
+def decode_ranges(ws: list, M: int):
+    """(ranges, strips per block, stages per block) of the persistent decode launch that
+    linear_group(x [M, K], ws) makes, by tern_decode_ranges: CTA b takes strips
+    [ranges[b], ranges[b + 1]); ([], 0, 0) when the call runs no persistent decode kernel."""
+    cap = 1024
+    arr = (ctypes.c_int32 * (cap + 1))()
+    n, sb, ns = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int32(0)
+    _lib.check("tern_decode_ranges", _lib.load().tern_decode_ranges(
+        _weight_array(ws), len(ws), M, arr, cap, ctypes.byref(n), ctypes.byref(sb), ctypes.byref(ns)))
+    return (list(arr[: n.value + 1]) if n.value else []), sb.value, ns.value
+
+
 def linear_group(x: torch.Tensor, ws: list, outs: list | None = None, workspace: torch.Tensor | None = None,
                  prefetch: list | None = None) -> list:
     """[x . W_i^T for W_i in ws]: weights that share the input x (same K), one decode launch for

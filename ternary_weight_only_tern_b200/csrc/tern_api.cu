@@ -223,6 +223,28 @@ extern "C" tern_status tern_linear_group(const tern_weight* const* w, int32_t n,
     return linear_group(w, n, x, M, y, workspace, workspace_bytes, next, n_next, stream);
 }
 
+extern "C" tern_status tern_decode_ranges(const tern_weight* const* w, int32_t n, int64_t M, int32_t* ranges,
+                                          int32_t max_ctas, int32_t* n_ctas, int32_t* strips_per_block,
+                                          int32_t* stages_per_block) {
+    if (n < 1 || n > kMaxGemvGroup || max_ctas < 1) return TERN_ERR_SHAPE;
+    if (!w || !ranges || !n_ctas) return TERN_ERR_NULL;
+    for (int i = 0; i < n; ++i) {
+        const tern_status ws = check_weight(w[i]);
+        if (ws != TERN_OK) return ws;
+        if (w[i]->K != w[0]->K) return TERN_ERR_SHAPE;
+        if ((w[i]->ecount != nullptr) != (w[0]->ecount != nullptr)) return TERN_ERR_SHAPE;
+    }
+    if (M < 1 || M > (int64_t(1) << 31)) return TERN_ERR_SHAPE;
+    int Sb = 0, nstage = 0, P = 0;
+    if (M == 1 && decode1_supported(w, n)) P = decode1_ranges(w, n, ranges, max_ctas, Sb, nstage);
+    else if (M >= 2 && decodem_supported(w, n, M, nullptr)) P = decodem_ranges(w, n, M, ranges, max_ctas, Sb, nstage);
+    if (P < 0) return TERN_ERR_SHAPE;
+    *n_ctas = P;
+    if (strips_per_block) *strips_per_block = Sb;
+    if (stages_per_block) *stages_per_block = nstage;
+    return TERN_OK;
+}
+
 extern "C" tern_status tern_linear(const tern_weight* w, const tern_half* x, int64_t M, tern_half* y,
                                    void* workspace, size_t workspace_bytes, tern_stream stream) {
     if (!w) return TERN_ERR_NULL;

@@ -734,6 +734,20 @@ bool decode1_supported(const tern_weight* const* ws, int nw) {
     return make_layout(int(K), per, res, has_mu, L);
 }
 
+int decode1_ranges(const tern_weight* const* ws, int nw, int32_t* jb, int max_ctas, int& Sb, int& nstage) {
+    int64_t S, P, per, res;
+    launch_strips(ws, nw, S, P, per, res);
+    bool has_mu = false;
+    for (int i = 0; i < nw; ++i) has_mu = has_mu || ws[i]->mu != nullptr;
+    Layout L;
+    if (P > max_ctas || !make_layout(int(ws[0]->K), per, res, has_mu, L)) return -1;
+    Sb = L.Sb;
+    nstage = L.nstage;
+    if (!balanced_ranges(ws, nw, S, P, L.Sb, L.nstage, kSegStrips, kMaxSegs, jb))
+        for (int64_t b = 0; b <= P; ++b) jb[b] = int32_t(uint32_t(b) * uint32_t(S) / uint32_t(P));
+    return int(P);
+}
+
 tern_status decode1_launch_group(const tern_weight* const* ws, int nw, const __half* x, __half* const* ys,
                                  const tern_weight* const* next, int nnext, cudaStream_t stream) {
     D1Maps maps;

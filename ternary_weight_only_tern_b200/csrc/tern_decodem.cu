@@ -801,6 +801,21 @@ void strips_m(const tern_weight* const* ws, int nw, int64_t& S, int64_t& P, int6
 
 }  // namespace
 
+int decodem_ranges(const tern_weight* const* ws, int nw, int64_t M, int32_t* jb, int max_ctas, int& Sb,
+                   int& nstage) {
+    int64_t S, P, per, res;
+    strips_m(ws, nw, S, P, per, res);
+    bool has_mu = false;
+    for (int i = 0; i < nw; ++i) has_mu = has_mu || ws[i]->mu != nullptr;
+    LayoutM L;
+    if (P > max_ctas || !make_layout_m(int(ws[0]->K), int(M), per, res, has_mu, L)) return -1;
+    Sb = L.Sb;
+    nstage = L.nstage;
+    if (!balanced_ranges(ws, nw, S, P, L.Sb, L.nstage, kSegStrips, kMaxSegs, jb))
+        for (int64_t b = 0; b <= P; ++b) jb[b] = int32_t(uint32_t(b) * uint32_t(S) / uint32_t(P));
+    return int(P);
+}
+
 bool decodem_supported(const tern_weight* const* ws, int nw, int64_t M, const void* x) {
     const int64_t K = ws[0]->K;
     if (M < 2 || M > 16 || K % 512 != 0 || K / 512 > 4096 || !aligned16(x)) return false;

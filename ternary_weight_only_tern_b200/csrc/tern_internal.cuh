@@ -48,6 +48,9 @@ bool balanced_ranges(const tern_weight* const* ws, int nw, int64_t S, int64_t P,
                      int seg_strips, int max_segs, int32_t* jb);
 constexpr int64_t kMaxLaunchStrips = int64_t(1) << 24;   // 16-row strips of one persistent decode launch
 bool decode1_supported(const tern_weight* const* ws, int nw);
+// The CTA strip ranges (jb[0..P]) and plan (strips per block, stages per block) the one-token
+// launch would use; P, or -1 when P > max_ctas or there is no layout.
+int decode1_ranges(const tern_weight* const* ws, int nw, int32_t* jb, int max_ctas, int& Sb, int& nstage);
 tern_status decode1_launch_group(const tern_weight* const* ws, int nw, const __half* x, __half* const* ys,
                                  const tern_weight* const* next, int nnext, cudaStream_t stream);
 
@@ -58,6 +61,8 @@ constexpr int64_t kDecodemMinStrips = 10;  // below it, from kDecodemStripsMinM 
 constexpr int64_t kDecodemStripsMinM = 4;  // least kDecodemMinStrips strips per CTA (measured: at 4 tokens the
                                             // 8B stack 2239 against 2420 us per step, at 2 tokens 2095 against 2080)
 bool decodem_supported(const tern_weight* const* ws, int nw, int64_t M, const void* x);
+int decodem_ranges(const tern_weight* const* ws, int nw, int64_t M, int32_t* jb, int max_ctas, int& Sb,
+                   int& nstage);
 tern_status decodem_launch_group(const tern_weight* const* ws, int nw, const __half* x, int64_t M, __half* const* ys,
                                  const tern_weight* const* next, int nnext, cudaStream_t stream);
 

@@ -299,3 +299,68 @@ def test_binding_caches_follow_the_weight(lib):
     a2 = api._weight_array([w, v])
     assert a2 is not a1 and a2[1] == ctypes.addressof(v.c_struct())
     assert w._ws is not None and v._ws is None
+
+
+def _ranges_cost(ranges, strips, Sb, nstage, seg_strips=16):
+    """Per-CTA stages of a split, on the kernels' walk: each CTA's strips in segments (one weight,
+    at most seg_strips strips, from the CTA's first strip), each ceil(main / Sb) blocks of main
+    strips and ceil(ceil(residual rows / 16) / Sb) of residual strips, nstage stages a block.
+    strips: [(weight, residual rows)] of the launch in order. Also the segment counts."""
+    costs, segs = [], []
+    for a, b in zip(ranges[:-1], ranges[1:]):
+        c, ns, j = 0, 0, a
+        while j < b:
+            e = j
+            while e < b and strips[e][0] == strips[j][0] and e - j < seg_strips:
+                e += 1
+            rows = sum(strips[k][1] for k in range(j, e))
+            c += (-(-(e - j) // Sb) + -(-(-(-rows // 16)) // Sb)) * nstage
+            ns += 1
+            j = e
+        costs.append(c)
+        segs.append(ns)
+    return costs, segs
+
+
+def test_decode_ranges_balance_residual_strips(lib):
+    """tern_decode_ranges on host descriptors: without res_per_strip the even split
+    [b S / P, (b + 1) S / P); with it a split that covers every strip in order, keeps each CTA
+    within 8 segments, and whose slowest CTA walks no more stages than the even split's, strictly
+    fewer when the residual rows are bunched at one end (gate and up of the 8B model)."""
+    import dataclasses
+    import numpy as np
+    import torch
+    from ternary_weight_only_tern_b200 import api
+
+    N, K, r = 12288, 4096, 1843
+    rng = np.random.default_rng(11)
+    ws, strips = [], []
+    for i in range(2):
+        rows = np.sort(rng.choice(N // 3, size=r, replace=False)).astype(np.int32)   # the first third
+        slot = np.full(N, -1, np.int32)
+        slot[rows] = np.arange(r, dtype=np.int32)
+        hint = torch.from_numpy(np.bincount(rows // 16, minlength=N // 16).astype(np.int16))
+        ws.append(api.TernWeight(N, K, torch.zeros((N, K // 16), dtype=torch.int32),
+                                 torch.zeros((N, K // 128), dtype=torch.float16), torch.from_numpy(rows),
+                                 torch.from_numpy(slot), torch.zeros((r, K // 16), dtype=torch.int32),
+                                 torch.zeros((r, K // 128), dtype=torch.float16), res_hint=hint))
+        strips += [(i, int(c)) for c in hint.numpy()]
+    S = len(strips)
+    even, Sb, nst = api.decode_ranges([dataclasses.replace(w, res_hint=None) for w in ws], 1)
+    P = len(even) - 1
+    assert P >= 1 and Sb >= 1 and nst >= 1
+    assert even == [b * S // P for b in range(P + 1)]
+    bal, Sb2, nst2 = api.decode_ranges(ws, 1)
+    assert (Sb2, nst2) == (Sb, nst) and len(bal) == P + 1
+    assert bal[0] == 0 and bal[-1] == S and all(x <= y for x, y in zip(bal, bal[1:]))
+    ce, _ = _ranges_cost(even, strips, Sb, nst)
+    cb, segs = _ranges_cost(bal, strips, Sb, nst)
+    assert max(segs) <= 8
+    assert max(cb) < max(ce), (max(cb), max(ce))
+    # 16 tokens: the multi-token kernel's split, with its own plan
+    bal16, Sb16, nst16 = api.decode_ranges(ws, 16)
+    even16, _, _ = api.decode_ranges([dataclasses.replace(w, res_hint=None) for w in ws], 16)
+    assert bal16[0] == 0 and bal16[-1] == S and len(bal16) == len(even16)
+    assert max(_ranges_cost(bal16, strips, Sb16, nst16)[0]) <= max(_ranges_cost(even16, strips, Sb16, nst16)[0])
+    # no persistent decode launch past 16 tokens
+    assert api.decode_ranges(ws, 17) == ([], 0, 0)
