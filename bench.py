@@ -50,7 +50,7 @@ KERNEL_TRAFFIC = {
     "gemv": {"sources": ["ternary_weight_only_tern_b200/csrc/tern_decode1.cu",
                          "ternary_weight_only_tern_b200/csrc/tern_device.cuh",
                          "ternary_weight_only_tern_b200/csrc/tern_stream.cuh"],
-             "sha256": "2559bec6f68d385a1ddbf6c0d83fe5b9282cc903381a1cc38ef912ea6aaba515",
+             "sha256": "45639663d5e346da78ff1653b6cb8d1c2dd802c6cc8bfa78cc8171310daecdb6",
              "bytes": 30926848},
 }
 
