@@ -184,6 +184,12 @@ tern_status tern_unpack_elem(const uint8_t* ecount, const int32_t* ebase, const 
 tern_status tern_pack_residual(const int32_t* res_rows, int64_t r, int64_t N, int32_t* res_slot,
                                uint8_t* row_bitmap, tern_stream stream);
 
+/* tern_residual_strip_counts: res_rows [r] (HOST; strictly increasing, in [0, N)) -> counts
+ * [ceil(N/16)] (host): the residual rows among rows 16 j .. 16 j + 15 of each strip j, the
+ * tern_weight.res_per_strip hint. Rows out of range or not strictly increasing return
+ * TERN_ERR_RESIDUAL (counts then undefined). Host function.                                */
+tern_status tern_residual_strip_counts(const int32_t* res_rows, int64_t r, int64_t N, uint16_t* counts);
+
 /* tern_unpack_residual: row bitmap [ceil(N/8)] (device) -> *r = |R| (host), and, when not
  * NULL, res_rows [r] (device, capacity r_cap entries) in increasing order and res_slot [N]
  * (device). Call with res_rows == NULL to learn *r. A bit set past row N - 1 is not a row and

@@ -27,6 +27,7 @@ EXPORTS = {
     "tern_weight_validate": (_c.c_int, [_c.c_void_p, _c.c_void_p]),
     "tern_decode_ranges": (_c.c_int, [_c.c_void_p, _c.c_int32, _c.c_int64, _c.c_void_p, _c.c_int32, _c.c_void_p,
                                      _c.c_void_p, _c.c_void_p]),
+    "tern_residual_strip_counts": (_c.c_int, [_c.c_void_p, _c.c_int64, _c.c_int64, _c.c_void_p]),
     "tern_linear_workspace_bytes": (_c.c_size_t, [_c.c_void_p, _c.c_int64]),
     "tern_linear": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_int64, _c.c_void_p, _c.c_void_p, _c.c_size_t,
                                _c.c_void_p]),

@@ -248,9 +248,14 @@ class TernWeight:
                 raise ValueError(f"s2e must have shape {(N, K // GROUP)}")
             elem = pack_elem(T2e.to(dev).contiguous())
             s2e = s2e.to(dev).contiguous()
-        # residual rows per 16-row strip, kept on the host for the decode launches' CTA split
-        hint = (torch.bincount(res_rows.long() // 16, minlength=(N + 15) // 16).to(torch.int16).cpu()
-                if r else None)
+        # residual rows per 16-row strip (tern_residual_strip_counts), kept on the host for the decode
+        # launches' CTA split
+        hint = None
+        if r:
+            rows_h = res_rows.cpu()
+            hint = torch.zeros((N + 15) // 16, dtype=torch.int16)
+            _lib.check("tern_residual_strip_counts", _lib.load().tern_residual_strip_counts(
+                _ptr(rows_h), r, N, _ptr(hint)))
         return cls(N, K, pack_exec(T1), s1.contiguous(), res_rows, slot, plane2,
                    s2.contiguous() if r else torch.zeros((0, K // GROUP), dtype=torch.float16, device=dev), mu=mu,
                    elem=elem, escale=s2e if elem is not None else None, res_hint=hint)

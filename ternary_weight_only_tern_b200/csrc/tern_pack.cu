@@ -420,6 +420,19 @@ extern "C" int tern_debug_build(void) {
 #endif
 }
 
+extern "C" tern_status tern_residual_strip_counts(const int32_t* res_rows, int64_t r, int64_t N, uint16_t* counts) {
+    if (r < 0 || N < 0 || r > N) return TERN_ERR_SHAPE;
+    if ((r > 0 && !res_rows) || (N > 0 && !counts)) return TERN_ERR_NULL;
+    const int64_t strips = (N + 15) / 16;
+    for (int64_t j = 0; j < strips; ++j) counts[j] = 0;
+    for (int64_t i = 0; i < r; ++i) {
+        const int64_t n = res_rows[i];
+        if (n < 0 || n >= N || (i > 0 && n <= res_rows[i - 1])) return TERN_ERR_RESIDUAL;
+        ++counts[n / 16];
+    }
+    return TERN_OK;
+}
+
 extern "C" tern_status tern_pack_residual(const int32_t* res_rows, int64_t r, int64_t N, int32_t* res_slot,
                                           uint8_t* row_bitmap, tern_stream s) {
     if (N < 0 || r < 0 || r > N || N > (int64_t(1) << 31) - 1) return TERN_ERR_SHAPE;

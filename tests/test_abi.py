@@ -364,3 +364,22 @@ def test_decode_ranges_balance_residual_strips(lib):
     assert max(_ranges_cost(bal16, strips, Sb16, nst16)[0]) <= max(_ranges_cost(even16, strips, Sb16, nst16)[0])
     # no persistent decode launch past 16 tokens
     assert api.decode_ranges(ws, 17) == ([], 0, 0)
+
+
+def test_residual_strip_counts(lib):
+    """tern_residual_strip_counts equals a per-strip count of the residual rows (ragged N), and
+    rejects rows out of range or out of order."""
+    import numpy as np
+
+    rng = np.random.default_rng(5)
+    for N, r in ((1, 1), (17, 5), (1000 + 9, 150), (12288, 1843)):
+        rows = np.sort(rng.choice(N, size=r, replace=False)).astype(np.int32)
+        out = np.full((N + 15) // 16, 999, np.uint16)
+        st = lib.tern_residual_strip_counts(rows.ctypes.data_as(ctypes.c_void_p), r, N,
+                                            out.ctypes.data_as(ctypes.c_void_p))
+        assert st == 0
+        assert np.array_equal(out, np.bincount(rows // 16, minlength=(N + 15) // 16))
+    out = np.zeros(2, np.uint16)
+    for bad in (np.array([3, 3], np.int32), np.array([5, 2], np.int32), np.array([0, 20], np.int32)):
+        assert lib.tern_residual_strip_counts(bad.ctypes.data_as(ctypes.c_void_p), 2, 20,
+                                              out.ctypes.data_as(ctypes.c_void_p)) == 6   # TERN_ERR_RESIDUAL
