@@ -383,3 +383,37 @@ def test_residual_strip_counts(lib):
     for bad in (np.array([3, 3], np.int32), np.array([5, 2], np.int32), np.array([0, 20], np.int32)):
         assert lib.tern_residual_strip_counts(bad.ctypes.data_as(ctypes.c_void_p), 2, 20,
                                               out.ctypes.data_as(ctypes.c_void_p)) == 6   # TERN_ERR_RESIDUAL
+
+
+def test_decode_dispatch_rules(lib):
+    """Which decode kernel a call takes, seen through tern_decode_ranges (host descriptors): one
+    token and 9-16 tokens always run a persistent kernel; 4-8 tokens only on launches of at least
+    10 strips per CTA (the 8B gate and up as one launch), else, like 2-3 tokens, the cluster kernel
+    (no split); no persistent kernel past 16 tokens or with an element plane's weights."""
+    import torch
+    from ternary_weight_only_tern_b200 import api
+
+    def weight(N, K):
+        return api.TernWeight(N, K, torch.zeros((N, K // 16), dtype=torch.int32),
+                              torch.zeros((N, K // 128), dtype=torch.float16), torch.zeros(0, dtype=torch.int32),
+                              torch.full((N,), -1, dtype=torch.int32), torch.zeros((0, K // 16), dtype=torch.int32),
+                              torch.zeros((0, K // 128), dtype=torch.float16))
+
+    big = [weight(12288, 4096), weight(12288, 4096)]      # 1536 strips: 11 per CTA
+    small = [weight(4096, 4096)]                          # 256 strips: 2 per CTA
+    persistent = lambda ws, M: len(api.decode_ranges(ws, M)[0]) > 0  # noqa: E731
+    for M in (1, 9, 12, 16):
+        assert persistent(big, M) and persistent(small, M), M
+    for M in (4, 5, 8):
+        assert persistent(big, M) and not persistent(small, M), M
+    for M in (2, 3):
+        assert not persistent(big, M) and not persistent(small, M), M
+    assert not persistent(big, 17)
+    import dataclasses
+    N, K = 12288, 4096
+    G = K // 128
+    elem = api.ElemPlane(N, K, torch.zeros((G, N), dtype=torch.uint8), torch.zeros(G * (N // 64) + 1, dtype=torch.int32),
+                         torch.zeros(16, dtype=torch.uint8), 0)
+    ew = [dataclasses.replace(w, elem=elem, escale=torch.zeros((N, G), dtype=torch.float16)) for w in big]
+    for M in (1, 8, 16):
+        assert not persistent(ew, M), M
