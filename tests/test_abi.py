@@ -417,3 +417,50 @@ def test_decode_dispatch_rules(lib):
     ew = [dataclasses.replace(w, elem=elem, escale=torch.zeros((N, G), dtype=torch.float16)) for w in big]
     for M in (1, 8, 16):
         assert not persistent(ew, M), M
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_balanced_split_random_groups(lib, seed):
+    """Random groups of 1-4 weights (ragged N, 0-100 % residual rows, bunched or spread): the
+    balanced split covers every strip in order, keeps each CTA within 8 segments, and its slowest
+    CTA walks no more stages than the even split's, for one token and for 16."""
+    import dataclasses
+    import numpy as np
+    import torch
+    from ternary_weight_only_tern_b200 import api
+
+    rng = np.random.default_rng(100 + seed)
+    K = int(rng.choice([1024, 2048, 4096]))
+    ws, strips = [], []
+    for i in range(int(rng.integers(1, 5))):
+        N = int(rng.integers(1, 9000))
+        r = int(rng.integers(0, N + 1)) if rng.random() < 0.8 else 0
+        span = N if rng.random() < 0.5 else max(r, N // 4)
+        rows = np.sort(rng.choice(span, size=r, replace=False)).astype(np.int32)
+        slot = np.full(N, -1, np.int32)
+        slot[rows] = np.arange(r, dtype=np.int32)
+        hint = None
+        if r:
+            h = np.zeros((N + 15) // 16, np.uint16)
+            assert lib.tern_residual_strip_counts(rows.ctypes.data_as(ctypes.c_void_p), r, N,
+                                                  h.ctypes.data_as(ctypes.c_void_p)) == 0
+            hint = torch.from_numpy(h.astype(np.int16))
+        ws.append(api.TernWeight(N, K, torch.zeros((N, K // 16), dtype=torch.int32),
+                                 torch.zeros((N, K // 128), dtype=torch.float16), torch.from_numpy(rows),
+                                 torch.from_numpy(slot), torch.zeros((r, K // 16), dtype=torch.int32),
+                                 torch.zeros((r, K // 128), dtype=torch.float16), res_hint=hint))
+        counts = np.bincount(rows // 16, minlength=(N + 15) // 16) if r else np.zeros((N + 15) // 16, int)
+        strips += [(i, int(c)) for c in counts]
+    S = len(strips)
+    for M in (1, 16):
+        bal, Sb, nst = api.decode_ranges(ws, M)
+        even, _, _ = api.decode_ranges([dataclasses.replace(w, res_hint=None) for w in ws], M)
+        if not bal:
+            assert not even
+            continue
+        assert bal[0] == 0 and bal[-1] == S and len(bal) == len(even)
+        assert all(a <= b for a, b in zip(bal, bal[1:]))
+        cb, segs = _ranges_cost(bal, strips, Sb, nst)
+        ce, _ = _ranges_cost(even, strips, Sb, nst)
+        assert max(segs) <= 8
+        assert max(cb) <= max(ce), (M, max(cb), max(ce))
